@@ -1,0 +1,151 @@
+"""ctypes wrapper of the fp64 CPU oracle of the BlockFFN chunk layer.
+
+TEST INFRASTRUCTURE: only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg import this package.  The CUDA path never does.  ``build()`` compiles ``blockffn_oracle.cpp``
+with the host C++ compiler into ``liboracle.so`` beside it; importing rebuilds it when the source is
+newer than the library.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "blockffn_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle (g++ -O2, no fast-math: fp64 results follow IEEE rounding)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fPIC", "-shared", "-pthread",
+                               "-ffp-contract=off", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            lib = C.CDLL(_LIB)
+            p, i, dptr = C.c_void_p, C.c_int, C.c_void_p
+            lib.oracle_set_mutation.argtypes = [i]
+            lib.oracle_get_mutation.restype = i
+            lib.oracle_swish.argtypes = [C.c_double]
+            lib.oracle_swish.restype = C.c_double
+            lib.oracle_router.argtypes = [p, i, i, p, p, p, i, dptr, dptr, p]
+            lib.oracle_union.argtypes = [p, i, i, p, p, p, p]
+            lib.oracle_expert.argtypes = [p, i, p, p, i, i, dptr]
+            lib.oracle_chunk_forward.argtypes = [p, i, i, p, p, p, p, p, i, i, i, dptr, dptr, p]
+            lib.oracle_tokens_forward_mt.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, dptr]
+            for f in ("oracle_router", "oracle_union", "oracle_expert", "oracle_chunk_forward",
+                      "oracle_tokens_forward_mt"):
+                getattr(lib, f).restype = i
+            _lib = lib
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(C.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_mutation(m: int) -> None:
+    """Plant mistake number m in the oracle (0 restores the correct oracle). Tests only."""
+    _load().oracle_set_mutation(int(m))
+
+
+def swish(u: float) -> float:
+    return float(_load().oracle_swish(float(u)))
+
+
+def router(x, Wr, br, g):
+    """x bf16 bits [L,d]; returns s fp64 [L,E], r fp64 [L,E], active bool [L,E]."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    Wr, g = _c(Wr, np.float32), _c(g, np.float32)
+    br = _c(br, np.float32)
+    L, d = x.shape
+    E = Wr.shape[1]
+    s = np.zeros((L, E)); r = np.zeros((L, E)); act = np.zeros((L, E), np.uint8)
+    rc = lib.oracle_router(_ptr(x), L, d, _ptr(Wr), _ptr(br), _ptr(g), E, _ptr(s), _ptr(r), _ptr(act))
+    assert rc == 0
+    return s, r, act.astype(bool)
+
+
+def union(active):
+    """active bool [L,E] -> (active_idx int32 [n], tls_zero, cls_zero)."""
+    lib = _load()
+    act = np.ascontiguousarray(active, dtype=np.uint8)
+    L, E = act.shape
+    idx = np.zeros(E, np.int32); n = np.zeros(1, np.int32)
+    tz = np.zeros(1, np.int64); cz = np.zeros(1, np.int64)
+    rc = lib.oracle_union(_ptr(act), L, E, _ptr(idx), _ptr(n), _ptr(tz), _ptr(cz))
+    assert rc == 0
+    return idx[: n[0]].copy(), int(tz[0]), int(cz[0])
+
+
+def expert(xt, W1, W2, i):
+    lib = _load()
+    xt = _c(xt, np.uint16); W1 = _c(W1, np.uint16); W2 = _c(W2, np.uint16)
+    E, de, d = W1.shape
+    out = np.zeros(d)
+    rc = lib.oracle_expert(_ptr(xt), d, _ptr(W1), _ptr(W2), de, int(i), _ptr(out))
+    assert rc == 0
+    return out
+
+
+def chunk_forward(x, Wr, br, g, W1, W2, sparse: bool = False):
+    """Full layer over one chunk -> (y fp64 [L,d], r fp64 [L,E], active bool [L,E])."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    Wr, g, br = _c(Wr, np.float32), _c(g, np.float32), _c(br, np.float32)
+    W1, W2 = _c(W1, np.uint16), _c(W2, np.uint16)
+    L, d = x.shape
+    E, de, _ = W1.shape
+    y = np.zeros((L, d)); r = np.zeros((L, E)); act = np.zeros((L, E), np.uint8)
+    rc = lib.oracle_chunk_forward(_ptr(x), L, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1), _ptr(W2),
+                                  E, de, int(bool(sparse)), _ptr(y), _ptr(r), _ptr(act))
+    assert rc == 0
+    return y, r, act.astype(bool)
+
+
+def tokens_forward_mt(x, Wr, br, g, W1, W2, threads: int, sparse: bool = False):
+    """Layer over n tokens [n,d] on `threads` host threads -> y fp64 [n,d]."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    Wr, g, br = _c(Wr, np.float32), _c(g, np.float32), _c(br, np.float32)
+    W1, W2 = _c(W1, np.uint16), _c(W2, np.uint16)
+    n, d = x.shape
+    E, de, _ = W1.shape
+    y = np.zeros((n, d))
+    rc = lib.oracle_tokens_forward_mt(_ptr(x), n, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1),
+                                      _ptr(W2), E, de, int(bool(sparse)), int(threads), _ptr(y))
+    assert rc == 0
+    return y
+
+
+def chunk_reference(x, Wr, br, g, W1, W2):
+    """Everything a parity test compares for one chunk: y, r, active flags, union and counts."""
+    y, r, act = chunk_forward(x, Wr, br, g, W1, W2, sparse=True)
+    idx, tz, cz = union(act)
+    return {"y": y, "r": r, "active": act, "active_idx": idx, "tls_zero": tz, "cls_zero": cz}
+
+
+def available_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1

@@ -1,0 +1,205 @@
+// BlockFFN chunk-layer oracle: plain, slow, fp64, on the CPU.
+//
+// TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the benchmark's CPU-baseline
+// leg may load this library. It shares no code, header, table or helper with the CUDA path; the
+// two meet only through the seeded input generator.
+//
+// What it computes, per token t of a chunk of L consecutive tokens (the BlockFFN layer as the
+// pages describe it; the pages print no equations, so each step names the passage it restates):
+//   s_{t,i} = sum_k x_{t,k} Wr[k,i] + b_i                     router projection
+//   a_{t,i} = max(s_{t,i}, 0)                                 ReLU  (lsdiaocha.cn BlockFFN article, section 2:
+//                                                             the router combines a ReLU activation with an RMSNorm layer)
+//   r_{t,i} = g_i a_{t,i} / sqrt((1/E) sum_i a_{t,i}^2)       RMSNorm over the E router outputs (same
+//                                                             passage, and the BlockFFN abstract, which names a
+//                                                             router built from ReLU followed by RMSNorm); r_t = 0
+//                                                             when every a is 0
+//   E_i(x) = W2_i Swish(W1_i x), Swish(u) = u / (1 + e^-u)    non-gated MLP expert with Swish (article, section 2)
+//   y_t = sum_i r_{t,i} E_i(x_t)                              router-weighted combination; the mask of
+//                                                             section 4 removes the terms with r = 0
+// Active sets: A_t = {i : s_{t,i} > 0}; the chunk's union U = U_t A_t (article, section 4: the union of
+// the experts the candidate tokens activate); token-level sparsity counts the (t,i) with i not in A_t,
+// chunk-level sparsity counts the experts outside U (article, section 1; BlockFFN abstract).
+//
+// Readings where the pages are silent: RMSNorm has no epsilon (a token with no active expert gets
+// r = 0 and y = 0); Swish has beta = 1; the RMSNorm mean runs over all E entries, zeros included;
+// the union is listed in ascending expert order.
+//
+// Storage: x is bf16 bit patterns [L,d]; Wr fp32 [d,E]; br fp32 [E] (may be null = no bias);
+// g fp32 [E]; W1 bf16 bits [E,de,d]; W2 bf16 bits [E,d,de]; everything row-major.
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+namespace {
+
+// Planted mistakes, used only by the tests that check each pin can fail (0 = the correct oracle).
+int g_mutation = 0;
+
+double widen_bf16(uint16_t bits) {
+  uint32_t u = static_cast<uint32_t>(bits) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return static_cast<double>(f);
+}
+
+double swish(double u) {
+  if (g_mutation == 2) return u / (1.0 + std::exp(u));  // planted: wrong sign in the sigmoid
+  return u / (1.0 + std::exp(-u));
+}
+
+// Router for one token: s (pre-activation), r (normalised weights), active flags.
+void router_token(const uint16_t* xt, int d, const float* Wr, const float* br, const float* g,
+                  int E, double* s, double* r, uint8_t* act) {
+  for (int i = 0; i < E; ++i) {
+    double acc = 0.0;
+    for (int k = 0; k < d; ++k) {
+      int kk = (g_mutation == 4) ? (d - 1 - k) : k;  // planted: reversed router input index
+      acc += widen_bf16(xt[kk]) * static_cast<double>(Wr[static_cast<size_t>(k) * E + i]);
+    }
+    if (br != nullptr && g_mutation != 1) acc += static_cast<double>(br[i]);  // planted 1: bias dropped
+    s[i] = acc;
+  }
+  double sumsq = 0.0;
+  int n_pos = 0;
+  for (int i = 0; i < E; ++i) {
+    double a = s[i] > 0.0 ? s[i] : 0.0;
+    sumsq += a * a;
+    if (a > 0.0) ++n_pos;
+  }
+  // planted 3: mean over the active entries only instead of over all E
+  double denom = (g_mutation == 3) ? static_cast<double>(n_pos > 0 ? n_pos : 1) : static_cast<double>(E);
+  double ms = sumsq / denom;
+  for (int i = 0; i < E; ++i) {
+    double a = s[i] > 0.0 ? s[i] : 0.0;
+    act[i] = s[i] > 0.0 ? 1 : 0;
+    r[i] = (ms > 0.0) ? static_cast<double>(g[i]) * a / std::sqrt(ms) : 0.0;
+  }
+}
+
+// One expert applied to one token: out[d] = W2_i Swish(W1_i x_t).
+void expert_token(const uint16_t* xt, int d, const uint16_t* W1, const uint16_t* W2, int de, int i,
+                  double* out) {
+  std::vector<double> h(de);
+  const uint16_t* W1i = W1 + static_cast<size_t>(i) * de * d;
+  const uint16_t* W2i = W2 + static_cast<size_t>(i) * d * de;
+  for (int j = 0; j < de; ++j) {
+    double u = 0.0;
+    for (int k = 0; k < d; ++k) u += widen_bf16(W1i[static_cast<size_t>(j) * d + k]) * widen_bf16(xt[k]);
+    h[j] = swish(u);
+  }
+  for (int k = 0; k < d; ++k) {
+    double acc = 0.0;
+    for (int j = 0; j < de; ++j) {
+      // planted 5: W2 read as if it were stored [de, d]
+      size_t idx = (g_mutation == 5) ? static_cast<size_t>(j) * d + k : static_cast<size_t>(k) * de + j;
+      acc += widen_bf16(W2i[idx]) * h[j];
+    }
+    out[k] = acc;
+  }
+}
+
+void forward_tokens(int t0, int t1, const uint16_t* x, int d, const float* Wr, const float* br,
+                    const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de, int sparse,
+                    double* y, double* r_out, uint8_t* act_out) {
+  std::vector<double> s(E), r(E), e(d);
+  std::vector<uint8_t> act(E);
+  for (int t = t0; t < t1; ++t) {
+    const uint16_t* xt = x + static_cast<size_t>(t) * d;
+    router_token(xt, d, Wr, br, g, E, s.data(), r.data(), act.data());
+    double* yt = y + static_cast<size_t>(t) * d;
+    for (int k = 0; k < d; ++k) yt[k] = 0.0;
+    for (int i = 0; i < E; ++i) {
+      if (sparse && !act[i]) continue;  // sparse evaluation: only experts in A_t
+      expert_token(xt, d, W1, W2, de, i, e.data());
+      for (int k = 0; k < d; ++k) yt[k] += r[i] * e[k];
+    }
+    if (r_out) for (int i = 0; i < E; ++i) r_out[static_cast<size_t>(t) * E + i] = r[i];
+    if (act_out) for (int i = 0; i < E; ++i) act_out[static_cast<size_t>(t) * E + i] = act[i];
+  }
+}
+
+bool bad_dims(int L, int d, int E, int de) { return L < 0 || d <= 0 || E <= 0 || de <= 0; }
+
+}  // namespace
+
+extern "C" {
+
+void oracle_set_mutation(int m) { g_mutation = m; }
+int oracle_get_mutation(void) { return g_mutation; }
+
+double oracle_swish(double u) { return swish(u); }
+
+// Router over a chunk: s, r as fp64 [L,E]; act as 0/1 bytes [L,E].
+int oracle_router(const uint16_t* x, int L, int d, const float* Wr, const float* br, const float* g,
+                  int E, double* s, double* r, uint8_t* act) {
+  if (bad_dims(L, d, E, 1)) return 1;
+  for (int t = 0; t < L; ++t)
+    router_token(x + static_cast<size_t>(t) * d, d, Wr, br, g, E, s + static_cast<size_t>(t) * E,
+                 r + static_cast<size_t>(t) * E, act + static_cast<size_t>(t) * E);
+  return 0;
+}
+
+// Chunk union and sparsity counts from the per-token active flags.
+//   active_idx: the experts of U in ascending order (first n_active entries written)
+//   tls_zero  : number of (t,i) with i not in A_t
+//   cls_zero  : number of experts not in U
+int oracle_union(const uint8_t* act, int L, int E, int32_t* active_idx, int32_t* n_active,
+                 int64_t* tls_zero, int64_t* cls_zero) {
+  if (bad_dims(L, 1, E, 1)) return 1;
+  int64_t zeros = 0;
+  int n = 0;
+  for (int i = 0; i < E; ++i) {
+    bool any = false;
+    for (int t = 0; t < L; ++t) {
+      if (act[static_cast<size_t>(t) * E + i]) any = true;
+      else ++zeros;
+    }
+    if (g_mutation == 6 && i == E - 1) any = false;  // planted: last expert never joins the union
+    if (any) active_idx[n++] = i;
+  }
+  *n_active = n;
+  if (tls_zero) *tls_zero = zeros;
+  if (cls_zero) *cls_zero = E - n;
+  return 0;
+}
+
+// One expert on one token (exposed for the special-case pins).
+int oracle_expert(const uint16_t* xt, int d, const uint16_t* W1, const uint16_t* W2, int de, int i,
+                  double* out) {
+  if (bad_dims(1, d, 1, de) || i < 0) return 1;
+  expert_token(xt, d, W1, W2, de, i, out);
+  return 0;
+}
+
+// Full layer over one chunk. sparse=0: every expert is evaluated and multiplied by its router
+// weight (zero for inactive experts); sparse=1: only the experts of A_t are evaluated.
+// y fp64 [L,d]; r_out fp64 [L,E] and act_out [L,E] may be null.
+int oracle_chunk_forward(const uint16_t* x, int L, int d, const float* Wr, const float* br,
+                         const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de,
+                         int sparse, double* y, double* r_out, uint8_t* act_out) {
+  if (bad_dims(L, d, E, de)) return 1;
+  forward_tokens(0, L, x, d, Wr, br, g, W1, W2, E, de, sparse, y, r_out, act_out);
+  return 0;
+}
+
+// The same over n_tok tokens split across `threads` host threads (tokens are independent, so the
+// result is identical to the single-threaded call). Used for the timed CPU baseline.
+int oracle_tokens_forward_mt(const uint16_t* x, int n_tok, int d, const float* Wr, const float* br,
+                             const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de,
+                             int sparse, int threads, double* y) {
+  if (bad_dims(n_tok, d, E, de) || threads < 1) return 1;
+  std::vector<std::thread> pool;
+  for (int w = 0; w < threads; ++w) {
+    int t0 = static_cast<int>(static_cast<int64_t>(n_tok) * w / threads);
+    int t1 = static_cast<int>(static_cast<int64_t>(n_tok) * (w + 1) / threads);
+    pool.emplace_back(forward_tokens, t0, t1, x, d, Wr, br, g, W1, W2, E, de, sparse, y,
+                      static_cast<double*>(nullptr), static_cast<uint8_t*>(nullptr));
+  }
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+}  // extern "C"
