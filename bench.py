@@ -1,0 +1,434 @@
+"""Benchmark of the BlockFFN chunk-layer forward on B200.
+
+One step = one pass of the hot path over one batch of synthetic input: `chunks` sequential chunk
+forwards (router + chunk union + sparse experts, two kernels per chunk) through the C ABI, chunk c
+using weight replica c % replicas.  The replicas stand for distinct layers of a stacked model and keep
+the weights (16 x 128 MiB for the default workload) well above the 126 MB L2, so every chunk streams
+its active experts from HBM ("inputs larger than L2").  A step is captured once into a CUDA graph
+and replayed; time is taken with CUDA events on the replay stream, with a barrier and a
+synchronize on both sides, max over ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode] [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the reference implementation of this build) on the
+host cores on a bounded sample of the same workload.  Multi-GPU runs (torchrun) shard chunks across
+ranks with no collective in the data path (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BlockFFN layer tokens/s at chunk L=8 and achieved HBM GB/s over active bytes"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ---------------------------------------------------------------------------------- helpers
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def shard_seed(seed: int, rank: int) -> int:
+    """Chunk stream of a rank: every rank draws its own chunks (weak scaling)."""
+    return seed * 1000003 + rank
+
+
+def reduce_max(value: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "chunk_sparse_moe_router_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """DRAM bytes per chunk from the committed ncu summary, only if the kernels are unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        rec = j.get(workload_name)
+        if rec and rec.get("kernel_source_hash") == kernel_source_hash():
+            return float(rec["dram_bytes_per_chunk"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bffn_clocks_{os.getpid()}_{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.fh,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i].lower() == "active"})
+        pw = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------------------------- workload
+def active_bytes(d, E, de, L, n_active):
+    """Algorithmic bytes of one chunk: router weights, gain and bias, x in, y out, and W1_i + W2_i of
+    every expert in the chunk's union (bf16)."""
+    return 4 * d * E + 4 * E * 2 + 2 * L * d + 4 * L * d + n_active * (2 * d * de * 2)
+
+
+def build_inputs(w, rank, device, chunks):
+    import numpy as np
+    import torch
+
+    import gen
+
+    def bf16(a):
+        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
+
+    layers = []
+    host_x = []
+    per = (chunks + w.replicas - 1) // w.replicas
+    for r in range(w.replicas):
+        lay = w.layer(r)
+        layers.append({
+            "lay": lay,
+            "Wr": torch.from_numpy(lay.Wr).to(device), "br": torch.from_numpy(lay.br).to(device),
+            "g": torch.from_numpy(lay.g).to(device), "W1": bf16(lay.W1), "W2": bf16(lay.W2)})
+        host_x.append(gen.make_chunks(shard_seed(w.seed, rank), lay, per, w.L, w.noise, stream=r))
+    # chunk c -> replica c % R, position c // R within that replica's stream
+    x_all = np.empty((chunks, w.L, w.d), dtype=np.uint16)
+    for c in range(chunks):
+        x_all[c] = host_x[c % w.replicas][c // w.replicas]
+    return layers, x_all
+
+
+# ---------------------------------------------------------------------------------- our arm
+def run_ours(args, w):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import chunk_sparse_moe_router_b200 as bffn
+
+    world, rank, local = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=device,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    chunks = args.chunks or w.n_chunks
+    t_gen = time.time()
+    layers, x_host_np = build_inputs(w, rank, device, chunks)
+    gen_s = time.time() - t_gen
+    L, d, E, de = w.L, w.d, w.E, w.de
+    x_dev = torch.from_numpy(x_host_np.view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((chunks, L, d), dtype=torch.float32, device=device)
+    idx = torch.empty((chunks, E), dtype=torch.int32, device=device)
+    nact = torch.empty((chunks, 4), dtype=torch.int32, device=device)  # [c, 0] used
+
+    def step(stream_handle):
+        for c in range(chunks):
+            lay = layers[c % w.replicas]
+            rc = bffn.blockffn_chunk_forward_ex(
+                x_dev[c].data_ptr(), L, d, lay["Wr"].data_ptr(), lay["g"].data_ptr(), lay["W1"].data_ptr(),
+                lay["W2"].data_ptr(), E, de, y[c].data_ptr(), idx[c].data_ptr(), nact[c].data_ptr(),
+                lay["br"].data_ptr(), None, None, None, 0, None, 0, stream_handle)
+            if rc != 0:
+                raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_ex")
+
+    s = torch.cuda.Stream(device)
+    with torch.cuda.stream(s):
+        step(s.cuda_stream)  # first call allocates the library workspace (before capture)
+        s.synchronize()
+        if bffn.device_status(stream=s.cuda_stream) != 0:
+            raise RuntimeError("device-side wait ran out")
+        graph = torch.cuda.CUDAGraph()
+        graph.capture_begin()
+        step(s.cuda_stream)
+        graph.capture_end()
+        s.synchronize()
+        for _ in range(args.warmup):
+            graph.replay()
+        s.synchronize()
+
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        with ClockSampler(local) as clk:
+            e0.record(s)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(s)
+            e1.synchronize()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        t_ms = e0.elapsed_time(e1)
+        if bffn.device_status(stream=s.cuda_stream) != 0:
+            raise RuntimeError("device-side wait ran out during the timed region")
+
+        # end to end: x from pinned host memory in, y and the active sets back, every step
+        x_pin = torch.from_numpy(x_host_np.view(np.int16)).pin_memory()
+        y_pin = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        idx_pin = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+        n_pin = torch.empty(nact.shape, dtype=nact.dtype).pin_memory()
+        x_dev_i16 = x_dev.view(torch.int16)
+
+        def e2e_step():
+            x_dev_i16.copy_(x_pin, non_blocking=True)
+            graph.replay()
+            y_pin.copy_(y, non_blocking=True)
+            idx_pin.copy_(idx, non_blocking=True)
+            n_pin.copy_(nact, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        s.synchronize()
+        barrier(device)
+        torch.cuda.synchronize(device)
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(3, args.steps // 2)
+        f0.record(s)
+        for _ in range(e2e_steps):
+            e2e_step()
+        f1.record(s)
+        f1.synchronize()
+        barrier(device)
+        e2e_ms = f0.elapsed_time(f1)
+
+    t_max = reduce_max(t_ms, device)
+    e2e_max = reduce_max(e2e_ms, device)
+    n_act_host = nact[:, 0].cpu().numpy()
+    total_active = float(sum(active_bytes(d, E, de, L, int(n)) for n in n_act_host))
+    ms_per_step = t_max / args.steps
+    tokens_step = chunks * L * world
+    value = tokens_step / (ms_per_step * 1e-3)
+    achieved_gbs = total_active / (ms_per_step * 1e-3) / 1e9  # per GPU: every rank streams its own
+    peak, peak_kind = measured_peaks()
+    traffic = recorded_traffic(w.name)
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {**w.describe(), "chunks_per_step": chunks,
+                   "l2": f"inputs larger than L2: {w.replicas} weight replicas, "
+                         f"{w.replicas * E * 2 * d * de * 2 / 1e9:.2f} GB of expert weights",
+                   "mean_n_active": round(float(n_act_host.mean()), 3),
+                   "cls": round(1.0 - float(n_act_host.mean()) / E, 4),
+                   "parallelism": f"dp{world} (chunks sharded, no collective in the data path)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind,
+                     "kernel": "one chunk forward (router kernel + expert kernel, PDL-chained)",
+                     "bytes_per_chunk": round(total_active / chunks, 1),
+                     "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3),
+                     "traffic": None if traffic is None else round(traffic, 1)},
+        "e2e": {"value": round(tokens_step / (e2e_max / e2e_steps * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": int(x_host_np.nbytes),
+                "d2h_bytes_per_step": int(y.numel() * 4 + idx.numel() * 4 + nact.numel() * 4),
+                "steps": e2e_steps},
+        "gpu_launches": 2 * chunks * args.steps,
+        "clocks": clk.summary(),
+        "gen_seconds": round(gen_s, 1),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, layers[0]["lay"], x_host_np, args.cpu_seconds,
+                                           y_gpu=y, n_gpu=n_act_host)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del graph
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
+    """The fp64 dense oracle timed on this host's cores on a bounded sample of the workload (chunks
+    of replica 0).  Also checks that sample against the GPU's output when one is given."""
+    import numpy as np
+
+    import oracle
+
+    cores = oracle.available_cores()
+    L, d = w.L, w.d
+    chunk_ids = list(range(0, x_host_np.shape[0], w.replicas))  # chunks that use replica 0
+    # calibrate on one chunk, then size the sample to about `seconds`
+    t0 = time.time()
+    oracle.tokens_forward_mt(x_host_np[chunk_ids[0]], lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
+    t1 = time.time() - t0
+    n_chunks = max(1, min(len(chunk_ids), int(seconds / max(t1, 1e-6))))
+    xs = x_host_np[chunk_ids[:n_chunks]].reshape(n_chunks * L, d)
+    t0 = time.time()
+    y_ref = oracle.tokens_forward_mt(xs, lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
+    dt = time.time() - t0
+    res = {"value": round(n_chunks * L / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{n_chunks} chunks x {L} tokens of weight replica 0 "
+                     f"(dense fp64: all {w.E} experts per token), {dt:.1f} s"}
+    if y_gpu is not None:
+        yg = y_gpu[chunk_ids[:n_chunks]].cpu().numpy().reshape(n_chunks * L, d).astype(np.float64)
+        bad = 0
+        for c in range(n_chunks):
+            yr = y_ref[c * L:(c + 1) * L]
+            bound = 2e-2 * np.abs(yr) + 1e-3 * np.sqrt(np.mean(yr ** 2))
+            bad += int((np.abs(yg[c * L:(c + 1) * L] - yr) > bound).sum())
+        res["parity_sample"] = {"y_elements_out_of_tolerance": bad, "elements": int(yg.size)}
+    return res
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    import numpy as np
+
+    import gen
+    import oracle
+
+    lay = w.layer(0)
+    L = w.L
+    cores = oracle.available_cores()
+    per_step_chunks = max(1, args.ref_chunks)
+    x = gen.make_chunks(w.seed, lay, per_step_chunks, L, w.noise, stream=0)
+    xs = x.reshape(per_step_chunks * L, w.d)
+    oracle.tokens_forward_mt(xs[:L], lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores)  # warm-up
+    t0 = time.time()
+    for _ in range(args.steps):
+        oracle.tokens_forward_mt(xs, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores)
+    dt = time.time() - t0
+    value = args.steps * per_step_chunks * L / dt
+    sample = (f"each step: {per_step_chunks} chunk(s) x {L} tokens of the workload, dense fp64 oracle "
+              f"(all {w.E} experts per token)")
+    out = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "impl": "reference",
+           "config": {**w.describe(), "chunks_per_step": per_step_chunks},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="decode", choices=["decode", "tiny", "lsweep", "tls_sweep"])
+    ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
+    ap.add_argument("--tls", type=float, default=None, help="token-level sparsity for --workload tls_sweep")
+    ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-chunks", type=int, default=1)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    import gen
+
+    kw = {}
+    if args.workload == "lsweep" and args.L:
+        kw["L"] = args.L
+    if args.workload == "tls_sweep" and args.tls:
+        kw["tls"] = args.tls
+    w = gen.workload(args.workload, **kw)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

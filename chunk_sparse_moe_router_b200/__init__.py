@@ -1,0 +1,155 @@
+"""Python binding of the BlockFFN chunk-layer C ABI (include/blockffn.h).
+
+The functions named like the C entry points take plain integers (device pointers, sizes, a
+cudaStream_t handle) and only marshal arguments; every step of the layer runs in the CUDA kernels of
+libblockffn.so.  `chunk_forward` is the same call taking torch CUDA tensors (it checks dtypes,
+shapes, devices and contiguity, then passes data pointers).  Importing this package fails loudly when
+the extension has not been built: there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libblockffn.so")
+
+BFFN_OK, BFFN_EINVAL, BFFN_ECUDA, BFFN_ENOMEM, BFFN_ETIMEOUT, BFFN_EUNSUPPORTED = range(6)
+BFFN_PATH_AUTO, BFFN_PATH_DECODE, BFFN_PATH_PREFILL = 0, 1, 2
+
+# Every symbol include/blockffn.h declares: name -> (restype, argtypes)
+_P, _I, _S = C.c_void_p, C.c_int, C.c_size_t
+SIGNATURES = {
+    "blockffn_chunk_forward": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
+    "blockffn_chunk_forward_ex": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P,
+                                       _P, _I, _P, _S, _P]),
+    "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
+    "blockffn_workspace_init": (_I, [_P, _S, _P]),
+    "blockffn_device_status": (_I, [_P, _P]),
+    "blockffn_status_string": (C.c_char_p, [_I]),
+    "blockffn_abi_version": (_I, []),
+}
+
+
+class BlockFFNError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build the CUDA extension first "
+            "(python -c 'import __graft_entry__ as g; g.build()'); there is no fallback path")
+    lib = C.CDLL(LIB_PATH)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+# ------------------------------------------------------------------- C entry points, same names
+def blockffn_chunk_forward(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, stream):
+    return _lib.blockffn_chunk_forward(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, stream)
+
+
+def blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask,
+                              counts, r_out, flags, workspace, workspace_bytes, stream):
+    return _lib.blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br,
+                                          tok_mask, counts, r_out, flags, workspace, workspace_bytes,
+                                          stream)
+
+
+def blockffn_workspace_size(L, d, E, de):
+    return _lib.blockffn_workspace_size(L, d, E, de)
+
+
+def blockffn_workspace_init(workspace, workspace_bytes, stream):
+    return _lib.blockffn_workspace_init(workspace, workspace_bytes, stream)
+
+
+def blockffn_device_status(workspace, stream):
+    return _lib.blockffn_device_status(workspace, stream)
+
+
+def blockffn_status_string(status):
+    return _lib.blockffn_status_string(status).decode()
+
+
+def blockffn_abi_version():
+    return _lib.blockffn_abi_version()
+
+
+status_string = blockffn_status_string
+
+
+# ------------------------------------------------------------------- torch-tensor marshalling
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _check(t, name, dtype, shape, device):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or t.device != device or not t.is_contiguous():
+        raise ValueError(f"{name}: want {dtype} {tuple(shape)} contiguous on {device}, "
+                         f"got {t.dtype} {tuple(t.shape)} on {t.device}")
+
+
+def chunk_forward(x, Wr, g, W1, W2, y, active_idx, n_active, br=None, tok_mask=None, counts=None,
+                  r_out=None, path=BFFN_PATH_AUTO, workspace=None, stream=None):
+    """One chunk: x bf16 [L,d], Wr fp32 [d,E], g fp32 [E], W1 bf16 [E,de,d], W2 bf16 [E,d,de];
+    outputs y fp32 [L,d], active_idx int32 [E], n_active int32 [1] (+ optional tok_mask int32
+    [L,ceil(E/32)] (bit patterns), counts int32 [2], r_out fp32 [L,E]).  Raises BlockFFNError."""
+    import torch
+
+    L, d = x.shape
+    E, de = W1.shape[0], W1.shape[1]
+    dev = x.device
+    _check(x, "x", torch.bfloat16, (L, d), dev)
+    _check(Wr, "Wr", torch.float32, (d, E), dev)
+    _check(g, "g", torch.float32, (E,), dev)
+    _check(W1, "W1", torch.bfloat16, (E, de, d), dev)
+    _check(W2, "W2", torch.bfloat16, (E, d, de), dev)
+    _check(y, "y", torch.float32, (L, d), dev)
+    _check(active_idx, "active_idx", torch.int32, (E,), dev)
+    _check(n_active, "n_active", torch.int32, (1,), dev)
+    if br is not None:
+        _check(br, "br", torch.float32, (E,), dev)
+    if tok_mask is not None:
+        _check(tok_mask, "tok_mask", torch.int32, (L, (E + 31) // 32), dev)
+    if counts is not None:
+        _check(counts, "counts", torch.int32, (2,), dev)
+    if r_out is not None:
+        _check(r_out, "r_out", torch.float32, (L, E), dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    rc = blockffn_chunk_forward_ex(_ptr(x), L, d, _ptr(Wr), _ptr(g), _ptr(W1), _ptr(W2), E, de, _ptr(y),
+                                   _ptr(active_idx), _ptr(n_active), _ptr(br), _ptr(tok_mask),
+                                   _ptr(counts), _ptr(r_out), int(path), ws_ptr, ws_bytes, stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_chunk_forward_ex")
+
+
+def device_status(workspace=None, stream=None):
+    import torch
+
+    if stream is None:
+        stream = torch.cuda.current_stream().cuda_stream
+    return blockffn_device_status(None if workspace is None else workspace.data_ptr(), stream)
+
+
+def new_workspace(L, d, E, de, device="cuda"):
+    """A zero-filled caller-owned workspace for blockffn_chunk_forward_ex."""
+    import torch
+
+    n = blockffn_workspace_size(L, d, E, de)
+    if n == 0:
+        raise BlockFFNError(BFFN_EINVAL, "blockffn_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)

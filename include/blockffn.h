@@ -1,0 +1,121 @@
+/*
+ * blockffn.h — C ABI of the B200 (sm_100a) BlockFFN chunk-layer forward.
+ *
+ * The operation (BlockFFN, as described by the lsdiaocha.cn BlockFFN article, sections 2 and 4, and the
+ * BlockFFN abstract on arxivdaily 2507.08771): for a chunk of L consecutive tokens x_t (the chunk a
+ * speculative-decoding verification step feeds in),
+ *   s_{t,i} = x_t . Wr[:,i] + b_i                        router projection (b = 0 unless given)
+ *   r_{t,i} = g_i relu(s_{t,i}) / sqrt(mean_i relu(s_{t,i})^2)    ReLU + RMSNorm router (section 2);
+ *                                                        r_t = 0 when no s_{t,i} is positive
+ *   U       = { i : s_{t,i} > 0 for some t }            the chunk's union of active experts (section 4)
+ *   y_t     = sum_{i in U} r_{t,i} W2_i Swish(W1_i x_t)   non-gated Swish MLP experts (section 2);
+ *                                                        Swish(u) = u / (1 + e^-u)
+ * Only the experts in U are read from memory and evaluated.
+ *
+ * Layouts (row-major, no padding):
+ *   x   bf16 [L, d]           Wr fp32 [d, E]      g fp32 [E]       br fp32 [E]
+ *   W1  bf16 [E, de, d]       W2 bf16 [E, d, de]
+ *   y   fp32 [L, d]           active_idx int32 [E]   n_active int32 [1]
+ *   tok_mask uint32 [L, ceil(E/32)]  (bit i%32 of word i/32 of row t = 1 iff s_{t,i} > 0)
+ *   counts int32 [2]  = { number of (t,i) with s_{t,i} <= 0,  number of experts outside U }
+ *   r_out fp32 [L, E]
+ *
+ * Ownership and execution: every pointer argument is a DEVICE pointer owned by the caller; the
+ * library keeps none of them after the call returns. Work is enqueued on `stream` (a cudaStream_t,
+ * NULL = the legacy default stream) and the call returns without synchronising; outputs are valid
+ * once the stream has reached the enqueued work. y is fully overwritten (rows of tokens with no
+ * active expert are exactly 0). active_idx[0 .. n_active) lists U in ascending order; entries past
+ * n_active are unspecified. n_active stays on the device.
+ *
+ * Requirements, checked before anything is enqueued (BFFN_EINVAL otherwise):
+ *   1 <= L, 1 <= E <= 1024, d >= 16 and d % 16 == 0, de >= 16 and de % 16 == 0;
+ *   x, Wr, W1, W2 16-byte aligned (they are read with bulk copies), a workspace 256-byte aligned,
+ *   every other pointer 4-byte aligned; required pointers non-NULL.
+ * Paths: L <= 32 runs the decode path (weights streamed from HBM, memory-bound); larger L runs the
+ * prefill path. A shape a path cannot take returns BFFN_EUNSUPPORTED.
+ *
+ * Errors: BFFN_ECUDA when a CUDA call fails (the CUDA error is cleared); BFFN_ENOMEM when the
+ * internal workspace cannot be allocated. Device-side waits are bounded (about 2 s); a wait that
+ * runs out records an error in the workspace instead of hanging, which blockffn_device_status
+ * reports as BFFN_ETIMEOUT.
+ */
+#ifndef BLOCKFFN_H
+#define BLOCKFFN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define BFFN_API __attribute__((visibility("default")))
+#else
+#define BFFN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  BFFN_OK = 0,
+  BFFN_EINVAL = 1,       /* bad argument: nothing was enqueued */
+  BFFN_ECUDA = 2,        /* a CUDA runtime call failed */
+  BFFN_ENOMEM = 3,       /* workspace allocation failed or the given workspace is too small */
+  BFFN_ETIMEOUT = 4,     /* a bounded device-side wait ran out (reported by blockffn_device_status) */
+  BFFN_EUNSUPPORTED = 5  /* valid arguments, but no path of this build takes the shape */
+};
+
+/* Path selection for blockffn_chunk_forward_ex's `flags` (low two bits). */
+enum { BFFN_PATH_AUTO = 0, BFFN_PATH_DECODE = 1, BFFN_PATH_PREFILL = 2 };
+
+/*
+ * The layer forward over one chunk, with no router bias.  Uses a per-device workspace that the
+ * library allocates on the first call (and grows when a later call needs more); make that first
+ * call before capturing the stream into a CUDA graph.  Calls that share the internal workspace must
+ * be ordered (one stream, or synchronised streams).
+ */
+BFFN_API int blockffn_chunk_forward(const void* x, int L, int d, const float* Wr, const float* g,
+                           const void* W1, const void* W2, int E, int de, float* y,
+                           int32_t* active_idx, int32_t* n_active, void* stream);
+
+/*
+ * The same with optional inputs and outputs:
+ *   br        router bias fp32 [E], or NULL for none
+ *   tok_mask  per-token active-expert bit mask out, or NULL
+ *   counts    int32[2] out (zero router entries, experts outside the union), or NULL
+ *   r_out     router output r fp32 [L, E] out, or NULL
+ *   flags     BFFN_PATH_* (0 = choose by L)
+ *   workspace caller-owned device scratch of at least blockffn_workspace_size(L, d, E, de) bytes,
+ *             zero-filled before its first use (blockffn_workspace_init), or NULL to use the
+ *             library's per-device workspace.  Two calls may run concurrently only with
+ *             different workspaces.
+ */
+BFFN_API int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, const float* g,
+                              const void* W1, const void* W2, int E, int de, float* y,
+                              int32_t* active_idx, int32_t* n_active, const float* br,
+                              uint32_t* tok_mask, int32_t* counts, float* r_out, int flags,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace a call with these sizes needs (0 for invalid sizes). */
+BFFN_API size_t blockffn_workspace_size(int L, int d, int E, int de);
+
+/* Zero-fill a caller-owned workspace on `stream` (required once before its first use). */
+BFFN_API int blockffn_workspace_init(void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device error word of `workspace` (NULL = the
+ * library's workspace of the current device).  Returns BFFN_OK, BFFN_ETIMEOUT when a bounded
+ * device wait ran out since the last check, or BFFN_ECUDA.
+ */
+BFFN_API int blockffn_device_status(void* workspace, void* stream);
+
+/* Static description of a status code. */
+BFFN_API const char* blockffn_status_string(int status);
+
+/* ABI version (major * 100 + minor). */
+BFFN_API int blockffn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BLOCKFFN_H */

@@ -15,3 +15,20 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(scope="session")
+def bffn():
+    """The CUDA extension's binding (built in-tree first when it is missing or stale)."""
+    from chunk_sparse_moe_router_b200 import _build
+    _build.build()
+    import chunk_sparse_moe_router_b200 as m
+    return m
+
+
+@pytest.fixture(scope="session")
+def cuda_device():
+    import torch
+    if not torch.cuda.is_available():
+        pytest.fail("GPU test selected but no CUDA device is visible")
+    return torch.device("cuda", 0)

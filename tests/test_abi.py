@@ -1,0 +1,82 @@
+"""The C-ABI library: it loads, exports every symbol include/blockffn.h declares, and rejects bad
+arguments before touching the GPU (these checks need no device)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "blockffn.h")).read()
+    return sorted(set(re.findall(r"BFFN_API\s+[\w\s\*]+?\b(blockffn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = _declared_symbols()
+    assert "blockffn_chunk_forward" in syms and "blockffn_chunk_forward_ex" in syms
+    assert "blockffn_workspace_size" in syms and "blockffn_status_string" in syms
+
+
+def test_library_exports_every_declared_symbol(bffn):
+    lib = C.CDLL(bffn.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    assert set(_declared_symbols()) == set(bffn.SIGNATURES), "binding and header disagree"
+
+
+def test_only_c_symbols_are_exported(bffn):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bffn.LIB_PATH], capture_output=True, text=True).stdout
+    ours = [l.split()[-1] for l in out.splitlines() if l.split()[-1].startswith("blockffn_")]
+    assert sorted(ours) == _declared_symbols()
+
+
+def test_status_strings(bffn):
+    assert bffn.blockffn_status_string(0) == "ok"
+    assert "invalid" in bffn.blockffn_status_string(1)
+    assert bffn.blockffn_status_string(99) == "unknown status"
+    assert bffn.blockffn_abi_version() >= 100
+
+
+def test_workspace_size(bffn):
+    assert bffn.blockffn_workspace_size(8, 2048, 64, 256) > 256
+    big = bffn.blockffn_workspace_size(32, 4096, 128, 256)
+    assert big >= 128 * 64 * 256 * 2  # h: E x 2L x de bf16
+    for bad in [(0, 256, 16, 64), (8, 250, 16, 64), (8, 256, 0, 64), (8, 256, 2000, 64), (8, 256, 16, 8)]:
+        assert bffn.blockffn_workspace_size(*bad) == 0
+
+
+FAKE = 1 << 20  # aligned, never dereferenced: every case below must fail validation first
+
+
+def _call(bffn, **kw):
+    a = dict(x=FAKE, L=8, d=256, Wr=FAKE, g=FAKE, W1=FAKE, W2=FAKE, E=16, de=64, y=FAKE,
+             active_idx=FAKE, n_active=FAKE, br=None, tok_mask=None, counts=None, r_out=None,
+             flags=0, workspace=None, workspace_bytes=0, stream=None)
+    a.update(kw)
+    return bffn.blockffn_chunk_forward_ex(**a)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(L=0), dict(L=-3), dict(d=250), dict(d=0), dict(de=24), dict(E=0), dict(E=1025),
+    dict(x=None), dict(Wr=None), dict(g=None), dict(W1=None), dict(W2=None), dict(y=None),
+    dict(active_idx=None), dict(n_active=None),
+    dict(x=FAKE + 2), dict(W1=FAKE + 8), dict(W2=FAKE + 4), dict(Wr=FAKE + 4), dict(y=FAKE + 2),
+    dict(n_active=FAKE + 1), dict(br=FAKE + 2), dict(r_out=FAKE + 1), dict(workspace=FAKE + 16),
+    dict(flags=3),
+])
+def test_invalid_arguments_rejected_before_launch(bffn, kw):
+    assert _call(bffn, **kw) == bffn.BFFN_EINVAL
+
+
+def test_unsupported_path_rejected_before_launch(bffn):
+    # a decode-path request for a chunk longer than the decode path takes
+    assert _call(bffn, L=33, flags=bffn.BFFN_PATH_DECODE) == bffn.BFFN_EUNSUPPORTED
+
+
+def test_plain_entry_point_validates(bffn):
+    assert bffn.blockffn_chunk_forward(None, 8, 256, FAKE, FAKE, FAKE, FAKE, 16, 64, FAKE, FAKE, FAKE,
+                                       None) == bffn.BFFN_EINVAL
