@@ -23,6 +23,7 @@ SIGNATURES = {
     "blockffn_chunk_forward": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
     "blockffn_chunk_forward_ex": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P,
                                        _P, _I, _P, _S, _P]),
+    "blockffn_chunk_forward_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_init": (_I, [_P, _S, _P]),
     "blockffn_device_status": (_I, [_P, _P]),
@@ -63,6 +64,14 @@ def blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_ac
     return _lib.blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br,
                                           tok_mask, counts, r_out, flags, workspace, workspace_bytes,
                                           stream)
+
+
+def blockffn_chunk_forward_noalloc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, stream):
+    return _lib.blockffn_chunk_forward_noalloc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br,
+                                               stream)
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20  # BFFN_NOALLOC_SCRATCH_BYTES in include/blockffn.h
 
 
 def blockffn_workspace_size(L, d, E, de):

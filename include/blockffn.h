@@ -108,6 +108,32 @@ BFFN_API int blockffn_workspace_init(void* workspace, size_t workspace_bytes, vo
  */
 BFFN_API int blockffn_device_status(void* workspace, void* stream);
 
+/*
+ * blockffn_chunk_forward_noalloc — no counterpart on the BlockFFN pages; this is a deployment aid.
+ *
+ * The same forward as blockffn_chunk_forward (plus the optional router bias `br`, may be NULL) for
+ * callers that cannot call cudaMalloc: for example a serving engine that has already reserved all
+ * of device memory for weights and KV cache and hands out no scratch, or code that must not
+ * synchronise the device (cudaMalloc and cudaFree may wait for outstanding GPU work).  It allocates
+ * nothing: its scratch is a fixed array of BFFN_NOALLOC_SCRATCH_BYTES compiled into the library,
+ * which every GPU that loads the library holds until the process exits.
+ *   - Sizes whose workspace (blockffn_workspace_size) exceeds BFFN_NOALLOC_SCRATCH_BYTES return
+ *     BFFN_ENOMEM before anything is enqueued.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *     that device current); make that first call before capturing the stream into a CUDA graph.
+ *   - Every call on a device shares the one array and leaves its contents behind: calls whose GPU
+ *     work overlaps (different streams, or several host threads) race on it and must be ordered
+ *     by the caller.
+ *   - Device-side timeouts of this entry point are recorded in its own array, not in the
+ *     workspace blockffn_device_status(NULL, ...) reads.
+ * Inputs and outputs are the caller's device buffers, as for blockffn_chunk_forward.
+ */
+#define BFFN_NOALLOC_SCRATCH_BYTES (8u << 20)
+BFFN_API int blockffn_chunk_forward_noalloc(const void* x, int L, int d, const float* Wr,
+                                            const float* g, const void* W1, const void* W2, int E,
+                                            int de, float* y, int32_t* active_idx,
+                                            int32_t* n_active, const float* br, void* stream);
+
 /* Static description of a status code. */
 BFFN_API const char* blockffn_status_string(int status);
 
