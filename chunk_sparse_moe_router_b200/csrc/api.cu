@@ -88,6 +88,43 @@ bool shapes_ok(int L, int d, int E, int de) {
          (long long)L * d < (1ll << 31) && (long long)E * de * d < (1ll << 40);
 }
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link against the driver library).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+    (void)cudaGetLastError();
+  });
+  return fn;
+}
+
+// bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, out-of-bounds elements read as 0.
+bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
+                 const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[5], gstride[4];
+  cuuint32_t bdim[5], estride[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
+  return fn(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, cuuint32_t(rank), const_cast<void*>(base), gdim, gstride, bdim,
+            estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 int forward_decode(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
@@ -100,42 +137,76 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
   rp.x = static_cast<const __nv_bfloat16*>(x);
   rp.Wr = Wr;
   rp.br = br;
-  rp.g = g;
   rp.L = L;
   rp.d = d;
   rp.E = E;
   rp.s_ws = reinterpret_cast<float*>(base + lay.s_off);
-  rp.r_ws = reinterpret_cast<float*>(base + lay.r_off);
-  rp.r_out = r_out;
-  rp.tok_mask = tok_mask;
-  rp.counts = counts;
-  rp.active_idx = active_idx;
-  rp.n_active = n_active;
   rp.hdr = hdr;
   RouterLaunch rl;
-  if (!router_decode_plan(L, d, E, di.max_smem, &rl, &rp.Rq)) return BFFN_EUNSUPPORTED;
-  rp.wreg_floats = rl.wreg_floats;
+  if (!router_decode_plan(L, d, E, di.max_smem, &rl)) return BFFN_EUNSUPPORTED;
+  rp.xt = rl.xt;
 
   DecodeParams dp;
-  dp.x = rp.x;
-  dp.W1 = static_cast<const __nv_bfloat16*>(W1);
-  dp.W2 = static_cast<const __nv_bfloat16*>(W2);
+  dp.s = rp.s_ws;
+  dp.g = g;
   dp.y = y;
   dp.active_idx = active_idx;
   dp.n_active = n_active;
-  dp.r = rp.r_ws;
-  dp.h = reinterpret_cast<__nv_bfloat16*>(base + lay.h_off);
+  dp.tok_mask = tok_mask;
+  dp.counts = counts;
+  dp.r_out = r_out;
+  dp.h = base + lay.h_off;
   dp.hdr = hdr;
   dp.L = L;
   dp.d = d;
   dp.E = E;
   dp.de = de;
   DecodeLaunch dl;
-  if (!expert_decode_plan(L, d, de, di.num_sms, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
+  if (!expert_decode_plan(L, d, E, de, di.num_sms, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
+
+  TensorMaps tm;
+  {
+    const uint64_t xrow = uint64_t(d) * 2, w1e = uint64_t(d) * de * 2;
+    const uint64_t w2row = uint64_t(de) * 2, w2e = uint64_t(d) * de * 2;
+    const int KC = dp.nKf / dp.KP;
+    // plain views: the ragged last chunk of d (and every stage when d < 64)
+    const uint64_t x2d[2] = {uint64_t(d), uint64_t(L)}, x2s[1] = {xrow};
+    const uint32_t x2b[2] = {64, uint32_t(dp.LB)};
+    if (!encode_bf16(&tm.x_2d, x, 2, x2d, x2s, x2b)) return BFFN_ECUDA;
+    const uint64_t w13d[3] = {uint64_t(d), uint64_t(de), uint64_t(E)}, w13s[2] = {xrow, w1e};
+    for (int k = 0; k < 4; ++k) {
+      const uint32_t b[3] = {64, uint32_t(1u << k), 1};
+      if (!encode_bf16(&tm.w1_3d[k], W1, 3, w13d, w13s, b)) return BFFN_ECUDA;
+    }
+    // chunked views over the full chunks: a box is whole rows of one K pass
+    if (KC > 0) {
+      const uint64_t xcd[3] = {64, uint64_t(L), uint64_t(dp.nKf)}, xcs[2] = {xrow, 128};
+      const uint32_t xcb[3] = {64, uint32_t(dp.LB), uint32_t(KC)};
+      if (!encode_bf16(&tm.x_ch, x, 3, xcd, xcs, xcb)) return BFFN_ECUDA;
+      const uint64_t w1cd[4] = {64, uint64_t(de), uint64_t(dp.nKf), uint64_t(E)}, w1cs[3] = {xrow, 128, w1e};
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t b[4] = {64, uint32_t(1u << k), uint32_t(KC), 1};
+        if (!encode_bf16(&tm.w1_ch[k], W1, 4, w1cd, w1cs, b)) return BFFN_ECUDA;
+      }
+    } else {
+      tm.x_ch = tm.x_2d;
+      for (int k = 0; k < 4; ++k) tm.w1_ch[k] = tm.w1_3d[k];
+    }
+    const uint64_t w23d[3] = {uint64_t(de), uint64_t(d), uint64_t(E)}, w23s[2] = {w2row, w2e};
+    const uint32_t w2b3[3] = {64, uint32_t(dp.RBB), 1};
+    if (!encode_bf16(&tm.w2_3d, W2, 3, w23d, w23s, w2b3)) return BFFN_ECUDA;
+    if (dp.nJf > 0) {
+      const uint64_t w2cd[4] = {64, uint64_t(d), uint64_t(dp.nJf), uint64_t(E)}, w2cs[3] = {w2row, 128, w2e};
+      const uint32_t w2cb[4] = {64, uint32_t(dp.RBB), uint32_t(dp.KWB), 1};
+      if (!encode_bf16(&tm.w2_ch, W2, 4, w2cd, w2cs, w2cb)) return BFFN_ECUDA;
+    } else {
+      tm.w2_ch = tm.w2_3d;
+    }
+  }
 
   cudaError_t err = router_decode_launch(rp, rl, st, di.pdl);
   if (err != cudaSuccess) return cuda_fail(err);
-  err = expert_decode_launch(dp, dl, st, di.pdl);
+  err = expert_decode_launch(dp, tm, dl, st, di.pdl);
   if (err != cudaSuccess) return cuda_fail(err);
   return BFFN_OK;
 }

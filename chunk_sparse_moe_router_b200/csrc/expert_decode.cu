@@ -1,81 +1,72 @@
 // Sparse expert kernel of the BlockFFN chunk layer for decode-sized chunks (L <= 32).
 //
-// The chunk's union U of active experts (lsdiaocha.cn BlockFFN article, section 4) is evaluated for all L
-// tokens as one batch, outer loop over active experts and inner batched product (article, section 7),
-// and each (token, expert) term is weighted by the router output r, which is zero for the pairs
-// the mask removes.  Only the rows of W1/W2 that belong to experts in U are read.
+// Prologue (every CTA, from the router projection s in L2): ReLU and RMSNorm statistics per token
+// (one warp per token, shuffle reduction), the per-token active masks with __ballot_sync, and the
+// chunk's union of active experts as an ascending list built with __popc and a warp scan
+// (lsdiaocha.cn BlockFFN article, sections 2 and 4).  CTA 0 also writes the active list, n_active, the
+// sparsity counts and the optional masks / router outputs.
 //
-// The kernel is memory-bound: every weight byte is used by L tokens (2L flop per bf16 weight), so
-// it is built around keeping HBM busy:
-//  * one persistent CTA per SM; the work of each phase is split over the CTAs in contiguous row
-//    ranges balanced to within one row, so every SM streams the same number of bytes;
-//  * weights move with bulk (TMA) copies into a ring of shared-memory slots guarded by mbarriers,
-//    one producer warp keeping up to S slots in flight, with an L2 evict-first hint;
-//  * 4 consumer warps run mma.sync m16n8k16 (bf16 in, fp32 accumulate) with tokens as the M
-//    dimension and 8 weight rows as N, reading operands from shared memory with ldmatrix.
+// Body: the union is evaluated for all L tokens as one batch, outer loop over active experts and
+// inner batched product (article, section 7); each (token, expert) term is weighted by the router
+// output r, which is zero for the pairs the mask removes.  Only the W1/W2 rows of experts in the
+// union are read.  The kernel is HBM-bound (2L flop per bf16 weight), so everything serves the
+// memory stream:
+//  * one persistent CTA per SM; each phase's rows are split over the CTAs in contiguous ranges
+//    balanced to within one row, so every SM streams the same number of bytes;
+//  * weights are read in long contiguous runs, as HBM wants them: the up-projection streams whole
+//    W1 rows (a CTA's rows of one expert are one contiguous block), the down-projection whole
+//    blocks of consecutive W2 rows; copies are TMA bulk copies / tensor boxes of several KB issued
+//    from several lanes into a ring of shared-memory stages guarded by mbarriers;
+//  * 4 consumer warps run mma.sync m16n8k16 (bf16 in, fp32 accumulate) with tokens as M and weight
+//    rows as N, reading operands with conflict-free ldmatrix (padded rows / 128-byte swizzle).
 //
-// Phase A (up-projection): the CTA owns rows [rA0, rA1) of the flattened (active expert, j) space;
-//   u[t, row] = W1[e, j, :] . x_t,  h = r[t, e] * Swish(u)  (Swish(u) = u / (1 + e^-u), article
-//   section 2), stored to the workspace as a high and a low bf16 part so the down-projection keeps
-//   ~16 mantissa bits of h on bf16 tensor cores.
-// Grid barrier: every CTA's h must be visible before any down-projection (bounded wait).  The
-//   producer keeps prefetching W2 tiles while the barrier is pending; only the h tiles wait for it.
+// Phase A (up-projection): the CTA owns rows [rA0, rA1) of the flattened (active expert, j) space,
+//   taken in groups of RS rows, one group per stage; a consumer warp owns whole groups and computes
+//   u = W1[e, j, :] . x_t over all of K (x stays resident in shared memory, in K passes when it is
+//   large), then h = r[t, e] * Swish(u), Swish(u) = u / (1 + e^-u) (article, section 2).  h goes to
+//   the workspace as a high and a low bf16 part (so the bf16 down-projection keeps about 16 mantissa
+//   bits of h), already in the swizzled tile layout the down-projection loads.
+// Grid barrier: all h are written before any CTA reads h (bounded wait).  W2 tiles keep streaming
+//   in while it is pending; only the h tiles wait for it.
 // Phase B (down-projection): the CTA owns output rows [rB0, rB1) of y and sums over every active
-//   expert:  y[t, k] = sum_a sum_j W2[e_a, k, j] (h_hi + h_lo)[a, t, j].  The hi and lo parts are
-//   two stacks of L rows of the MMA's M dimension, added in the epilogue.  Each y element is written
-//   exactly once, in a fixed summation order, so y is bit-reproducible run to run.
+//   expert, y[t, k] = sum_a sum_j W2[e_a, k, j] (h_hi + h_lo)[a, t, j], with the hi and lo parts as
+//   two stacks of L rows of the MMA's M dimension.  Each y element is written exactly once, in a
+//   fixed summation order, so y is bit-reproducible run to run.
 #include "blockffn_internal.cuh"
 #include "ptx.cuh"
 
 namespace bffn {
 namespace {
 
-constexpr int NCW = 4;                  // consumer warps
-constexpr int kThreads = (NCW + 2) * 32;
-constexpr int RB = 32;                  // weight rows per row-block: 4 n-tiles of 8
+constexpr int NCW = 4;                      // consumer warps
+constexpr int kThreads = (NCW + 2) * 32;    // + weight producer warp + x / h producer warp
+constexpr int GPW = 2;                      // row groups per consumer warp per row-block
+constexpr int GB = NCW * GPW;               // row groups per row-block
+constexpr int kMaxSpan = GB;                // experts one row-block can touch (a group never crosses one)
 constexpr uint64_t kWaitNs = 2000000000ull;
-constexpr int kMaxSpan = 3;             // experts a 32-row block can touch when de >= 16
 
+// ------------------------------------------------------------------------------------- smem
 struct Smem {
-  uint8_t* ring;
-  int32_t* act;        // [E] the chunk's active expert ids (copied once per CTA)
-  float* rs;           // [kMaxSpan][L] router outputs of the experts of the current row-block
-  float* red;          // [NCW][MT][4][32][4]
+  uint8_t* xbuf;       // resident x part [L][PX]
+  uint8_t* ring;       // S slots
+  float* red;          // [NCW][MT][4][32][4] phase-B cross-warp partials (aliases xbuf when it fits)
+  uint8_t* zero;       // 16 zero bytes
+  volatile int* abort_flag;
   uint64_t* fullW;     // [S]
   uint64_t* fullH;     // [S]
   uint64_t* empty;     // [S]
-  uint8_t* zero;       // 16 zero bytes
-  volatile int* abort_flag;
+  uint64_t* xfull;     // x part landed
+  uint64_t* xfree;     // consumers done with the x part
+  int32_t* act;        // [E] active experts, ascending
+  int* n_act;          // [1]
+  float* rms;          // [32] per-token sqrt(mean relu(s)^2)
+  uint32_t* maskw;     // [32][32] per-token active bits
+  float* pre_s;        // [kMaxSpan][32] s of the current row-block's experts
+  float* pre_g;        // [kMaxSpan]
 };
 
-struct Work {
-  int nA;              // phase A rows of this CTA
-  int rA0;
-  int nB;              // phase B rows of this CTA
-  int rB0;
-  int nRBA, nRBB;      // row-blocks
-  int nKA;             // stages per phase-A row-block
-  int nJB;             // j-chunks per expert in phase B
-  int n_act;
-  int stagesA, stagesB;
-};
-
-__device__ __forceinline__ Work make_work(const DecodeParams& p, int n_act) {
-  Work w;
-  const int G = gridDim.x, c = blockIdx.x;
-  const long long RA = (long long)n_act * p.de;
-  w.rA0 = int(RA * c / G);
-  w.nA = int(RA * (c + 1) / G) - w.rA0;
-  w.rB0 = int((long long)p.d * c / G);
-  w.nB = int((long long)p.d * (c + 1) / G) - w.rB0;
-  w.nRBA = (w.nA + RB - 1) / RB;
-  w.nRBB = (w.nB + RB - 1) / RB;
-  w.nKA = (p.d + p.KcA - 1) / p.KcA;
-  w.nJB = (p.de + p.KcB - 1) / p.KcB;
-  w.n_act = n_act;
-  w.stagesA = w.nRBA * w.nKA;
-  w.stagesB = w.nRBB * n_act * w.nJB;
-  return w;
+__device__ __forceinline__ uint32_t swz(int row, int chunk16) {
+  return uint32_t(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
 __device__ __forceinline__ void set_error(const DecodeParams& p, const Smem& sm, uint32_t bit, uint32_t info) {
@@ -84,188 +75,8 @@ __device__ __forceinline__ void set_error(const DecodeParams& p, const Smem& sm,
   *sm.abort_flag = 1;
 }
 
-// ----------------------------------------------------------------------------------------- producers
-// Weight producer: phase A stages (x rows + W1 rows) then phase B stages (W2 rows), in order.
-__device__ void produce_weights(const DecodeParams& p, const Smem& sm, const Work& w) {
-  const int lane = threadIdx.x % 32;
-  const uint64_t pol_w = policy_evict_first();
-  const uint64_t pol_x = policy_evict_last();
-  const int total = w.stagesA + w.stagesB;
-  int i = 0;
-  for (; i < total; ++i) {
-    if (*sm.abort_flag) break;
-    const int slot = i % p.S;
-    if (i >= p.S) {
-      if (!mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
-        if (lane == 0) set_error(p, sm, kErrRingWait, 1);
-        break;
-      }
-    }
-    uint8_t* base = sm.ring + size_t(slot) * p.slot_bytes;
-    if (i < w.stagesA) {
-      const int rb = i / w.nKA, kc = i % w.nKA;
-      const int r0 = w.rA0 + rb * RB, nrows = min(RB, w.nA - rb * RB);
-      const int k0 = kc * p.KcA, kw = min(p.KcA, p.d - k0);
-      const uint32_t rowb = uint32_t(kw) * 2;
-      if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[slot], rowb * uint32_t(p.L + nrows));
-      __syncwarp();
-      for (int c = lane; c < p.L + nrows; c += 32) {
-        if (c < p.L) {
-          bulk_g2s(base + size_t(c) * p.pitchA, p.x + size_t(c) * p.d + k0, rowb, &sm.fullW[slot], pol_x);
-        } else {
-          const int row = r0 + (c - p.L);
-          const int a = row / p.de, j = row % p.de;
-          const int e = sm.act[a];
-          const __nv_bfloat16* src = p.W1 + (size_t(e) * p.de + j) * p.d + k0;
-          bulk_g2s(base + p.woff + size_t(c - p.L) * p.pitchA, src, rowb, &sm.fullW[slot], pol_w);
-        }
-      }
-    } else {
-      const int jb = i - w.stagesA;
-      const int per_rb = w.n_act * w.nJB;
-      const int rb = jb / per_rb, rem = jb % per_rb;
-      const int a = rem / w.nJB, jc = rem % w.nJB;
-      const int k0 = w.rB0 + rb * RB, nrows = min(RB, w.nB - rb * RB);
-      const int j0 = jc * p.KcB, jw = min(p.KcB, p.de - j0);
-      const uint32_t rowb = uint32_t(jw) * 2;
-      const int e = sm.act[a];
-      if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[slot], rowb * uint32_t(nrows));
-      __syncwarp();
-      for (int c = lane; c < nrows; c += 32) {
-        const __nv_bfloat16* src = p.W2 + (size_t(e) * p.d + k0 + c) * p.de + j0;
-        bulk_g2s(base + p.woff + size_t(c) * p.pitchB, src, rowb, &sm.fullW[slot], pol_w);
-      }
-    }
-    __syncwarp();
-  }
-  // Drain: every copy this warp issued must land before the CTA may exit.
-  const int issued = i;
-  for (int k = max(0, issued - p.S); k < issued; ++k) {
-    mbar_wait_bounded(&sm.fullW[k % p.S], (k / p.S) & 1, kWaitNs / 10);
-  }
-}
-
-// h producer: after the grid barrier, the h tiles of every phase-B stage.
-__device__ void produce_h(const DecodeParams& p, const Smem& sm, const Work& w) {
-  const int lane = threadIdx.x % 32;
-  if (w.stagesB == 0) return;
-  {
-    const uint64_t t0 = globaltimer_ns();
-    bool ok = true;
-    while (ld_acquire_gpu(&p.hdr->grid_bar) < gridDim.x) {
-      if (*sm.abort_flag || globaltimer_ns() - t0 > kWaitNs) { ok = false; break; }
-      __nanosleep(64);
-    }
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) {
-      if (lane == 0) set_error(p, sm, kErrGridBarrier, uint32_t(blockIdx.x));
-      return;
-    }
-    fence_proxy_async_global();
-  }
-  const uint64_t pol_h = policy_evict_last();
-  const int L2 = 2 * p.L;
-  uint32_t hphase = 0;  // bit s = parity of the next fullH phase of slot s
-  int issued = 0;
-  for (int jb = 0; jb < w.stagesB; ++jb) {
-    if (*sm.abort_flag) break;
-    const int i = w.stagesA + jb;
-    const int slot = i % p.S;
-    if (i >= p.S) {
-      if (!mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
-        if (lane == 0) set_error(p, sm, kErrRingWait, 2);
-        break;
-      }
-    }
-    const int per_rb = w.n_act * w.nJB;
-    const int rem = jb % per_rb;
-    const int a = rem / w.nJB, jc = rem % w.nJB;
-    const int j0 = jc * p.KcB, jw = min(p.KcB, p.de - j0);
-    const uint32_t rowb = uint32_t(jw) * 2;
-    uint8_t* base = sm.ring + size_t(slot) * p.slot_bytes;
-    if (lane == 0) mbar_arrive_expect_tx(&sm.fullH[slot], rowb * uint32_t(L2));
-    __syncwarp();
-    for (int c = lane; c < L2; c += 32) {
-      const __nv_bfloat16* src = p.h + (size_t(a) * L2 + c) * p.de + j0;
-      bulk_g2s(base + size_t(c) * p.pitchB, src, rowb, &sm.fullH[slot], pol_h);
-    }
-    __syncwarp();
-    hphase ^= 1u << slot;
-    ++issued;
-  }
-  // Drain this warp's copies.
-  uint32_t ph = hphase;
-  for (int k = issued - 1; k >= 0 && k >= issued - p.S; --k) {
-    const int slot = (w.stagesA + k) % p.S;
-    ph ^= 1u << slot;  // parity of that stage's phase
-    mbar_wait_bounded(&sm.fullH[slot], (ph >> slot) & 1u, kWaitNs / 10);
-  }
-}
-
-// ----------------------------------------------------------------------------------------- consumers
-template <int MT>
-__device__ __forceinline__ void mma_stage(const uint8_t* abase, int rowsA, int pitch, const uint8_t* wbase,
-                                          int kw, const uint8_t* zero, float (&acc)[MT][4][4], int mtn) {
-  const int cw = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nks = kw / 16;
-  const uint32_t zaddr = smem_u32(zero);
-  const uint32_t abase_u = smem_u32(abase), wbase_u = smem_u32(wbase);
-  for (int ks = cw; ks < nks; ks += NCW) {
-    uint32_t a[MT][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      if (mt < mtn) {
-        const int row = mt * 16 + (lane & 15);
-        const int kcol = ks * 16 + (lane >> 4) * 8;
-        const uint32_t addr = (row < rowsA) ? abase_u + uint32_t(row * pitch + kcol * 2) : zaddr;
-        ldmatrix_x4(addr, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-      }
-    }
-    uint32_t b[4][2];
-#pragma unroll
-    for (int np = 0; np < 2; ++np) {
-      const int nrow = np * 16 + (lane & 7) + (lane >> 4) * 8;
-      const int kcol = ks * 16 + ((lane >> 3) & 1) * 8;
-      ldmatrix_x4(wbase_u + uint32_t(nrow * pitch + kcol * 2), b[2 * np][0], b[2 * np][1], b[2 * np + 1][0],
-                  b[2 * np + 1][1]);
-    }
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-      if (mt < mtn) {
-#pragma unroll
-        for (int nt = 0; nt < 4; ++nt) mma_bf16_16816(acc[mt][nt], a[mt], b[nt][0], b[nt][1]);
-      }
-    }
-  }
-}
-
-// Value of output (row, col) of the row-block, summed over the consumer warps' partials.
-template <int MT>
-__device__ __forceinline__ float red_value(const float* red, int row, int col) {
-  const int mt = row >> 4, r16 = row & 15;
-  const int lane = (r16 & 7) * 4 + ((col & 7) >> 1);
-  const int reg = (r16 >> 3) * 2 + (col & 1);
-  const int nt = col >> 3;
-  float v = 0.f;
-#pragma unroll
-  for (int w = 0; w < NCW; ++w) v += red[((((w * MT + mt) * 4 + nt) * 32 + lane) * 4) + reg];
-  return v;
-}
-
-template <int MT>
-__device__ __forceinline__ void stash(float* red, const float (&acc)[MT][4][4]) {
-  const int cw = threadIdx.x / 32, lane = threadIdx.x % 32;
-#pragma unroll
-  for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
-      *reinterpret_cast<float4*>(red + ((((cw * MT + mt) * 4 + nt) * 32 + lane) * 4)) =
-          make_float4(acc[mt][nt][0], acc[mt][nt][1], acc[mt][nt][2], acc[mt][nt][3]);
-}
-
-// Wait for a ring barrier; on timeout record the error and mark the CTA aborted.  Once aborted,
-// waits are skipped (the caller skips the work) so every consumer warp still reaches the same
-// named barriers and the CTA can finish.
+// A wait that records a timeout and marks the CTA aborted; once aborted, waits are skipped (callers
+// skip the work) so that every warp still reaches the same named barriers and the CTA can finish.
 __device__ __forceinline__ bool ring_wait(const DecodeParams& p, const Smem& sm, uint64_t* bar, uint32_t parity,
                                           uint32_t where) {
   if (*sm.abort_flag) return false;
@@ -275,65 +86,377 @@ __device__ __forceinline__ bool ring_wait(const DecodeParams& p, const Smem& sm,
   return false;
 }
 
+// ------------------------------------------------------------------------------------- work split
+struct Work {
+  int rA0, rA1;        // phase-A rows (flattened over active experts)
+  int rB0, nB;         // phase-B rows of y
+  int nRBB;            // phase-B row-blocks of RBB rows
+  int nEg;             // phase-B expert groups of NEB
+  int nJs;             // phase-B j-stages per expert group
+  int n_act;
+};
+
+__device__ __forceinline__ Work make_work(const DecodeParams& p, int n_act) {
+  Work w;
+  const int G = gridDim.x, c = blockIdx.x;
+  const long long RA = (long long)n_act * p.de;
+  w.rA0 = int(RA * c / G);
+  w.rA1 = int(RA * (c + 1) / G);
+  w.rB0 = int((long long)p.d * c / G);
+  w.nB = int((long long)p.d * (c + 1) / G) - w.rB0;
+  w.nRBB = (w.nB + p.RBB - 1) / p.RBB;
+  w.nEg = (n_act + p.NEB - 1) / p.NEB;
+  w.nJs = (p.nJc + p.KWB - 1) / p.KWB;
+  w.n_act = n_act;
+  return w;
+}
+
+// Phase-A row group: h (a power of two <= RSM) adjacent rows of one expert, starting at flattened row
+// r.  Groups never cross an expert or the CTA's range, so one box fetches exactly the group.
+struct Group {
+  int a, j0, h;
+};
+
+__device__ __forceinline__ Group group_at(const DecodeParams& p, int r, int r_end) {
+  Group gr;
+  gr.a = r / p.de;
+  gr.j0 = r - gr.a * p.de;
+  const int room = min(p.de - gr.j0, r_end - r);
+  int h = p.RSM;
+  while (h > room) h >>= 1;
+  gr.h = h;
+  return gr;
+}
+
+// Groups [g_begin, g_begin + GB) of the CTA, walking from cursor r: the first group's row, their
+// count, and the cursor after them.
+__device__ __forceinline__ int rowblock_walk(const DecodeParams& p, int r, int r_end, int* ngroups) {
+  int n = 0;
+  while (r < r_end && n < GB) {
+    r += group_at(p, r, r_end).h;
+    ++n;
+  }
+  *ngroups = n;
+  return r;
+}
+
+// The k-th group of the row-block starting at cursor r (k < number of groups).
+__device__ __forceinline__ Group group_k(const DecodeParams& p, int r, int r_end, int k, int* row0) {
+  Group gr = group_at(p, r, r_end);
+  for (int q = 0; q < k; ++q) {
+    r += gr.h;
+    gr = group_at(p, r, r_end);
+  }
+  *row0 = r;
+  return gr;
+}
+
+__device__ __forceinline__ bool stage_is_chunked(int c0, int nc, int nfull) { return c0 + nc <= nfull; }
+
+// ------------------------------------------------------------------------------------- producers
+// Weight producer (one warp): W1 row groups, then W2 expert tiles, in stage order.
+__device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol_w = policy_evict_first();
+  int i = 0;
+  bool ok = true;
+  // ---- phase A: stage = one box of a group's whole rows over the pass's columns
+  const int KC = p.nKf / p.KP;                 // full chunks per pass
+  const bool tail = p.nKc > p.nKf;             // only with one pass
+  for (int r = w.rA0; r < w.rA1 && ok;) {
+    int ngr;
+    const int r_next = rowblock_walk(p, r, w.rA1, &ngr);
+    int row0 = 0;
+    const Group mine = group_k(p, r, w.rA1, lane < ngr ? lane : 0, &row0);  // lane k: group k
+    const int hsel = __ffs(mine.h) - 1;
+    const int e = sm.act[mine.a];
+    for (int ps = 0; ps < p.KP && ok; ++ps) {
+      for (int gl = 0; gl < ngr; ++gl, ++i) {
+        if (*sm.abort_flag) { ok = false; break; }
+        const int slot = i % p.S;
+        if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+          if (lane == 0) set_error(p, sm, kErrRingWait, 1);
+          ok = false;
+          break;
+        }
+        const int h = __shfl_sync(0xffffffffu, mine.h, gl);
+        if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[slot], uint32_t(KC + (tail ? 1 : 0)) * h * 128);
+        __syncwarp();
+        if (lane == gl) {
+          uint8_t* dst = sm.ring + size_t(slot) * p.slot_bytes;
+          if (KC > 0) tma_load_4d(dst, &tm.w1_ch[hsel], 0, mine.j0, ps * KC, e, &sm.fullW[slot], pol_w);
+          if (tail)
+            tma_load_3d(dst + p.w1_tail_off, &tm.w1_3d[hsel], p.nKf * 64, mine.j0, e, &sm.fullW[slot], pol_w);
+        }
+        __syncwarp();
+      }
+    }
+    r = r_next;
+  }
+  // ---- phase B: stage = NEB experts x KWB chunks of W2 rows [k0, k0 + RBB)
+  for (int rb = 0; rb < w.nRBB && ok; ++rb) {
+    const int k0 = w.rB0 + rb * p.RBB;
+    for (int eg = 0; eg < w.nEg && ok; ++eg) {
+      const int a0 = eg * p.NEB, nq = min(p.NEB, w.n_act - a0);
+      for (int js = 0; js < w.nJs; ++js, ++i) {
+        if (*sm.abort_flag) { ok = false; break; }
+        const int slot = i % p.S;
+        if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+          if (lane == 0) set_error(p, sm, kErrRingWait, 2);
+          ok = false;
+          break;
+        }
+        const int c0 = js * p.KWB, nc = min(p.KWB, p.nJc - c0);
+        const bool chunked = stage_is_chunked(c0, nc, p.nJf);
+        if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[slot], uint32_t(nq) * (chunked ? p.KWB : nc) * p.RBB * 128);
+        __syncwarp();
+        if (lane < nq) {
+          uint8_t* dst = sm.ring + size_t(slot) * p.slot_bytes + size_t(lane) * p.eB;
+          const int e = sm.act[a0 + lane];
+          if (chunked) {
+            tma_load_4d(dst, &tm.w2_ch, 0, k0, c0, e, &sm.fullW[slot], pol_w);
+          } else {
+            for (int c = 0; c < nc; ++c)
+              tma_load_3d(dst + size_t(c) * p.RBB * 128, &tm.w2_3d, (c0 + c) * 64, k0, e, &sm.fullW[slot], pol_w);
+          }
+        }
+        __syncwarp();
+      }
+    }
+  }
+  // every copy this warp issued lands before the CTA may exit
+  for (int k = max(0, i - p.S); k < i; ++k) mbar_wait_bounded(&sm.fullW[k % p.S], (k / p.S) & 1, kWaitNs / 10);
+}
+
+// x / h producer (one warp): the resident x parts of phase A, then (after the grid barrier) the h
+// tiles of phase B.
+__device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
+  const int lane = threadIdx.x & 31;
+  const uint64_t pol_x = policy_evict_last();
+  // ---- x parts: once, or once per (row-block, pass) when K is split in passes
+  const int KC = p.nKf / p.KP;
+  const bool tail = p.nKc > p.nKf;
+  int nrb = 0;
+  for (int r = w.rA0; r < w.rA1; ++nrb) {
+    int ngr;
+    r = rowblock_walk(p, r, w.rA1, &ngr);
+  }
+  int xloads = 0;
+  const int nparts = (p.KP > 1) ? nrb * p.KP : (nrb > 0 ? 1 : 0);
+  for (int part = 0; part < nparts; ++part) {
+    if (*sm.abort_flag) break;
+    if (xloads > 0 && !mbar_wait_bounded(sm.xfree, (xloads - 1) & 1, kWaitNs)) {
+      if (lane == 0) set_error(p, sm, kErrRingWait, 8);
+      break;
+    }
+    const int ps = part % p.KP;
+    if (lane == 0) {
+      mbar_arrive_expect_tx(sm.xfull, uint32_t(KC + (tail ? 1 : 0)) * p.LB * 128);
+      if (KC > 0) tma_load_3d(sm.xbuf, &tm.x_ch, 0, 0, ps * KC, sm.xfull, pol_x);
+      if (tail) tma_load_2d(sm.xbuf + size_t(KC) * p.LB * 128, &tm.x_2d, p.nKf * 64, 0, sm.xfull, pol_x);
+    }
+    __syncwarp();
+    ++xloads;
+  }
+  if (xloads > 0) mbar_wait_bounded(sm.xfull, (xloads - 1) & 1, kWaitNs / 10);  // the last x copies landed
+
+  // ---- h tiles after the grid barrier
+  int nG = 0;
+  for (int r = w.rA0; r < w.rA1; ++nG) r += group_at(p, r, w.rA1).h;
+  const int stagesA = p.KP * nG;
+  const int stagesB = w.nRBB * w.nEg * w.nJs;
+  if (stagesB == 0) return;
+  {
+    const uint64_t t0 = globaltimer_ns();
+    bool ok = true;
+    while (ld_acquire_gpu(&p.hdr->grid_bar) < gridDim.x) {
+      if (*sm.abort_flag || globaltimer_ns() - t0 > kWaitNs) { ok = false; break; }
+      __nanosleep(32);
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) {
+      if (lane == 0) set_error(p, sm, kErrGridBarrier, uint32_t(blockIdx.x));
+      return;
+    }
+    fence_proxy_async_global();
+  }
+  const uint64_t pol_h = policy_evict_last();
+  uint32_t hphase = 0;
+  int issued = 0;
+  int eg = 0, js = 0;
+  for (int jb = 0; jb < stagesB; ++jb) {
+    if (*sm.abort_flag) break;
+    const int i = stagesA + jb;
+    const int slot = i % p.S;
+    if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+      if (lane == 0) set_error(p, sm, kErrRingWait, 6);
+      break;
+    }
+    const int a0 = eg * p.NEB, nq = min(p.NEB, w.n_act - a0);
+    const int c0 = js * p.KWB, nc = min(p.KWB, p.nJc - c0);
+    const uint32_t bytes = uint32_t(nc) * p.HR * 128;
+    if (lane == 0) mbar_arrive_expect_tx(&sm.fullH[slot], bytes * nq);
+    __syncwarp();
+    if (lane < nq)
+      bulk_g2s(sm.ring + size_t(slot) * p.slot_bytes + size_t(lane) * p.eB + p.hoff,
+               p.h + size_t(a0 + lane) * p.h_expert_bytes + size_t(c0) * p.HR * 128, bytes, &sm.fullH[slot], pol_h);
+    __syncwarp();
+    hphase ^= 1u << slot;
+    ++issued;
+    if (++js == w.nJs) {
+      js = 0;
+      if (++eg == w.nEg) eg = 0;
+    }
+  }
+  uint32_t ph = hphase;
+  for (int k = issued - 1; k >= 0 && k >= issued - p.S; --k) {
+    const int slot = (stagesA + k) % p.S;
+    ph ^= 1u << slot;
+    mbar_wait_bounded(&sm.fullH[slot], (ph >> slot) & 1u, kWaitNs / 10);
+  }
+}
+
+// ------------------------------------------------------------------------------------- consumers
 template <int LC>
 __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
-  constexpr int MT = (2 * LC + 15) / 16;  // m-tiles of the down-projection (2L rows: h hi + lo)
-  const int ctid = threadIdx.x;           // consumers are threads [0, NCW*32)
-  const int lane = ctid % 32;
-  const int mtA = (p.L + 15) / 16, mtB = (2 * p.L + 15) / 16;
-  float acc[MT][4][4];
-  uint32_t hphase = 0;
-  int i = 0;  // global stage index, same order as the producers
+  constexpr int MTA = (LC + 15) / 16;
+  constexpr int MT = (2 * LC + 15) / 16;
+  const int ctid = threadIdx.x;
+  const int cw = ctid >> 5, lane = ctid & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int mtA = (p.L + 15) / 16, mtB = (p.HR + 15) / 16;
+  const uint32_t zaddr = smem_u32(sm.zero);
+  int i = 0, xloads = 0;
 
-  // ---------------- phase A: up-projection, Swish, router scale
-  for (int rb = 0; rb < w.nRBA; ++rb) {
-#pragma unroll
-    for (int a = 0; a < MT; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
-    const int r0 = w.rA0 + rb * RB, nrows = min(RB, w.nA - rb * RB);
-    const int a_first = r0 / p.de;
-    {
-      // r of the (at most kMaxSpan) experts this row-block touches, fetched while the stages stream
-      const int a_last = (r0 + nrows - 1) / p.de;
+  // ---------------- phase A
+  const int KC = p.nKf / p.KP;
+  const int nck = KC + (p.nKc > p.nKf ? 1 : 0);  // chunk tiles per stage
+  for (int r = w.rA0; r < w.rA1;) {
+    int ngr;
+    const int r_next = rowblock_walk(p, r, w.rA1, &ngr);
+    const int rb_r1 = r_next;
+    const int a_first = r / p.de;
+    {  // s and g of this row-block's experts, fetched while its stages stream in
+      const int a_last = (rb_r1 - 1) / p.de;
       for (int o = ctid; o < (a_last - a_first + 1) * p.L; o += NCW * 32) {
-        const int aa = o / p.L, t = o % p.L;
-        const float* src = p.r + size_t(t) * p.E + sm.act[a_first + aa];
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.rs + aa * p.L + t)), "l"(src)
+        const int aa = o / p.L, t = o - aa * p.L;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_s + aa * 32 + t)),
+                     "l"(p.s + size_t(t) * p.E + sm.act[a_first + aa])
                      : "memory");
       }
+      for (int aa = ctid; aa <= a_last - a_first; aa += NCW * 32)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_g + aa)),
+                     "l"(p.g + sm.act[a_first + aa])
+                     : "memory");
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    for (int kc = 0; kc < w.nKA; ++kc, ++i) {
-      const int slot = i % p.S;
-      if (ring_wait(p, sm, &sm.fullW[slot], (i / p.S) & 1, 3)) {
-        const uint8_t* base = sm.ring + size_t(slot) * p.slot_bytes;
-        const int kw = min(p.KcA, p.d - kc * p.KcA);
-        mma_stage<MT>(base, p.L, p.pitchA, base + p.woff, kw, sm.zero, acc, mtA);
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    // this warp's groups gl = cw + NCW q
+    Group gq[GPW];
+    int grow[GPW];
+#pragma unroll
+    for (int q = 0; q < GPW; ++q) {
+      const int gl = cw + q * NCW;
+      gq[q] = group_k(p, r, w.rA1, gl < ngr ? gl : 0, &grow[q]);
     }
-    stash<MT>(sm.red, acc);
+    float acc[GPW][MTA][4];
+#pragma unroll
+    for (int q = 0; q < GPW; ++q)
+#pragma unroll
+      for (int a = 0; a < MTA; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) acc[q][a][c] = 0.f;
+    for (int ps = 0; ps < p.KP; ++ps) {
+      if (p.KP > 1 || xloads == 0) {
+        ring_wait(p, sm, sm.xfull, xloads & 1, 7);
+        ++xloads;
+      }
+      const uint32_t xb = smem_u32(sm.xbuf);
+      for (int gl = 0; gl < ngr; ++gl, ++i) {
+        if ((gl % NCW) != cw) continue;
+        const int slot = i % p.S;
+        const int q = gl / NCW;
+        if (ring_wait(p, sm, &sm.fullW[slot], (i / p.S) & 1, 3)) {
+          int h = gq[0].h;
+#pragma unroll
+          for (int qq = 1; qq < GPW; ++qq)
+            if (qq == q) h = gq[qq].h;
+          const uint32_t wb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
+          const int brow = (lane & 7) < h ? (lane & 7) : 0;  // rows past the group: never used
+          float ak[4][MTA][4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+#pragma unroll
+            for (int mt = 0; mt < MTA; ++mt)
+#pragma unroll
+              for (int v = 0; v < 4; ++v) ak[k][mt][v] = 0.f;
+          for (int c = 0; c < nck; ++c) {
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16) {
+              uint32_t b0, b1, b2, b3;
+              const int wq = (c < KC ? c * h : (p.w1_tail_off >> 7)) + brow;  // tile row (1024-aligned tiles)
+              ldmatrix_x4(wb + swz(wq, k16 * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+#pragma unroll
+              for (int mt = 0; mt < MTA; ++mt) {
+                if (mt < mtA) {
+                  uint32_t a[4];
+                  const int row = mt * 16 + (lane & 15);
+                  const uint32_t ad = row < p.L ? xb + swz(c * p.LB + row, k16 * 2 + (lane >> 4)) : zaddr;
+                  ldmatrix_x4(ad, a[0], a[1], a[2], a[3]);
+                  mma_bf16_16816(ak[k16][mt], a, b0, b1);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int qq = 0; qq < GPW; ++qq)
+            if (qq == q)
+#pragma unroll
+              for (int mt = 0; mt < MTA; ++mt)
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                  acc[qq][mt][v] += (ak[0][mt][v] + ak[1][mt][v]) + (ak[2][mt][v] + ak[3][mt][v]);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cnt(&sm.empty[slot], NCW);  // the only warp that reads this stage
+      }
+      if (p.KP > 1) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.xfree);  // this warp is done with the x part
+      }
+    }
+    // epilogue of the row-block: h = r * Swish(u) as bf16 hi + lo, for this warp's groups
     asm volatile("cp.async.wait_all;" ::: "memory");
     named_bar_sync(1, NCW * 32);
-    for (int o = ctid; o < p.L * nrows; o += NCW * 32) {
-      const int t = o / nrows, c = o % nrows;
-      const float u = red_value<MT>(sm.red, t, c);
-      const int row = r0 + c;
-      const int a = row / p.de, j = row % p.de;
-      const float rr = sm.rs[(a - a_first) * p.L + t];
-      const float hv = rr * (u / (1.f + expf(-u)));
-      const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
-      p.h[(size_t(a) * 2 * p.L + t) * p.de + j] = hi;
-      p.h[(size_t(a) * 2 * p.L + p.L + t) * p.de + j] = lo;
+#pragma unroll
+    for (int qq = 0; qq < GPW; ++qq) {
+      const int gl = qq * NCW + cw;
+      if (gl >= ngr) continue;
+#pragma unroll
+      for (int mt = 0; mt < MTA; ++mt) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int t = mt * 16 + gid + (v >> 1) * 8;
+          const int n = tig * 2 + (v & 1);
+          if (t >= p.L || n >= gq[qq].h) continue;
+          const int a = gq[qq].a, j = gq[qq].j0 + n;
+          const float sv = sm.pre_s[(a - a_first) * 32 + t];
+          const float rms = sm.rms[t];
+          const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
+          const float u = acc[qq][mt][v];
+          const float hv = rr * (u / (1.f + expf(-u)));
+          const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
+          uint8_t* himg = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
+          const int col = j & 63;
+          *reinterpret_cast<__nv_bfloat16*>(himg + swz(t, col >> 3) + (col & 7) * 2) = hi;
+          *reinterpret_cast<__nv_bfloat16*>(himg + swz(p.L + t, col >> 3) + (col & 7) * 2) = lo;
+        }
+      }
     }
     named_bar_sync(1, NCW * 32);
+    r = r_next;
   }
-  // publish this CTA's h before any CTA starts reading h
+  // publish this CTA's h before any CTA reads h
   __threadfence();
   named_bar_sync(1, NCW * 32);
   if (ctid == 0) {
@@ -342,91 +465,257 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
     pdl_launch_dependents();
   }
 
-  // ---------------- phase B: down-projection over every active expert
+  // ---------------- phase B
+  const int ntB = p.RBB >> 3;  // RBB is a multiple of 8 (<= 32)
+  uint32_t hphase = 0;
   for (int rb = 0; rb < w.nRBB; ++rb) {
+    float acc[MT][4][4];
 #pragma unroll
     for (int a = 0; a < MT; ++a)
 #pragma unroll
       for (int b = 0; b < 4; ++b)
 #pragma unroll
         for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
-    for (int s = 0; s < w.n_act * w.nJB; ++s, ++i) {
+    for (int s = 0; s < w.nEg * w.nJs; ++s, ++i) {
       const int slot = i % p.S;
       const bool okW = ring_wait(p, sm, &sm.fullW[slot], (i / p.S) & 1, 4);
       const bool okH = okW && ring_wait(p, sm, &sm.fullH[slot], (hphase >> slot) & 1u, 5);
       hphase ^= 1u << slot;
       if (okH) {
-        const uint8_t* base = sm.ring + size_t(slot) * p.slot_bytes;
-        const int jc = s % w.nJB;
-        const int jw = min(p.KcB, p.de - jc * p.KcB);
-        mma_stage<MT>(base, 2 * p.L, p.pitchB, base + p.woff, jw, sm.zero, acc, mtB);
+        const int eg = s / w.nJs, js = s - eg * w.nJs;
+        const int nq = min(p.NEB, w.n_act - eg * p.NEB);
+        const int nc = min(p.KWB, p.nJc - js * p.KWB);
+        for (int qe = 0; qe < nq; ++qe) {
+          const uint32_t part = smem_u32(sm.ring + size_t(slot) * p.slot_bytes + size_t(qe) * p.eB);
+          // k-steps of 16 columns of j, split over the consumer warps (at most 4 per warp per chunk)
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            const int kk = cw + kq * NCW;
+            if (kk >= nc * 4) break;
+            const int c = kk >> 2, k16 = kk & 3;
+            const uint32_t ht = part + uint32_t(p.hoff + c * p.HR * 128);
+            uint32_t a[MT][4];
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+              if (mt < mtB) {
+                const int row = mt * 16 + (lane & 15);
+                const uint32_t addr = row < p.HR ? ht + swz(row, k16 * 2 + (lane >> 4)) : zaddr;
+                ldmatrix_x4(addr, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
+              }
+            }
+#pragma unroll
+            for (int np2 = 0; np2 < 2; ++np2) {
+              if (np2 * 2 < ntB) {
+                uint32_t b0, b1, b2, b3;
+                int row = np2 * 16 + (lane & 7) + (lane >> 4) * 8;
+                if (row >= p.RBB) row = 0;  // a second n-tile beyond the tile: loaded, never accumulated
+                ldmatrix_x4(part + swz(c * p.RBB + row, k16 * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                  if (mt < mtB) {
+                    mma_bf16_16816(acc[mt][np2 * 2], a[mt], b0, b1);
+                    if (np2 * 2 + 1 < ntB) mma_bf16_16816(acc[mt][np2 * 2 + 1], a[mt], b2, b3);
+                  }
+                }
+              }
+            }
+          }
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
     }
-    stash<MT>(sm.red, acc);
+    // sum the warps' partials in a fixed order; y = (hi part) + (lo part)
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+      for (int nt = 0; nt < 4; ++nt)
+        *reinterpret_cast<float4*>(sm.red + ((((cw * MT + mt) * 4 + nt) * 32 + lane) * 4)) =
+            make_float4(acc[mt][nt][0], acc[mt][nt][1], acc[mt][nt][2], acc[mt][nt][3]);
     named_bar_sync(1, NCW * 32);
-    const int k0 = w.rB0 + rb * RB, nrows = min(RB, w.nB - rb * RB);
+    const int k0 = w.rB0 + rb * p.RBB, nrows = min(p.RBB, w.nB - rb * p.RBB);
     for (int o = ctid; o < p.L * nrows; o += NCW * 32) {
-      const int t = o / nrows, c = o % nrows;
-      const float v = red_value<MT>(sm.red, t, c) + red_value<MT>(sm.red, p.L + t, c);
+      const int t = o / nrows, c = o - t * nrows;
+      float v = 0.f;
+      for (int half = 0; half < 2; ++half) {
+        const int row = half * p.L + t;
+        const int mt = row >> 4, r16 = row & 15;
+        const int ln = (r16 & 7) * 4 + ((c & 7) >> 1);
+        const int reg = (r16 >> 3) * 2 + (c & 1);
+        const int nt = c >> 3;
+#pragma unroll
+        for (int ww = 0; ww < NCW; ++ww) v += sm.red[((((ww * MT + mt) * 4 + nt) * 32 + ln) * 4) + reg];
+      }
       p.y[size_t(t) * p.d + k0 + c] = v;
     }
     named_bar_sync(1, NCW * 32);
   }
 }
 
+// ------------------------------------------------------------------------------------- prologue
+// Per token: RMS of relu(s) over the E experts and the active bits; then the union (ascending).
+__device__ void prologue_router_stats(const DecodeParams& p, const Smem& sm, float* sbuf) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nW = (p.E + 31) >> 5;
+  const int tg = p.sbuf_floats / p.E;  // tokens per staging group (>= 1)
+  for (int t0 = 0; t0 < p.L; t0 += tg) {
+    const int nt = min(tg, p.L - t0);
+    for (int o = tid; o < nt * p.E; o += kThreads)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sbuf + o)),
+                   "l"(p.s + size_t(t0) * p.E + o)
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    for (int tt = warp; tt < nt; tt += kThreads / 32) {
+      const float* st = sbuf + size_t(tt) * p.E;
+      float sumsq = 0.f;
+      for (int ww = 0; ww < nW; ++ww) {
+        const int e = ww * 32 + lane;
+        const float sv = e < p.E ? st[e] : -1.f;
+        const float a = fmaxf(sv, 0.f);
+        sumsq = fmaf(a, a, sumsq);
+        const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
+        if (lane == 0) sm.maskw[(t0 + tt) * 32 + ww] = bits;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+      if (lane == 0) sm.rms[t0 + tt] = sqrtf(sumsq / float(p.E));
+    }
+    __syncthreads();
+  }
+  if (warp == 0) {
+    uint32_t u = 0;
+    int tok_active = 0;
+    if (lane < nW)
+      for (int t = 0; t < p.L; ++t) {
+        const uint32_t m = sm.maskw[t * 32 + lane];
+        u |= m;
+        tok_active += __popc(m);
+      }
+    const int c = __popc(u);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    int pos = incl - c;
+    uint32_t rest = u;
+    while (rest) {
+      const int b = __ffs(rest) - 1;
+      rest &= rest - 1;
+      sm.act[pos++] = lane * 32 + b;
+    }
+    int act_sum = tok_active;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) act_sum += __shfl_xor_sync(0xffffffffu, act_sum, o);
+    if (lane == 0) {
+      *sm.n_act = total;
+      if (blockIdx.x == 0) {
+        *p.n_active = total;
+        if (p.counts) {
+          p.counts[0] = p.L * p.E - act_sum;
+          p.counts[1] = p.E - total;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {  // the chunk's outputs besides y
+    for (int a = tid; a < *sm.n_act; a += kThreads) p.active_idx[a] = sm.act[a];
+    if (p.tok_mask)
+      for (int o = tid; o < p.L * nW; o += kThreads) p.tok_mask[o] = sm.maskw[(o / nW) * 32 + (o % nW)];
+  }
+}
+
+__device__ void write_router_outputs(const DecodeParams& p, const Smem& sm) {
+  // r = g * relu(s) / rms, the same expression the up-projection epilogue uses
+  for (int o = threadIdx.x; o < p.L * p.E; o += kThreads) {
+    const int t = o / p.E, e = o - t * p.E;
+    const float rms = sm.rms[t];
+    p.r_out[o] = rms > 0.f ? (p.g[e] * fmaxf(p.s[o], 0.f)) / rms : 0.f;
+  }
+}
+
 template <int LC>
-__global__ void __launch_bounds__(kThreads, 1) expert_decode_kernel(DecodeParams p) {
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
+__global__ void __launch_bounds__(kThreads, 1)
+    expert_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TensorMaps tm) {
+  extern __shared__ uint8_t smem_raw[];
   constexpr int MT = (2 * LC + 15) / 16;
+  constexpr int kRedBytes = NCW * MT * 4 * 32 * 4 * 4;
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem sm;
-  sm.ring = smem_raw;
-  sm.red = reinterpret_cast<float*>(smem_raw + size_t(p.S) * p.slot_bytes);
-  // tail (16-byte aligned): zero block [16] | abort flag [16] | fullW[S] | fullH[S] | empty[S] |
-  // act[E] | rs[kMaxSpan][L]
-  uint8_t* tail = reinterpret_cast<uint8_t*>(sm.red + NCW * MT * 4 * 32 * 4);
+  sm.xbuf = base;
+  sm.ring = base + p.xbuf_bytes;
+  uint8_t* after_ring = sm.ring + size_t(p.S) * p.slot_bytes;
+  const bool red_alias = p.xbuf_bytes >= kRedBytes;  // x is no longer needed in phase B
+  sm.red = reinterpret_cast<float*>(red_alias ? sm.xbuf : after_ring);
+  uint8_t* tail = red_alias ? after_ring : after_ring + kRedBytes;
   sm.zero = tail;
   sm.abort_flag = reinterpret_cast<volatile int*>(tail + 16);
   sm.fullW = reinterpret_cast<uint64_t*>(tail + 32);
   sm.fullH = sm.fullW + p.S;
   sm.empty = sm.fullH + p.S;
-  sm.act = reinterpret_cast<int32_t*>(sm.empty + p.S);
-  sm.rs = reinterpret_cast<float*>(sm.act + p.E);
+  sm.xfull = sm.empty + p.S;
+  sm.xfree = sm.xfull + 1;
+  sm.act = reinterpret_cast<int32_t*>(sm.xfree + 1);
+  sm.n_act = sm.act + kMaxE;
+  sm.rms = reinterpret_cast<float*>(sm.n_act + 4);
+  sm.maskw = reinterpret_cast<uint32_t*>(sm.rms + 32);
+  sm.pre_s = reinterpret_cast<float*>(sm.maskw + 32 * 32);
+  sm.pre_g = sm.pre_s + kMaxSpan * 32;
 
-  if (threadIdx.x == 0) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
     for (int s = 0; s < p.S; ++s) {
       mbar_init(&sm.fullW[s], 1);
       mbar_init(&sm.fullH[s], 1);
       mbar_init(&sm.empty[s], NCW);
     }
+    mbar_init(sm.xfull, 1);
+    mbar_init(sm.xfree, NCW);
     *reinterpret_cast<uint4*>(sm.zero) = make_uint4(0, 0, 0, 0);
     *sm.abort_flag = 0;
     fence_mbar_init();
   }
+  if (warp == NCW && lane == 0) {
+    for (int k = 0; k < 4; ++k) {
+      prefetch_tensormap(&tm.w1_ch[k]);
+      prefetch_tensormap(&tm.w1_3d[k]);
+    }
+    prefetch_tensormap(&tm.w2_ch);
+    prefetch_tensormap(&tm.w2_3d);
+    prefetch_tensormap(&tm.x_ch);
+    prefetch_tensormap(&tm.x_2d);
+  }
   __syncthreads();
 
-  // the router (previous kernel) wrote the active list, r and reset the grid barrier
+  // the router wrote s and reset the grid barrier
   pdl_wait();
-  // one round trip: the count and the whole list (entries past the count are not used)
-  const int n_raw = *p.n_active;
-  for (int a = threadIdx.x; a < p.E; a += kThreads) sm.act[a] = min(max(p.active_idx[a], 0), p.E - 1);
-  const int n_act = min(max(n_raw, 0), p.E);  // never index past the active list
+  prologue_router_stats(p, sm, reinterpret_cast<float*>(sm.ring));
+  fence_proxy_async_smem();  // the ring held s (generic writes) before bulk copies write into it
   __syncthreads();
+  const int n_act = *sm.n_act;
   const Work w = make_work(p, n_act);
 
-  const int warp = threadIdx.x / 32;
   if (warp < NCW) {
     consume<LC>(p, sm, w);
   } else if (warp == NCW) {
-    produce_weights(p, sm, w);
+    produce_weights(p, tm, sm, w);
   } else {
-    produce_h(p, sm, w);
+    produce_x_h(p, tm, sm, w);
+  }
+  if (blockIdx.x == 0 && p.r_out) {
+    __syncthreads();
+    write_router_outputs(p, sm);
   }
 }
 
 template <int LC>
-cudaError_t launch_lc(const DecodeParams& p, const DecodeLaunch& plan, cudaStream_t st, bool pdl) {
+cudaError_t launch_lc(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan, cudaStream_t st,
+                      bool pdl) {
   auto kfn = expert_decode_kernel<LC>;
   cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
@@ -440,46 +729,89 @@ cudaError_t launch_lc(const DecodeParams& p, const DecodeLaunch& plan, cudaStrea
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, kfn, p);
+  return cudaLaunchKernelEx(&cfg, kfn, p, tm);
 }
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 }  // namespace
 
-bool expert_decode_plan(int L, int d, int de, int num_sms, int max_smem, DecodeParams* p,
+size_t decode_h_bytes(int L, int E, int de) { return size_t(E) * ((de + 63) / 64) * size_t(2 * L) * 128; }
+
+bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, DecodeParams* p,
                         DecodeLaunch* out) {
-  if (L < 1 || L > kDecodeMaxL) return false;
+  if (L < 1 || L > kDecodeMaxL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
   const int lc = L <= 8 ? 8 : L <= 16 ? 16 : 32;
   const int mt = (2 * lc + 15) / 16;
-  p->KcA = d < 256 ? d : 256;
-  p->KcB = de < 256 ? de : 256;
-  p->pitchA = round_up(p->KcA * 2, 128) + 16;
-  p->pitchB = round_up(p->KcB * 2, 128) + 16;
-  const int pitch_max = p->pitchA > p->pitchB ? p->pitchA : p->pitchB;
-  const int areg = round_up(L * p->pitchA > 2 * L * p->pitchB ? L * p->pitchA : 2 * L * p->pitchB, 128);
-  p->woff = areg;
-  p->slot_bytes = round_up(areg + RB * pitch_max, 128);
-  const size_t red_bytes = size_t(NCW) * mt * 4 * 32 * 4 * 4;
-  const size_t extra = size_t(kMaxE) * 4 + size_t(kMaxSpan) * kDecodeMaxL * 4;  // act + rs
-  const size_t fixed = red_bytes + 3 * 8 * 32 + 64 + extra;
-  if (size_t(max_smem) <= fixed) return false;
+  const int G = num_sms;
+  if (d > 256 * 64) return false;  // a box spans at most 256 chunks
+  // up-projection: x resident per pass of KC full 64-column chunks (plus the ragged chunk, which
+  // needs a single pass); stages of one box of up to RSM whole rows
+  p->nKf = d / 64;
+  p->nKc = (d + 63) / 64;
+  p->LB = round_up(L, 8);
+  const int xbudget = 100 * 1024;
+  p->KP = 1;
+  if (p->nKc > p->nKf) {
+    if (size_t(p->nKc) * p->LB * 128 > size_t(xbudget)) return false;
+  } else {
+    while (size_t(p->nKf / p->KP) * p->LB * 128 > size_t(xbudget) || p->nKf % p->KP != 0) {
+      if (++p->KP > p->nKf) return false;
+    }
+  }
+  const int KC = p->nKf / p->KP;
+  const int nck = KC + (p->nKc > p->nKf ? 1 : 0);
+  p->Kp = KC * 64;
+  p->xbuf_bytes = round_up(nck * p->LB * 128, 1024);
+  const int target = 32 * 1024;
+  p->RSM = 8;
+  while (p->RSM > 1 && p->RSM * nck * 128 > target) p->RSM >>= 1;
+  // the ragged chunk's tile sits at a 1024-byte aligned offset after the full chunks
+  p->w1_tail_off = round_up(KC * p->RSM * 128, 1024);
+  const int slotA = round_up(nck > KC ? p->w1_tail_off + p->RSM * 128 : KC * p->RSM * 128, 1024);
+  // down-projection: W2 boxes of RBB rows x KWB chunks per expert, NEB experts per stage
+  p->HR = 2 * L;
+  p->nJc = (de + 63) / 64;
+  p->nJf = de / 64;
+  p->h_expert_bytes = p->nJc * p->HR * 128;
+  const int rbmax = (d + G - 1) / G;
+  p->RBB = round_up(rbmax < 1 ? 1 : (rbmax > 32 ? 32 : rbmax), 8);
+  auto part_bytes = [&](int kwb) {
+    const int w2 = p->RBB * kwb * 128;  // multiple of 1024
+    return round_up(w2 + round_up(p->HR * kwb * 128, 16), 1024);
+  };
+  p->KWB = p->nJc;
+  if (p->nJf >= 1 && p->KWB > p->nJf) p->KWB = p->nJf;
+  while (p->KWB > 1 && part_bytes(p->KWB) > (slotA > 8192 ? slotA : 8192)) --p->KWB;
+  p->hoff = p->RBB * p->KWB * 128;
+  p->eB = part_bytes(p->KWB);
+  const int slot = round_up(slotA > p->eB ? slotA : p->eB, 1024);
+  p->NEB = slot / p->eB;
+  if (p->NEB < 1) p->NEB = 1;
+  p->slot_bytes = slot;
+  const size_t red = size_t(NCW) * mt * 4 * 32 * 4 * 4;
+  const size_t red_extra = size_t(p->xbuf_bytes) >= red ? 0 : red;
+  const size_t tail = 32 + 3 * 8 * 32 + 16 + size_t(kMaxE + 4) * 4 + 32 * 4 + 32 * 32 * 4 + (kMaxSpan * 33) * 4;
+  const size_t fixed = 1024 + size_t(p->xbuf_bytes) + red_extra + tail;
+  if (fixed >= size_t(max_smem)) return false;
   int S = int((size_t(max_smem) - fixed) / size_t(p->slot_bytes));
-  if (S > 16) S = 16;
+  if (S > 32) S = 32;
   if (S < 2) return false;
   p->S = S;
-  out->grid = num_sms;
+  p->sbuf_floats = int(size_t(S) * p->slot_bytes / 4);  // the prologue stages s in the ring
+  if (p->sbuf_floats < E) return false;
+  out->grid = G;
   out->lclass = lc;
-  out->smem = size_t(S) * p->slot_bytes + red_bytes + 3 * 8 * size_t(S) + 64 + extra;
+  out->smem = fixed + size_t(S) * p->slot_bytes;
   return true;
 }
 
-cudaError_t expert_decode_launch(const DecodeParams& p, const DecodeLaunch& plan, cudaStream_t st,
-                                 bool pdl) {
+cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
+                                 cudaStream_t st, bool pdl) {
   switch (plan.lclass) {
-    case 8: return launch_lc<8>(p, plan, st, pdl);
-    case 16: return launch_lc<16>(p, plan, st, pdl);
-    default: return launch_lc<32>(p, plan, st, pdl);
+    case 8: return launch_lc<8>(p, tm, plan, st, pdl);
+    case 16: return launch_lc<16>(p, tm, plan, st, pdl);
+    default: return launch_lc<32>(p, tm, plan, st, pdl);
   }
 }
 

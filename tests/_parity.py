@@ -9,9 +9,11 @@ import oracle
 # y tolerance: |y - y_ref| <= 2e-2 |y_ref| + 1e-3 rms(y_ref), per element (rms over the call's y_ref)
 Y_RTOL = 2e-2
 Y_ATOL_RMS = 1e-3
-# router output r: fp32 arithmetic against fp64
-R_RTOL = 2e-5
-R_ATOL = 1e-6
+# router output r = g relu(s) / rms: s is an fp32 dot product over d ~ 2-4K terms of size O(1/sqrt(d)),
+# so its absolute rounding error is ~1e-6..1e-5 whatever the summation order, and rms(r/g) = 1 puts
+# r on the same O(1) scale: |r - r_ref| <= 1e-5 + 1e-5 |r_ref|.
+R_RTOL = 1e-5
+R_ATOL = 1e-5
 
 
 class DeviceLayer:
