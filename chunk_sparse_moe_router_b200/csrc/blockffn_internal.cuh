@@ -94,6 +94,8 @@ struct DecodeParams {
   int LB;           // x tile rows (L rounded up to 8)
   int xbuf_bytes;   // resident x tiles [chunks of a pass][LB][128 B]
   int w1_tail_off;  // offset of the ragged-chunk tile in an up-projection stage (1024-aligned)
+  int ustage_bytes; // shared-memory staging of a CTA's up-projection sums (K split only)
+  int ksplit;       // 1: L <= 8 and one pass: the consumer warps split K inside every up-projection stage
   // down-projection: stages of NEB experts, each a W2 box of RBB rows x KWB 64-column chunks
   int NEB;
   int nJc, nJf;     // 64-column chunks of de (all / full)

@@ -38,11 +38,12 @@
 namespace bffn {
 namespace {
 
-constexpr int NCW = 4;                      // consumer warps
+constexpr int NCW = 8;                      // consumer warps
 constexpr int kThreads = (NCW + 2) * 32;    // + weight producer warp + x / h producer warp
-constexpr int GPW = 2;                      // row groups per consumer warp per row-block
-constexpr int GB = NCW * GPW;               // row groups per row-block
-constexpr int kMaxSpan = GB;                // experts one row-block can touch (a group never crosses one)
+constexpr int GPW = 2;                      // row groups per consumer warp per row-block (x in smem)
+constexpr int GB = NCW * GPW;               // row groups per row-block (x in smem)
+constexpr int kMaxSpan = 16;                // experts a CTA's up-projection rows touch (<= E / G + 2)
+constexpr int kXregChunks = 4;              // 64-column chunks of x one warp keeps in registers
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 // ------------------------------------------------------------------------------------- smem
@@ -61,29 +62,49 @@ struct Smem {
   int* n_act;          // [1]
   float* rms;          // [32] per-token sqrt(mean relu(s)^2)
   uint32_t* maskw;     // [32][32] per-token active bits
-  float* pre_s;        // [kMaxSpan][32] s of the current row-block's experts
+  float* pre_s;        // [kMaxSpan][32] s of the experts of this CTA's up-projection rows
   float* pre_g;        // [kMaxSpan]
+  float* red_s;        // [S][NCW][32][2] per-stage partial sums (K split)
+  uint64_t* rbar;      // [S] partial sums of a stage written (NCW arrivals)
+  float* ustage;       // [(rA1 - rA0) / 8][L][8] this CTA's up-projection sums u, until the end of phase A (K split)
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk16) {
   return uint32_t(row * 128 + ((chunk16 ^ (row & 7)) << 4));
 }
 
+// The CTA's abort flag, read and written with explicit shared-memory instructions.
+__device__ __forceinline__ bool aborted(const Smem& sm) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)sm.abort_flag)) : "memory");
+  return v != 0;
+}
+__device__ __forceinline__ void set_abort(const Smem& sm) {
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(smem_u32((const void*)sm.abort_flag)), "r"(1u) : "memory");
+}
+
 __device__ __forceinline__ void set_error(const DecodeParams& p, const Smem& sm, uint32_t bit, uint32_t info) {
   atomicOr(&p.hdr->err, bit);
   p.hdr->err_info = info;
-  *sm.abort_flag = 1;
+  set_abort(sm);
 }
 
 // A wait that records a timeout and marks the CTA aborted; once aborted, waits are skipped (callers
 // skip the work) so that every warp still reaches the same named barriers and the CTA can finish.
+// The first try is inline, the rest out of line.
+__device__ __noinline__ bool ring_wait_slow(const DecodeParams& p, const Smem& sm, uint64_t* bar, uint32_t parity,
+                                            uint32_t where) {
+  if (aborted(sm)) return false;
+  if (mbar_wait_slow(bar, parity, kWaitNs)) return true;
+  if ((threadIdx.x & 31) == 0) set_error(p, sm, kErrRingWait, where);
+  set_abort(sm);
+  return false;
+}
+
 __device__ __forceinline__ bool ring_wait(const DecodeParams& p, const Smem& sm, uint64_t* bar, uint32_t parity,
                                           uint32_t where) {
-  if (*sm.abort_flag) return false;
-  if (mbar_wait_bounded(bar, parity, kWaitNs)) return true;
-  if ((threadIdx.x & 31) == 0) set_error(p, sm, kErrRingWait, where);
-  *sm.abort_flag = 1;
-  return false;
+  if (mbar_try_wait(bar, parity) && !aborted(sm)) return true;
+  return ring_wait_slow(p, sm, bar, parity, where);
 }
 
 // ------------------------------------------------------------------------------------- work split
@@ -99,9 +120,10 @@ struct Work {
 __device__ __forceinline__ Work make_work(const DecodeParams& p, int n_act) {
   Work w;
   const int G = gridDim.x, c = blockIdx.x;
-  const long long RA = (long long)n_act * p.de;
-  w.rA0 = int(RA * c / G);
-  w.rA1 = int(RA * (c + 1) / G);
+  // in units of 8 rows, so a 16-byte piece of the h image (8 consecutive j) belongs to one CTA
+  const long long RA8 = (long long)n_act * p.de / 8;
+  w.rA0 = int(RA8 * c / G) * 8;
+  w.rA1 = int(RA8 * (c + 1) / G) * 8;
   w.rB0 = int((long long)p.d * c / G);
   w.nB = int((long long)p.d * (c + 1) / G) - w.rB0;
   w.nRBB = (w.nB + p.RBB - 1) / p.RBB;
@@ -153,12 +175,28 @@ __device__ __forceinline__ Group group_k(const DecodeParams& p, int r, int r_end
 
 __device__ __forceinline__ bool stage_is_chunked(int c0, int nc, int nfull) { return c0 + nc <= nfull; }
 
+// Position in the stage ring: stage index, its slot, and the parity of the slot's barrier phase that
+// the stage uses (advanced incrementally: no division per stage).
+struct RingPos {
+  int i = 0, slot = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next(int S) {
+    ++i;
+    if (++slot == S) slot = 0, ph ^= 1u;
+  }
+  __device__ __forceinline__ void seek(int k, int S) {
+    i = k;
+    slot = k % S;
+    ph = uint32_t(k / S) & 1u;
+  }
+};
+
 // ------------------------------------------------------------------------------------- producers
 // Weight producer (one warp): W1 row groups, then W2 expert tiles, in stage order.
 __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_w = policy_evict_first();
-  int i = 0;
+  RingPos rp;
   bool ok = true;
   // ---- phase A: stage = one box of a group's whole rows over the pass's columns
   const int KC = p.nKf / p.KP;                 // full chunks per pass
@@ -171,10 +209,10 @@ __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, con
     const int hsel = __ffs(mine.h) - 1;
     const int e = sm.act[mine.a];
     for (int ps = 0; ps < p.KP && ok; ++ps) {
-      for (int gl = 0; gl < ngr; ++gl, ++i) {
-        if (*sm.abort_flag) { ok = false; break; }
-        const int slot = i % p.S;
-        if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+      for (int gl = 0; gl < ngr; ++gl, rp.next(p.S)) {
+        if (aborted(sm)) { ok = false; break; }
+        const int slot = rp.slot;
+        if (rp.i >= p.S && !mbar_wait_bounded(&sm.empty[slot], rp.ph ^ 1u, kWaitNs)) {
           if (lane == 0) set_error(p, sm, kErrRingWait, 1);
           ok = false;
           break;
@@ -198,10 +236,10 @@ __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, con
     const int k0 = w.rB0 + rb * p.RBB;
     for (int eg = 0; eg < w.nEg && ok; ++eg) {
       const int a0 = eg * p.NEB, nq = min(p.NEB, w.n_act - a0);
-      for (int js = 0; js < w.nJs; ++js, ++i) {
-        if (*sm.abort_flag) { ok = false; break; }
-        const int slot = i % p.S;
-        if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+      for (int js = 0; js < w.nJs; ++js, rp.next(p.S)) {
+        if (aborted(sm)) { ok = false; break; }
+        const int slot = rp.slot;
+        if (rp.i >= p.S && !mbar_wait_bounded(&sm.empty[slot], rp.ph ^ 1u, kWaitNs)) {
           if (lane == 0) set_error(p, sm, kErrRingWait, 2);
           ok = false;
           break;
@@ -225,7 +263,7 @@ __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, con
     }
   }
   // every copy this warp issued lands before the CTA may exit
-  for (int k = max(0, i - p.S); k < i; ++k) mbar_wait_bounded(&sm.fullW[k % p.S], (k / p.S) & 1, kWaitNs / 10);
+  for (int k = max(0, rp.i - p.S); k < rp.i; ++k) mbar_wait_bounded(&sm.fullW[k % p.S], (k / p.S) & 1, kWaitNs / 10);
 }
 
 // x / h producer (one warp): the resident x parts of phase A, then (after the grid barrier) the h
@@ -244,7 +282,7 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
   int xloads = 0;
   const int nparts = (p.KP > 1) ? nrb * p.KP : (nrb > 0 ? 1 : 0);
   for (int part = 0; part < nparts; ++part) {
-    if (*sm.abort_flag) break;
+    if (aborted(sm)) break;
     if (xloads > 0 && !mbar_wait_bounded(sm.xfree, (xloads - 1) & 1, kWaitNs)) {
       if (lane == 0) set_error(p, sm, kErrRingWait, 8);
       break;
@@ -270,7 +308,7 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
     const uint64_t t0 = globaltimer_ns();
     bool ok = true;
     while (ld_acquire_gpu(&p.hdr->grid_bar) < gridDim.x) {
-      if (*sm.abort_flag || globaltimer_ns() - t0 > kWaitNs) { ok = false; break; }
+      if (aborted(sm) || globaltimer_ns() - t0 > kWaitNs) { ok = false; break; }
       __nanosleep(32);
     }
     ok = __all_sync(0xffffffffu, ok);
@@ -284,11 +322,12 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
   uint32_t hphase = 0;
   int issued = 0;
   int eg = 0, js = 0;
-  for (int jb = 0; jb < stagesB; ++jb) {
-    if (*sm.abort_flag) break;
-    const int i = stagesA + jb;
-    const int slot = i % p.S;
-    if (i >= p.S && !mbar_wait_bounded(&sm.empty[slot], ((i / p.S) - 1) & 1, kWaitNs)) {
+  RingPos rp;
+  rp.seek(stagesA, p.S);
+  for (int jb = 0; jb < stagesB; ++jb, rp.next(p.S)) {
+    if (aborted(sm)) break;
+    const int slot = rp.slot;
+    if (rp.i >= p.S && !mbar_wait_bounded(&sm.empty[slot], rp.ph ^ 1u, kWaitNs)) {
       if (lane == 0) set_error(p, sm, kErrRingWait, 6);
       break;
     }
@@ -317,40 +356,170 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
 }
 
 // ------------------------------------------------------------------------------------- consumers
-template <int LC>
-__device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
-  constexpr int MTA = (LC + 15) / 16;
-  constexpr int MT = (2 * LC + 15) / 16;
-  const int ctid = threadIdx.x;
-  const int cw = ctid >> 5, lane = ctid & 31;
-  const int gid = lane >> 2, tig = lane & 3;
-  const int mtA = (p.L + 15) / 16, mtB = (p.HR + 15) / 16;
-  const uint32_t zaddr = smem_u32(sm.zero);
-  int i = 0, xloads = 0;
+// The epilogue of one up-projection value: h = r * Swish(u), stored as bf16 hi and lo parts in the
+// down-projection's tile layout.
+__device__ __forceinline__ void store_h(const DecodeParams& p, const Smem& sm, int a_first, int a, int j, int t,
+                                        float u) {
+  const float sv = sm.pre_s[(a - a_first) * 32 + t];
+  const float rms = sm.rms[t];
+  const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
+  const float hv = rr * (u / (1.f + expf(-u)));
+  const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
+  uint8_t* himg = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
+  const int col = j & 63;
+  *reinterpret_cast<__nv_bfloat16*>(himg + swz(t, col >> 3) + (col & 7) * 2) = hi;
+  *reinterpret_cast<__nv_bfloat16*>(himg + swz(p.L + t, col >> 3) + (col & 7) * 2) = lo;
+}
 
-  // ---------------- phase A
+// Up-projection split over K (L <= 8, one pass): every consumer warp works on every stage over its
+// own 64-column chunks c = cw + NCW q, writes its partial sums, and the stage's designated warp adds
+// the NCW partials in warp order, finishes the group and frees the slot.  The x fragments of the
+// first kXregChunks chunks of a warp stay in registers; further chunks read them from shared memory.
+// Only tokens 0-7 are real rows of the MMA (rows 8-15 are zero).  Every group has RSM rows (the CTA's
+// rows are whole multiples of 8 and RSM <= 8), so a warp's operand offsets inside a stage are the
+// same for every stage and are computed once; chunks past the end read a zero row, so loads and
+// MMAs run unconditionally.
+__device__ void phase_a_ksplit(const DecodeParams& p, const Smem& sm, const Work& w, int a_first, RingPos& rp) {
+  const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int KC = p.nKf;
+  const int nck = p.nKc;
+  const int h = p.RSM;
+  const uint32_t xb = smem_u32(sm.xbuf), zaddr = smem_u32(sm.zero);
+  const int lrow = lane & 7, lhalf = (lane >> 3) & 1;  // ldmatrix .x2 addressing: rows 0-7, two k halves
+  if (w.rA0 >= w.rA1) return;  // no up-projection rows: x is not loaded
+  // the offset inside a stage of this lane's 16-byte piece for chunk c, k16 = 0 (k16 adds 32 bytes
+  // before the swizzle: the swizzled chunk index is (2 k16 + lhalf) ^ (row & 7))
+  auto w_row = [&](int c) { return (c < KC ? c * h : (p.w1_tail_off >> 7)) + (lrow < h ? lrow : 0); };
+  ring_wait(p, sm, sm.xfull, 0, 7);
+  uint32_t xf[kXregChunks][4][2];
+  int wrow[kXregChunks];
+#pragma unroll
+  for (int q = 0; q < kXregChunks; ++q) {
+    const int c = cw + q * NCW;
+    wrow[q] = c < nck ? w_row(c) : -1;
+#pragma unroll
+    for (int k16 = 0; k16 < 4; ++k16) {
+      const uint32_t ad = c < nck ? xb + swz(c * p.LB + lrow, k16 * 2 + lhalf) : zaddr;
+      ldmatrix_x2(ad, xf[q][k16][0], xf[q][k16][1]);
+    }
+  }
+  for (int r = w.rA0; r < w.rA1; r += h, rp.next(p.S)) {
+    const int slot = rp.slot;
+    if (ring_wait(p, sm, &sm.fullW[slot], rp.ph, 3)) {
+      const uint32_t wb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
+      // all fragment loads of a batch first, then its MMAs: one k16 chain per accumulator
+      float ak[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) ak[k][v] = 0.f;
+#pragma unroll
+      for (int q0 = 0; q0 < kXregChunks; q0 += 2) {  // two chunks per batch
+        uint32_t wf[2][4][2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const int wr = wrow[q0 + q];
+            const uint32_t ad = wr >= 0 ? wb + swz(wr, k16 * 2 + lhalf) : zaddr;
+            ldmatrix_x2(ad, wf[q][k16][0], wf[q][k16][1]);
+          }
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+#pragma unroll
+          for (int k16 = 0; k16 < 4; ++k16) {
+            const uint32_t a[4] = {xf[q0 + q][k16][0], 0u, xf[q0 + q][k16][1], 0u};
+            mma_bf16_16816(ak[k16], a, wf[q][k16][0], wf[q][k16][1]);
+          }
+      }
+      for (int c = cw + kXregChunks * NCW; c < nck; c += NCW) {  // chunks whose x stays in smem
+        const int wr = w_row(c);
+        uint32_t wf[4][2], xs[4][2];
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          ldmatrix_x2(wb + swz(wr, k16 * 2 + lhalf), wf[k16][0], wf[k16][1]);
+          ldmatrix_x2(xb + swz(c * p.LB + lrow, k16 * 2 + lhalf), xs[k16][0], xs[k16][1]);
+        }
+#pragma unroll
+        for (int k16 = 0; k16 < 4; ++k16) {
+          const uint32_t a[4] = {xs[k16][0], 0u, xs[k16][1], 0u};
+          mma_bf16_16816(ak[k16], a, wf[k16][0], wf[k16][1]);
+        }
+      }
+      float2* red = reinterpret_cast<float2*>(sm.red_s) + size_t(slot) * NCW * 32;
+      red[cw * 32 + lane] = make_float2((ak[0][0] + ak[1][0]) + (ak[2][0] + ak[3][0]),
+                                        (ak[0][1] + ak[1][1]) + (ak[2][1] + ak[3][1]));
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.rbar[slot]);
+    if ((rp.i % NCW) == cw) {  // this warp finishes the stage
+      const bool ok = ring_wait(p, sm, &sm.rbar[slot], rp.ph, 9);
+      float u0 = 0.f, u1 = 0.f;
+      if (ok) {
+        const float2* red = reinterpret_cast<const float2*>(sm.red_s) + size_t(slot) * NCW * 32;
+#pragma unroll
+        for (int ww = 0; ww < NCW; ++ww) {
+          const float2 v = red[ww * 32 + lane];
+          u0 += v.x;
+          u1 += v.y;
+        }
+      }
+      // the slot and its partial sums are free once read; u waits in shared memory for the epilogue
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cnt(&sm.empty[slot], NCW);
+      const int t = gid, loc = r - w.rA0 + tig * 2;  // rows loc, loc + 1 of the CTA (loc even)
+      if (ok && t < p.L && tig * 2 < h)
+        *reinterpret_cast<float2*>(sm.ustage + ((loc >> 3) * p.L + t) * 8 + (loc & 7)) = make_float2(u0, u1);
+    }
+  }
+  // Epilogue, once per CTA: h = r Swish(u) with r = g relu(s) / rms, split into bf16 hi and lo parts and
+  // written to the global h image as 16-byte pieces of 8 consecutive j (one expert each: the CTA's
+  // rows are whole multiples of 8 and de is a multiple of 16).
+  named_bar_sync(1, NCW * 32);
+  const int units = (w.rA1 - w.rA0) >> 3;
+  for (int o = threadIdx.x; o < units * p.L; o += NCW * 32) {
+    const int u = o / p.L, t = o - u * p.L;
+    const int row = w.rA0 + u * 8;
+    const int a = row / p.de, j = row - a * p.de;
+    const float rms = sm.rms[t];
+    const float sv = sm.pre_s[(a - a_first) * 32 + t];
+    const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
+    const float4* us = reinterpret_cast<const float4*>(sm.ustage + (u * p.L + t) * 8);
+    const float4 ua = us[0], ub = us[1];
+    const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float h0 = rr * (uv[2 * k] / (1.f + expf(-uv[2 * k])));
+      const float h1 = rr * (uv[2 * k + 1] / (1.f + expf(-uv[2 * k + 1])));
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(h0, h1);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(h0 - __low2float(hh), h1 - __high2float(hh));
+      hi[k] = *reinterpret_cast<const uint32_t*>(&hh);
+      lo[k] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    uint8_t* img = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
+    *reinterpret_cast<uint4*>(img + swz(t, (j & 63) >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(img + swz(p.L + t, (j & 63) >> 3)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
+// Up-projection with x resident in shared memory (any L, K in passes): a consumer warp owns whole
+// row groups (gl = cw + NCW q within a row-block of GB groups) over all of K.
+template <int MTA>
+__device__ void phase_a_smem(const DecodeParams& p, const Smem& sm, const Work& w, int a_first, RingPos& rp) {
+  const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gid = lane >> 2, tig = lane & 3;
+  const int mtA = (p.L + 15) / 16;
+  const uint32_t zaddr = smem_u32(sm.zero);
   const int KC = p.nKf / p.KP;
-  const int nck = KC + (p.nKc > p.nKf ? 1 : 0);  // chunk tiles per stage
+  const int nck = KC + (p.nKc > p.nKf ? 1 : 0);
+  const int tail_q = p.w1_tail_off >> 7;
+  int xloads = 0;
   for (int r = w.rA0; r < w.rA1;) {
     int ngr;
     const int r_next = rowblock_walk(p, r, w.rA1, &ngr);
-    const int rb_r1 = r_next;
-    const int a_first = r / p.de;
-    {  // s and g of this row-block's experts, fetched while its stages stream in
-      const int a_last = (rb_r1 - 1) / p.de;
-      for (int o = ctid; o < (a_last - a_first + 1) * p.L; o += NCW * 32) {
-        const int aa = o / p.L, t = o - aa * p.L;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_s + aa * 32 + t)),
-                     "l"(p.s + size_t(t) * p.E + sm.act[a_first + aa])
-                     : "memory");
-      }
-      for (int aa = ctid; aa <= a_last - a_first; aa += NCW * 32)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_g + aa)),
-                     "l"(p.g + sm.act[a_first + aa])
-                     : "memory");
-      asm volatile("cp.async.commit_group;" ::: "memory");
-    }
-    // this warp's groups gl = cw + NCW q
     Group gq[GPW];
     int grow[GPW];
 #pragma unroll
@@ -371,11 +540,12 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
         ++xloads;
       }
       const uint32_t xb = smem_u32(sm.xbuf);
-      for (int gl = 0; gl < ngr; ++gl, ++i) {
-        if ((gl % NCW) != cw) continue;
-        const int slot = i % p.S;
+      // every warp waits for and releases every stage in order (one barrier phase at a time, so the
+      // parity of a wait is never ambiguous whatever S is); only the stage's owner computes
+      for (int gl = 0; gl < ngr; ++gl, rp.next(p.S)) {
+        const int slot = rp.slot;
         const int q = gl / NCW;
-        if (ring_wait(p, sm, &sm.fullW[slot], (i / p.S) & 1, 3)) {
+        if (ring_wait(p, sm, &sm.fullW[slot], rp.ph, 3) && (gl % NCW) == cw) {
           int h = gq[0].h;
 #pragma unroll
           for (int qq = 1; qq < GPW; ++qq)
@@ -390,10 +560,10 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
 #pragma unroll
               for (int v = 0; v < 4; ++v) ak[k][mt][v] = 0.f;
           for (int c = 0; c < nck; ++c) {
+            const int wq = (c < KC ? c * h : tail_q) + brow;
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16) {
               uint32_t b0, b1, b2, b3;
-              const int wq = (c < KC ? c * h : (p.w1_tail_off >> 7)) + brow;  // tile row (1024-aligned tiles)
               ldmatrix_x4(wb + swz(wq, k16 * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
 #pragma unroll
               for (int mt = 0; mt < MTA; ++mt) {
@@ -417,16 +587,13 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
                   acc[qq][mt][v] += (ak[0][mt][v] + ak[1][mt][v]) + (ak[2][mt][v] + ak[3][mt][v]);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive_cnt(&sm.empty[slot], NCW);  // the only warp that reads this stage
+        if (lane == 0) mbar_arrive(&sm.empty[slot]);
       }
       if (p.KP > 1) {
         __syncwarp();
         if (lane == 0) mbar_arrive(sm.xfree);  // this warp is done with the x part
       }
     }
-    // epilogue of the row-block: h = r * Swish(u) as bf16 hi + lo, for this warp's groups
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    named_bar_sync(1, NCW * 32);
 #pragma unroll
     for (int qq = 0; qq < GPW; ++qq) {
       const int gl = qq * NCW + cw;
@@ -438,23 +605,47 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
           const int t = mt * 16 + gid + (v >> 1) * 8;
           const int n = tig * 2 + (v & 1);
           if (t >= p.L || n >= gq[qq].h) continue;
-          const int a = gq[qq].a, j = gq[qq].j0 + n;
-          const float sv = sm.pre_s[(a - a_first) * 32 + t];
-          const float rms = sm.rms[t];
-          const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
-          const float u = acc[qq][mt][v];
-          const float hv = rr * (u / (1.f + expf(-u)));
-          const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
-          uint8_t* himg = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
-          const int col = j & 63;
-          *reinterpret_cast<__nv_bfloat16*>(himg + swz(t, col >> 3) + (col & 7) * 2) = hi;
-          *reinterpret_cast<__nv_bfloat16*>(himg + swz(p.L + t, col >> 3) + (col & 7) * 2) = lo;
+          store_h(p, sm, a_first, gq[qq].a, gq[qq].j0 + n, t, acc[qq][mt][v]);
         }
       }
     }
-    named_bar_sync(1, NCW * 32);
     r = r_next;
+  }
+}
+
+template <int LC, bool KSPLIT>
+__device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
+  constexpr int MTA = (LC + 15) / 16;
+  constexpr int MT = (2 * LC + 15) / 16;
+  const int ctid = threadIdx.x;
+  const int cw = ctid >> 5, lane = ctid & 31;
+  const uint32_t zaddr = smem_u32(sm.zero);
+  RingPos rp;
+
+  // s and g of every expert this CTA's up-projection rows touch
+  const int a_first = w.rA0 / p.de;
+  if (w.rA0 < w.rA1) {
+    const int a_last = (w.rA1 - 1) / p.de;
+    for (int o = ctid; o < (a_last - a_first + 1) * p.L; o += NCW * 32) {
+      const int aa = o / p.L, t = o - aa * p.L;
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_s + aa * 32 + t)),
+                   "l"(p.s + size_t(t) * p.E + sm.act[a_first + aa])
+                   : "memory");
+    }
+    for (int aa = ctid; aa <= a_last - a_first; aa += NCW * 32)
+      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_g + aa)),
+                   "l"(p.g + sm.act[a_first + aa])
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  named_bar_sync(1, NCW * 32);
+
+  // ---------------- phase A
+  if constexpr (KSPLIT) {
+    phase_a_ksplit(p, sm, w, a_first, rp);
+  } else {
+    phase_a_smem<MTA>(p, sm, w, a_first, rp);
   }
   // publish this CTA's h before any CTA reads h
   __threadfence();
@@ -466,72 +657,103 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
   }
 
   // ---------------- phase B
-  const int ntB = p.RBB >> 3;  // RBB is a multiple of 8 (<= 32)
+  // A stage holds nq <= NEB experts x nc <= KWB chunks of 64 j; its k-steps (16 j each) in
+  // expert-major order g = qe * 4 KWB + kk go to warp g % NCW, at most kKS per warp (the plan keeps
+  // NEB KWB <= 8).  The offsets of a warp's k-steps inside a stage are the same for every stage, so
+  // they are computed once; a k-step outside the stage, or an operand row outside the tile, reads the
+  // zero row, and loads and MMAs run unconditionally (zero fragments add nothing).
+  constexpr int kKS = 4;
+  constexpr int KB = MT == 4 ? 2 : 4;  // k-steps per batch: all loads of a batch, then its MMAs
+  constexpr int NSET = MT == 4 ? 1 : 2;
+  int ks_qe[kKS], ks_c[kKS], offA[kKS][MT], offB[kKS][2];
+#pragma unroll
+  for (int b = 0; b < kKS; ++b) {
+    const int g = cw + NCW * b;
+    const int qe = g / (4 * p.KWB), kk = g - qe * 4 * p.KWB;
+    const int c = kk >> 2, k16 = kk & 3;
+    ks_qe[b] = qe;
+    ks_c[b] = c;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+      const int row = mt * 16 + (lane & 15);
+      offA[b][mt] = row < p.HR ? qe * p.eB + p.hoff + c * p.HR * 128 + int(swz(row, k16 * 2 + (lane >> 4))) : -1;
+    }
+#pragma unroll
+    for (int np2 = 0; np2 < 2; ++np2) {
+      const int row = np2 * 16 + (lane & 7) + (lane >> 4) * 8;
+      offB[b][np2] = row < p.RBB ? qe * p.eB + int(swz(c * p.RBB + row, k16 * 2 + ((lane >> 3) & 1))) : -1;
+    }
+  }
   uint32_t hphase = 0;
   for (int rb = 0; rb < w.nRBB; ++rb) {
-    float acc[MT][4][4];
+    float acc[NSET][MT][4][4];
 #pragma unroll
-    for (int a = 0; a < MT; ++a)
+    for (int e = 0; e < NSET; ++e)
 #pragma unroll
-      for (int b = 0; b < 4; ++b)
+      for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[a][b][c] = 0.f;
-    for (int s = 0; s < w.nEg * w.nJs; ++s, ++i) {
-      const int slot = i % p.S;
-      const bool okW = ring_wait(p, sm, &sm.fullW[slot], (i / p.S) & 1, 4);
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[e][a][b][c] = 0.f;
+    int eg = 0, js = 0;
+    for (int s = 0; s < w.nEg * w.nJs; ++s, rp.next(p.S)) {
+      const int slot = rp.slot;
+      const bool okW = ring_wait(p, sm, &sm.fullW[slot], rp.ph, 4);
       const bool okH = okW && ring_wait(p, sm, &sm.fullH[slot], (hphase >> slot) & 1u, 5);
       hphase ^= 1u << slot;
       if (okH) {
-        const int eg = s / w.nJs, js = s - eg * w.nJs;
         const int nq = min(p.NEB, w.n_act - eg * p.NEB);
         const int nc = min(p.KWB, p.nJc - js * p.KWB);
-        for (int qe = 0; qe < nq; ++qe) {
-          const uint32_t part = smem_u32(sm.ring + size_t(slot) * p.slot_bytes + size_t(qe) * p.eB);
-          // k-steps of 16 columns of j, split over the consumer warps (at most 4 per warp per chunk)
+        const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
 #pragma unroll
-          for (int kq = 0; kq < 4; ++kq) {
-            const int kk = cw + kq * NCW;
-            if (kk >= nc * 4) break;
-            const int c = kk >> 2, k16 = kk & 3;
-            const uint32_t ht = part + uint32_t(p.hoff + c * p.HR * 128);
-            uint32_t a[MT][4];
+        for (int b0 = 0; b0 < kKS; b0 += KB) {
+          uint32_t af[KB][MT][4], bf[KB][2][4];
+#pragma unroll
+          for (int b = 0; b < KB; ++b) {
+            const bool in = ks_qe[b0 + b] < nq && ks_c[b0 + b] < nc;
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-              if (mt < mtB) {
-                const int row = mt * 16 + (lane & 15);
-                const uint32_t addr = row < p.HR ? ht + swz(row, k16 * 2 + (lane >> 4)) : zaddr;
-                ldmatrix_x4(addr, a[mt][0], a[mt][1], a[mt][2], a[mt][3]);
-              }
+              const int o = offA[b0 + b][mt];
+              ldmatrix_x4(in && o >= 0 ? sb + uint32_t(o) : zaddr, af[b][mt][0], af[b][mt][1], af[b][mt][2],
+                          af[b][mt][3]);
             }
 #pragma unroll
             for (int np2 = 0; np2 < 2; ++np2) {
-              if (np2 * 2 < ntB) {
-                uint32_t b0, b1, b2, b3;
-                int row = np2 * 16 + (lane & 7) + (lane >> 4) * 8;
-                if (row >= p.RBB) row = 0;  // a second n-tile beyond the tile: loaded, never accumulated
-                ldmatrix_x4(part + swz(c * p.RBB + row, k16 * 2 + ((lane >> 3) & 1)), b0, b1, b2, b3);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                  if (mt < mtB) {
-                    mma_bf16_16816(acc[mt][np2 * 2], a[mt], b0, b1);
-                    if (np2 * 2 + 1 < ntB) mma_bf16_16816(acc[mt][np2 * 2 + 1], a[mt], b2, b3);
-                  }
-                }
-              }
+              const int o = offB[b0 + b][np2];
+              ldmatrix_x4(in && o >= 0 ? sb + uint32_t(o) : zaddr, bf[b][np2][0], bf[b][np2][1], bf[b][np2][2],
+                          bf[b][np2][3]);
             }
           }
+#pragma unroll
+          for (int b = 0; b < KB; ++b)
+#pragma unroll
+            for (int np2 = 0; np2 < 2; ++np2)
+#pragma unroll
+              for (int mt = 0; mt < MT; ++mt) {
+                mma_bf16_16816(acc[b % NSET][mt][np2 * 2], af[b][mt], bf[b][np2][0], bf[b][np2][1]);
+                mma_bf16_16816(acc[b % NSET][mt][np2 * 2 + 1], af[b][mt], bf[b][np2][2], bf[b][np2][3]);
+              }
         }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[slot]);
+      if (++js == w.nJs) js = 0, ++eg;
     }
+#pragma unroll
+    for (int e = 1; e < NSET; ++e)
+#pragma unroll
+      for (int a = 0; a < MT; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int c = 0; c < 4; ++c) acc[0][a][b][c] += acc[e][a][b][c];
     // sum the warps' partials in a fixed order; y = (hi part) + (lo part)
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt)
         *reinterpret_cast<float4*>(sm.red + ((((cw * MT + mt) * 4 + nt) * 32 + lane) * 4)) =
-            make_float4(acc[mt][nt][0], acc[mt][nt][1], acc[mt][nt][2], acc[mt][nt][3]);
+            make_float4(acc[0][mt][nt][0], acc[0][mt][nt][1], acc[0][mt][nt][2], acc[0][mt][nt][3]);
     named_bar_sync(1, NCW * 32);
     const int k0 = w.rB0 + rb * p.RBB, nrows = min(p.RBB, w.nB - rb * p.RBB);
     for (int o = ctid; o < p.L * nrows; o += NCW * 32) {
@@ -639,7 +861,7 @@ __device__ void write_router_outputs(const DecodeParams& p, const Smem& sm) {
   }
 }
 
-template <int LC>
+template <int LC, bool KSPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     expert_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TensorMaps tm) {
   extern __shared__ uint8_t smem_raw[];
@@ -666,6 +888,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm.maskw = reinterpret_cast<uint32_t*>(sm.rms + 32);
   sm.pre_s = reinterpret_cast<float*>(sm.maskw + 32 * 32);
   sm.pre_g = sm.pre_s + kMaxSpan * 32;
+  sm.red_s = reinterpret_cast<float*>(reinterpret_cast<uintptr_t>(sm.pre_g + kMaxSpan + 3) & ~uintptr_t(15));
+  sm.rbar = reinterpret_cast<uint64_t*>(sm.red_s + (p.ksplit ? size_t(p.S) * NCW * 32 * 2 : 0));
+  sm.ustage = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(sm.rbar + p.S) + 15) & ~uintptr_t(15));
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
@@ -676,6 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(sm.xfull, 1);
     mbar_init(sm.xfree, NCW);
+    for (int s2 = 0; s2 < p.S; ++s2) mbar_init(&sm.rbar[s2], NCW);
     *reinterpret_cast<uint4*>(sm.zero) = make_uint4(0, 0, 0, 0);
     *sm.abort_flag = 0;
     fence_mbar_init();
@@ -701,7 +927,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Work w = make_work(p, n_act);
 
   if (warp < NCW) {
-    consume<LC>(p, sm, w);
+    consume<LC, KSPLIT>(p, sm, w);
   } else if (warp == NCW) {
     produce_weights(p, tm, sm, w);
   } else {
@@ -713,10 +939,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int LC>
+template <int LC, bool KSPLIT>
 cudaError_t launch_lc(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan, cudaStream_t st,
                       bool pdl) {
-  auto kfn = expert_decode_kernel<LC>;
+  auto kfn = expert_decode_kernel<LC, KSPLIT>;
   cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
@@ -745,6 +971,7 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   const int mt = (2 * lc + 15) / 16;
   const int G = num_sms;
   if (d > 256 * 64) return false;  // a box spans at most 256 chunks
+  if ((E + G - 1) / G + 2 > kMaxSpan) return false;  // experts one CTA's up-projection rows touch
   // up-projection: x resident per pass of KC full 64-column chunks (plus the ragged chunk, which
   // needs a single pass); stages of one box of up to RSM whole rows
   p->nKf = d / 64;
@@ -763,6 +990,7 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   const int nck = KC + (p->nKc > p->nKf ? 1 : 0);
   p->Kp = KC * 64;
   p->xbuf_bytes = round_up(nck * p->LB * 128, 1024);
+  p->ksplit = (L <= 8 && p->KP == 1) ? 1 : 0;
   const int target = 32 * 1024;
   p->RSM = 8;
   while (p->RSM > 1 && p->RSM * nck * 128 > target) p->RSM >>= 1;
@@ -788,13 +1016,17 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   const int slot = round_up(slotA > p->eB ? slotA : p->eB, 1024);
   p->NEB = slot / p->eB;
   if (p->NEB < 1) p->NEB = 1;
+  while (p->NEB > 1 && p->NEB * p->KWB > 8) --p->NEB;  // a stage has at most 32 k-steps of 16 j
   p->slot_bytes = slot;
   const size_t red = size_t(NCW) * mt * 4 * 32 * 4 * 4;
   const size_t red_extra = size_t(p->xbuf_bytes) >= red ? 0 : red;
-  const size_t tail = 32 + 3 * 8 * 32 + 16 + size_t(kMaxE + 4) * 4 + 32 * 4 + 32 * 32 * 4 + (kMaxSpan * 33) * 4;
-  const size_t fixed = 1024 + size_t(p->xbuf_bytes) + red_extra + tail;
+  const size_t tail = 32 + 3 * 8 * 32 + 16 + size_t(kMaxE + 4) * 4 + 32 * 4 + 32 * 32 * 4 + (kMaxSpan * 33) * 4 + 16;
+  const size_t per_slot = (p->ksplit ? size_t(NCW) * 32 * 2 * 4 : 0) + 16;  // red_s and rbar of one slot
+  // staged u of one CTA: at most ceil(E de / 8 / G) units of 8 rows, L tokens x 8 floats each
+  p->ustage_bytes = p->ksplit ? int((size_t(E) * de / 8 + G - 1) / G) * L * 32 : 0;
+  const size_t fixed = 1024 + size_t(p->xbuf_bytes) + red_extra + tail + size_t(p->ustage_bytes);
   if (fixed >= size_t(max_smem)) return false;
-  int S = int((size_t(max_smem) - fixed) / size_t(p->slot_bytes));
+  int S = int((size_t(max_smem) - fixed) / (size_t(p->slot_bytes) + per_slot));
   if (S > 32) S = 32;
   if (S < 2) return false;
   p->S = S;
@@ -802,16 +1034,16 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   if (p->sbuf_floats < E) return false;
   out->grid = G;
   out->lclass = lc;
-  out->smem = fixed + size_t(S) * p->slot_bytes;
+  out->smem = fixed + size_t(S) * (p->slot_bytes + per_slot);
   return true;
 }
 
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl) {
   switch (plan.lclass) {
-    case 8: return launch_lc<8>(p, tm, plan, st, pdl);
-    case 16: return launch_lc<16>(p, tm, plan, st, pdl);
-    default: return launch_lc<32>(p, tm, plan, st, pdl);
+    case 8: return p.ksplit ? launch_lc<8, true>(p, tm, plan, st, pdl) : launch_lc<8, false>(p, tm, plan, st, pdl);
+    case 16: return launch_lc<16, false>(p, tm, plan, st, pdl);
+    default: return launch_lc<32, false>(p, tm, plan, st, pdl);
   }
 }
 
