@@ -87,15 +87,16 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name: str):
-    """DRAM bytes per chunk from the committed ncu summary, only if the kernels are unchanged."""
+def recorded_traffic_ratio(workload_name: str):
+    """DRAM bytes per algorithmic (active) byte from the committed ncu summary, only if the kernel
+    sources are unchanged since the counters were taken."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             j = json.load(f)
         rec = j.get(workload_name)
         if rec and rec.get("kernel_source_hash") == kernel_source_hash():
-            return float(rec["dram_bytes_per_chunk"])
+            return float(rec["dram_bytes_per_active_byte"])
     except Exception:
         pass
     return None
@@ -294,7 +295,8 @@ def run_ours(args, w):
     value = tokens_step / (ms_per_step * 1e-3)
     achieved_gbs = total_active / (ms_per_step * 1e-3) / 1e9  # per GPU: every rank streams its own
     peak, peak_kind = measured_peaks()
-    traffic = recorded_traffic(w.name)
+    ratio = recorded_traffic_ratio(w.name)
+    traffic = None if ratio is None else ratio * total_active / chunks
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -341,10 +343,12 @@ def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
     cores = oracle.available_cores()
     L, d = w.L, w.d
     chunk_ids = list(range(0, x_host_np.shape[0], w.replicas))  # chunks that use replica 0
-    # calibrate on one chunk, then size the sample to about `seconds`
-    t0 = time.time()
+    # warm up on one chunk, calibrate on two, then size the sample to about `seconds`
     oracle.tokens_forward_mt(x_host_np[chunk_ids[0]], lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
-    t1 = time.time() - t0
+    t0 = time.time()
+    oracle.tokens_forward_mt(x_host_np[chunk_ids[0]].repeat(2, axis=0), lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2,
+                             cores)
+    t1 = (time.time() - t0) / 2
     n_chunks = max(1, min(len(chunk_ids), int(seconds / max(t1, 1e-6))))
     xs = x_host_np[chunk_ids[:n_chunks]].reshape(n_chunks * L, d)
     t0 = time.time()
@@ -409,6 +413,8 @@ def main():
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
     ap.add_argument("--tls", type=float, default=None, help="token-level sparsity for --workload tls_sweep")
     ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")
+    ap.add_argument("--replicas", type=int, default=None,
+                    help="weight replicas (default: the workload's; keep their weights above the 126 MB L2)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-chunks", type=int, default=1)
@@ -423,6 +429,8 @@ def main():
         kw["L"] = args.L
     if args.workload == "tls_sweep" and args.tls:
         kw["tls"] = args.tls
+    if args.replicas:
+        kw["replicas"] = args.replicas
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":
         run_reference(args, w)

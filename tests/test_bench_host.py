@@ -1,0 +1,73 @@
+"""Host-side logic of bench.py that needs no GPU: the max-over-ranks timing reduction and the per-rank
+chunk streams (world size 2 over gloo, on the CPU), the active-bytes formula, and the clock-sample
+summary."""
+import os
+import socket
+
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        got_world, got_rank, _ = bench.dist_env()
+        # every rank contributes its own event time; all must see the largest
+        t = bench.reduce_max(10.0 + 5.0 * rank)
+        bench.barrier()
+        out.put((got_rank, got_world, t, bench.shard_seed(0, got_rank)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_reduce_max_and_distinct_streams():
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(out.get(timeout=10) for _ in range(2))
+    assert [r[0] for r in res] == [0, 1] and all(r[1] == 2 for r in res)
+    assert all(r[2] == 15.0 for r in res)          # max over ranks, seen by every rank
+    assert res[0][3] != res[1][3]                    # each rank draws its own chunks (weak scaling)
+
+
+def test_single_process_helpers_without_a_process_group():
+    assert bench.reduce_max(3.5) == 3.5
+    bench.barrier()  # no process group: a no-op
+
+
+def test_active_bytes_formula():
+    # decode layer, 17 active experts: router weights + gain/bias + x + y + W1_i and W2_i in bf16
+    d, E, de, L = 2048, 64, 256, 8
+    assert bench.active_bytes(d, E, de, L, 17) == 4 * d * E + 8 * E + 2 * L * d + 4 * L * d + 17 * 4 * d * de
+    assert bench.active_bytes(d, E, de, L, 0) == 4 * d * E + 8 * E + 6 * L * d
+
+
+def test_clock_summary_parses_samples(tmp_path):
+    cs = bench.ClockSampler(0)
+    cs.proc = object()  # pretend nvidia-smi ran
+    cs.path = str(tmp_path / "clk.csv")
+    with open(cs.path, "w") as f:
+        f.write("1965, 1965, 500.1, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+        f.write("1860, 1965, 990.0, 0x4, Not Active, Not Active, Not Active, Active\n")
+        f.write("1950, 1965, 700.0, 0x0, Not Active, Not Active, Not Active, Not Active\n")
+    s = cs.summary()
+    assert s["sm_mhz"] == 1950 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
