@@ -62,7 +62,8 @@ struct RouterParams {
 struct RouterLaunch {
   int cluster;      // CTAs per cluster (split of d)
   int grid;         // clusters (32 router columns each)
-  int xt;
+  int xt;           // d rows per CTA
+  int lt;           // tokens rounded up to 8, 16 or 32 (accumulators per thread)
   size_t smem;
 };
 

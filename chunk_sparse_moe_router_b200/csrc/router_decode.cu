@@ -3,11 +3,13 @@
 // s = x Wr + b in fp32 (lsdiaocha.cn BlockFFN article, section 2: the router's linear map, before its
 // ReLU and RMSNorm).  The work is spread over many SMs with thread-block clusters: cluster y owns 32
 // router columns (experts), and its C CTAs split the d rows.  Each CTA stages its [rows x 32] slice of
-// Wr and its [L x rows] slice of x in shared memory with cp.async (one memory round trip), computes
-// its partial sums (one output per thread and token group), and the cluster then adds the C partials
-// through distributed shared memory in rank order, every rank finishing a 1/C share of the outputs
-// with all of its remote loads in flight at once.  The order of every sum is fixed, so s is
-// bit-reproducible.  The ReLU, the RMSNorm and the chunk union run in the expert kernel's prologue.
+// Wr (issued before the dependent-launch wait: weights never depend on the previous kernel) and its
+// [L x rows] slice of x in shared memory with cp.async.  Each warp takes a contiguous share of the
+// rows with one accumulator per token (lane = column), the CTA adds its warps' shares in warp order,
+// and the cluster then adds the C partials through distributed shared memory in rank order, every
+// rank finishing a 1/C share of the outputs with all of its remote loads in flight at once.  The
+// order of every sum is fixed, so s is bit-reproducible.  The ReLU, the RMSNorm and the chunk union
+// run in the expert kernel's prologue.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -24,27 +26,25 @@ constexpr int kRouterThreads = 256;
 constexpr int kCols = 32;         // router columns per cluster
 constexpr int kMaxCluster = 16;
 
+template <int LT>
 __global__ void __launch_bounds__(kRouterThreads) router_decode_kernel(RouterParams p) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   cg::cluster_group cluster = cg::this_cluster();
   const int q = int(cluster.block_rank());
   const int C = int(cluster.num_blocks());
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = kRouterThreads / 32;
   const int e0 = blockIdx.y * kCols;
   const int Ec = min(kCols, p.E - e0);
   const int k0 = q * p.xt;  // xt holds the rows per rank here
   const int nk = max(0, min(p.d, k0 + p.xt) - k0);
-  const int LP = (p.L + 7) & ~7;
 
   float* W_s = reinterpret_cast<float*>(smem_raw);                                      // [rows][32]
-  __nv_bfloat16* X_s = reinterpret_cast<__nv_bfloat16*>(W_s + size_t(p.xt) * kCols);   // [LP][rows]
-  float* part = reinterpret_cast<float*>(X_s + size_t(LP) * p.xt);                      // [LP][32]
+  __nv_bfloat16* X_s = reinterpret_cast<__nv_bfloat16*>(W_s + size_t(p.xt) * kCols);   // [LT][rows]
+  float* wpart = reinterpret_cast<float*>(X_s + size_t(LT) * p.xt);                     // [NW][LT][32]
+  float* part = wpart + NW * LT * kCols;                                                // [LT][32]
 
-  // x may come from the previous kernel in the stream, and the workspace is shared with it.
-  pdl_wait();
-  pdl_launch_dependents();
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.hdr->grid_bar = 0u;  // expert kernel barrier
-
+  // The router weights do not depend on the previous kernel in the stream: start their copies first.
   if ((p.E & 3) == 0) {
     constexpr int q4 = kCols / 4;
     for (int o = tid; o < nk * q4; o += kRouterThreads) {
@@ -69,6 +69,11 @@ __global__ void __launch_bounds__(kRouterThreads) router_decode_kernel(RouterPar
         *dst = 0.f;
     }
   }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  // x may come from the previous kernel in the stream, and the workspace is shared with it.
+  pdl_wait();
+  pdl_launch_dependents();
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) p.hdr->grid_bar = 0u;  // expert kernel barrier
   {
     const int q8 = nk / 8;  // nk and k0 are multiples of 8
     for (int o = tid; o < p.L * q8; o += kRouterThreads) {
@@ -77,20 +82,36 @@ __global__ void __launch_bounds__(kRouterThreads) router_decode_kernel(RouterPar
                    "l"(p.x + size_t(t) * p.d + k0 + c8)
                    : "memory");
     }
+    for (int o = p.L * p.xt + tid; o < LT * p.xt; o += kRouterThreads)  // padding tokens read as 0
+      X_s[o] = __float2bfloat16_rn(0.f);
   }
   asm volatile("cp.async.commit_group;" ::: "memory");
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
 
-  // warp w handles tokens w, w+8, ...; lane = column.  x is a broadcast, Wr a conflict-free row.
-  for (int t = warp; t < LP; t += kRouterThreads / 32) {
-    float acc = 0.f;
-    if (t < p.L) {
-      const __nv_bfloat16* xr = X_s + size_t(t) * p.xt;
-#pragma unroll 8
-      for (int kk = 0; kk < nk; ++kk) acc = fmaf(__bfloat162float(xr[kk]), W_s[kk * kCols + lane], acc);
+  // warp w takes a contiguous share of the CTA's rows for every token, lane = column: LT independent
+  // accumulators per thread; x is a broadcast, W_s a conflict-free row.
+  {
+    const int per = (nk + NW - 1) / NW;
+    const int r0 = warp * per, r1 = min(nk, r0 + per);
+    float acc[LT];
+#pragma unroll
+    for (int t = 0; t < LT; ++t) acc[t] = 0.f;
+#pragma unroll 4
+    for (int kk = r0; kk < r1; ++kk) {
+      const float wv = W_s[kk * kCols + lane];
+#pragma unroll
+      for (int t = 0; t < LT; ++t) acc[t] = fmaf(__bfloat162float(X_s[t * p.xt + kk]), wv, acc[t]);
     }
-    part[t * kCols + lane] = acc;
+#pragma unroll
+    for (int t = 0; t < LT; ++t) wpart[(warp * LT + t) * kCols + lane] = acc[t];
+  }
+  __syncthreads();
+  for (int o = tid; o < LT * kCols; o += kRouterThreads) {  // the warps' shares, in warp order
+    float v = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) v += wpart[w * LT * kCols + o];
+    part[o] = v;
   }
   cluster.sync();
   {
@@ -116,28 +137,31 @@ __global__ void __launch_bounds__(kRouterThreads) router_decode_kernel(RouterPar
 
 bool router_decode_plan(int L, int d, int E, int max_smem, RouterLaunch* out) {
   if (L < 1 || L > kDecodeMaxL || E < 1 || E > kMaxE || d % 8 != 0) return false;
-  const int LP = (L + 7) & ~7;
+  const int LT = L <= 8 ? 8 : L <= 16 ? 16 : 32;
   for (int cluster : {8, 16}) {
     int rows = (d + cluster - 1) / cluster;
     rows = (rows + 7) & ~7;
-    const size_t smem = size_t(rows) * kCols * 4 + size_t(LP) * rows * 2 + size_t(LP) * kCols * 4;
+    const size_t smem = size_t(rows) * kCols * 4 + size_t(LT) * rows * 2 +
+                        size_t(kRouterThreads / 32 + 1) * LT * kCols * 4;
     if (smem <= size_t(max_smem) && (cluster == 16 || rows <= 256)) {
       out->cluster = cluster;
       out->xt = rows;
       out->smem = smem;
       out->grid = (E + kCols - 1) / kCols;
+      out->lt = LT;
       return true;
     }
   }
   return false;
 }
 
-cudaError_t router_decode_launch(const RouterParams& p, const RouterLaunch& plan, cudaStream_t st, bool pdl) {
-  cudaError_t err =
-      cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
+template <int LT>
+static cudaError_t launch_lt(const RouterParams& p, const RouterLaunch& plan, cudaStream_t st, bool pdl) {
+  auto kfn = router_decode_kernel<LT>;
+  cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
   if (plan.cluster > 8) {
-    err = cudaFuncSetAttribute(router_decode_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    err = cudaFuncSetAttribute(kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (err != cudaSuccess) return err;
   }
   cudaLaunchConfig_t cfg = {};
@@ -154,7 +178,15 @@ cudaError_t router_decode_launch(const RouterParams& p, const RouterLaunch& plan
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl ? 2 : 1;
-  return cudaLaunchKernelEx(&cfg, router_decode_kernel, p);
+  return cudaLaunchKernelEx(&cfg, kfn, p);
+}
+
+cudaError_t router_decode_launch(const RouterParams& p, const RouterLaunch& plan, cudaStream_t st, bool pdl) {
+  switch (plan.lt) {
+    case 8: return launch_lt<8>(p, plan, st, pdl);
+    case 16: return launch_lt<16>(p, plan, st, pdl);
+    default: return launch_lt<32>(p, plan, st, pdl);
+  }
 }
 
 }  // namespace bffn
