@@ -211,6 +211,63 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
   return BFFN_OK;
 }
 
+int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
+                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
+                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
+                    const DeviceInfo& di, cudaStream_t st) {
+  if (!aligned16(y)) return BFFN_EINVAL;  // the down-projection adds into y 16 bytes at a time
+  const WsLayout lay = ws_layout(L, d, E, de);
+  const PrefillLayout pl = prefill_layout(lay.h_off, L, E, de);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  PrefillParams p;
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.Wr = Wr;
+  p.br = br;
+  p.g = g;
+  p.y = y;
+  p.active_idx = active_idx;
+  p.n_active = n_active;
+  p.tok_mask = tok_mask;
+  p.counts = counts;
+  p.r_out = r_out;
+  p.L = L;
+  p.d = d;
+  p.E = E;
+  p.de = de;
+  p.s = reinterpret_cast<float*>(base + lay.s_off);
+  p.mask = reinterpret_cast<uint32_t*>(base + pl.mask_off);
+  p.rms = reinterpret_cast<float*>(base + pl.rms_off);
+  p.cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);
+  p.off = reinterpret_cast<int32_t*>(base + pl.off_off);
+  p.toff = reinterpret_cast<int32_t*>(base + pl.toff_off);
+  p.n_pos = reinterpret_cast<int32_t*>(base + pl.npos_off);
+  p.tok = reinterpret_cast<int32_t*>(base + pl.tok_off);
+  p.rv = reinterpret_cast<float*>(base + pl.rv_off);
+  p.H = reinterpret_cast<__nv_bfloat16*>(base + pl.h_off);
+  p.hdr = reinterpret_cast<WsHeader*>(base);
+  PrefillLaunch launch;
+  if (!prefill_plan(L, d, E, de, di.num_sms, di.max_smem, &p, &launch)) return BFFN_EUNSUPPORTED;
+
+  PrefillMaps m;
+  {
+    const uint64_t xd[2] = {uint64_t(d), uint64_t(L)}, xs[1] = {uint64_t(d) * 2};
+    const uint32_t xb[2] = {64, 1};
+    if (!encode_bf16(&m.xg, x, 2, xd, xs, xb)) return BFFN_ECUDA;
+    const uint64_t w1d[2] = {uint64_t(d), uint64_t(E) * de}, w1s[1] = {uint64_t(d) * 2};
+    const uint32_t w1b[2] = {64, uint32_t(p.N1)};
+    if (!encode_bf16(&m.w1, W1, 2, w1d, w1s, w1b)) return BFFN_ECUDA;
+    const uint64_t hd[2] = {uint64_t(2 * de), uint64_t(L) * E}, hs[1] = {uint64_t(2 * de) * 2};
+    const uint32_t hb[2] = {64, 128};
+    if (!encode_bf16(&m.h, p.H, 2, hd, hs, hb)) return BFFN_ECUDA;
+    const uint64_t w2d[2] = {uint64_t(de), uint64_t(E) * d}, w2s[1] = {uint64_t(de) * 2};
+    const uint32_t w2b[2] = {64, uint32_t(p.N2)};
+    if (!encode_bf16(&m.w2, W2, 2, w2d, w2s, w2b)) return BFFN_ECUDA;
+  }
+  const cudaError_t err = prefill_launch(p, m, launch, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  return BFFN_OK;
+}
+
 }  // namespace
 }  // namespace bffn
 
@@ -263,8 +320,10 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   const int path = flags & 3;
   if (path == 3) return BFFN_EINVAL;
   const bool decode = (path == BFFN_PATH_DECODE) || (path == BFFN_PATH_AUTO && L <= kDecodeMaxL);
-  if (!decode) return BFFN_EUNSUPPORTED;
-  if (L > kDecodeMaxL) return BFFN_EUNSUPPORTED;
+  if (decode && L > kDecodeMaxL) return BFFN_EUNSUPPORTED;
+  if (!decode && L <= kDecodeMaxL) return BFFN_EUNSUPPORTED;  // the prefill path takes L > 32
+  if (!decode && (d % 64 != 0 || de % 64 != 0 || de > 256)) return BFFN_EUNSUPPORTED;
+  if (!decode && !aligned16(y)) return BFFN_EINVAL;  // the down-projection adds into y 16 bytes at a time
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   DeviceInfo di;
@@ -279,8 +338,11 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   } else if (workspace_bytes < need) {
     return BFFN_ENOMEM;
   }
-  return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                        r_out, ws, di, st);
+  if (decode)
+    return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
+                          r_out, ws, di, st);
+  return forward_prefill(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts, r_out,
+                         ws, di, st);
 }
 
 int blockffn_chunk_forward(const void* x, int L, int d, const float* Wr, const float* g,

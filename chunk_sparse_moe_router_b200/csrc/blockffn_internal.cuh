@@ -16,6 +16,7 @@ constexpr int kDecodeMaxL = 32;
 enum : uint32_t {
   kErrGridBarrier = 1u,   // expert kernel: waiting for every CTA to finish the up-projection
   kErrRingWait = 2u,      // expert kernel: waiting on a shared-memory ring barrier
+  kErrPrefillWait = 4u,   // prefill GEMMs: waiting on a shared-memory barrier
 };
 
 // First 256 bytes of every workspace.
@@ -34,17 +35,39 @@ __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_
 // lo rows) in the 128-byte-swizzled layout the down-projection loads.
 size_t decode_h_bytes(int L, int E, int de);
 
+// Prefill workspace regions (L > 32), after s: per-token masks and RMS, per-expert counts and
+// offsets, the pair lists (token, r) in expert-major order, and H = [pairs][2 de] bf16 (hi | lo).
+struct PrefillLayout {
+  size_t mask_off, rms_off, cnt_off, off_off, toff_off, npos_off, tok_off, rv_off, h_off, end;
+};
+
+inline PrefillLayout prefill_layout(size_t start, int L, int E, int de) {
+  PrefillLayout p;
+  const size_t W = size_t(E + 31) / 32, P = size_t(L) * E;
+  p.mask_off = start;
+  p.rms_off = p.mask_off + align256(size_t(L) * W * 4);
+  p.cnt_off = p.rms_off + align256(size_t(L) * 4);
+  p.off_off = p.cnt_off + align256(size_t(E) * 4);
+  p.toff_off = p.off_off + align256(size_t(E + 1) * 4);
+  p.npos_off = p.toff_off + align256(size_t(E + 1) * 4);
+  p.tok_off = p.npos_off + 256;
+  p.rv_off = p.tok_off + align256(P * 4);
+  p.h_off = p.rv_off + align256(P * 4);
+  p.end = p.h_off + align256(P * size_t(2 * de) * 2);
+  return p;
+}
+
 struct WsLayout {
   size_t s_off, h_off, total;
 };
 
-// Workspace: header | s fp32 [L,E] (router projection) | h (decode only)
+// Workspace: header | s fp32 [L,E] (router projection) | decode h (L <= 32) or the prefill regions
 inline WsLayout ws_layout(int L, int d, int E, int de) {
   (void)d;
   WsLayout w;
   w.s_off = sizeof(WsHeader);
   w.h_off = w.s_off + align256(size_t(L) * E * sizeof(float));
-  w.total = w.h_off + (L <= kDecodeMaxL ? align256(decode_h_bytes(L, E, de)) : 0);
+  w.total = L <= kDecodeMaxL ? w.h_off + align256(decode_h_bytes(L, E, de)) : prefill_layout(w.h_off, L, E, de).end;
   return w;
 }
 
@@ -133,5 +156,48 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
                         DecodeLaunch* out);
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------------------------------ prefill
+struct PrefillParams {
+  const __nv_bfloat16* x;   // [L,d]
+  const float* Wr;          // [d,E]
+  const float* br;          // [E] or null
+  const float* g;           // [E]
+  float* y;                 // [L,d] out (zeroed before the down-projection adds into it)
+  int32_t* active_idx;
+  int32_t* n_active;
+  uint32_t* tok_mask;       // optional
+  int32_t* counts;          // optional
+  float* r_out;             // optional
+  int L, d, E, de, W;       // W = ceil(E / 32)
+  float* s;                 // [L,E]
+  uint32_t* mask;           // [L,W]
+  float* rms;               // [L]
+  int32_t* cnt;             // [E] tokens per expert
+  int32_t* off;             // [E+1] pair offset per expert
+  int32_t* toff;            // [E+1] 128-row tile offset per expert (toff[E] = tiles)
+  int32_t* n_pos;           // positive (t, e) entries of the call
+  int32_t* tok;             // [L*E] pair -> token
+  float* rv;                // [L*E] pair -> r_{t,e}
+  __nv_bfloat16* H;         // [L*E][2 de] hi | lo
+  WsHeader* hdr;
+  int N1, S1;               // GEMM1: N (= de), pipeline stages
+  int N2, S2;               // GEMM2: N tile of d, pipeline stages
+};
+
+struct PrefillMaps {
+  CUtensorMap xg;   // x [L rows, d] box 64 x 1 (gather4 of token rows)
+  CUtensorMap w1;   // W1 [E*de rows, d] box 64 x N1
+  CUtensorMap h;    // H [L*E rows, 2 de] box 64 x 128
+  CUtensorMap w2;   // W2 [E*d rows, de] box 64 x N2
+};
+
+struct PrefillLaunch {
+  int grid;
+  size_t smem1, smem2;
+};
+
+bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, PrefillParams* p, PrefillLaunch* out);
+cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st);
 
 }  // namespace bffn

@@ -1,0 +1,561 @@
+// Prefill variant of the BlockFFN chunk layer (L in the hundreds to thousands of tokens).
+//
+// At this size the layer is a dense contraction per expert, so it runs as grouped GEMMs on the
+// tcgen05 tensor cores (lsdiaocha.cn BlockFFN article, sections 2 and 4: the same router and experts;
+// the tokens of the chunk are grouped per active expert instead of evaluated as one batch):
+//   P1 router       s = x Wr + b, fp32 FFMA tiles (the mask decisions need fp32 accuracy)
+//   P2 stats        per token: RMS of relu(s), active bits, optional r and masks
+//   P3 grouping     per expert: its tokens in ascending order with r_{t,e}, 128-row tiles
+//   P4 GEMM1        per (expert, 128-token tile): U = X[T_e] W1_e^T on tcgen05 (A rows gathered with
+//                   TMA gather4), h = r Swish(U) split into bf16 hi + lo parts
+//   P5 GEMM2        per (expert tile, 256 columns of d): Y[T_e] += (H_hi + H_lo) W2_e^T on tcgen05,
+//                   added into y with vector reductions
+#include <cuda_bf16.h>
+
+#include "blockffn_internal.cuh"
+#include "ptx.cuh"
+#include "tc.cuh"
+
+namespace bffn {
+namespace {
+
+constexpr uint64_t kPWaitNs = 2000000000ull;
+
+// ---------------------------------------------------------------------------------- P1 router
+constexpr int kRtT = 32, kRtE = 64, kRtK = 32;  // tile: 32 tokens x 64 experts, K step 32
+
+__global__ void __launch_bounds__(256) prefill_router_kernel(PrefillParams p) {
+  __shared__ float Xs[kRtK][kRtT + 1];
+  __shared__ __align__(16) float Ws[kRtK][kRtE];
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *p.n_pos = 0;  // positive (t, e) count of this call
+  float acc[2][4] = {};
+  for (int k0 = 0; k0 < p.d; k0 += kRtK) {
+    for (int o = tid; o < kRtT * kRtK; o += 256) {
+      const int t = o / kRtK, k = o - t * kRtK;
+      Xs[k][t] = (t0 + t < p.L) ? __bfloat162float(p.x[size_t(t0 + t) * p.d + k0 + k]) : 0.f;
+    }
+    for (int o = tid; o < kRtK * kRtE; o += 256) {
+      const int k = o / kRtE, e = o - k * kRtE;
+      Ws[k][e] = (e0 + e < p.E) ? p.Wr[size_t(k0 + k) * p.E + e0 + e] : 0.f;
+    }
+    __syncthreads();
+    // a partial sum per K tile, added to the running total: a two-level sum keeps the rounding of a
+    // d-term dot product near that of its (d / 32 + 32)-term levels rather than of one d-term chain
+    float part[2][4] = {};
+#pragma unroll 8
+    for (int k = 0; k < kRtK; ++k) {
+      const float a0 = Xs[k][ty * 2], a1 = Xs[k][ty * 2 + 1];
+      const float4 b = *reinterpret_cast<const float4*>(&Ws[k][tx * 4]);
+      part[0][0] = fmaf(a0, b.x, part[0][0]);
+      part[0][1] = fmaf(a0, b.y, part[0][1]);
+      part[0][2] = fmaf(a0, b.z, part[0][2]);
+      part[0][3] = fmaf(a0, b.w, part[0][3]);
+      part[1][0] = fmaf(a1, b.x, part[1][0]);
+      part[1][1] = fmaf(a1, b.y, part[1][1]);
+      part[1][2] = fmaf(a1, b.z, part[1][2]);
+      part[1][3] = fmaf(a1, b.w, part[1][3]);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const int t = t0 + ty * 2 + i;
+    if (t >= p.L) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < p.E) p.s[size_t(t) * p.E + e] = acc[i][j] + (p.br ? p.br[e] : 0.f);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------- P2 stats
+// One warp per token: RMS over the E router entries of relu(s), the active bits, r if asked for.
+__global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int t = warp;
+  if (t >= p.L) return;
+  const float* st = p.s + size_t(t) * p.E;
+  float sumsq = 0.f;
+  int n_pos = 0;
+  for (int w = 0; w < p.W; ++w) {
+    const int e = w * 32 + lane;
+    const float sv = e < p.E ? st[e] : -1.f;
+    const float a = fmaxf(sv, 0.f);
+    sumsq = fmaf(a, a, sumsq);
+    const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
+    if (lane == 0) {
+      p.mask[size_t(t) * p.W + w] = bits;
+      if (p.tok_mask) p.tok_mask[size_t(t) * p.W + w] = bits;
+    }
+    n_pos += __popc(bits);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+  const float rms = sqrtf(sumsq / float(p.E));
+  if (lane == 0) {
+    p.rms[t] = rms;
+    atomicAdd(p.n_pos, n_pos);  // an integer sum: the same in any order
+  }
+  if (p.r_out)
+    for (int e = lane; e < p.E; e += 32)
+      p.r_out[size_t(t) * p.E + e] = rms > 0.f ? (p.g[e] * fmaxf(st[e], 0.f)) / rms : 0.f;
+}
+
+// ---------------------------------------------------------------------------------- P3 grouping
+__device__ __forceinline__ bool active_bit(const PrefillParams& p, int t, int e) {
+  return t < p.L && ((p.mask[size_t(t) * p.W + (e >> 5)] >> (e & 31)) & 1u);
+}
+
+// One warp per expert: the number of its tokens.
+__global__ void __launch_bounds__(256) prefill_count_kernel(PrefillParams p) {
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (e >= p.E) return;
+  int n = 0;
+  for (int t0 = 0; t0 < p.L; t0 += 32) n += __popc(__ballot_sync(0xffffffffu, active_bit(p, t0 + lane, e)));
+  if (lane == 0) p.cnt[e] = n;
+}
+
+// One warp per expert: its token list (ascending) and r values at its pair offset.  CTA 0 also
+// writes the pair and tile offsets, the union (active experts ascending), n_active and the counts.
+__global__ void __launch_bounds__(256) prefill_fill_kernel(PrefillParams p) {
+  const int lane = threadIdx.x & 31;
+  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    // exclusive scans over the experts (pairs and 128-row tiles) and the union, in one warp
+    int pairs = 0, tiles = 0, nact = 0;
+    for (int e0 = 0; e0 < p.E; e0 += 32) {
+      const int ee = e0 + lane;
+      const int c = ee < p.E ? p.cnt[ee] : 0;
+      const int mt = (c + 127) >> 7;
+      int ic = c, im = mt, ia = c > 0 ? 1 : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int vc = __shfl_up_sync(0xffffffffu, ic, o), vm = __shfl_up_sync(0xffffffffu, im, o),
+                  va = __shfl_up_sync(0xffffffffu, ia, o);
+        if (lane >= o) ic += vc, im += vm, ia += va;
+      }
+      if (ee < p.E) {
+        p.off[ee] = pairs + ic - c;
+        p.toff[ee] = tiles + im - mt;
+        if (c > 0) p.active_idx[nact + ia - 1] = ee;
+      }
+      pairs += __shfl_sync(0xffffffffu, ic, 31);
+      tiles += __shfl_sync(0xffffffffu, im, 31);
+      nact += __shfl_sync(0xffffffffu, ia, 31);
+    }
+    if (lane == 0) {
+      p.off[p.E] = pairs;
+      p.toff[p.E] = tiles;
+      *p.n_active = nact;
+      if (p.counts) {
+        p.counts[0] = p.L * p.E - *p.n_pos;
+        p.counts[1] = p.E - nact;
+      }
+    }
+  }
+  if (e >= p.E) return;
+  int base = 0;  // this expert's pair offset: the tokens of every lower expert
+  for (int e2 = lane; e2 < e; e2 += 32) base += p.cnt[e2];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
+  const float ge = p.g[e];
+  for (int t0 = 0; t0 < p.L; t0 += 32) {
+    const int t = t0 + lane;
+    const bool on = active_bit(p, t, e);
+    const uint32_t b = __ballot_sync(0xffffffffu, on);
+    if (on) {
+      const int pos = base + __popc(b & ((1u << lane) - 1u));
+      p.tok[pos] = t;
+      p.rv[pos] = (ge * p.s[size_t(t) * p.E + e]) / p.rms[t];  // s > 0, so relu(s) = s and rms > 0
+    }
+    base += __popc(b);
+  }
+}
+
+}  // namespace
+
+namespace {
+
+// ---------------------------------------------------------------------------------- P4/P5 GEMMs
+constexpr int kGThreads = 192;  // warp 0: TMA producer, warp 1: MMA issuer (owns TMEM), warps 2-5: epilogue
+constexpr int kTileM = 128;
+
+struct GemmSmem {
+  uint8_t* stages;
+  uint64_t* full;   // [S] operands of a stage landed
+  uint64_t* empty;  // [S] MMAs of a stage done reading it
+  uint64_t* accf;   // [2] accumulator buffer complete
+  uint64_t* acce;   // [2] accumulator buffer drained by the epilogue (4 warps)
+  uint64_t* drain;  // every MMA of this CTA complete (before TMEM is freed)
+  uint32_t* tmem_slot;
+  volatile int* abort_flag;
+};
+
+__device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_bytes) {
+  GemmSmem g;
+  g.stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+  g.full = reinterpret_cast<uint64_t*>(g.stages + size_t(S) * stage_bytes);
+  g.empty = g.full + S;
+  g.accf = g.empty + S;
+  g.acce = g.accf + 2;
+  g.drain = g.acce + 2;
+  g.tmem_slot = reinterpret_cast<uint32_t*>(g.drain + 1);
+  g.abort_flag = reinterpret_cast<volatile int*>(g.tmem_slot + 1);
+  return g;
+}
+
+__device__ __forceinline__ bool g_aborted(const GemmSmem& g) {
+  uint32_t v;
+  asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32((const void*)g.abort_flag)) : "memory");
+  return v != 0;
+}
+
+// A bounded wait; on timeout the CTA records the error and stops (every role then skips its work).
+__device__ __noinline__ bool g_wait_slow(const PrefillParams& p, const GemmSmem& g, uint64_t* bar, uint32_t parity,
+                                         uint32_t where) {
+  if (g_aborted(g)) return false;
+  if (mbar_wait_slow(bar, parity, kPWaitNs)) return true;
+  if ((threadIdx.x & 31) == 0) {
+    atomicOr(&p.hdr->err, kErrPrefillWait);
+    p.hdr->err_info = where;
+  }
+  asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(smem_u32((const void*)g.abort_flag)), "r"(1u) : "memory");
+  return false;
+}
+__device__ __forceinline__ bool g_wait(const PrefillParams& p, const GemmSmem& g, uint64_t* bar, uint32_t parity,
+                                       uint32_t where) {
+  if (mbar_try_wait(bar, parity) && !g_aborted(g)) return true;
+  return g_wait_slow(p, g, bar, parity, where);
+}
+
+struct Ring {
+  int i = 0, slot = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void next(int S) {
+    ++i;
+    if (++slot == S) slot = 0, ph ^= 1u;
+  }
+};
+
+// The expert owning 128-row tile `tile`: the largest e with toff[e] <= tile (experts without tokens
+// share their successor's offset, so the expert found has at least one tile).
+__device__ __forceinline__ int tile_expert(const int32_t* toff, int E, int tile) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (toff[mid] <= tile) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t tmem_cols(int n) {
+  uint32_t c = 32;
+  while (c < uint32_t(2 * n)) c <<= 1;
+  return c;
+}
+
+__device__ void gemm_setup(const GemmSmem& g, int S, int N) {
+  const int tid = threadIdx.x, warp = tid >> 5;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&g.full[s], 1);
+      mbar_init(&g.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&g.accf[b], 1);
+      mbar_init(&g.acce[b], 4);
+    }
+    mbar_init(g.drain, 1);
+    *g.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(g.tmem_slot, tmem_cols(N));
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+}
+
+__device__ void gemm_teardown(const PrefillParams& p, const GemmSmem& g, int N) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 1) {  // every MMA issued by this CTA has completed before the columns are freed
+    if (lane == 0) tc::commit(g.drain);
+    __syncwarp();
+    mbar_wait_bounded(g.drain, 0, kPWaitNs / 10);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(*g.tmem_slot, tmem_cols(N));
+  (void)p;
+}
+
+// The producer's copies land before the CTA may exit.
+__device__ void producer_drain(const GemmSmem& g, const Ring& rp, int S) {
+  for (int k = rp.i - S > 0 ? rp.i - S : 0; k < rp.i; ++k)
+    mbar_wait_bounded(&g.full[k % S], uint32_t(k / S) & 1u, kPWaitNs / 10);
+}
+
+// GEMM1: per tile of 128 pairs of expert e, U = X[tokens] W1_e^T (N = de), then h = r Swish(U) as
+// bf16 hi and lo parts into H[pair][0, de) and H[pair][de, 2 de).
+__global__ void __launch_bounds__(kGThreads, 1)
+    prefill_gemm1_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
+  extern __shared__ uint8_t smem_raw[];
+  const int N = p.N1, S = p.S1;
+  const uint32_t a_bytes = kTileM * 128, stage_bytes = a_bytes + uint32_t(N) * 128;
+  const GemmSmem g = carve(smem_raw, S, stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&m.xg);
+    prefetch_tensormap(&m.w1);
+  }
+  gemm_setup(g, S, N);
+  const uint32_t tmem = *g.tmem_slot;
+  const int T = p.toff[p.E];
+  const int KB = p.d / 64;
+
+  if (warp == 0) {
+    const uint64_t pol = policy_evict_last();
+    Ring rp;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
+      const int e = tile_expert(p.toff, p.E, tile);
+      const int m0 = (tile - p.toff[e]) * kTileM, ne = p.cnt[e], pb = p.off[e] + m0;
+      int tk[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int r = lane * 4 + i;
+        tk[i] = p.tok[pb + (m0 + r < ne ? r : 0)];  // rows past the expert repeat its first row
+      }
+      for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
+        if (rp.i >= S && !g_wait(p, g, &g.empty[rp.slot], rp.ph ^ 1u, 21)) { ok = false; break; }
+        uint8_t* st = g.stages + size_t(rp.slot) * stage_bytes;
+        if (lane == 0) mbar_arrive_expect_tx(&g.full[rp.slot], stage_bytes);
+        __syncwarp();
+        tc::tma_gather4(st + lane * 512, &m.xg, kb * 64, tk[0], tk[1], tk[2], tk[3], &g.full[rp.slot]);
+        if (lane == 0) tma_load_2d(st + a_bytes, &m.w1, kb * 64, e * p.de, &g.full[rp.slot], pol);
+        __syncwarp();
+      }
+    }
+    producer_drain(g, rp, S);
+  } else if (warp == 1) {
+    const uint32_t idesc = tc::idesc_bf16_f32(kTileM, N);
+    Ring rp;
+    int tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x, ++tcount) {
+      const int ab = tcount & 1;
+      if (tcount >= 2 && !g_wait(p, g, &g.acce[ab], uint32_t((tcount >> 1) - 1) & 1u, 22)) { ok = false; break; }
+      tc::fence_after_sync();
+      for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
+        if (!g_wait(p, g, &g.full[rp.slot], rp.ph, 23)) { ok = false; break; }
+        tc::fence_after_sync();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(g.stages + size_t(rp.slot) * stage_bytes);
+          const uint64_t ad = tc::smem_desc_k128(sa), bd = tc::smem_desc_k128(sa + a_bytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            tc::mma_bf16(tmem + uint32_t(ab * N), ad + 2 * k, bd + 2 * k, idesc, uint32_t(kb | k));
+          tc::commit(&g.empty[rp.slot]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc::commit(&g.accf[ab]);
+      __syncwarp();
+    }
+  } else {
+    const int q = warp & 3;  // this warp's quarter of the tensor-memory lanes (rows)
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++tcount) {
+      const int ab = tcount & 1;
+      if (!g_wait(p, g, &g.accf[ab], uint32_t(tcount >> 1) & 1u, 24)) break;
+      tc::fence_after_sync();
+      const int e = tile_expert(p.toff, p.E, tile);
+      const int m0 = (tile - p.toff[e]) * kTileM, ne = p.cnt[e];
+      const int row = q * 32 + lane;
+      const bool valid = m0 + row < ne;
+      const size_t pair = size_t(p.off[e] + m0 + row);
+      const float r = valid ? p.rv[pair] : 0.f;
+      __nv_bfloat16* hrow = p.H + pair * size_t(2 * p.de);
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        float v[32];
+        tc::ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * N + c0), v);
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float h0 = r * (v[2 * i] / (1.f + expf(-v[2 * i])));
+          const float h1 = r * (v[2 * i + 1] / (1.f + expf(-v[2 * i + 1])));
+          const __nv_bfloat162 hh = __floats2bfloat162_rn(h0, h1);
+          const __nv_bfloat162 ll = __floats2bfloat162_rn(h0 - __low2float(hh), h1 - __high2float(hh));
+          hi[i] = *reinterpret_cast<const uint32_t*>(&hh);
+          lo[i] = *reinterpret_cast<const uint32_t*>(&ll);
+        }
+        if (valid) {
+          uint4* dh = reinterpret_cast<uint4*>(hrow + c0);
+          uint4* dl = reinterpret_cast<uint4*>(hrow + p.de + c0);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            dh[k] = make_uint4(hi[4 * k], hi[4 * k + 1], hi[4 * k + 2], hi[4 * k + 3]);
+            dl[k] = make_uint4(lo[4 * k], lo[4 * k + 1], lo[4 * k + 2], lo[4 * k + 3]);
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&g.acce[ab]);
+    }
+  }
+  gemm_teardown(p, g, N);
+}
+
+// GEMM2: per tile of 128 pairs of expert e and N2 columns of d, Y = H_hi W2_e^T + H_lo W2_e^T, added
+// into y[token] with vector reductions (every pair's row goes to its token's row).
+__global__ void __launch_bounds__(kGThreads, 1)
+    prefill_gemm2_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
+  extern __shared__ uint8_t smem_raw[];
+  const int N = p.N2, S = p.S2;
+  const uint32_t a_bytes = kTileM * 128, stage_bytes = 2 * a_bytes + uint32_t(N) * 128;
+  const GemmSmem g = carve(smem_raw, S, stage_bytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&m.h);
+    prefetch_tensormap(&m.w2);
+  }
+  gemm_setup(g, S, N);
+  const uint32_t tmem = *g.tmem_slot;
+  const int NT = p.d / N;
+  const int T = p.toff[p.E] * NT;
+  const int KB = p.de / 64;
+
+  if (warp == 0) {
+    const uint64_t pol = policy_evict_last();
+    Ring rp;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
+      const int mt = tile / NT, jn = tile - mt * NT;
+      const int e = tile_expert(p.toff, p.E, mt);
+      const int row0 = p.off[e] + (mt - p.toff[e]) * kTileM;
+      for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
+        if (rp.i >= S && !g_wait(p, g, &g.empty[rp.slot], rp.ph ^ 1u, 31)) { ok = false; break; }
+        uint8_t* st = g.stages + size_t(rp.slot) * stage_bytes;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&g.full[rp.slot], stage_bytes);
+          tma_load_2d(st, &m.h, kb * 64, row0, &g.full[rp.slot], pol);
+          tma_load_2d(st + a_bytes, &m.h, p.de + kb * 64, row0, &g.full[rp.slot], pol);
+          tma_load_2d(st + 2 * a_bytes, &m.w2, kb * 64, e * p.d + jn * N, &g.full[rp.slot], pol);
+        }
+        __syncwarp();
+      }
+    }
+    producer_drain(g, rp, S);
+  } else if (warp == 1) {
+    const uint32_t idesc = tc::idesc_bf16_f32(kTileM, N);
+    Ring rp;
+    int tcount = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x, ++tcount) {
+      const int ab = tcount & 1;
+      if (tcount >= 2 && !g_wait(p, g, &g.acce[ab], uint32_t((tcount >> 1) - 1) & 1u, 32)) { ok = false; break; }
+      tc::fence_after_sync();
+      for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
+        if (!g_wait(p, g, &g.full[rp.slot], rp.ph, 33)) { ok = false; break; }
+        tc::fence_after_sync();
+        if (lane == 0) {
+          const uint32_t sa = smem_u32(g.stages + size_t(rp.slot) * stage_bytes);
+          const uint64_t dhi = tc::smem_desc_k128(sa), dlo = tc::smem_desc_k128(sa + a_bytes),
+                         db = tc::smem_desc_k128(sa + 2 * a_bytes);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            tc::mma_bf16(tmem + uint32_t(ab * N), dhi + 2 * k, db + 2 * k, idesc, uint32_t(kb | k));
+            tc::mma_bf16(tmem + uint32_t(ab * N), dlo + 2 * k, db + 2 * k, idesc, 1u);
+          }
+          tc::commit(&g.empty[rp.slot]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc::commit(&g.accf[ab]);
+      __syncwarp();
+    }
+  } else {
+    const int q = warp & 3;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++tcount) {
+      const int ab = tcount & 1;
+      if (!g_wait(p, g, &g.accf[ab], uint32_t(tcount >> 1) & 1u, 34)) break;
+      tc::fence_after_sync();
+      const int mt = tile / NT, jn = tile - mt * NT;
+      const int e = tile_expert(p.toff, p.E, mt);
+      const int m0 = (mt - p.toff[e]) * kTileM, ne = p.cnt[e];
+      const int row = q * 32 + lane;
+      const bool valid = m0 + row < ne;
+      const int tok = valid ? p.tok[p.off[e] + m0 + row] : 0;
+      float* yrow = p.y + size_t(tok) * p.d + size_t(jn) * N;
+      for (int c0 = 0; c0 < N; c0 += 32) {
+        float v[32];
+        tc::ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * N + c0), v);
+        if (valid) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            atomicAdd(reinterpret_cast<float4*>(yrow + c0 + 4 * k),
+                      make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+        }
+      }
+      tc::fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&g.acce[ab]);
+    }
+  }
+  gemm_teardown(p, g, N);
+}
+
+}  // namespace
+
+bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, PrefillParams* p, PrefillLaunch* out) {
+  if (L <= kDecodeMaxL || d % 64 != 0 || de % 64 != 0 || de > 256 || E < 1 || E > kMaxE) return false;
+  if ((long long)L * E >= (1ll << 31) / 2) return false;  // pair indices, and H rows as TMA coordinates
+  p->W = (E + 31) / 32;
+  p->N1 = de;
+  p->N2 = d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
+  const size_t fixed = 1024 + 256;  // alignment slack, barriers, tensor-memory slot, abort flag
+  const size_t st1 = size_t(kTileM) * 128 + size_t(p->N1) * 128;
+  const size_t st2 = 2 * size_t(kTileM) * 128 + size_t(p->N2) * 128;
+  p->S1 = int((size_t(max_smem) - fixed) / st1);
+  p->S2 = int((size_t(max_smem) - fixed) / st2);
+  if (p->S1 > 6) p->S1 = 6;
+  if (p->S2 > 6) p->S2 = 6;
+  if (p->S1 < 2 || p->S2 < 2) return false;
+  out->grid = num_sms;
+  out->smem1 = fixed + size_t(p->S1) * st1;
+  out->smem2 = fixed + size_t(p->S2) * st2;
+  return true;
+}
+
+cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st) {
+  cudaError_t err = cudaMemsetAsync(p.y, 0, size_t(p.L) * p.d * sizeof(float), st);
+  if (err != cudaSuccess) return err;
+  prefill_router_kernel<<<dim3((p.L + kRtT - 1) / kRtT, (p.E + kRtE - 1) / kRtE), 256, 0, st>>>(p);
+  prefill_stats_kernel<<<(p.L + 7) / 8, 256, 0, st>>>(p);
+  prefill_count_kernel<<<(p.E + 7) / 8, 256, 0, st>>>(p);
+  prefill_fill_kernel<<<(p.E + 7) / 8, 256, 0, st>>>(p);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = cudaFuncSetAttribute(prefill_gemm1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(pl.smem1))) != cudaSuccess)
+    return err;
+  if ((err = cudaFuncSetAttribute(prefill_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(pl.smem2))) != cudaSuccess)
+    return err;
+  prefill_gemm1_kernel<<<pl.grid, kGThreads, pl.smem1, st>>>(p, m);
+  prefill_gemm2_kernel<<<pl.grid, kGThreads, pl.smem2, st>>>(p, m);
+  return cudaGetLastError();
+}
+
+}  // namespace bffn

@@ -75,6 +75,16 @@ def test_invalid_arguments_rejected_before_launch(bffn, kw):
 def test_unsupported_path_rejected_before_launch(bffn):
     # a decode-path request for a chunk longer than the decode path takes
     assert _call(bffn, L=33, flags=bffn.BFFN_PATH_DECODE) == bffn.BFFN_EUNSUPPORTED
+    # a prefill-path request for a decode-sized chunk
+    assert _call(bffn, L=32, flags=bffn.BFFN_PATH_PREFILL) == bffn.BFFN_EUNSUPPORTED
+    # prefill widths: d and de multiples of 64, de <= 256
+    assert _call(bffn, L=64, de=96) == bffn.BFFN_EUNSUPPORTED
+    assert _call(bffn, L=64, de=320) == bffn.BFFN_EUNSUPPORTED
+    assert _call(bffn, L=64, d=272) == bffn.BFFN_EUNSUPPORTED
+
+
+def test_prefill_needs_a_16_byte_aligned_y(bffn):
+    assert _call(bffn, L=64, y=FAKE + 4) == bffn.BFFN_EINVAL
 
 
 def test_plain_entry_point_validates(bffn):
