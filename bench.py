@@ -30,6 +30,8 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "BlockFFN layer tokens/s at chunk L=8 and achieved HBM GB/s over active bytes"
+METRIC_PREFILL = "BlockFFN layer tokens/s on a prefill chunk and achieved TFLOP/s (tcgen05 grouped GEMMs)"
+DECODE_MAX_L = 32
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -67,14 +69,14 @@ def barrier(device=None):
             dist.barrier()
 
 
-def measured_peaks():
+def measured_peaks(key="hbm_gbs"):
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             j = json.load(f)
-        return float(j["hbm_gbs"]), "measured"
+        return float(j[key]), "measured"
     except Exception:
-        return FALLBACK_HBM_GBS, "fallback"
+        return (FALLBACK_HBM_GBS if key == "hbm_gbs" else 1590.0), "fallback"
 
 
 def kernel_source_hash() -> str:
@@ -160,6 +162,12 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------------------------- workload
+def prefill_flops(d, E, de, L, pairs):
+    """Algorithmic FLOPs of a prefill chunk: both expert projections over the (token, expert) pairs
+    with r > 0, plus the router projection."""
+    return 4.0 * d * de * pairs + 2.0 * L * d * E
+
+
 def active_bytes(d, E, de, L, n_active):
     """Algorithmic bytes of one chunk: router weights, gain and bias, x in, y out, and W1_i + W2_i of
     every expert in the chunk's union (bf16)."""
@@ -216,6 +224,7 @@ def run_ours(args, w):
     y = torch.empty((chunks, L, d), dtype=torch.float32, device=device)
     idx = torch.empty((chunks, E), dtype=torch.int32, device=device)
     nact = torch.empty((chunks, 4), dtype=torch.int32, device=device)  # [c, 0] used
+    cnts = torch.empty((chunks, 2), dtype=torch.int32, device=device)  # TLS / CLS zero counts
 
     def step(stream_handle):
         for c in range(chunks):
@@ -223,7 +232,7 @@ def run_ours(args, w):
             rc = bffn.blockffn_chunk_forward_ex(
                 x_dev[c].data_ptr(), L, d, lay["Wr"].data_ptr(), lay["g"].data_ptr(), lay["W1"].data_ptr(),
                 lay["W2"].data_ptr(), E, de, y[c].data_ptr(), idx[c].data_ptr(), nact[c].data_ptr(),
-                lay["br"].data_ptr(), None, None, None, 0, None, 0, stream_handle)
+                lay["br"].data_ptr(), None, cnts[c].data_ptr(), None, 0, None, 0, stream_handle)
             if rc != 0:
                 raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_ex")
 
@@ -289,6 +298,8 @@ def run_ours(args, w):
     t_max = reduce_max(t_ms, device)
     e2e_max = reduce_max(e2e_ms, device)
     n_act_host = nact[:, 0].cpu().numpy()
+    pairs_host = L * E - cnts[:, 0].cpu().numpy().astype(np.int64)
+    prefill = L > DECODE_MAX_L
     total_active = float(sum(active_bytes(d, E, de, L, int(n)) for n in n_act_host))
     ms_per_step = t_max / args.steps
     tokens_step = chunks * L * world
@@ -297,8 +308,25 @@ def run_ours(args, w):
     peak, peak_kind = measured_peaks()
     ratio = recorded_traffic_ratio(w.name)
     traffic = None if ratio is None else ratio * total_active / chunks
+    if prefill:
+        flops = float(sum(prefill_flops(d, E, de, L, int(p)) for p in pairs_host))
+        achieved_tf = flops / (ms_per_step * 1e-3) / 1e12
+        tpeak, tpeak_kind = measured_peaks("bf16_tflops")
+        roofline = {"bound": "tensor", "achieved": round(achieved_tf, 1), "peak": tpeak, "unit": "TFLOP/s",
+                    "frac": round(achieved_tf / tpeak, 4), "peak_kind": tpeak_kind + " (bf16 burst)",
+                    "kernel": "one prefill chunk forward (router, grouping, tcgen05 GEMM1 and GEMM2)",
+                    "flops_per_chunk": round(flops / chunks, 1),
+                    "pairs_per_chunk": round(float(pairs_host.mean()), 1),
+                    "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3), "traffic": None}
+    else:
+        roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
+                    "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind,
+                    "kernel": "one chunk forward (router kernel + expert kernel, PDL-chained)",
+                    "bytes_per_chunk": round(total_active / chunks, 1),
+                    "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3),
+                    "traffic": None if traffic is None else round(traffic, 1)}
     out = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC_PREFILL if prefill else METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
@@ -308,17 +336,12 @@ def run_ours(args, w):
                    "mean_n_active": round(float(n_act_host.mean()), 3),
                    "cls": round(1.0 - float(n_act_host.mean()) / E, 4),
                    "parallelism": f"dp{world} (chunks sharded, no collective in the data path)"},
-        "roofline": {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind,
-                     "kernel": "one chunk forward (router kernel + expert kernel, PDL-chained)",
-                     "bytes_per_chunk": round(total_active / chunks, 1),
-                     "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3),
-                     "traffic": None if traffic is None else round(traffic, 1)},
+        "roofline": roofline,
         "e2e": {"value": round(tokens_step / (e2e_max / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host_np.nbytes),
                 "d2h_bytes_per_step": int(y.numel() * 4 + idx.numel() * 4 + nact.numel() * 4),
                 "steps": e2e_steps},
-        "gpu_launches": 2 * chunks * args.steps,
+        "gpu_launches": (6 if prefill else 2) * chunks * args.steps,
         "clocks": clk.summary(),
         "gen_seconds": round(gen_s, 1),
     }
@@ -334,8 +357,9 @@ def run_ours(args, w):
 
 # ---------------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
-    """The fp64 dense oracle timed on this host's cores on a bounded sample of the workload (chunks
-    of replica 0).  Also checks that sample against the GPU's output when one is given."""
+    """The fp64 dense oracle timed on this host's cores on a bounded sample of the workload (tokens
+    of the chunks that use replica 0, in groups of up to 8).  Also checks that sample against the
+    GPU's output when one is given."""
     import numpy as np
 
     import oracle
@@ -343,27 +367,28 @@ def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
     cores = oracle.available_cores()
     L, d = w.L, w.d
     chunk_ids = list(range(0, x_host_np.shape[0], w.replicas))  # chunks that use replica 0
-    # warm up on one chunk, calibrate on two, then size the sample to about `seconds`
-    oracle.tokens_forward_mt(x_host_np[chunk_ids[0]], lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
+    toks = x_host_np[chunk_ids].reshape(len(chunk_ids) * L, d)
+    group = min(L, 8)
+    # warm up on one group, calibrate on two, then size the sample to about `seconds`
+    oracle.tokens_forward_mt(toks[:group], lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
     t0 = time.time()
-    oracle.tokens_forward_mt(x_host_np[chunk_ids[0]].repeat(2, axis=0), lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2,
-                             cores)
-    t1 = (time.time() - t0) / 2
-    n_chunks = max(1, min(len(chunk_ids), int(seconds / max(t1, 1e-6))))
-    xs = x_host_np[chunk_ids[:n_chunks]].reshape(n_chunks * L, d)
+    oracle.tokens_forward_mt(np.repeat(toks[:group], 2, axis=0), lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
+    t_group = (time.time() - t0) / 2
+    n_groups = max(1, min(toks.shape[0] // group, int(seconds / max(t_group, 1e-6))))
+    n_tok = n_groups * group
     t0 = time.time()
-    y_ref = oracle.tokens_forward_mt(xs, lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
+    y_ref = oracle.tokens_forward_mt(toks[:n_tok], lay0.Wr, lay0.br, lay0.g, lay0.W1, lay0.W2, cores)
     dt = time.time() - t0
-    res = {"value": round(n_chunks * L / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-           "sample": f"{n_chunks} chunks x {L} tokens of weight replica 0 "
+    res = {"value": round(n_tok / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{n_tok} tokens of weight replica 0's chunks "
                      f"(dense fp64: all {w.E} experts per token), {dt:.1f} s"}
     if y_gpu is not None:
-        yg = y_gpu[chunk_ids[:n_chunks]].cpu().numpy().reshape(n_chunks * L, d).astype(np.float64)
+        yg = y_gpu[chunk_ids].reshape(len(chunk_ids) * L, d)[:n_tok].cpu().numpy().astype(np.float64)
         bad = 0
-        for c in range(n_chunks):
-            yr = y_ref[c * L:(c + 1) * L]
+        for a in range(0, n_tok, L):  # the tolerance's rms is taken per chunk
+            yr, yc = y_ref[a:a + L], yg[a:a + L]
             bound = 2e-2 * np.abs(yr) + 1e-3 * np.sqrt(np.mean(yr ** 2))
-            bad += int((np.abs(yg[c * L:(c + 1) * L] - yr) > bound).sum())
+            bad += int((np.abs(yc - yr) > bound).sum())
         res["parity_sample"] = {"y_elements_out_of_tolerance": bad, "elements": int(yg.size)}
     return res
 
@@ -380,22 +405,22 @@ def run_reference(args, w):
     lay = w.layer(0)
     L = w.L
     cores = oracle.available_cores()
-    per_step_chunks = max(1, args.ref_chunks)
-    x = gen.make_chunks(w.seed, lay, per_step_chunks, L, w.noise, stream=0)
-    xs = x.reshape(per_step_chunks * L, w.d)
-    oracle.tokens_forward_mt(xs[:L], lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores)  # warm-up
+    per_step_tokens = max(1, args.ref_chunks) * min(L, 8)  # decode: whole chunks; prefill: 8 tokens each
+    x = gen.make_chunks(w.seed, lay, 1 if L > 8 else max(1, args.ref_chunks), L, w.noise, stream=0)
+    xs = x.reshape(-1, w.d)[:per_step_tokens]
+    oracle.tokens_forward_mt(xs[:min(L, 8)], lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores)  # warm-up
     t0 = time.time()
     for _ in range(args.steps):
         oracle.tokens_forward_mt(xs, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores)
     dt = time.time() - t0
-    value = args.steps * per_step_chunks * L / dt
-    sample = (f"each step: {per_step_chunks} chunk(s) x {L} tokens of the workload, dense fp64 oracle "
+    value = args.steps * per_step_tokens / dt
+    sample = (f"each step: {per_step_tokens} tokens of the workload, dense fp64 oracle "
               f"(all {w.E} experts per token)")
-    out = {"metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
+    out = {"metric": METRIC_PREFILL if L > DECODE_MAX_L else METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
            "data": "synthetic", "impl": "reference",
-           "config": {**w.describe(), "chunks_per_step": per_step_chunks},
+           "config": {**w.describe(), "tokens_per_step": per_step_tokens},
            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
                             "sample": sample},
            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
@@ -409,7 +434,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=["decode", "tiny", "lsweep", "tls_sweep"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill"])
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
     ap.add_argument("--tls", type=float, default=None, help="token-level sparsity for --workload tls_sweep")
     ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")

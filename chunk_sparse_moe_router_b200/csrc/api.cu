@@ -224,6 +224,8 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
   p.Wr = Wr;
   p.br = br;
   p.g = g;
+  p.W1 = static_cast<const __nv_bfloat16*>(W1);
+  p.W2 = static_cast<const __nv_bfloat16*>(W2);
   p.y = y;
   p.active_idx = active_idx;
   p.n_active = n_active;
@@ -235,6 +237,7 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
   p.E = E;
   p.de = de;
   p.s = reinterpret_cast<float*>(base + lay.s_off);
+  p.s_part = reinterpret_cast<float*>(base + pl.spart_off);
   p.mask = reinterpret_cast<uint32_t*>(base + pl.mask_off);
   p.rms = reinterpret_cast<float*>(base + pl.rms_off);
   p.cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);

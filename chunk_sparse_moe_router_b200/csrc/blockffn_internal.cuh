@@ -35,16 +35,20 @@ __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_
 // lo rows) in the 128-byte-swizzled layout the down-projection loads.
 size_t decode_h_bytes(int L, int E, int de);
 
-// Prefill workspace regions (L > 32), after s: per-token masks and RMS, per-expert counts and
+// Prefill workspace regions (L > 32), after s: the router's K-split partial projections, per-token
+// masks and RMS, per-expert counts and
 // offsets, the pair lists (token, r) in expert-major order, and H = [pairs][2 de] bf16 (hi | lo).
+constexpr int kPrefillRouterSplit = 4;  // K parts of the prefill router projection
+
 struct PrefillLayout {
-  size_t mask_off, rms_off, cnt_off, off_off, toff_off, npos_off, tok_off, rv_off, h_off, end;
+  size_t spart_off, mask_off, rms_off, cnt_off, off_off, toff_off, npos_off, tok_off, rv_off, h_off, end;
 };
 
 inline PrefillLayout prefill_layout(size_t start, int L, int E, int de) {
   PrefillLayout p;
   const size_t W = size_t(E + 31) / 32, P = size_t(L) * E;
-  p.mask_off = start;
+  p.spart_off = start;
+  p.mask_off = p.spart_off + align256(size_t(kPrefillRouterSplit) * L * E * 4);
   p.rms_off = p.mask_off + align256(size_t(L) * W * 4);
   p.cnt_off = p.rms_off + align256(size_t(L) * 4);
   p.off_off = p.cnt_off + align256(size_t(E) * 4);
@@ -163,6 +167,8 @@ struct PrefillParams {
   const float* Wr;          // [d,E]
   const float* br;          // [E] or null
   const float* g;           // [E]
+  const __nv_bfloat16* W1;  // [E,de,d] (L2 prefetches; the GEMM reads it through its tensor map)
+  const __nv_bfloat16* W2;  // [E,d,de]
   float* y;                 // [L,d] out (zeroed before the down-projection adds into it)
   int32_t* active_idx;
   int32_t* n_active;
@@ -171,6 +177,8 @@ struct PrefillParams {
   float* r_out;             // optional
   int L, d, E, de, W;       // W = ceil(E / 32)
   float* s;                 // [L,E]
+  float* s_part;            // [ksplit][L,E] partial router projections
+  int ksplit;               // K parts of the router projection (d / ksplit a multiple of 32)
   uint32_t* mask;           // [L,W]
   float* rms;               // [L]
   int32_t* cnt;             // [E] tokens per expert

@@ -22,55 +22,72 @@ namespace {
 constexpr uint64_t kPWaitNs = 2000000000ull;
 
 // ---------------------------------------------------------------------------------- P1 router
-constexpr int kRtT = 32, kRtE = 64, kRtK = 32;  // tile: 32 tokens x 64 experts, K step 32
+// Tile: 64 tokens x 64 experts x (d / ksplit) of K per CTA, 256 threads with 4 x 4 outputs each.
+// The ksplit partial projections go to the workspace; the stats kernel adds them in fixed order.
+constexpr int kRtT = 64, kRtE = 64, kRtK = 32;
 
 __global__ void __launch_bounds__(256) prefill_router_kernel(PrefillParams p) {
-  __shared__ float Xs[kRtK][kRtT + 1];
+  __shared__ __align__(16) float Xs[kRtK][kRtT];
   __shared__ __align__(16) float Ws[kRtK][kRtE];
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *p.n_pos = 0;  // positive (t, e) count of this call
-  float acc[2][4] = {};
-  for (int k0 = 0; k0 < p.d; k0 += kRtK) {
-    for (int o = tid; o < kRtT * kRtK; o += 256) {
-      const int t = o / kRtK, k = o - t * kRtK;
-      Xs[k][t] = (t0 + t < p.L) ? __bfloat162float(p.x[size_t(t0 + t) * p.d + k0 + k]) : 0.f;
+  const int kper = p.d / p.ksplit, kbeg = blockIdx.z * kper;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0) *p.n_pos = 0;
+  const bool e_vec = (p.E & 3) == 0;
+  float acc[4][4] = {};
+  for (int k0 = kbeg; k0 < kbeg + kper; k0 += kRtK) {
+    {  // x: 64 tokens x 32 columns of bf16, one 16-byte load per thread, stored transposed as fp32
+      const int t = tid >> 2, k8 = (tid & 3) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t0 + t < p.L) v = *reinterpret_cast<const uint4*>(p.x + size_t(t0 + t) * p.d + k0 + k8);
+      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) Xs[k8 + i][t] = __bfloat162float(hv[i]);
     }
-    for (int o = tid; o < kRtK * kRtE; o += 256) {
-      const int k = o / kRtE, e = o - k * kRtE;
-      Ws[k][e] = (e0 + e < p.E) ? p.Wr[size_t(k0 + k) * p.E + e0 + e] : 0.f;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // Wr: 32 rows x 64 experts of fp32, two 16-byte loads per thread
+      const int o = tid + h * 256, k = o >> 4, e4 = (o & 15) * 4;
+      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+      const float* src = p.Wr + size_t(k0 + k) * p.E + e0 + e4;
+      if (e_vec && e0 + e4 + 3 < p.E) {
+        w = *reinterpret_cast<const float4*>(src);
+      } else {
+        if (e0 + e4 + 0 < p.E) w.x = src[0];
+        if (e0 + e4 + 1 < p.E) w.y = src[1];
+        if (e0 + e4 + 2 < p.E) w.z = src[2];
+        if (e0 + e4 + 3 < p.E) w.w = src[3];
+      }
+      *reinterpret_cast<float4*>(&Ws[k][e4]) = w;
     }
     __syncthreads();
     // a partial sum per K tile, added to the running total: a two-level sum keeps the rounding of a
-    // d-term dot product near that of its (d / 32 + 32)-term levels rather than of one d-term chain
-    float part[2][4] = {};
+    // d-term dot product near that of its shorter levels rather than of one long chain
+    float part[4][4] = {};
 #pragma unroll 8
     for (int k = 0; k < kRtK; ++k) {
-      const float a0 = Xs[k][ty * 2], a1 = Xs[k][ty * 2 + 1];
+      const float4 a = *reinterpret_cast<const float4*>(&Xs[k][ty * 4]);
       const float4 b = *reinterpret_cast<const float4*>(&Ws[k][tx * 4]);
-      part[0][0] = fmaf(a0, b.x, part[0][0]);
-      part[0][1] = fmaf(a0, b.y, part[0][1]);
-      part[0][2] = fmaf(a0, b.z, part[0][2]);
-      part[0][3] = fmaf(a0, b.w, part[0][3]);
-      part[1][0] = fmaf(a1, b.x, part[1][0]);
-      part[1][1] = fmaf(a1, b.y, part[1][1]);
-      part[1][2] = fmaf(a1, b.z, part[1][2]);
-      part[1][3] = fmaf(a1, b.w, part[1][3]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
     }
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
     __syncthreads();
   }
+  float* out = p.s_part + size_t(blockIdx.z) * p.L * p.E;
 #pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const int t = t0 + ty * 2 + i;
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
     if (t >= p.L) continue;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int e = e0 + tx * 4 + j;
-      if (e < p.E) p.s[size_t(t) * p.E + e] = acc[i][j] + (p.br ? p.br[e] : 0.f);
+      if (e < p.E) out[size_t(t) * p.E + e] = acc[i][j];
     }
   }
 }
@@ -81,7 +98,13 @@ __global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int t = warp;
   if (t >= p.L) return;
-  const float* st = p.s + size_t(t) * p.E;
+  float* st = p.s + size_t(t) * p.E;
+  for (int e = lane; e < p.E; e += 32) {  // s = the split-K parts in order, plus the bias
+    float v = 0.f;
+    for (int k = 0; k < p.ksplit; ++k) v += p.s_part[(size_t(k) * p.L + t) * p.E + e];
+    st[e] = v + (p.br ? p.br[e] : 0.f);
+  }
+  __syncwarp();
   float sumsq = 0.f;
   int n_pos = 0;
   for (int w = 0; w < p.W; ++w) {
@@ -113,67 +136,86 @@ __device__ __forceinline__ bool active_bit(const PrefillParams& p, int t, int e)
   return t < p.L && ((p.mask[size_t(t) * p.W + (e >> 5)] >> (e & 31)) & 1u);
 }
 
-// One warp per expert: the number of its tokens.
-__global__ void __launch_bounds__(256) prefill_count_kernel(PrefillParams p) {
-  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (e >= p.E) return;
-  int n = 0;
-  for (int t0 = 0; t0 < p.L; t0 += 32) n += __popc(__ballot_sync(0xffffffffu, active_bit(p, t0 + lane, e)));
-  if (lane == 0) p.cnt[e] = n;
+// Tokens [t0, t1) of warp w when 8 warps split L tokens into 32-token groups.
+__device__ __forceinline__ void warp_token_range(int L, int w, int* t0, int* t1) {
+  const int groups = (L + 31) / 32, per = (groups + 7) / 8;
+  *t0 = min(L, w * per * 32);
+  *t1 = min(L, (w + 1) * per * 32);
 }
 
-// One warp per expert: its token list (ascending) and r values at its pair offset.  CTA 0 also
-// writes the pair and tile offsets, the union (active experts ascending), n_active and the counts.
-__global__ void __launch_bounds__(256) prefill_fill_kernel(PrefillParams p) {
-  const int lane = threadIdx.x & 31;
-  const int e = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (blockIdx.x == 0 && threadIdx.x < 32) {
-    // exclusive scans over the experts (pairs and 128-row tiles) and the union, in one warp
-    int pairs = 0, tiles = 0, nact = 0;
-    for (int e0 = 0; e0 < p.E; e0 += 32) {
-      const int ee = e0 + lane;
-      const int c = ee < p.E ? p.cnt[ee] : 0;
-      const int mt = (c + 127) >> 7;
-      int ic = c, im = mt, ia = c > 0 ? 1 : 0;
+// One CTA per expert: the number of its tokens (8 warps count a share each).
+__global__ void __launch_bounds__(256) prefill_count_kernel(PrefillParams p) {
+  __shared__ int wc[8];
+  const int e = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int t0, t1;
+  warp_token_range(p.L, warp, &t0, &t1);
+  int n = 0;
+#pragma unroll 4
+  for (int t = t0; t < t1; t += 32) n += __popc(__ballot_sync(0xffffffffu, active_bit(p, t + lane, e)));
+  if (lane == 0) wc[warp] = n;
+  __syncthreads();
+  if (threadIdx.x == 0) p.cnt[e] = wc[0] + wc[1] + wc[2] + wc[3] + wc[4] + wc[5] + wc[6] + wc[7];
+}
+
+// Pair and tile offsets of every expert, the union (active experts ascending), n_active and the
+// counts: one warp.
+__global__ void __launch_bounds__(32) prefill_scan_kernel(PrefillParams p) {
+  const int lane = threadIdx.x;
+  int pairs = 0, tiles = 0, nact = 0;
+  for (int e0 = 0; e0 < p.E; e0 += 32) {
+    const int ee = e0 + lane;
+    const int c = ee < p.E ? p.cnt[ee] : 0;
+    const int mt = (c + 127) >> 7;
+    int ic = c, im = mt, ia = c > 0 ? 1 : 0;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int vc = __shfl_up_sync(0xffffffffu, ic, o), vm = __shfl_up_sync(0xffffffffu, im, o),
-                  va = __shfl_up_sync(0xffffffffu, ia, o);
-        if (lane >= o) ic += vc, im += vm, ia += va;
-      }
-      if (ee < p.E) {
-        p.off[ee] = pairs + ic - c;
-        p.toff[ee] = tiles + im - mt;
-        if (c > 0) p.active_idx[nact + ia - 1] = ee;
-      }
-      pairs += __shfl_sync(0xffffffffu, ic, 31);
-      tiles += __shfl_sync(0xffffffffu, im, 31);
-      nact += __shfl_sync(0xffffffffu, ia, 31);
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xffffffffu, ic, o), vm = __shfl_up_sync(0xffffffffu, im, o),
+                va = __shfl_up_sync(0xffffffffu, ia, o);
+      if (lane >= o) ic += vc, im += vm, ia += va;
     }
-    if (lane == 0) {
-      p.off[p.E] = pairs;
-      p.toff[p.E] = tiles;
-      *p.n_active = nact;
-      if (p.counts) {
-        p.counts[0] = p.L * p.E - *p.n_pos;
-        p.counts[1] = p.E - nact;
-      }
+    if (ee < p.E) {
+      p.off[ee] = pairs + ic - c;
+      p.toff[ee] = tiles + im - mt;
+      if (c > 0) p.active_idx[nact + ia - 1] = ee;
+    }
+    pairs += __shfl_sync(0xffffffffu, ic, 31);
+    tiles += __shfl_sync(0xffffffffu, im, 31);
+    nact += __shfl_sync(0xffffffffu, ia, 31);
+  }
+  if (lane == 0) {
+    p.off[p.E] = pairs;
+    p.toff[p.E] = tiles;
+    *p.n_active = nact;
+    if (p.counts) {
+      p.counts[0] = p.L * p.E - *p.n_pos;
+      p.counts[1] = p.E - nact;
     }
   }
-  if (e >= p.E) return;
-  int base = 0;  // this expert's pair offset: the tokens of every lower expert
-  for (int e2 = lane; e2 < e; e2 += 32) base += p.cnt[e2];
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) base += __shfl_xor_sync(0xffffffffu, base, o);
+}
+
+// One CTA per expert: its token list (ascending) and r values at its pair offset.  8 warps take a
+// share of the tokens each; a warp's position is the expert's offset plus the lower warps' counts.
+__global__ void __launch_bounds__(256) prefill_fill_kernel(PrefillParams p) {
+  __shared__ int wc[8];
+  const int e = blockIdx.x, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int t0, t1;
+  warp_token_range(p.L, warp, &t0, &t1);
+  int n = 0;
+#pragma unroll 4
+  for (int t = t0; t < t1; t += 32) n += __popc(__ballot_sync(0xffffffffu, active_bit(p, t + lane, e)));
+  if (lane == 0) wc[warp] = n;
+  __syncthreads();
+  int base = p.off[e];
+  for (int w = 0; w < warp; ++w) base += wc[w];
   const float ge = p.g[e];
-  for (int t0 = 0; t0 < p.L; t0 += 32) {
-    const int t = t0 + lane;
-    const bool on = active_bit(p, t, e);
+  for (int t = t0; t < t1; t += 32) {
+    const int tt = t + lane;
+    const bool on = active_bit(p, tt, e);
     const uint32_t b = __ballot_sync(0xffffffffu, on);
     if (on) {
       const int pos = base + __popc(b & ((1u << lane) - 1u));
-      p.tok[pos] = t;
-      p.rv[pos] = (ge * p.s[size_t(t) * p.E + e]) / p.rms[t];  // s > 0, so relu(s) = s and rms > 0
+      p.tok[pos] = tt;
+      p.rv[pos] = (ge * p.s[size_t(tt) * p.E + e]) / p.rms[tt];  // s > 0, so relu(s) = s and rms > 0
     }
     base += __popc(b);
   }
@@ -184,8 +226,22 @@ __global__ void __launch_bounds__(256) prefill_fill_kernel(PrefillParams p) {
 namespace {
 
 // ---------------------------------------------------------------------------------- P4/P5 GEMMs
-constexpr int kGThreads = 192;  // warp 0: TMA producer, warp 1: MMA issuer (owns TMEM), warps 2-5: epilogue
+constexpr int kGThreads = 192;   // warp 0: TMA producer, warp 1: MMA issuer (owns TMEM), warps 2-5: epilogue
+constexpr int kG1Threads = 320;  // GEMM1 adds warps 6-9: the gathered A rows, one token row per thread
 constexpr int kTileM = 128;
+constexpr int kPf1 = 12;  // GEMM1: W1 rows are prefetched into L2 this many stages ahead
+
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// y[0..3] += v, a reduction performed at L2; the line is marked to stay in L2 (y takes every pair's
+// contribution while W2 streams past).
+__device__ __forceinline__ void red_add_v4(float* y, float a, float b, float c, float d, uint64_t policy) {
+  asm volatile("red.global.add.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(y), "f"(a), "f"(b), "f"(c),
+               "f"(d), "l"(policy)
+               : "memory");
+}
 
 struct GemmSmem {
   uint8_t* stages;
@@ -196,9 +252,12 @@ struct GemmSmem {
   uint64_t* drain;  // every MMA of this CTA complete (before TMEM is freed)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
+  int* toff;        // [E+1] copies of the per-expert tile offsets, pair offsets and token counts
+  int* off;         // [E+1]
+  int* cnt;         // [E]
 };
 
-__device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_bytes) {
+__device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_bytes, int E) {
   GemmSmem g;
   g.stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
   g.full = reinterpret_cast<uint64_t*>(g.stages + size_t(S) * stage_bytes);
@@ -208,6 +267,10 @@ __device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_by
   g.drain = g.acce + 2;
   g.tmem_slot = reinterpret_cast<uint32_t*>(g.drain + 1);
   g.abort_flag = reinterpret_cast<volatile int*>(g.tmem_slot + 1);
+  g.toff = reinterpret_cast<int*>(g.tmem_slot + 4);
+  g.off = g.toff + (E + 1);
+  g.cnt = g.off + (E + 1);
+  (void)E;
   return g;
 }
 
@@ -256,17 +319,38 @@ __device__ __forceinline__ int tile_expert(const int32_t* toff, int E, int tile)
   return lo;
 }
 
+// GEMM2 tile -> (expert e, N tile jn, 128-row tile of the expert): the tiles of one expert are
+// contiguous, N-tile-major, so the CTAs working on one W2_e slice at a time read it once from HBM
+// and the expert's (few) rows of H repeat from L2.
+struct Tile2 {
+  int e, jn, m0;
+};
+__device__ __forceinline__ Tile2 tile2_at(const GemmSmem& g, int E, int NT, int tile) {
+  Tile2 t;
+  t.e = tile_expert(g.toff, E, tile / NT);  // the expert's tiles are [toff[e] NT, toff[e+1] NT)
+  const int nm = g.toff[t.e + 1] - g.toff[t.e];
+  const int li = tile - g.toff[t.e] * NT;
+  t.jn = li / nm;
+  t.m0 = (li - t.jn * nm) * kTileM;
+  return t;
+}
+
 __device__ __forceinline__ uint32_t tmem_cols(int n) {
   uint32_t c = 32;
   while (c < uint32_t(2 * n)) c <<= 1;
   return c;
 }
 
-__device__ void gemm_setup(const GemmSmem& g, int S, int N) {
+__device__ void gemm_setup(const PrefillParams& p, const GemmSmem& g, int S, int N, int full_count) {
   const int tid = threadIdx.x, warp = tid >> 5;
+  for (int i = tid; i <= p.E; i += blockDim.x) {  // the tables every tile lookup reads
+    g.toff[i] = p.toff[i];
+    g.off[i] = p.off[i];
+    if (i < p.E) g.cnt[i] = p.cnt[i];
+  }
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&g.full[s], 1);
+      mbar_init(&g.full[s], full_count);
       mbar_init(&g.empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -305,46 +389,79 @@ __device__ void producer_drain(const GemmSmem& g, const Ring& rp, int S) {
 
 // GEMM1: per tile of 128 pairs of expert e, U = X[tokens] W1_e^T (N = de), then h = r Swish(U) as
 // bf16 hi and lo parts into H[pair][0, de) and H[pair][de, 2 de).
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kG1Threads, 1)
     prefill_gemm1_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
   extern __shared__ uint8_t smem_raw[];
   const int N = p.N1, S = p.S1;
   const uint32_t a_bytes = kTileM * 128, stage_bytes = a_bytes + uint32_t(N) * 128;
-  const GemmSmem g = carve(smem_raw, S, stage_bytes);
+  const GemmSmem g = carve(smem_raw, S, stage_bytes, p.E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    prefetch_tensormap(&m.xg);
-    prefetch_tensormap(&m.w1);
-  }
-  gemm_setup(g, S, N);
+  if (threadIdx.x == 0) prefetch_tensormap(&m.w1);
+  gemm_setup(p, g, S, N, 1 + kTileM);  // the W1 box (expect_tx) and one row-copy arrival per A row
   const uint32_t tmem = *g.tmem_slot;
-  const int T = p.toff[p.E];
+  const int T = g.toff[p.E];
   const int KB = p.d / 64;
 
   if (warp == 0) {
-    const uint64_t pol = policy_evict_last();
+    const uint64_t pol_w = policy_evict_first();  // W1 streams through once
     Ring rp;
     bool ok = true;
     for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
-      const int e = tile_expert(p.toff, p.E, tile);
-      const int m0 = (tile - p.toff[e]) * kTileM, ne = p.cnt[e], pb = p.off[e] + m0;
-      int tk[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int r = lane * 4 + i;
-        tk[i] = p.tok[pb + (m0 + r < ne ? r : 0)];  // rows past the expert repeat its first row
-      }
+      const int e = tile_expert(g.toff, p.E, tile);
       for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
         if (rp.i >= S && !g_wait(p, g, &g.empty[rp.slot], rp.ph ^ 1u, 21)) { ok = false; break; }
         uint8_t* st = g.stages + size_t(rp.slot) * stage_bytes;
-        if (lane == 0) mbar_arrive_expect_tx(&g.full[rp.slot], stage_bytes);
-        __syncwarp();
-        tc::tma_gather4(st + lane * 512, &m.xg, kb * 64, tk[0], tk[1], tk[2], tk[3], &g.full[rp.slot]);
-        if (lane == 0) tma_load_2d(st + a_bytes, &m.w1, kb * 64, e * p.de, &g.full[rp.slot], pol);
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&g.full[rp.slot], uint32_t(N) * 128);
+          tma_load_2d(st + a_bytes, &m.w1, kb * 64, e * p.de, &g.full[rp.slot], pol_w);
+        }
         __syncwarp();
       }
     }
     producer_drain(g, rp, S);
+  } else if (warp >= 6) {
+    // A rows: lanes 8q..8q+7 of a loader warp copy the eight 16-byte pieces of one token row (128
+    // bytes: 64 bf16 of the K block), so a warp-wide copy covers 4 whole rows; loader warp w takes rows
+    // 32w..32w+31 in 8 such steps.  Pieces land in the 128-byte-swizzled layout; a thread's arrival on
+    // the stage barrier fires when its copies complete.
+    const int lw = warp - 6, c = lane & 7, rq = lane >> 3;
+    const int tpr = threadIdx.x - 6 * 32;  // W1 L2 prefetch: rows 2 tpr, 2 tpr + 1 of a future stage
+    Ring rp;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
+      const int e = tile_expert(g.toff, p.E, tile);
+      const int m0 = (tile - g.toff[e]) * kTileM, ne = g.cnt[e];
+      const __nv_bfloat16* src[8];
+#pragma unroll
+      for (int it = 0; it < 8; ++it) {
+        const int r = lw * 32 + it * 4 + rq;
+        const int tok = p.tok[g.off[e] + m0 + (m0 + r < ne ? r : 0)];  // rows past the expert repeat row 0
+        src[it] = p.x + size_t(tok) * p.d + c * 8;
+      }
+      const int tile_nx = tile + int(gridDim.x);
+      const int e_nx = tile_nx < T ? tile_expert(g.toff, p.E, tile_nx) : -1;
+      for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
+        if (rp.i >= S && !g_wait(p, g, &g.empty[rp.slot], rp.ph ^ 1u, 25)) { ok = false; break; }
+        const uint32_t st = smem_u32(g.stages + size_t(rp.slot) * stage_bytes);
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int r = lw * 32 + it * 4 + rq;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(st + uint32_t(r * 128 + ((c ^ (r & 7)) << 4))),
+                       "l"(src[it] + kb * 64)
+                       : "memory");
+        }
+        asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(&g.full[rp.slot]))
+                     : "memory");
+        // the W1 lines of the stage kPf1 ahead into L2
+        const int kf = kb + kPf1;
+        const int ef = kf < KB ? e : e_nx, kbf = kf < KB ? kf : kf - KB;
+        if (ef >= 0 && kbf < KB)
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            if (2 * tpr + h < N) prefetch_l2(p.W1 + (size_t(ef) * p.de + 2 * tpr + h) * p.d + kbf * 64);
+      }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // every row copy has landed before the CTA may exit
   } else if (warp == 1) {
     const uint32_t idesc = tc::idesc_bf16_f32(kTileM, N);
     Ring rp;
@@ -357,6 +474,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
       for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
         if (!g_wait(p, g, &g.full[rp.slot], rp.ph, 23)) { ok = false; break; }
         tc::fence_after_sync();
+        fence_proxy_async_smem();  // the A rows were written by ordinary (non-bulk) copies
         if (lane == 0) {
           const uint32_t sa = smem_u32(g.stages + size_t(rp.slot) * stage_bytes);
           const uint64_t ad = tc::smem_desc_k128(sa), bd = tc::smem_desc_k128(sa + a_bytes);
@@ -378,11 +496,11 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int ab = tcount & 1;
       if (!g_wait(p, g, &g.accf[ab], uint32_t(tcount >> 1) & 1u, 24)) break;
       tc::fence_after_sync();
-      const int e = tile_expert(p.toff, p.E, tile);
-      const int m0 = (tile - p.toff[e]) * kTileM, ne = p.cnt[e];
+      const int e = tile_expert(g.toff, p.E, tile);
+      const int m0 = (tile - g.toff[e]) * kTileM, ne = g.cnt[e];
       const int row = q * 32 + lane;
       const bool valid = m0 + row < ne;
-      const size_t pair = size_t(p.off[e] + m0 + row);
+      const size_t pair = size_t(g.off[e] + m0 + row);
       const float r = valid ? p.rv[pair] : 0.f;
       __nv_bfloat16* hrow = p.H + pair * size_t(2 * p.de);
       for (int c0 = 0; c0 < N; c0 += 32) {
@@ -423,34 +541,35 @@ __global__ void __launch_bounds__(kGThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   const int N = p.N2, S = p.S2;
   const uint32_t a_bytes = kTileM * 128, stage_bytes = 2 * a_bytes + uint32_t(N) * 128;
-  const GemmSmem g = carve(smem_raw, S, stage_bytes);
+  const GemmSmem g = carve(smem_raw, S, stage_bytes, p.E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     prefetch_tensormap(&m.h);
     prefetch_tensormap(&m.w2);
   }
-  gemm_setup(g, S, N);
+  gemm_setup(p, g, S, N, 1);
   const uint32_t tmem = *g.tmem_slot;
   const int NT = p.d / N;
-  const int T = p.toff[p.E] * NT;
+  const int T = g.toff[p.E] * NT;
   const int KB = p.de / 64;
 
   if (warp == 0) {
-    const uint64_t pol = policy_evict_last();
+    const uint64_t pol_h = policy_evict_normal();  // an expert's H rows repeat over its N tiles, soon
+    const uint64_t pol_w = policy_evict_first();  // W2 streams through (y stays in L2 for the adds)
     Ring rp;
     bool ok = true;
     for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
-      const int mt = tile / NT, jn = tile - mt * NT;
-      const int e = tile_expert(p.toff, p.E, mt);
-      const int row0 = p.off[e] + (mt - p.toff[e]) * kTileM;
+      const Tile2 tl = tile2_at(g, p.E, NT, tile);
+      const int e = tl.e, jn = tl.jn;
+      const int row0 = g.off[e] + tl.m0;
       for (int kb = 0; kb < KB; ++kb, rp.next(S)) {
         if (rp.i >= S && !g_wait(p, g, &g.empty[rp.slot], rp.ph ^ 1u, 31)) { ok = false; break; }
         uint8_t* st = g.stages + size_t(rp.slot) * stage_bytes;
         if (lane == 0) {
           mbar_arrive_expect_tx(&g.full[rp.slot], stage_bytes);
-          tma_load_2d(st, &m.h, kb * 64, row0, &g.full[rp.slot], pol);
-          tma_load_2d(st + a_bytes, &m.h, p.de + kb * 64, row0, &g.full[rp.slot], pol);
-          tma_load_2d(st + 2 * a_bytes, &m.w2, kb * 64, e * p.d + jn * N, &g.full[rp.slot], pol);
+          tma_load_2d(st, &m.h, kb * 64, row0, &g.full[rp.slot], pol_h);
+          tma_load_2d(st + a_bytes, &m.h, p.de + kb * 64, row0, &g.full[rp.slot], pol_h);
+          tma_load_2d(st + 2 * a_bytes, &m.w2, kb * 64, e * p.d + jn * N, &g.full[rp.slot], pol_w);
         }
         __syncwarp();
       }
@@ -487,17 +606,17 @@ __global__ void __launch_bounds__(kGThreads, 1)
     }
   } else {
     const int q = warp & 3;
+    const uint64_t pol_y = policy_evict_last();
     int tcount = 0;
     for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++tcount) {
       const int ab = tcount & 1;
       if (!g_wait(p, g, &g.accf[ab], uint32_t(tcount >> 1) & 1u, 34)) break;
       tc::fence_after_sync();
-      const int mt = tile / NT, jn = tile - mt * NT;
-      const int e = tile_expert(p.toff, p.E, mt);
-      const int m0 = (mt - p.toff[e]) * kTileM, ne = p.cnt[e];
+      const Tile2 tl = tile2_at(g, p.E, NT, tile);
+      const int e = tl.e, jn = tl.jn, m0 = tl.m0, ne = g.cnt[e];
       const int row = q * 32 + lane;
       const bool valid = m0 + row < ne;
-      const int tok = valid ? p.tok[p.off[e] + m0 + row] : 0;
+      const int tok = valid ? p.tok[g.off[e] + m0 + row] : 0;
       float* yrow = p.y + size_t(tok) * p.d + size_t(jn) * N;
       for (int c0 = 0; c0 < N; c0 += 32) {
         float v[32];
@@ -505,8 +624,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
         if (valid) {
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            atomicAdd(reinterpret_cast<float4*>(yrow + c0 + 4 * k),
-                      make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]));
+            red_add_v4(yrow + c0 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], pol_y);
         }
       }
       tc::fence_before_sync();
@@ -523,9 +641,11 @@ bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, Prefil
   if (L <= kDecodeMaxL || d % 64 != 0 || de % 64 != 0 || de > 256 || E < 1 || E > kMaxE) return false;
   if ((long long)L * E >= (1ll << 31) / 2) return false;  // pair indices, and H rows as TMA coordinates
   p->W = (E + 31) / 32;
+  p->ksplit = d % (kPrefillRouterSplit * 32) == 0 ? kPrefillRouterSplit : 2;  // d / ksplit: whole K tiles
   p->N1 = de;
   p->N2 = d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
-  const size_t fixed = 1024 + 256;  // alignment slack, barriers, tensor-memory slot, abort flag
+  // alignment slack, barriers, tensor-memory slot, abort flag, the three per-expert tables
+  const size_t fixed = 1024 + 256 + (3 * size_t(E) + 2) * 4;
   const size_t st1 = size_t(kTileM) * 128 + size_t(p->N1) * 128;
   const size_t st2 = 2 * size_t(kTileM) * 128 + size_t(p->N2) * 128;
   p->S1 = int((size_t(max_smem) - fixed) / st1);
@@ -542,10 +662,11 @@ bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, Prefil
 cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st) {
   cudaError_t err = cudaMemsetAsync(p.y, 0, size_t(p.L) * p.d * sizeof(float), st);
   if (err != cudaSuccess) return err;
-  prefill_router_kernel<<<dim3((p.L + kRtT - 1) / kRtT, (p.E + kRtE - 1) / kRtE), 256, 0, st>>>(p);
+  prefill_router_kernel<<<dim3((p.L + kRtT - 1) / kRtT, (p.E + kRtE - 1) / kRtE, p.ksplit), 256, 0, st>>>(p);
   prefill_stats_kernel<<<(p.L + 7) / 8, 256, 0, st>>>(p);
-  prefill_count_kernel<<<(p.E + 7) / 8, 256, 0, st>>>(p);
-  prefill_fill_kernel<<<(p.E + 7) / 8, 256, 0, st>>>(p);
+  prefill_count_kernel<<<p.E, 256, 0, st>>>(p);
+  prefill_scan_kernel<<<1, 32, 0, st>>>(p);
+  prefill_fill_kernel<<<p.E, 256, 0, st>>>(p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   if ((err = cudaFuncSetAttribute(prefill_gemm1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(pl.smem1))) != cudaSuccess)
@@ -553,7 +674,7 @@ cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const P
   if ((err = cudaFuncSetAttribute(prefill_gemm2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(pl.smem2))) != cudaSuccess)
     return err;
-  prefill_gemm1_kernel<<<pl.grid, kGThreads, pl.smem1, st>>>(p, m);
+  prefill_gemm1_kernel<<<pl.grid, kG1Threads, pl.smem1, st>>>(p, m);
   prefill_gemm2_kernel<<<pl.grid, kGThreads, pl.smem2, st>>>(p, m);
   return cudaGetLastError();
 }
