@@ -31,8 +31,12 @@
  *   1 <= L, 1 <= E <= 1024, d >= 16 and d % 16 == 0, de >= 16 and de % 16 == 0;
  *   x, Wr, W1, W2 16-byte aligned (they are read with bulk copies), a workspace 256-byte aligned,
  *   every other pointer 4-byte aligned; required pointers non-NULL.
- * Paths: L <= 32 runs the decode path (weights streamed from HBM, memory-bound); larger L runs the
- * prefill path. A shape a path cannot take returns BFFN_EUNSUPPORTED.
+ * Paths: L <= 32 runs the decode path (the union's weights streamed from HBM once for the whole chunk,
+ * memory-bound, deterministic: y is bit-identical run to run). Larger L runs the prefill path (tokens
+ * grouped per active expert, grouped GEMMs on the tcgen05 tensor cores); it additionally needs d and de
+ * multiples of 64, de <= 256 and y 16-byte aligned, and it adds each (token, expert) row into y with
+ * hardware reductions, so y may differ in the last bits between runs (masks, union, counts and r do
+ * not). A shape a path cannot take returns BFFN_EUNSUPPORTED (nothing is enqueued).
  *
  * Errors: BFFN_ECUDA when a CUDA call fails (the CUDA error is cleared); BFFN_ENOMEM when the
  * internal workspace cannot be allocated. Device-side waits are bounded (about 2 s); a wait that
