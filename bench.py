@@ -1,8 +1,10 @@
 """Benchmark of the BlockFFN chunk-layer forward on B200.
 
-One step = one pass of the hot path over one batch of synthetic input: `chunks` sequential chunk
-forwards (router + chunk union + sparse experts, two kernels per chunk) through the C ABI, chunk c
-using weight replica c % replicas.  The replicas stand for distinct layers of a stacked model and keep
+One step = one pass of the hot path over one batch of synthetic input: `chunks` chunk forwards
+(router + chunk union + sparse experts, two kernels per chunk) through the C ABI, chunk c using
+weight replica c % replicas.  The chunks are independent: chunk c is issued on stream c % K (--streams,
+default 8) with its own workspace and the concurrency hint, so K chunks run side by side, each on
+1/K of the SMs, and one chunk's fixed latencies overlap the others' weight streaming.  The replicas stand for distinct layers of a stacked model and keep
 the weights (16 x 128 MiB for the default workload) well above the 126 MB L2, so every chunk streams
 its active experts from HBM ("inputs larger than L2").  A step is captured once into a CUDA graph
 and replayed; time is taken with CUDA events on the replay stream, with a barrier and a
@@ -226,25 +228,48 @@ def run_ours(args, w):
     nact = torch.empty((chunks, 4), dtype=torch.int32, device=device)  # [c, 0] used
     cnts = torch.empty((chunks, 2), dtype=torch.int32, device=device)  # TLS / CLS zero counts
 
-    def step(stream_handle):
+    # K streams, each with its own workspace: chunk c goes to stream c % K, and with K > 1 each call
+    # takes 1/K of the SMs (decode), so K independent chunks run side by side.
+    K = max(1, args.streams if L <= DECODE_MAX_L else 1)
+    flags = bffn.BFFN_FLAGS_SHARE(K) if K > 1 else 0
+    ws_bytes = bffn.blockffn_workspace_size(L, d, E, de)
+    workspaces = [bffn.new_workspace(L, d, E, de, device) for _ in range(K)]  # zero-filled, 512-byte aligned
+    ws_ptrs = [t.data_ptr() for t in workspaces]
+
+    def step(streams):
+        if K > 1:  # fork: the side streams start after everything queued on the main one
+            ev = torch.cuda.Event()
+            ev.record(streams[0])
+            for sk in streams[1:]:
+                sk.wait_event(ev)
         for c in range(chunks):
             lay = layers[c % w.replicas]
+            k = c % K
             rc = bffn.blockffn_chunk_forward_ex(
                 x_dev[c].data_ptr(), L, d, lay["Wr"].data_ptr(), lay["g"].data_ptr(), lay["W1"].data_ptr(),
                 lay["W2"].data_ptr(), E, de, y[c].data_ptr(), idx[c].data_ptr(), nact[c].data_ptr(),
-                lay["br"].data_ptr(), None, cnts[c].data_ptr(), None, 0, None, 0, stream_handle)
+                lay["br"].data_ptr(), None, cnts[c].data_ptr(), None, flags, ws_ptrs[k], ws_bytes,
+                streams[k].cuda_stream)
             if rc != 0:
                 raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_ex")
+        if K > 1:  # join
+            for sk in streams[1:]:
+                ev = torch.cuda.Event()
+                ev.record(sk)
+                streams[0].wait_event(ev)
 
     s = torch.cuda.Stream(device)
+    side = [torch.cuda.Stream(device) for _ in range(K - 1)]
+    streams = [s] + side
     with torch.cuda.stream(s):
-        step(s.cuda_stream)  # first call allocates the library workspace (before capture)
+        step(streams)
         s.synchronize()
-        if bffn.device_status(stream=s.cuda_stream) != 0:
-            raise RuntimeError("device-side wait ran out")
+        for k in range(K):
+            if bffn.device_status(workspace=workspaces[k], stream=s.cuda_stream) != 0:
+                raise RuntimeError("device-side wait ran out")
         graph = torch.cuda.CUDAGraph()
         graph.capture_begin()
-        step(s.cuda_stream)
+        step(streams)
         graph.capture_end()
         s.synchronize()
         for _ in range(args.warmup):
@@ -263,8 +288,9 @@ def run_ours(args, w):
         torch.cuda.synchronize(device)
         barrier(device)
         t_ms = e0.elapsed_time(e1)
-        if bffn.device_status(stream=s.cuda_stream) != 0:
-            raise RuntimeError("device-side wait ran out during the timed region")
+        for k in range(K):
+            if bffn.device_status(workspace=workspaces[k], stream=s.cuda_stream) != 0:
+                raise RuntimeError("device-side wait ran out during the timed region")
 
         # end to end: x from pinned host memory in, y and the active sets back, every step
         x_pin = torch.from_numpy(x_host_np.view(np.int16)).pin_memory()
@@ -335,7 +361,8 @@ def run_ours(args, w):
                          f"{w.replicas * E * 2 * d * de * 2 / 1e9:.2f} GB of expert weights",
                    "mean_n_active": round(float(n_act_host.mean()), 3),
                    "cls": round(1.0 - float(n_act_host.mean()) / E, 4),
-                   "parallelism": f"dp{world} (chunks sharded, no collective in the data path)"},
+                   "parallelism": f"dp{world} (chunks sharded, no collective in the data path)",
+                   "concurrent_chunks": K},
         "roofline": roofline,
         "e2e": {"value": round(tokens_step / (e2e_max / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host_np.nbytes),
@@ -440,6 +467,8 @@ def main():
     ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")
     ap.add_argument("--replicas", type=int, default=None,
                     help="weight replicas (default: the workload's; keep their weights above the 126 MB L2)")
+    ap.add_argument("--streams", type=int, default=8,
+                    help="decode: independent chunks in flight at once, each on 1/streams of the SMs")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-chunks", type=int, default=1)

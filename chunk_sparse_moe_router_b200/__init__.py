@@ -17,6 +17,12 @@ LIB_PATH = os.path.join(_PKG, "libblockffn.so")
 BFFN_OK, BFFN_EINVAL, BFFN_ECUDA, BFFN_ENOMEM, BFFN_ETIMEOUT, BFFN_EUNSUPPORTED = range(6)
 BFFN_PATH_AUTO, BFFN_PATH_DECODE, BFFN_PATH_PREFILL = 0, 1, 2
 
+
+def BFFN_FLAGS_SHARE(k: int) -> int:
+    """Concurrency hint (decode path): the call takes 1/k of the SMs; k calls on k streams with k
+    workspaces run side by side."""
+    return int(k) << 4
+
 # Every symbol include/blockffn.h declares: name -> (restype, argtypes)
 _P, _I, _S = C.c_void_p, C.c_int, C.c_size_t
 SIGNATURES = {

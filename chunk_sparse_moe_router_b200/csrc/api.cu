@@ -128,7 +128,7 @@ bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* di
 int forward_decode(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                   const DeviceInfo& di, cudaStream_t st) {
+                   const DeviceInfo& di, int share, cudaStream_t st) {
   const WsLayout lay = ws_layout(L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
@@ -162,7 +162,8 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
   dp.E = E;
   dp.de = de;
   DecodeLaunch dl;
-  if (!expert_decode_plan(L, d, E, de, di.num_sms, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
+  const int grid = di.num_sms / share;  // one persistent CTA per SM of this call's share
+  if (grid < 1 || !expert_decode_plan(L, d, E, de, grid, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
 
   TensorMaps tm;
   {
@@ -322,6 +323,8 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   if (workspace != nullptr && !aligned256(workspace)) return BFFN_EINVAL;
   const int path = flags & 3;
   if (path == 3) return BFFN_EINVAL;
+  const int share = ((flags >> 4) & 15) == 0 ? 1 : ((flags >> 4) & 15);
+  if ((flags & ~0xF3) != 0) return BFFN_EINVAL;
   const bool decode = (path == BFFN_PATH_DECODE) || (path == BFFN_PATH_AUTO && L <= kDecodeMaxL);
   if (decode && L > kDecodeMaxL) return BFFN_EUNSUPPORTED;
   if (!decode && L <= kDecodeMaxL) return BFFN_EUNSUPPORTED;  // the prefill path takes L > 32
@@ -343,7 +346,7 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   }
   if (decode)
     return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                          r_out, ws, di, st);
+                          r_out, ws, di, share, st);
   return forward_prefill(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts, r_out,
                          ws, di, st);
 }

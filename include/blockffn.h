@@ -71,6 +71,13 @@ enum {
 /* Path selection for blockffn_chunk_forward_ex's `flags` (low two bits). */
 enum { BFFN_PATH_AUTO = 0, BFFN_PATH_DECODE = 1, BFFN_PATH_PREFILL = 2 };
 
+/* Concurrency hint in `flags` bits 4-7 (decode path): k in 1..15 (0 = 1).  The call's persistent expert
+ * kernel then takes 1/k of the GPU's SMs, so that k calls for independent chunks, issued on k streams
+ * with k different workspaces, run side by side and one chunk's fixed latencies (router, pipeline fill,
+ * the up-projection's grid barrier) overlap another chunk's weight streaming.  At most k such calls may
+ * be in flight at once.  The results do not depend on k. */
+#define BFFN_FLAGS_SHARE(k) ((int)(k) << 4)
+
 /*
  * The layer forward over one chunk, with no router bias.  Uses a per-device workspace that the
  * library allocates on the first call (and grows when a later call needs more); make that first

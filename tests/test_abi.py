@@ -66,7 +66,7 @@ def _call(bffn, **kw):
     dict(active_idx=None), dict(n_active=None),
     dict(x=FAKE + 2), dict(W1=FAKE + 8), dict(W2=FAKE + 4), dict(Wr=FAKE + 4), dict(y=FAKE + 2),
     dict(n_active=FAKE + 1), dict(br=FAKE + 2), dict(r_out=FAKE + 1), dict(workspace=FAKE + 16),
-    dict(flags=3),
+    dict(flags=3), dict(flags=1 << 8), dict(flags=1 << 2),
 ])
 def test_invalid_arguments_rejected_before_launch(bffn, kw):
     assert _call(bffn, **kw) == bffn.BFFN_EINVAL

@@ -113,3 +113,46 @@ def test_caller_workspace_and_repeatability(bffn, cuda_device):
     c = run_chunk(bffn, dl, x)
     assert np.array_equal(a["y"], b["y"]) and np.array_equal(a["y"], c["y"])  # bitwise reproducible
     assert np.array_equal(a["active_idx"], c["active_idx"])
+
+
+@pytest.mark.parametrize("share", [2, 4])
+def test_concurrency_hint_keeps_parity(bffn, cuda_device, share):
+    # flags bits 4-7 = k: the expert kernel takes 1/k of the SMs (a different work split); k calls on
+    # k streams with their own workspaces run side by side, each still exact against the oracle
+    import torch
+    from _parity import assert_parity, bf16_tensor, reference
+    w = gen.workload("decode")
+    from _parity import DeviceLayer
+    dl = DeviceLayer(w.layer(0))
+    xs = w.chunks(dl.lay, share)
+    L, d, E, de = w.L, w.d, w.E, w.de
+    streams = [torch.cuda.Stream() for _ in range(share)]
+    wss = [bffn.new_workspace(L, d, E, de) for _ in range(share)]
+    outs = []
+    torch.cuda.synchronize()
+    for k in range(share):
+        x = bf16_tensor(xs[k])
+        y = torch.full((L, d), float("nan"), dtype=torch.float32, device="cuda")
+        idx = torch.full((E,), -7, dtype=torch.int32, device="cuda")
+        n = torch.full((1,), -7, dtype=torch.int32, device="cuda")
+        mask = torch.zeros((L, (E + 31) // 32), dtype=torch.int32, device="cuda")
+        counts = torch.full((2,), -7, dtype=torch.int32, device="cuda")
+        r = torch.full((L, E), float("nan"), dtype=torch.float32, device="cuda")
+        rc = bffn.blockffn_chunk_forward_ex(x.data_ptr(), L, d, dl.Wr.data_ptr(), dl.g.data_ptr(), dl.W1.data_ptr(),
+                                            dl.W2.data_ptr(), E, de, y.data_ptr(), idx.data_ptr(), n.data_ptr(),
+                                            dl.br.data_ptr(), mask.data_ptr(), counts.data_ptr(), r.data_ptr(),
+                                            bffn.BFFN_FLAGS_SHARE(share), wss[k].data_ptr(), wss[k].numel(),
+                                            streams[k].cuda_stream)
+        assert rc == 0, bffn.blockffn_status_string(rc)
+        outs.append((x, y, idx, n, mask, counts, r))
+    torch.cuda.synchronize()
+    for k in range(share):
+        assert bffn.device_status(workspace=wss[k]) == 0
+        x, y, idx, n, mask, counts, r = outs[k]
+        nn = int(n.item())
+        words = mask.cpu().numpy().view(np.uint32)
+        bits = ((words[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).astype(bool).reshape(L, -1)[:, :E]
+        got = {"y": y.cpu().numpy().astype(np.float64), "active_idx": idx.cpu().numpy()[:nn], "n_active": nn,
+               "active": bits, "counts": tuple(int(v) for v in counts.cpu().numpy()),
+               "r": r.cpu().numpy().astype(np.float64)}
+        assert_parity(got, reference(dl, xs[k]), L, E)
