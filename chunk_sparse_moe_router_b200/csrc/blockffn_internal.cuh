@@ -123,6 +123,7 @@ struct DecodeParams {
   int xbuf_bytes;   // resident x tiles [chunks of a pass][LB][128 B]
   int w1_tail_off;  // offset of the ragged-chunk tile in an up-projection stage (1024-aligned)
   int ustage_bytes; // shared-memory staging of a CTA's up-projection sums (K split only)
+  int ustage_units; // its capacity in units of 8 rows; the epilogue runs once per full block
   int ksplit;       // 1: L <= 8 and one pass: the consumer warps split K inside every up-projection stage
   // down-projection: stages of NEB experts, each a W2 box of RBB rows x KWB 64-column chunks
   int NEB;

@@ -45,6 +45,11 @@ constexpr int GB = NCW * GPW;               // row groups per row-block (x in sm
 constexpr int kMaxSpan = 16;                // experts a CTA's up-projection rows touch (<= E / G + 2)
 constexpr int kXregChunks = 4;              // 64-column chunks of x one warp keeps in registers
 constexpr uint64_t kWaitNs = 2000000000ull;
+// 16-row n groups of a down-projection row block: up to 48 rows (with 8 tokens a row block of W2 then
+// fills a 32 KB stage with the h tiles), 32 for the longer token classes (accumulator registers)
+template <int LC>
+constexpr int kNP2 = LC == 8 ? 3 : 2;
+constexpr int np2_of(int lc) { return lc == 8 ? 3 : 2; }
 
 // ------------------------------------------------------------------------------------- smem
 struct Smem {
@@ -66,7 +71,7 @@ struct Smem {
   float* pre_g;        // [kMaxSpan]
   float* red_s;        // [S][NCW][32][2] per-stage partial sums (K split)
   uint64_t* rbar;      // [S] partial sums of a stage written (NCW arrivals)
-  float* ustage;       // [(rA1 - rA0) / 8][L][8] this CTA's up-projection sums u, until the end of phase A (K split)
+  float* ustage;       // [ustage_units][L][8] up-projection sums u of a block of rows until its epilogue (K split)
 };
 
 __device__ __forceinline__ uint32_t swz(int row, int chunk16) {
@@ -372,6 +377,38 @@ __device__ __forceinline__ void store_h(const DecodeParams& p, const Smem& sm, i
   *reinterpret_cast<__nv_bfloat16*>(himg + swz(p.L + t, col >> 3) + (col & 7) * 2) = lo;
 }
 
+// Epilogue of a block of the CTA's up-projection rows [r0, r1) (multiples of 8): h = r Swish(u) with
+// r = g relu(s) / rms, split into bf16 hi and lo parts and written to the global h image as 16-byte
+// pieces of 8 consecutive j (one expert each: row blocks are multiples of 8 and de of 16).  u of
+// row r0 + i waits in unit i / 8 of the staging buffer.
+__device__ void flush_u(const DecodeParams& p, const Smem& sm, int a_first, int r0, int r1) {
+  const int units = (r1 - r0) >> 3;
+  for (int o = threadIdx.x; o < units * p.L; o += NCW * 32) {
+    const int u = o / p.L, t = o - u * p.L;
+    const int row = r0 + u * 8;
+    const int a = row / p.de, j = row - a * p.de;
+    const float rms = sm.rms[t];
+    const float sv = sm.pre_s[(a - a_first) * 32 + t];
+    const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
+    const float4* us = reinterpret_cast<const float4*>(sm.ustage + (u * p.L + t) * 8);
+    const float4 ua = us[0], ub = us[1];
+    const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float h0 = rr * (uv[2 * k] / (1.f + expf(-uv[2 * k])));
+      const float h1 = rr * (uv[2 * k + 1] / (1.f + expf(-uv[2 * k + 1])));
+      const __nv_bfloat162 hh = __floats2bfloat162_rn(h0, h1);
+      const __nv_bfloat162 ll = __floats2bfloat162_rn(h0 - __low2float(hh), h1 - __high2float(hh));
+      hi[k] = *reinterpret_cast<const uint32_t*>(&hh);
+      lo[k] = *reinterpret_cast<const uint32_t*>(&ll);
+    }
+    uint8_t* img = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
+    *reinterpret_cast<uint4*>(img + swz(t, (j & 63) >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(img + swz(p.L + t, (j & 63) >> 3)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+}
+
 // Up-projection split over K (L <= 8, one pass): every consumer warp works on every stage over its
 // own 64-column chunks c = cw + NCW q, writes its partial sums, and the stage's designated warp adds
 // the NCW partials in warp order, finishes the group and frees the slot.  The x fragments of the
@@ -405,6 +442,8 @@ __device__ void phase_a_ksplit(const DecodeParams& p, const Smem& sm, const Work
       ldmatrix_x2(ad, xf[q][k16][0], xf[q][k16][1]);
     }
   }
+  const int blk_rows = p.ustage_units * 8;  // rows whose u fit the staging buffer
+  int blk0 = w.rA0;
   for (int r = w.rA0; r < w.rA1; r += h, rp.next(p.S)) {
     const int slot = rp.slot;
     if (ring_wait(p, sm, &sm.fullW[slot], rp.ph, 3)) {
@@ -469,39 +508,16 @@ __device__ void phase_a_ksplit(const DecodeParams& p, const Smem& sm, const Work
       // the slot and its partial sums are free once read; u waits in shared memory for the epilogue
       __syncwarp();
       if (lane == 0) mbar_arrive_cnt(&sm.empty[slot], NCW);
-      const int t = gid, loc = r - w.rA0 + tig * 2;  // rows loc, loc + 1 of the CTA (loc even)
+      const int t = gid, loc = r - blk0 + tig * 2;  // rows loc, loc + 1 of the block (loc even)
       if (ok && t < p.L && tig * 2 < h)
         *reinterpret_cast<float2*>(sm.ustage + ((loc >> 3) * p.L + t) * 8 + (loc & 7)) = make_float2(u0, u1);
     }
-  }
-  // Epilogue, once per CTA: h = r Swish(u) with r = g relu(s) / rms, split into bf16 hi and lo parts and
-  // written to the global h image as 16-byte pieces of 8 consecutive j (one expert each: the CTA's
-  // rows are whole multiples of 8 and de is a multiple of 16).
-  named_bar_sync(1, NCW * 32);
-  const int units = (w.rA1 - w.rA0) >> 3;
-  for (int o = threadIdx.x; o < units * p.L; o += NCW * 32) {
-    const int u = o / p.L, t = o - u * p.L;
-    const int row = w.rA0 + u * 8;
-    const int a = row / p.de, j = row - a * p.de;
-    const float rms = sm.rms[t];
-    const float sv = sm.pre_s[(a - a_first) * 32 + t];
-    const float rr = (rms > 0.f) ? (sm.pre_g[a - a_first] * fmaxf(sv, 0.f)) / rms : 0.f;
-    const float4* us = reinterpret_cast<const float4*>(sm.ustage + (u * p.L + t) * 8);
-    const float4 ua = us[0], ub = us[1];
-    const float uv[8] = {ua.x, ua.y, ua.z, ua.w, ub.x, ub.y, ub.z, ub.w};
-    uint32_t hi[4], lo[4];
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const float h0 = rr * (uv[2 * k] / (1.f + expf(-uv[2 * k])));
-      const float h1 = rr * (uv[2 * k + 1] / (1.f + expf(-uv[2 * k + 1])));
-      const __nv_bfloat162 hh = __floats2bfloat162_rn(h0, h1);
-      const __nv_bfloat162 ll = __floats2bfloat162_rn(h0 - __low2float(hh), h1 - __high2float(hh));
-      hi[k] = *reinterpret_cast<const uint32_t*>(&hh);
-      lo[k] = *reinterpret_cast<const uint32_t*>(&ll);
+    if (r + h - blk0 == blk_rows || r + h >= w.rA1) {  // the block is full, or the CTA's rows end
+      named_bar_sync(1, NCW * 32);  // every u of the block is staged
+      flush_u(p, sm, a_first, blk0, r + h);
+      named_bar_sync(1, NCW * 32);  // the staging buffer is free for the next block
+      blk0 = r + h;
     }
-    uint8_t* img = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
-    *reinterpret_cast<uint4*>(img + swz(t, (j & 63) >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    *reinterpret_cast<uint4*>(img + swz(p.L + t, (j & 63) >> 3)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
   }
 }
 
@@ -663,9 +679,10 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
   // they are computed once; a k-step outside the stage, or an operand row outside the tile, reads the
   // zero row, and loads and MMAs run unconditionally (zero fragments add nothing).
   constexpr int kKS = 4;
-  constexpr int KB = MT == 4 ? 2 : 4;  // k-steps per batch: all loads of a batch, then its MMAs
-  constexpr int NSET = MT == 4 ? 1 : 2;
-  int ks_qe[kKS], ks_c[kKS], offA[kKS][MT], offB[kKS][2];
+  constexpr int KB = MT == 1 ? 4 : 2;  // k-steps per batch: all loads of a batch, then its MMAs
+  constexpr int NP2 = kNP2<LC>;        // 16-row n groups of a row block (RBB <= 16 NP2)
+  constexpr int NSET = 1;
+  int ks_qe[kKS], ks_c[kKS], offA[kKS][MT], offB[kKS][NP2];
 #pragma unroll
   for (int b = 0; b < kKS; ++b) {
     const int g = cw + NCW * b;
@@ -679,20 +696,20 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
       offA[b][mt] = row < p.HR ? qe * p.eB + p.hoff + c * p.HR * 128 + int(swz(row, k16 * 2 + (lane >> 4))) : -1;
     }
 #pragma unroll
-    for (int np2 = 0; np2 < 2; ++np2) {
+    for (int np2 = 0; np2 < NP2; ++np2) {
       const int row = np2 * 16 + (lane & 7) + (lane >> 4) * 8;
       offB[b][np2] = row < p.RBB ? qe * p.eB + int(swz(c * p.RBB + row, k16 * 2 + ((lane >> 3) & 1))) : -1;
     }
   }
   uint32_t hphase = 0;
   for (int rb = 0; rb < w.nRBB; ++rb) {
-    float acc[NSET][MT][4][4];
+    float acc[NSET][MT][2 * NP2][4];
 #pragma unroll
     for (int e = 0; e < NSET; ++e)
 #pragma unroll
       for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < 2 * NP2; ++b)
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[e][a][b][c] = 0.f;
     int eg = 0, js = 0;
@@ -707,7 +724,7 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
         const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
 #pragma unroll
         for (int b0 = 0; b0 < kKS; b0 += KB) {
-          uint32_t af[KB][MT][4], bf[KB][2][4];
+          uint32_t af[KB][MT][4], bf[KB][NP2][4];
 #pragma unroll
           for (int b = 0; b < KB; ++b) {
             const bool in = ks_qe[b0 + b] < nq && ks_c[b0 + b] < nc;
@@ -718,7 +735,7 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
                           af[b][mt][3]);
             }
 #pragma unroll
-            for (int np2 = 0; np2 < 2; ++np2) {
+            for (int np2 = 0; np2 < NP2; ++np2) {
               const int o = offB[b0 + b][np2];
               ldmatrix_x4(in && o >= 0 ? sb + uint32_t(o) : zaddr, bf[b][np2][0], bf[b][np2][1], bf[b][np2][2],
                           bf[b][np2][3]);
@@ -727,7 +744,7 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
 #pragma unroll
           for (int b = 0; b < KB; ++b)
 #pragma unroll
-            for (int np2 = 0; np2 < 2; ++np2)
+            for (int np2 = 0; np2 < NP2; ++np2)
 #pragma unroll
               for (int mt = 0; mt < MT; ++mt) {
                 mma_bf16_16816(acc[b % NSET][mt][np2 * 2], af[b][mt], bf[b][np2][0], bf[b][np2][1]);
@@ -744,15 +761,16 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
 #pragma unroll
       for (int a = 0; a < MT; ++a)
 #pragma unroll
-        for (int b = 0; b < 4; ++b)
+        for (int b = 0; b < 2 * NP2; ++b)
 #pragma unroll
           for (int c = 0; c < 4; ++c) acc[0][a][b][c] += acc[e][a][b][c];
     // sum the warps' partials in a fixed order; y = (hi part) + (lo part)
+    constexpr int NT8 = 2 * NP2;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-      for (int nt = 0; nt < 4; ++nt)
-        *reinterpret_cast<float4*>(sm.red + ((((cw * MT + mt) * 4 + nt) * 32 + lane) * 4)) =
+      for (int nt = 0; nt < NT8; ++nt)
+        *reinterpret_cast<float4*>(sm.red + ((((cw * MT + mt) * NT8 + nt) * 32 + lane) * 4)) =
             make_float4(acc[0][mt][nt][0], acc[0][mt][nt][1], acc[0][mt][nt][2], acc[0][mt][nt][3]);
     named_bar_sync(1, NCW * 32);
     const int k0 = w.rB0 + rb * p.RBB, nrows = min(p.RBB, w.nB - rb * p.RBB);
@@ -766,7 +784,7 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
         const int reg = (r16 >> 3) * 2 + (c & 1);
         const int nt = c >> 3;
 #pragma unroll
-        for (int ww = 0; ww < NCW; ++ww) v += sm.red[((((ww * MT + mt) * 4 + nt) * 32 + ln) * 4) + reg];
+        for (int ww = 0; ww < NCW; ++ww) v += sm.red[((((ww * MT + mt) * NT8 + nt) * 32 + ln) * 4) + reg];
       }
       p.y[size_t(t) * p.d + k0 + c] = v;
     }
@@ -866,7 +884,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     expert_decode_kernel(const __grid_constant__ DecodeParams p, const __grid_constant__ TensorMaps tm) {
   extern __shared__ uint8_t smem_raw[];
   constexpr int MT = (2 * LC + 15) / 16;
-  constexpr int kRedBytes = NCW * MT * 4 * 32 * 4 * 4;
+  constexpr int kRedBytes = NCW * MT * 2 * kNP2<LC> * 32 * 4 * 4;
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem sm;
   sm.xbuf = base;
@@ -1003,14 +1021,17 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   p->nJf = de / 64;
   p->h_expert_bytes = p->nJc * p->HR * 128;
   const int rbmax = (d + G - 1) / G;
-  p->RBB = round_up(rbmax < 1 ? 1 : (rbmax > 32 ? 32 : rbmax), 8);
+  const int rbb_cap = 16 * np2_of(lc);
+  p->RBB = round_up(rbmax < 1 ? 1 : (rbmax > rbb_cap ? rbb_cap : rbmax), 8);
   auto part_bytes = [&](int kwb) {
     const int w2 = p->RBB * kwb * 128;  // multiple of 1024
     return round_up(w2 + round_up(p->HR * kwb * 128, 16), 1024);
   };
   p->KWB = p->nJc;
   if (p->nJf >= 1 && p->KWB > p->nJf) p->KWB = p->nJf;
-  while (p->KWB > 1 && part_bytes(p->KWB) > (slotA > 8192 ? slotA : 8192)) --p->KWB;
+  const int slot_cap = slotA > 8192 ? slotA : 8192;
+  while (p->RBB > 32 && part_bytes(p->KWB) > slot_cap) p->RBB -= 8;  // keep the stage at the A size
+  while (p->KWB > 1 && part_bytes(p->KWB) > slot_cap) --p->KWB;
   p->hoff = p->RBB * p->KWB * 128;
   p->eB = part_bytes(p->KWB);
   const int slot = round_up(slotA > p->eB ? slotA : p->eB, 1024);
@@ -1018,12 +1039,17 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   if (p->NEB < 1) p->NEB = 1;
   while (p->NEB > 1 && p->NEB * p->KWB > 8) --p->NEB;  // a stage has at most 32 k-steps of 16 j
   p->slot_bytes = slot;
-  const size_t red = size_t(NCW) * mt * 4 * 32 * 4 * 4;
+  const size_t red = size_t(NCW) * mt * 2 * np2_of(lc) * 32 * 4 * 4;
   const size_t red_extra = size_t(p->xbuf_bytes) >= red ? 0 : red;
   const size_t tail = 32 + 3 * 8 * 32 + 16 + size_t(kMaxE + 4) * 4 + 32 * 4 + 32 * 32 * 4 + (kMaxSpan * 33) * 4 + 16;
   const size_t per_slot = (p->ksplit ? size_t(NCW) * 32 * 2 * 4 : 0) + 16;  // red_s and rbar of one slot
-  // staged u of one CTA: at most ceil(E de / 8 / G) units of 8 rows, L tokens x 8 floats each
-  p->ustage_bytes = p->ksplit ? int((size_t(E) * de / 8 + G - 1) / G) * L * 32 : 0;
+  // staged u: blocks of ustage_units units of 8 rows, L tokens x 8 floats each
+  {
+    const int worst = int((size_t(E) * de / 8 + G - 1) / G);  // units of 8 rows a CTA may get
+    const int cap = 8192 / (L * 32) > 0 ? 8192 / (L * 32) : 1;   // about 8 KB of staging
+    p->ustage_units = p->ksplit ? (worst < cap ? worst : cap) : 0;
+    p->ustage_bytes = p->ustage_units * L * 32;
+  }
   const size_t fixed = 1024 + size_t(p->xbuf_bytes) + red_extra + tail + size_t(p->ustage_bytes);
   if (fixed >= size_t(max_smem)) return false;
   int S = int((size_t(max_smem) - fixed) / (size_t(p->slot_bytes) + per_slot));
