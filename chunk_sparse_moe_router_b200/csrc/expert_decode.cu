@@ -198,6 +198,7 @@ struct RingPos {
 
 // ------------------------------------------------------------------------------------- producers
 // Weight producer (one warp): W1 row groups, then W2 expert tiles, in stage order.
+template <bool KSPLIT>
 __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_w = policy_evict_first();
@@ -206,6 +207,28 @@ __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, con
   // ---- phase A: stage = one box of a group's whole rows over the pass's columns
   const int KC = p.nKf / p.KP;                 // full chunks per pass
   const bool tail = p.nKc > p.nKf;             // only with one pass
+  if constexpr (KSPLIT) {
+    // one pass, and every group is RSM adjacent rows of one expert (the CTA's rows are whole multiples
+    // of 8): stage s holds rows [rA0 + s RSM, + RSM)
+    const int h = p.RSM, hsel = __ffs(h) - 1;
+    for (int r = w.rA0; r < w.rA1; r += h, rp.next(p.S)) {
+      if (aborted(sm)) { ok = false; break; }
+      const int slot = rp.slot;
+      if (rp.i >= p.S && !mbar_wait_bounded(&sm.empty[slot], rp.ph ^ 1u, kWaitNs)) {
+        if (lane == 0) set_error(p, sm, kErrRingWait, 1);
+        ok = false;
+        break;
+      }
+      if (lane == 0) {
+        const int a = r / p.de, j0 = r - a * p.de, e = sm.act[a];
+        uint8_t* dst = sm.ring + size_t(slot) * p.slot_bytes;
+        mbar_arrive_expect_tx(&sm.fullW[slot], uint32_t(KC + (tail ? 1 : 0)) * h * 128);
+        if (KC > 0) tma_load_4d(dst, &tm.w1_ch[hsel], 0, j0, 0, e, &sm.fullW[slot], pol_w);
+        if (tail) tma_load_3d(dst + p.w1_tail_off, &tm.w1_3d[hsel], p.nKf * 64, j0, e, &sm.fullW[slot], pol_w);
+      }
+      __syncwarp();
+    }
+  } else
   for (int r = w.rA0; r < w.rA1 && ok;) {
     int ngr;
     const int r_next = rowblock_walk(p, r, w.rA1, &ngr);
@@ -273,6 +296,7 @@ __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, con
 
 // x / h producer (one warp): the resident x parts of phase A, then (after the grid barrier) the h
 // tiles of phase B.
+template <bool KSPLIT>
 __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
   const int lane = threadIdx.x & 31;
   const uint64_t pol_x = policy_evict_last();
@@ -280,9 +304,13 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
   const int KC = p.nKf / p.KP;
   const bool tail = p.nKc > p.nKf;
   int nrb = 0;
-  for (int r = w.rA0; r < w.rA1; ++nrb) {
-    int ngr;
-    r = rowblock_walk(p, r, w.rA1, &ngr);
+  if constexpr (KSPLIT) {
+    nrb = w.rA0 < w.rA1 ? 1 : 0;  // one pass: x is loaded once
+  } else {
+    for (int r = w.rA0; r < w.rA1; ++nrb) {
+      int ngr;
+      r = rowblock_walk(p, r, w.rA1, &ngr);
+    }
   }
   int xloads = 0;
   const int nparts = (p.KP > 1) ? nrb * p.KP : (nrb > 0 ? 1 : 0);
@@ -305,7 +333,11 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
 
   // ---- h tiles after the grid barrier
   int nG = 0;
-  for (int r = w.rA0; r < w.rA1; ++nG) r += group_at(p, r, w.rA1).h;
+  if constexpr (KSPLIT) {
+    nG = (w.rA1 - w.rA0) / p.RSM;
+  } else {
+    for (int r = w.rA0; r < w.rA1; ++nG) r += group_at(p, r, w.rA1).h;
+  }
   const int stagesA = p.KP * nG;
   const int stagesB = w.nRBB * w.nEg * w.nJs;
   if (stagesB == 0) return;
@@ -410,8 +442,8 @@ __device__ void flush_u(const DecodeParams& p, const Smem& sm, int a_first, int 
 }
 
 // Up-projection split over K (L <= 8, one pass): every consumer warp works on every stage over its
-// own 64-column chunks c = cw + NCW q, writes its partial sums, and the stage's designated warp adds
-// the NCW partials in warp order, finishes the group and frees the slot.  The x fragments of the
+// own 64-column chunks c = cw + NCW q and writes its partial sums; then each warp adds the NCW
+// partials of one token in warp order and frees the slot.  The x fragments of the
 // first kXregChunks chunks of a warp stay in registers; further chunks read them from shared memory.
 // Only tokens 0-7 are real rows of the MMA (rows 8-15 are zero).  Every group has RSM rows (the CTA's
 // rows are whole multiples of 8 and RSM <= 8), so a warp's operand offsets inside a stage are the
@@ -493,23 +525,27 @@ __device__ void phase_a_ksplit(const DecodeParams& p, const Smem& sm, const Work
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.rbar[slot]);
-    if ((rp.i % NCW) == cw) {  // this warp finishes the stage
+    // Every warp finishes one token of the stage: the MMA fragment's lanes 4 cw .. 4 cw + 3 hold token
+    // cw (rows 2 (lane & 3) and + 1), so lanes 0-3 of warp cw add the NCW partial sums of those lanes in
+    // warp order.  All warps run this every stage, then release the slot (NCW arrivals).
+    {
       const bool ok = ring_wait(p, sm, &sm.rbar[slot], rp.ph, 9);
       float u0 = 0.f, u1 = 0.f;
-      if (ok) {
+      const int src = cw * 4 + (lane & 3);
+      if (ok && lane < 4) {
         const float2* red = reinterpret_cast<const float2*>(sm.red_s) + size_t(slot) * NCW * 32;
 #pragma unroll
         for (int ww = 0; ww < NCW; ++ww) {
-          const float2 v = red[ww * 32 + lane];
+          const float2 v = red[ww * 32 + src];
           u0 += v.x;
           u1 += v.y;
         }
       }
       // the slot and its partial sums are free once read; u waits in shared memory for the epilogue
       __syncwarp();
-      if (lane == 0) mbar_arrive_cnt(&sm.empty[slot], NCW);
-      const int t = gid, loc = r - blk0 + tig * 2;  // rows loc, loc + 1 of the block (loc even)
-      if (ok && t < p.L && tig * 2 < h)
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);
+      const int t = cw, loc = r - blk0 + lane * 2;  // rows loc, loc + 1 of the block (loc even)
+      if (ok && lane < 4 && t < p.L && lane * 2 < h)
         *reinterpret_cast<float2*>(sm.ustage + ((loc >> 3) * p.L + t) * 8 + (loc & 7)) = make_float2(u0, u1);
     }
     if (r + h - blk0 == blk_rows || r + h >= w.rA1) {  // the block is full, or the CTA's rows end
@@ -947,9 +983,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp < NCW) {
     consume<LC, KSPLIT>(p, sm, w);
   } else if (warp == NCW) {
-    produce_weights(p, tm, sm, w);
+    produce_weights<KSPLIT>(p, tm, sm, w);
   } else {
-    produce_x_h(p, tm, sm, w);
+    produce_x_h<KSPLIT>(p, tm, sm, w);
   }
   if (blockIdx.x == 0 && p.r_out) {
     __syncthreads();
