@@ -1,10 +1,11 @@
 """Benchmark of the BlockFFN chunk-layer forward on B200.
 
 One step = one pass of the hot path over one batch of synthetic input: `chunks` chunk forwards
-(router + chunk union + sparse experts, two kernels per chunk) through the C ABI, chunk c using
-weight replica c % replicas.  The chunks are independent: chunk c is issued on stream c % K (--streams,
-default 8) with its own workspace and the concurrency hint, so K chunks run side by side, each on
-1/K of the SMs, and one chunk's fixed latencies overlap the others' weight streaming.  The replicas stand for distinct layers of a stacked model and keep
+(router + chunk union + sparse experts: one kernel per decode chunk, seven per prefill chunk) through
+the C ABI, chunk c using weight replica c % replicas.  The chunks are independent: chunk c is issued
+on stream c % K (--streams, default 8) with its own workspace and the concurrency hint, so K chunks
+run side by side, each on 1/K of the SMs, and one chunk's fixed latencies overlap the others' weight
+streaming.  The replicas stand for distinct layers of a stacked model and keep
 the weights (16 x 128 MiB for the default workload) well above the 126 MB L2, so every chunk streams
 its active experts from HBM ("inputs larger than L2").  A step is captured once into a CUDA graph
 and replayed; time is taken with CUDA events on the replay stream, with a barrier and a
@@ -347,7 +348,7 @@ def run_ours(args, w):
     else:
         roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
                     "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind,
-                    "kernel": "one chunk forward (router kernel + expert kernel, PDL-chained)",
+                    "kernel": "expert_decode_kernel: one chunk forward, router included",
                     "bytes_per_chunk": round(total_active / chunks, 1),
                     "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3),
                     "traffic": None if traffic is None else round(traffic, 1)}
@@ -368,7 +369,7 @@ def run_ours(args, w):
                 "h2d_bytes_per_step": int(x_host_np.nbytes),
                 "d2h_bytes_per_step": int(y.numel() * 4 + idx.numel() * 4 + nact.numel() * 4),
                 "steps": e2e_steps},
-        "gpu_launches": (6 if prefill else 2) * chunks * args.steps,
+        "gpu_launches": (7 if prefill else 1) * chunks * args.steps,
         "clocks": clk.summary(),
         "gen_seconds": round(gen_s, 1),
     }

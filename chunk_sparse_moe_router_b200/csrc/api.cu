@@ -133,21 +133,11 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
 
-  RouterParams rp;
-  rp.x = static_cast<const __nv_bfloat16*>(x);
-  rp.Wr = Wr;
-  rp.br = br;
-  rp.L = L;
-  rp.d = d;
-  rp.E = E;
-  rp.s_ws = reinterpret_cast<float*>(base + lay.s_off);
-  rp.hdr = hdr;
-  RouterLaunch rl;
-  if (!router_decode_plan(L, d, E, di.max_smem, &rl)) return BFFN_EUNSUPPORTED;
-  rp.xt = rl.xt;
-
   DecodeParams dp;
-  dp.s = rp.s_ws;
+  dp.x = static_cast<const __nv_bfloat16*>(x);
+  dp.Wr = Wr;
+  dp.br = br;
+  dp.s_part = reinterpret_cast<float*>(base + lay.s_off);
   dp.g = g;
   dp.y = y;
   dp.active_idx = active_idx;
@@ -205,9 +195,7 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
     }
   }
 
-  cudaError_t err = router_decode_launch(rp, rl, st, di.pdl);
-  if (err != cudaSuccess) return cuda_fail(err);
-  err = expert_decode_launch(dp, tm, dl, st, di.pdl);
+  const cudaError_t err = expert_decode_launch(dp, tm, dl, st, di.pdl);
   if (err != cudaSuccess) return cuda_fail(err);
   return BFFN_OK;
 }

@@ -17,15 +17,18 @@ enum : uint32_t {
   kErrGridBarrier = 1u,   // expert kernel: waiting for every CTA to finish the up-projection
   kErrRingWait = 2u,      // expert kernel: waiting on a shared-memory ring barrier
   kErrPrefillWait = 4u,   // prefill GEMMs: waiting on a shared-memory barrier
+  kErrRouterBarrier = 8u, // expert kernel: waiting for every CTA's router partial sums
 };
 
 // First 256 bytes of every workspace.
 struct alignas(256) WsHeader {
   uint32_t ticket;     // reserved
-  uint32_t grid_bar;   // expert kernel: CTAs past the up-projection (reset by the router, per call)
+  uint32_t grid_bar;   // expert kernel: CTAs past the up-projection
   uint32_t err;        // error bits, cleared by blockffn_device_status
   uint32_t err_info;
-  uint32_t pad[60];
+  uint32_t router_bar; // expert kernel: CTAs whose router partial sums are written
+  uint32_t exit_ctr;   // expert kernel: CTAs done; the last one sets the three counters back to 0
+  uint32_t pad[58];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
 
@@ -61,45 +64,36 @@ inline PrefillLayout prefill_layout(size_t start, int L, int E, int de) {
   return p;
 }
 
+// Decode router split: d is cut into parts of R rows (a multiple of 8, at most 256); the expert
+// kernel's CTAs write one fp32 partial projection [L,E] per part and add the parts in part order.
+// Both numbers depend on d only, so the order of every sum does too.
+inline int decode_router_rows(int d) {
+  const int q0 = (d + 255) / 256;
+  return (((d + q0 - 1) / q0) + 7) & ~7;
+}
+inline int decode_router_parts(int d) { return (d + decode_router_rows(d) - 1) / decode_router_rows(d); }
+
 struct WsLayout {
   size_t s_off, h_off, total;
 };
 
-// Workspace: header | s fp32 [L,E] (router projection) | decode h (L <= 32) or the prefill regions
+// Workspace: header | router projection (decode: per-part partials [parts][L,E]; prefill: s [L,E]) |
+// decode h (L <= 32) or the prefill regions
 inline WsLayout ws_layout(int L, int d, int E, int de) {
-  (void)d;
   WsLayout w;
+  const size_t parts = L <= kDecodeMaxL ? size_t(decode_router_parts(d)) : 1;
   w.s_off = sizeof(WsHeader);
-  w.h_off = w.s_off + align256(size_t(L) * E * sizeof(float));
+  w.h_off = w.s_off + align256(parts * size_t(L) * E * sizeof(float));
   w.total = L <= kDecodeMaxL ? w.h_off + align256(decode_h_bytes(L, E, de)) : prefill_layout(w.h_off, L, E, de).end;
   return w;
 }
 
-// ------------------------------------------------------------------------------------ router
-struct RouterParams {
-  const __nv_bfloat16* x;   // [L,d]
-  const float* Wr;          // [d,E]
-  const float* br;          // [E] or null
-  int L, d, E;
-  int xt;                   // Wr rows per cluster rank (multiple of 8)
-  float* s_ws;              // [L,E] out
-  WsHeader* hdr;
-};
-
-struct RouterLaunch {
-  int cluster;      // CTAs per cluster (split of d)
-  int grid;         // clusters (32 router columns each)
-  int xt;           // d rows per CTA
-  int lt;           // tokens rounded up to 8, 16 or 32 (accumulators per thread)
-  size_t smem;
-};
-
-bool router_decode_plan(int L, int d, int E, int max_smem, RouterLaunch* out);
-cudaError_t router_decode_launch(const RouterParams& p, const RouterLaunch& plan, cudaStream_t st, bool pdl);
-
 // ------------------------------------------------------------------------------------ experts
 struct DecodeParams {
-  const float* s;             // [L,E] router projection (workspace)
+  const __nv_bfloat16* x;     // [L,d]
+  const float* Wr;            // [d,E]
+  const float* br;            // [E] or null
+  float* s_part;              // [rq][L,E] router partial projections (workspace)
   const float* g;             // [E]
   float* y;                   // [L,d]
   int32_t* active_idx;        // [E]
@@ -134,7 +128,12 @@ struct DecodeParams {
   int h_expert_bytes;
   int eB;           // bytes of one expert's part of a down-projection stage (W2 tile, then h tile)
   int hoff;         // offset of the h tile within that part
-  int sbuf_floats;  // floats of the ring the prologue may use to stage s
+  // router: units of (part of rrows rows of d, block of 32 experts), unit u on CTA u mod G
+  int rq;           // parts of d
+  int rrows;        // rows per part (multiple of 8, <= 256)
+  int rcb;          // blocks of 32 experts
+  int pre_bytes;    // shared memory before the phase-B partials and the barriers: x, the ring, and room
+                    // for the router's staging and the chunk's s [L,E]
 };
 
 // Tensor maps (128-byte swizzle, out-of-bounds elements read as zero).  The chunked views put the

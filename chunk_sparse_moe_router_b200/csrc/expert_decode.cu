@@ -1,10 +1,17 @@
-// Sparse expert kernel of the BlockFFN chunk layer for decode-sized chunks (L <= 32).
+// Sparse expert kernel of the BlockFFN chunk layer for decode-sized chunks (L <= 32): one launch
+// per chunk, router included.
 //
-// Prologue (every CTA, from the router projection s in L2): ReLU and RMSNorm statistics per token
-// (one warp per token, shuffle reduction), the per-token active masks with __ballot_sync, and the
-// chunk's union of active experts as an ascending list built with __popc and a warp scan
-// (lsdiaocha.cn BlockFFN article, sections 2 and 4).  CTA 0 also writes the active list, n_active, the
-// sparsity counts and the optional masks / router outputs.
+// Router (lsdiaocha.cn BlockFFN article, section 2: the router's linear map s = x Wr + b, before its
+// ReLU and RMSNorm): d is cut into parts of at most 256 rows and E into blocks of 32 experts; each
+// (part, block) unit runs on one CTA, which stages its Wr rows (copied before the dependent-launch
+// wait: weights never depend on the previous kernel in the stream) and its x columns in shared
+// memory and writes a partial projection.  After a grid-wide barrier (bounded wait) every CTA adds
+// the parts in part order.  The split depends on d only, so s is the same bits for every grid size.
+//
+// Prologue (every CTA): ReLU and RMSNorm statistics per token (one warp per token, shuffle
+// reduction), the per-token active masks with __ballot_sync, and the chunk's union of active experts
+// as an ascending list built with __popc and a warp scan (article, sections 2 and 4).  CTA 0 also
+// writes the active list, n_active, the sparsity counts and the optional masks / router outputs.
 //
 // Body: the union is evaluated for all L tokens as one batch, outer loop over active experts and
 // inner batched product (article, section 7); each (token, expert) term is weighted by the router
@@ -17,7 +24,7 @@
 //    W1 rows (a CTA's rows of one expert are one contiguous block), the down-projection whole
 //    blocks of consecutive W2 rows; copies are TMA bulk copies / tensor boxes of several KB issued
 //    from several lanes into a ring of shared-memory stages guarded by mbarriers;
-//  * 4 consumer warps run mma.sync m16n8k16 (bf16 in, fp32 accumulate) with tokens as M and weight
+//  * 8 consumer warps run mma.sync m16n8k16 (bf16 in, fp32 accumulate) with tokens as M and weight
 //    rows as N, reading operands with conflict-free ldmatrix (padded rows / 128-byte swizzle).
 //
 // Phase A (up-projection): the CTA owns rows [rA0, rA1) of the flattened (active expert, j) space,
@@ -674,24 +681,7 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
   const uint32_t zaddr = smem_u32(sm.zero);
   RingPos rp;
 
-  // s and g of every expert this CTA's up-projection rows touch
-  const int a_first = w.rA0 / p.de;
-  if (w.rA0 < w.rA1) {
-    const int a_last = (w.rA1 - 1) / p.de;
-    for (int o = ctid; o < (a_last - a_first + 1) * p.L; o += NCW * 32) {
-      const int aa = o / p.L, t = o - aa * p.L;
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_s + aa * 32 + t)),
-                   "l"(p.s + size_t(t) * p.E + sm.act[a_first + aa])
-                   : "memory");
-    }
-    for (int aa = ctid; aa <= a_last - a_first; aa += NCW * 32)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sm.pre_g + aa)),
-                   "l"(p.g + sm.act[a_first + aa])
-                   : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  named_bar_sync(1, NCW * 32);
+  const int a_first = w.rA0 / p.de;  // pre_s / pre_g hold s and g of experts a_first ..
 
   // ---------------- phase A
   if constexpr (KSPLIT) {
@@ -828,38 +818,162 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
   }
 }
 
-// ------------------------------------------------------------------------------------- prologue
-// Per token: RMS of relu(s) over the E experts and the active bits; then the union (ascending).
-__device__ void prologue_router_stats(const DecodeParams& p, const Smem& sm, float* sbuf) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nW = (p.E + 31) >> 5;
-  const int tg = p.sbuf_floats / p.E;  // tokens per staging group (>= 1)
-  for (int t0 = 0; t0 < p.L; t0 += tg) {
-    const int nt = min(tg, p.L - t0);
-    for (int o = tid; o < nt * p.E; o += kThreads)
-      asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(sbuf + o)),
-                   "l"(p.s + size_t(t0) * p.E + o)
-                   : "memory");
-    asm volatile("cp.async.commit_group;" ::: "memory");
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
-    for (int tt = warp; tt < nt; tt += kThreads / 32) {
-      const float* st = sbuf + size_t(tt) * p.E;
-      float sumsq = 0.f;
-      for (int ww = 0; ww < nW; ++ww) {
-        const int e = ww * 32 + lane;
-        const float sv = e < p.E ? st[e] : -1.f;
-        const float a = fmaxf(sv, 0.f);
-        sumsq = fmaf(a, a, sumsq);
-        const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
-        if (lane == 0) sm.maskw[(t0 + tt) * 32 + ww] = bits;
-      }
+// --------------------------------------------------------------------------------------- router
+// Unit u = (part q = u / rcb, expert block cb = u % rcb): rows [q rrows, + rrows) of d, experts
+// [32 cb, + 32).  Staging at the start of the dynamic shared memory (RouterStage): g and b [E] (copied
+// before the dependent-launch wait with this CTA's first Wr rows), Wr rows [rrows][32] fp32, x columns
+// [L][rrows] converted to fp32, warp sums [warps][8][32] fp32.
+constexpr int kRouterWarps = kThreads / 32;
+
+struct RouterStage {
+  float* g;
+  float* b;
+  float* W;
+  float* X;
+  float* wsum;
+};
+
+__device__ __forceinline__ RouterStage router_stage(const DecodeParams& p, uint8_t* base) {
+  RouterStage r;
+  const int E4 = (p.E + 3) & ~3;
+  r.g = reinterpret_cast<float*>(base);
+  r.b = r.g + E4;
+  r.W = r.b + E4;
+  r.X = r.W + size_t(p.rrows) * 32;
+  r.wsum = r.X + size_t(p.L) * p.rrows;
+  return r;
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+__device__ void router_copy_w(const DecodeParams& p, float* Ws, int u) {
+  const int cb = u % p.rcb, q = u / p.rcb;
+  const int k0 = q * p.rrows, nk = min(p.d - k0, p.rrows);
+  const int e0 = cb * 32, Ec = min(32, p.E - e0);
+  if ((p.E & 3) == 0) {  // Ec is then a multiple of 4 too
+    for (int o = threadIdx.x; o < nk * 8; o += kThreads) {
+      const int kk = o >> 3, c4 = (o & 7) * 4;
+      float* dst = Ws + kk * 32 + c4;
+      if (c4 < Ec)
+        cp_async16(dst, p.Wr + size_t(k0 + kk) * p.E + e0 + c4);
+      else
+        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  } else {
+    for (int o = threadIdx.x; o < nk * 32; o += kThreads) {
+      const int kk = o >> 5, c = o & 31;
+      if (c < Ec)
+        cp_async4(Ws + kk * 32 + c, p.Wr + size_t(k0 + kk) * p.E + e0 + c);
+      else
+        Ws[kk * 32 + c] = 0.f;
+    }
+  }
+}
+
+// x columns of unit u, bf16 -> fp32 (exact)
+__device__ void router_load_x(const DecodeParams& p, float* Xs, int u) {
+  const int k0 = (u / p.rcb) * p.rrows, nk = min(p.d - k0, p.rrows);
+  const int q8 = nk >> 3;  // k0 and nk are multiples of 8
+  for (int o = threadIdx.x; o < p.L * q8; o += kThreads) {
+    const int t = o / q8, c8 = (o - t * q8) * 8;
+    const uint4 v = *reinterpret_cast<const uint4*>(p.x + size_t(t) * p.d + k0 + c8);
+    float4* dst = reinterpret_cast<float4*>(Xs + size_t(t) * p.rrows + c8);
+    dst[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    dst[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
+                         __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+  }
+}
+
+// Partial projection of unit u from the staged operands.  Warp w takes rows [w R4, w R4 + R4) of the
+// part (R4 = rrows / warps rounded up to 4), lane = expert column, 8 tokens at a time; each sum runs
+// over its rows in increasing order, then the CTA adds the warps' sums in warp order.
+__device__ void router_unit(const DecodeParams& p, const RouterStage& rs, int u) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int cb = u % p.rcb, q = u / p.rcb;
+  const int k0 = q * p.rrows, nk = min(p.d - k0, p.rrows);
+  const int e0 = cb * 32, Ec = min(32, p.E - e0);
+  const int per = ((p.rrows + kRouterWarps - 1) / kRouterWarps + 3) & ~3;
+  const int r0 = min(nk, warp * per), r1 = min(nk, r0 + per);
+  for (int t0 = 0; t0 < p.L; t0 += 8) {
+    float acc[8];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-      if (lane == 0) sm.rms[t0 + tt] = sqrtf(sumsq / float(p.E));
+    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
+    for (int k = r0; k < r1; k += 4) {
+      float wv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wv[i] = rs.W[(k + i) * 32 + lane];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (t0 + t < p.L) {
+          const float4 xv = *reinterpret_cast<const float4*>(rs.X + size_t(t0 + t) * p.rrows + k);
+          acc[t] = fmaf(xv.x, wv[0], acc[t]);
+          acc[t] = fmaf(xv.y, wv[1], acc[t]);
+          acc[t] = fmaf(xv.z, wv[2], acc[t]);
+          acc[t] = fmaf(xv.w, wv[3], acc[t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 8; ++t) rs.wsum[(warp * 8 + t) * 32 + lane] = acc[t];
+    __syncthreads();
+    for (int o = threadIdx.x; o < 8 * 32; o += kThreads) {
+      const int t = o >> 5, c = o & 31;
+      if (t0 + t < p.L && c < Ec) {
+        float v = 0.f;
+#pragma unroll
+        for (int w = 0; w < kRouterWarps; ++w) v += rs.wsum[(w * 8 + t) * 32 + c];
+        p.s_part[(size_t(q) * p.L + t0 + t) * p.E + e0 + c] = v;
+      }
     }
     __syncthreads();
   }
+}
+
+// ------------------------------------------------------------------------------------- prologue
+// s = the parts in part order plus b, into sbuf [L][E]; per token the RMS of relu(s) over the E
+// experts and the active bits; then the union (ascending).  CTA 0 writes the chunk's outputs besides y.
+__device__ void prologue_router_stats(const DecodeParams& p, const Smem& sm, const RouterStage& rs, float* sbuf) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nW = (p.E + 31) >> 5;
+  const size_t qs = size_t(p.L) * p.E;
+  for (int o = tid; o < p.L * p.E; o += kThreads) {
+    const float* src = p.s_part + o;
+    float v = 0.f;
+    int q = 0;
+    for (; q + 8 <= p.rq; q += 8) {  // written by other CTAs of this grid: L2 loads, not L1
+      float a[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a[i] = __ldcg(src + (q + i) * qs);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v += a[i];
+    }
+    for (; q < p.rq; ++q) v += __ldcg(src + q * qs);
+    if (p.br) v += rs.b[o % p.E];
+    sbuf[o] = v;
+  }
+  __syncthreads();
+  for (int t = warp; t < p.L; t += kThreads / 32) {
+    const float* st = sbuf + size_t(t) * p.E;
+    float sumsq = 0.f;
+    for (int ww = 0; ww < nW; ++ww) {
+      const int e = ww * 32 + lane;
+      const float sv = e < p.E ? st[e] : -1.f;
+      const float a = fmaxf(sv, 0.f);
+      sumsq = fmaf(a, a, sumsq);
+      const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
+      if (lane == 0) sm.maskw[t * 32 + ww] = bits;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+    if (lane == 0) sm.rms[t] = sqrtf(sumsq / float(p.E));
+  }
+  __syncthreads();
   if (warp == 0) {
     uint32_t u = 0;
     int tok_active = 0;
@@ -903,15 +1017,12 @@ __device__ void prologue_router_stats(const DecodeParams& p, const Smem& sm, flo
     for (int a = tid; a < *sm.n_act; a += kThreads) p.active_idx[a] = sm.act[a];
     if (p.tok_mask)
       for (int o = tid; o < p.L * nW; o += kThreads) p.tok_mask[o] = sm.maskw[(o / nW) * 32 + (o % nW)];
-  }
-}
-
-__device__ void write_router_outputs(const DecodeParams& p, const Smem& sm) {
-  // r = g * relu(s) / rms, the same expression the up-projection epilogue uses
-  for (int o = threadIdx.x; o < p.L * p.E; o += kThreads) {
-    const int t = o / p.E, e = o - t * p.E;
-    const float rms = sm.rms[t];
-    p.r_out[o] = rms > 0.f ? (p.g[e] * fmaxf(p.s[o], 0.f)) / rms : 0.f;
+    if (p.r_out)  // r = g relu(s) / rms, the expression the up-projection epilogue uses
+      for (int o = tid; o < p.L * p.E; o += kThreads) {
+        const int t = o / p.E, e = o - t * p.E;
+        const float rms = sm.rms[t];
+        p.r_out[o] = rms > 0.f ? (rs.g[e] * fmaxf(sbuf[o], 0.f)) / rms : 0.f;
+      }
   }
 }
 
@@ -925,7 +1036,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem sm;
   sm.xbuf = base;
   sm.ring = base + p.xbuf_bytes;
-  uint8_t* after_ring = sm.ring + size_t(p.S) * p.slot_bytes;
+  uint8_t* after_ring = base + p.pre_bytes;  // >= the ring's end
   const bool red_alias = p.xbuf_bytes >= kRedBytes;  // x is no longer needed in phase B
   sm.red = reinterpret_cast<float*>(red_alias ? sm.xbuf : after_ring);
   uint8_t* tail = red_alias ? after_ring : after_ring + kRedBytes;
@@ -972,24 +1083,77 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
 
-  // the router wrote s and reset the grid barrier
-  pdl_wait();
-  prologue_router_stats(p, sm, reinterpret_cast<float*>(sm.ring));
-  fence_proxy_async_smem();  // the ring held s (generic writes) before bulk copies write into it
-  __syncthreads();
-  const int n_act = *sm.n_act;
-  const Work w = make_work(p, n_act);
-
-  if (warp < NCW) {
-    consume<LC, KSPLIT>(p, sm, w);
-  } else if (warp == NCW) {
-    produce_weights<KSPLIT>(p, tm, sm, w);
-  } else {
-    produce_x_h<KSPLIT>(p, tm, sm, w);
-  }
-  if (blockIdx.x == 0 && p.r_out) {
+  // ---- router: this CTA's units, then every CTA's partials
+  const RouterStage rs = router_stage(p, base);
+  {
+    const int U = p.rq * p.rcb;
+    for (int e = tid; e < p.E; e += kThreads) {
+      cp_async4(rs.g + e, p.g + e);
+      if (p.br) cp_async4(rs.b + e, p.br + e);
+    }
+    if (int(blockIdx.x) < U) router_copy_w(p, rs.W, blockIdx.x);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    // x may come from the previous kernel in the stream, and the workspace is shared with it
+    pdl_wait();
+    for (int u = blockIdx.x; u < U; u += gridDim.x) {
+      if (u != int(blockIdx.x)) {
+        router_copy_w(p, rs.W, u);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      router_load_x(p, rs.X, u);
+      asm volatile("cp.async.wait_all;" ::: "memory");
+      __syncthreads();
+      router_unit(p, rs, u);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    if (tid == 0) {
+      __threadfence();
+      red_release_gpu_add(&p.hdr->router_bar, 1u);
+      const uint64_t t0 = globaltimer_ns();
+      while (ld_acquire_gpu(&p.hdr->router_bar) < gridDim.x) {
+        if (globaltimer_ns() - t0 > kWaitNs) {
+          set_error(p, sm, kErrRouterBarrier, uint32_t(blockIdx.x));
+          break;
+        }
+        __nanosleep(32);
+      }
+    }
     __syncthreads();
-    write_router_outputs(p, sm);
+  }
+  if (!aborted(sm)) {
+    float* sbuf = rs.W;  // [L][E], over the router's staging
+    prologue_router_stats(p, sm, rs, sbuf);
+    __syncthreads();
+    const int n_act = *sm.n_act;
+    const Work w = make_work(p, n_act);
+    if (w.rA0 < w.rA1) {  // s and g of every expert this CTA's up-projection rows touch
+      const int a_first = w.rA0 / p.de, span = (w.rA1 - 1) / p.de - a_first + 1;
+      for (int o = tid; o < span * p.L; o += kThreads) {
+        const int aa = o / p.L, t = o - aa * p.L;
+        sm.pre_s[aa * 32 + t] = sbuf[size_t(t) * p.E + sm.act[a_first + aa]];
+      }
+      for (int aa = tid; aa < span; aa += kThreads) sm.pre_g[aa] = rs.g[sm.act[a_first + aa]];
+    }
+    fence_proxy_async_smem();  // the ring held generic data before bulk copies write into it
+    __syncthreads();
+
+    if (warp < NCW) {
+      consume<LC, KSPLIT>(p, sm, w);
+    } else if (warp == NCW) {
+      produce_weights<KSPLIT>(p, tm, sm, w);
+    } else {
+      produce_x_h<KSPLIT>(p, tm, sm, w);
+    }
+  }
+  // the last CTA out sets the grid's counters back for the next call on this workspace
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(&p.hdr->exit_ctr, 1u) == gridDim.x - 1) {
+      p.hdr->router_bar = 0u;
+      p.hdr->grid_bar = 0u;
+      p.hdr->exit_ctr = 0u;
+    }
   }
 }
 
@@ -1086,17 +1250,33 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
     p->ustage_units = p->ksplit ? (worst < cap ? worst : cap) : 0;
     p->ustage_bytes = p->ustage_units * L * 32;
   }
-  const size_t fixed = 1024 + size_t(p->xbuf_bytes) + red_extra + tail + size_t(p->ustage_bytes);
-  if (fixed >= size_t(max_smem)) return false;
-  int S = int((size_t(max_smem) - fixed) / (size_t(p->slot_bytes) + per_slot));
+  // router units, and the shared memory the router's staging and the chunk's s need before the ring
+  // is filled: at the start of the region of x and the ring, which is made at least that large
+  p->rrows = decode_router_rows(d);
+  p->rq = decode_router_parts(d);
+  p->rcb = (E + 31) / 32;
+  const size_t gb = size_t(2) * ((E + 3) & ~3) * 4;  // g and b
+  const size_t router_need = size_t(p->rrows) * 128 + size_t(L) * p->rrows * 4 + size_t(kThreads / 32) * 8 * 32 * 4;
+  const size_t s_need = size_t(L) * E * 4;
+  const size_t pre_need = gb + (router_need > s_need ? router_need : s_need);
+  const size_t fixed = 1024 + red_extra + tail + size_t(p->ustage_bytes);
+  if (fixed + pre_need >= size_t(max_smem)) return false;
+  int S = int((size_t(max_smem) - fixed - size_t(p->xbuf_bytes)) / (size_t(p->slot_bytes) + per_slot));
   if (S > 32) S = 32;
-  if (S < 2) return false;
-  p->S = S;
-  p->sbuf_floats = int(size_t(S) * p->slot_bytes / 4);  // the prologue stages s in the ring
-  if (p->sbuf_floats < E) return false;
+  for (;; --S) {
+    if (S < 2) return false;
+    size_t pre = size_t(p->xbuf_bytes) + size_t(S) * p->slot_bytes;
+    if (pre < pre_need) pre = round_up(int(pre_need), 1024);
+    const size_t smem = fixed + pre + size_t(S) * per_slot;
+    if (smem <= size_t(max_smem)) {
+      p->S = S;
+      p->pre_bytes = int(pre);
+      out->smem = smem;
+      break;
+    }
+  }
   out->grid = G;
   out->lclass = lc;
-  out->smem = fixed + size_t(S) * (p->slot_bytes + per_slot);
   return true;
 }
 
