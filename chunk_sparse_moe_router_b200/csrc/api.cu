@@ -125,6 +125,64 @@ bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* di
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Chunks of 9..32 tokens: the tcgen05 decode kernel (expert_decode_tc.cu).
+int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
+                      const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
+                      const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
+                      const DeviceInfo& di, int share, cudaStream_t st) {
+  const WsLayout lay = ws_layout(L, d, E, de);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  tcdec::Params dp;
+  dp.x = static_cast<const __nv_bfloat16*>(x);
+  dp.Wr = Wr;
+  dp.br = br;
+  dp.s_part = reinterpret_cast<float*>(base + lay.s_off);
+  dp.g = g;
+  dp.y = y;
+  dp.active_idx = active_idx;
+  dp.n_active = n_active;
+  dp.tok_mask = tok_mask;
+  dp.counts = counts;
+  dp.r_out = r_out;
+  dp.h = base + lay.h_off;
+  dp.part = reinterpret_cast<float*>(base + lay.part_off);
+  dp.cntA = reinterpret_cast<uint32_t*>(base + lay.cnt_off);
+  dp.cntB = dp.cntA + size_t(E) * ((de + 127) / 128);
+  dp.hdr = reinterpret_cast<WsHeader*>(base);
+  dp.L = L;
+  dp.d = d;
+  dp.E = E;
+  dp.de = de;
+  tcdec::Launch dl;
+  const int grid = di.num_sms / share;  // one persistent CTA per SM of this call's share
+  if (grid < 1 || !tcdec::plan(L, d, E, de, grid, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
+  {
+    // the kernel's grid barriers need every CTA resident at once
+    int per_sm = 0;
+    const cudaError_t oe = tcdec::occupancy(L, dl.smem, &per_sm);
+    if (oe != cudaSuccess) return cuda_fail(oe);
+    if (per_sm < 1) return BFFN_EUNSUPPORTED;
+  }
+  tcdec::Maps tm;
+  {
+    const uint64_t xrow = uint64_t(d) * 2, w1e = uint64_t(d) * de * 2;
+    const uint64_t w2row = uint64_t(de) * 2, w2e = uint64_t(d) * de * 2;
+    const uint64_t xd[2] = {uint64_t(d), uint64_t(L)}, xs[1] = {xrow};
+    const uint32_t xb[2] = {64, uint32_t(dp.LB)};
+    if (!encode_bf16(&tm.x, x, 2, xd, xs, xb)) return BFFN_ECUDA;
+    const uint64_t w1d[3] = {uint64_t(d), uint64_t(de), uint64_t(E)}, w1s[2] = {xrow, w1e};
+    const uint64_t w2d[3] = {uint64_t(de), uint64_t(d), uint64_t(E)}, w2s[2] = {w2row, w2e};
+    for (int k = 0; k < 5; ++k) {
+      const uint32_t b[3] = {64, uint32_t(8u << k), 1};
+      if (!encode_bf16(&tm.w1[k], W1, 3, w1d, w1s, b)) return BFFN_ECUDA;
+      if (!encode_bf16(&tm.w2[k], W2, 3, w2d, w2s, b)) return BFFN_ECUDA;
+    }
+  }
+  const cudaError_t err = tcdec::launch(dp, tm, dl, st, di.pdl);
+  if (err != cudaSuccess) return cuda_fail(err);
+  return BFFN_OK;
+}
+
 int forward_decode(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
@@ -332,9 +390,13 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   } else if (workspace_bytes < need) {
     return BFFN_ENOMEM;
   }
-  if (decode)
+  if (decode) {
+    if (L > kTcSmallL)
+      return forward_decode_tc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
+                               r_out, ws, di, share, st);
     return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
                           r_out, ws, di, share, st);
+  }
   return forward_prefill(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts, r_out,
                          ws, di, st);
 }

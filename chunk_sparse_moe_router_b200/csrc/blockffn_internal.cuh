@@ -38,6 +38,19 @@ __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_
 // lo rows) in the 128-byte-swizzled layout the down-projection loads.
 size_t decode_h_bytes(int L, int E, int de);
 
+// The tcgen05 decode path (8 < L <= 32; namespace tcdec): its h image has tiles of 2 LC rows
+// (LC = L rounded up to 16 or 32), and its stream-K scratch holds the partial accumulators of blocks
+// split between CTAs (two slots of 128 rows x LC fp32 per CTA) and one arrival counter per up- and
+// down-projection block.
+constexpr int kTcSmallL = 8;     // chunks of at most this many tokens take the mma.sync decode kernel
+constexpr int kTcMaxGrid = 160;  // CTAs of one tcgen05 decode launch
+namespace tcdec {
+inline int lc_of(int L) { return L <= 16 ? 16 : 32; }
+inline size_t h_bytes(int L, int E, int de) { return size_t(E) * ((de + 63) / 64) * size_t(2 * lc_of(L)) * 128; }
+inline size_t part_bytes(int L) { return size_t(kTcMaxGrid) * 2 * 128 * lc_of(L) * 4; }
+inline size_t cnt_words(int d, int E, int de) { return size_t(E) * ((de + 127) / 128) + (d + 127) / 128; }
+}  // namespace tcdec
+
 // Prefill workspace regions (L > 32), after s: the router's K-split partial projections, per-token
 // masks and RMS, per-expert counts and
 // offsets, the pair lists (token, r) in expert-major order, and H = [pairs][2 de] bf16 (hi | lo).
@@ -74,7 +87,7 @@ inline int decode_router_rows(int d) {
 inline int decode_router_parts(int d) { return (d + decode_router_rows(d) - 1) / decode_router_rows(d); }
 
 struct WsLayout {
-  size_t s_off, h_off, total;
+  size_t s_off, h_off, part_off, cnt_off, total;  // part / cnt: tcgen05 decode path only
 };
 
 // Workspace: header | router projection (decode: per-part partials [parts][L,E]; prefill: s [L,E]) |
@@ -84,7 +97,16 @@ inline WsLayout ws_layout(int L, int d, int E, int de) {
   const size_t parts = L <= kDecodeMaxL ? size_t(decode_router_parts(d)) : 1;
   w.s_off = sizeof(WsHeader);
   w.h_off = w.s_off + align256(parts * size_t(L) * E * sizeof(float));
-  w.total = L <= kDecodeMaxL ? w.h_off + align256(decode_h_bytes(L, E, de)) : prefill_layout(w.h_off, L, E, de).end;
+  w.part_off = w.cnt_off = 0;
+  if (L <= kTcSmallL) {
+    w.total = w.h_off + align256(decode_h_bytes(L, E, de));
+  } else if (L <= kDecodeMaxL) {
+    w.part_off = w.h_off + align256(tcdec::h_bytes(L, E, de));
+    w.cnt_off = w.part_off + align256(tcdec::part_bytes(L));
+    w.total = w.cnt_off + align256(tcdec::cnt_words(d, E, de) * 4);
+  } else {
+    w.total = prefill_layout(w.h_off, L, E, de).end;
+  }
   return w;
 }
 
@@ -160,6 +182,65 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
                         DecodeLaunch* out);
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl);
+
+// ------------------------------------------------------------------------ decode on tcgen05 (8 < L <= 32)
+namespace tcdec {
+struct Params {
+  const __nv_bfloat16* x;     // [L,d]
+  const float* Wr;            // [d,E]
+  const float* br;            // [E] or null
+  float* s_part;              // [rq][L,E] router partial projections (workspace)
+  const float* g;             // [E]
+  float* y;                   // [L,d]
+  int32_t* active_idx;        // [E]
+  int32_t* n_active;          // [1]
+  uint32_t* tok_mask;         // [L, ceil(E/32)] or null
+  int32_t* counts;            // [2] or null
+  float* r_out;               // [L,E] or null
+  uint8_t* h;                 // h_bytes(L, E, de)
+  float* part;                // part_bytes(L): [CTA][2][128][LC] partial accumulators
+  uint32_t* cntA;             // [E * nbpe] up-projection block arrivals (zeroed by every call)
+  uint32_t* cntB;             // [nrb] down-projection block arrivals, right after cntA
+  WsHeader* hdr;
+  int L, d, E, de;
+  int nck;          // 64-column chunks of d (the last may be ragged: the tensor maps read zeros past d)
+  int nbpe, HA;     // up-projection blocks per expert and their height (multiple of 8, <= 128)
+  int nrb, HB;      // down-projection blocks of y rows and their height (multiple of 8, <= 128)
+  int nJc;          // 64-column chunks of de
+  int LB;           // rows of an x tile (L rounded up to 8)
+  int NA;           // MMA N of the up-projection (LC)
+  int NB;           // MMA N of the down-projection (2 LC)
+  int HT;           // bytes of an h tile: 2 LC rows of 128 bytes
+  int h_expert_bytes;  // bytes of one expert's h image: nJc tiles
+  int S;            // ring slots
+  int slot_bytes;   // bytes per slot (multiple of 1024)
+  int tmem_cols;    // tensor-memory columns: two accumulators of each projection
+  int rq, rrows, rcb;  // router split (decode_router.cuh)
+  int pre_bytes;    // shared memory from the ring's start to the barriers: the ring, and room for the
+                    // router's staging and the chunk's s [L,E]
+  int tail_bytes;   // shared memory after that: barriers and per-CTA tables, at least the 16 KB that
+                    // an M = 128 operand read starting in the ring's last slot may reach
+};
+
+// Tensor maps (128-byte swizzle, out-of-bounds elements read as zero).  W1 and W2 boxes are 64
+// columns wide and 8 << k rows high (k = 0..4); a block of rows is loaded as a sum of such boxes.
+struct Maps {
+  CUtensorMap w1[5];     // [d, de, E]   box {64, 8 << k, 1}
+  CUtensorMap w2[5];     // [de, d, E]   box {64, 8 << k, 1}
+  CUtensorMap x;         // [d, L]       box {64, LB}
+};
+
+struct Launch {
+  int grid;
+  size_t smem;
+};
+
+bool plan(int L, int d, int E, int de, int grid, int max_smem, Params* p, Launch* out);
+cudaError_t launch(const Params& p, const Maps& tm, const Launch& plan, cudaStream_t st, bool pdl);
+// CTAs of the kernel for chunks of L tokens with `smem` bytes of dynamic shared memory that fit on one
+// SM at once.
+cudaError_t occupancy(int L, size_t smem, int* ctas_per_sm);
+}  // namespace tcdec
 
 // ------------------------------------------------------------------------------------ prefill
 struct PrefillParams {

@@ -1,5 +1,5 @@
-// Sparse expert kernel of the BlockFFN chunk layer for decode-sized chunks (L <= 32): one launch
-// per chunk, router included.
+// Sparse expert kernel of the BlockFFN chunk layer for chunks of up to 8 tokens: one launch per chunk,
+// router included.  (Chunks of 9 to 32 tokens take the tcgen05 kernel of expert_decode_tc.cu.)
 //
 // Router (lsdiaocha.cn BlockFFN article, section 2: the router's linear map s = x Wr + b, before its
 // ReLU and RMSNorm): d is cut into parts of at most 256 rows and E into blocks of 32 experts; each
@@ -40,6 +40,7 @@
 //   two stacks of L rows of the MMA's M dimension.  Each y element is written exactly once, in a
 //   fixed summation order, so y is bit-reproducible run to run.
 #include "blockffn_internal.cuh"
+#include "decode_router.cuh"
 #include "ptx.cuh"
 
 namespace bffn {
@@ -818,213 +819,10 @@ __device__ void consume(const DecodeParams& p, const Smem& sm, const Work& w) {
   }
 }
 
-// --------------------------------------------------------------------------------------- router
-// Unit u = (part q = u / rcb, expert block cb = u % rcb): rows [q rrows, + rrows) of d, experts
-// [32 cb, + 32).  Staging at the start of the dynamic shared memory (RouterStage): g and b [E] (copied
-// before the dependent-launch wait with this CTA's first Wr rows), Wr rows [rrows][32] fp32, x columns
-// [L][rrows] converted to fp32, warp sums [warps][8][32] fp32.
-constexpr int kRouterWarps = kThreads / 32;
-
-struct RouterStage {
-  float* g;
-  float* b;
-  float* W;
-  float* X;
-  float* wsum;
-};
-
-__device__ __forceinline__ RouterStage router_stage(const DecodeParams& p, uint8_t* base) {
-  RouterStage r;
-  const int E4 = (p.E + 3) & ~3;
-  r.g = reinterpret_cast<float*>(base);
-  r.b = r.g + E4;
-  r.W = r.b + E4;
-  r.X = r.W + size_t(p.rrows) * 32;
-  r.wsum = r.X + size_t(p.L) * p.rrows;
-  return r;
-}
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void* dst, const void* src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-
-__device__ void router_copy_w(const DecodeParams& p, float* Ws, int u) {
-  const int cb = u % p.rcb, q = u / p.rcb;
-  const int k0 = q * p.rrows, nk = min(p.d - k0, p.rrows);
-  const int e0 = cb * 32, Ec = min(32, p.E - e0);
-  if ((p.E & 3) == 0) {  // Ec is then a multiple of 4 too
-    for (int o = threadIdx.x; o < nk * 8; o += kThreads) {
-      const int kk = o >> 3, c4 = (o & 7) * 4;
-      float* dst = Ws + kk * 32 + c4;
-      if (c4 < Ec)
-        cp_async16(dst, p.Wr + size_t(k0 + kk) * p.E + e0 + c4);
-      else
-        *reinterpret_cast<float4*>(dst) = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-  } else {
-    for (int o = threadIdx.x; o < nk * 32; o += kThreads) {
-      const int kk = o >> 5, c = o & 31;
-      if (c < Ec)
-        cp_async4(Ws + kk * 32 + c, p.Wr + size_t(k0 + kk) * p.E + e0 + c);
-      else
-        Ws[kk * 32 + c] = 0.f;
-    }
-  }
-}
-
-// x columns of unit u, bf16 -> fp32 (exact)
-__device__ void router_load_x(const DecodeParams& p, float* Xs, int u) {
-  const int k0 = (u / p.rcb) * p.rrows, nk = min(p.d - k0, p.rrows);
-  const int q8 = nk >> 3;  // k0 and nk are multiples of 8
-  for (int o = threadIdx.x; o < p.L * q8; o += kThreads) {
-    const int t = o / q8, c8 = (o - t * q8) * 8;
-    const uint4 v = *reinterpret_cast<const uint4*>(p.x + size_t(t) * p.d + k0 + c8);
-    float4* dst = reinterpret_cast<float4*>(Xs + size_t(t) * p.rrows + c8);
-    dst[0] = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
-                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
-    dst[1] = make_float4(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u),
-                         __uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
-  }
-}
-
-// Partial projection of unit u from the staged operands.  Warp w takes rows [w R4, w R4 + R4) of the
-// part (R4 = rrows / warps rounded up to 4), lane = expert column, 8 tokens at a time; each sum runs
-// over its rows in increasing order, then the CTA adds the warps' sums in warp order.
-__device__ void router_unit(const DecodeParams& p, const RouterStage& rs, int u) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cb = u % p.rcb, q = u / p.rcb;
-  const int k0 = q * p.rrows, nk = min(p.d - k0, p.rrows);
-  const int e0 = cb * 32, Ec = min(32, p.E - e0);
-  const int per = ((p.rrows + kRouterWarps - 1) / kRouterWarps + 3) & ~3;
-  const int r0 = min(nk, warp * per), r1 = min(nk, r0 + per);
-  for (int t0 = 0; t0 < p.L; t0 += 8) {
-    float acc[8];
-#pragma unroll
-    for (int t = 0; t < 8; ++t) acc[t] = 0.f;
-    for (int k = r0; k < r1; k += 4) {
-      float wv[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) wv[i] = rs.W[(k + i) * 32 + lane];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (t0 + t < p.L) {
-          const float4 xv = *reinterpret_cast<const float4*>(rs.X + size_t(t0 + t) * p.rrows + k);
-          acc[t] = fmaf(xv.x, wv[0], acc[t]);
-          acc[t] = fmaf(xv.y, wv[1], acc[t]);
-          acc[t] = fmaf(xv.z, wv[2], acc[t]);
-          acc[t] = fmaf(xv.w, wv[3], acc[t]);
-        }
-      }
-    }
-#pragma unroll
-    for (int t = 0; t < 8; ++t) rs.wsum[(warp * 8 + t) * 32 + lane] = acc[t];
-    __syncthreads();
-    for (int o = threadIdx.x; o < 8 * 32; o += kThreads) {
-      const int t = o >> 5, c = o & 31;
-      if (t0 + t < p.L && c < Ec) {
-        float v = 0.f;
-#pragma unroll
-        for (int w = 0; w < kRouterWarps; ++w) v += rs.wsum[(w * 8 + t) * 32 + c];
-        p.s_part[(size_t(q) * p.L + t0 + t) * p.E + e0 + c] = v;
-      }
-    }
-    __syncthreads();
-  }
-}
-
-// ------------------------------------------------------------------------------------- prologue
-// s = the parts in part order plus b, into sbuf [L][E]; per token the RMS of relu(s) over the E
-// experts and the active bits; then the union (ascending).  CTA 0 writes the chunk's outputs besides y.
-__device__ void prologue_router_stats(const DecodeParams& p, const Smem& sm, const RouterStage& rs, float* sbuf) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nW = (p.E + 31) >> 5;
-  const size_t qs = size_t(p.L) * p.E;
-  for (int o = tid; o < p.L * p.E; o += kThreads) {
-    const float* src = p.s_part + o;
-    float v = 0.f;
-    int q = 0;
-    for (; q + 8 <= p.rq; q += 8) {  // written by other CTAs of this grid: L2 loads, not L1
-      float a[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) a[i] = __ldcg(src + (q + i) * qs);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v += a[i];
-    }
-    for (; q < p.rq; ++q) v += __ldcg(src + q * qs);
-    if (p.br) v += rs.b[o % p.E];
-    sbuf[o] = v;
-  }
-  __syncthreads();
-  for (int t = warp; t < p.L; t += kThreads / 32) {
-    const float* st = sbuf + size_t(t) * p.E;
-    float sumsq = 0.f;
-    for (int ww = 0; ww < nW; ++ww) {
-      const int e = ww * 32 + lane;
-      const float sv = e < p.E ? st[e] : -1.f;
-      const float a = fmaxf(sv, 0.f);
-      sumsq = fmaf(a, a, sumsq);
-      const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
-      if (lane == 0) sm.maskw[t * 32 + ww] = bits;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-    if (lane == 0) sm.rms[t] = sqrtf(sumsq / float(p.E));
-  }
-  __syncthreads();
-  if (warp == 0) {
-    uint32_t u = 0;
-    int tok_active = 0;
-    if (lane < nW)
-      for (int t = 0; t < p.L; ++t) {
-        const uint32_t m = sm.maskw[t * 32 + lane];
-        u |= m;
-        tok_active += __popc(m);
-      }
-    const int c = __popc(u);
-    int incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int total = __shfl_sync(0xffffffffu, incl, 31);
-    int pos = incl - c;
-    uint32_t rest = u;
-    while (rest) {
-      const int b = __ffs(rest) - 1;
-      rest &= rest - 1;
-      sm.act[pos++] = lane * 32 + b;
-    }
-    int act_sum = tok_active;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) act_sum += __shfl_xor_sync(0xffffffffu, act_sum, o);
-    if (lane == 0) {
-      *sm.n_act = total;
-      if (blockIdx.x == 0) {
-        *p.n_active = total;
-        if (p.counts) {
-          p.counts[0] = p.L * p.E - act_sum;
-          p.counts[1] = p.E - total;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {  // the chunk's outputs besides y
-    for (int a = tid; a < *sm.n_act; a += kThreads) p.active_idx[a] = sm.act[a];
-    if (p.tok_mask)
-      for (int o = tid; o < p.L * nW; o += kThreads) p.tok_mask[o] = sm.maskw[(o / nW) * 32 + (o % nW)];
-    if (p.r_out)  // r = g relu(s) / rms, the expression the up-projection epilogue uses
-      for (int o = tid; o < p.L * p.E; o += kThreads) {
-        const int t = o / p.E, e = o - t * p.E;
-        const float rms = sm.rms[t];
-        p.r_out[o] = rms > 0.f ? (rs.g[e] * fmaxf(sbuf[o], 0.f)) / rms : 0.f;
-      }
-  }
-}
+// ------------------------------------------------------------------------------ router and prologue
+// (decode_router.cuh, instantiated for this kernel's kThreads)
+using decode_router::RouterStage;
+using decode_router::cp_async4;
 
 template <int LC, bool KSPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1084,26 +882,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
 
   // ---- router: this CTA's units, then every CTA's partials
-  const RouterStage rs = router_stage(p, base);
+  const RouterStage rs = decode_router::router_stage<kThreads>(p, base);
   {
     const int U = p.rq * p.rcb;
     for (int e = tid; e < p.E; e += kThreads) {
       cp_async4(rs.g + e, p.g + e);
       if (p.br) cp_async4(rs.b + e, p.br + e);
     }
-    if (int(blockIdx.x) < U) router_copy_w(p, rs.W, blockIdx.x);
+    if (int(blockIdx.x) < U) decode_router::router_copy_w<kThreads>(p, rs.W, blockIdx.x);
     asm volatile("cp.async.commit_group;" ::: "memory");
     // x may come from the previous kernel in the stream, and the workspace is shared with it
     pdl_wait();
     for (int u = blockIdx.x; u < U; u += gridDim.x) {
       if (u != int(blockIdx.x)) {
-        router_copy_w(p, rs.W, u);
+        decode_router::router_copy_w<kThreads>(p, rs.W, u);
         asm volatile("cp.async.commit_group;" ::: "memory");
       }
-      router_load_x(p, rs.X, u);
+      decode_router::router_load_x<kThreads>(p, rs.X, u);
       asm volatile("cp.async.wait_all;" ::: "memory");
       __syncthreads();
-      router_unit(p, rs, u);
+      decode_router::router_unit<kThreads>(p, rs, u);
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
     if (tid == 0) {
@@ -1122,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (!aborted(sm)) {
     float* sbuf = rs.W;  // [L][E], over the router's staging
-    prologue_router_stats(p, sm, rs, sbuf);
+    decode_router::prologue_router_stats<kThreads>(p, sm, rs, sbuf);
     __syncthreads();
     const int n_act = *sm.n_act;
     const Work w = make_work(p, n_act);
@@ -1184,8 +982,8 @@ size_t decode_h_bytes(int L, int E, int de) { return size_t(E) * ((de + 63) / 64
 
 bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, DecodeParams* p,
                         DecodeLaunch* out) {
-  if (L < 1 || L > kDecodeMaxL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
-  const int lc = L <= 8 ? 8 : L <= 16 ? 16 : 32;
+  if (L < 1 || L > kTcSmallL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
+  const int lc = 8;
   const int mt = (2 * lc + 15) / 16;
   const int G = num_sms;
   if (d > 256 * 64) return false;  // a box spans at most 256 chunks
@@ -1282,11 +1080,9 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
 
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl) {
-  switch (plan.lclass) {
-    case 8: return p.ksplit ? launch_lc<8, true>(p, tm, plan, st, pdl) : launch_lc<8, false>(p, tm, plan, st, pdl);
-    case 16: return launch_lc<16, false>(p, tm, plan, st, pdl);
-    default: return launch_lc<32, false>(p, tm, plan, st, pdl);
-  }
+  // chunks of more than kTcSmallL tokens take the tcgen05 kernel (expert_decode_tc.cu)
+  if (plan.lclass != 8) return cudaErrorInvalidValue;
+  return p.ksplit ? launch_lc<8, true>(p, tm, plan, st, pdl) : launch_lc<8, false>(p, tm, plan, st, pdl);
 }
 
 }  // namespace bffn

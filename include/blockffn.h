@@ -32,7 +32,8 @@
  *   x, Wr, W1, W2 16-byte aligned (they are read with bulk copies), a workspace 256-byte aligned,
  *   every other pointer 4-byte aligned; required pointers non-NULL.
  * Paths: L <= 32 runs the decode path (the union's weights streamed from HBM once for the whole chunk,
- * memory-bound, deterministic: y is bit-identical run to run). Larger L runs the prefill path (tokens
+ * memory-bound, deterministic: y is bit-identical run to run); chunks of up to 8 tokens use warp MMAs,
+ * chunks of 9 to 32 tokens the tcgen05 tensor cores. Larger L runs the prefill path (tokens
  * grouped per active expert, grouped GEMMs on the tcgen05 tensor cores); it additionally needs d and de
  * multiples of 64, de <= 256 and y 16-byte aligned, and it adds each (token, expert) row into y with
  * hardware reductions, so y may differ in the last bits between runs (masks, union, counts and r do

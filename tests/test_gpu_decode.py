@@ -57,6 +57,12 @@ def test_chunk_size_sweep_width_4096(bffn, cuda_device, L):
     dict(d=128, E=1, de=32, L=3),      # a single expert
     dict(d=64, E=1024, de=16, L=3),    # maximum expert count
     dict(d=4112, E=24, de=272, L=7),   # K chunks with a ragged tail in both projections
+    # chunks of more than 8 tokens (tcgen05 kernel)
+    dict(d=16, E=16, de=16, L=9),      # minimum widths
+    dict(d=128, E=1, de=32, L=31),     # a single expert
+    dict(d=64, E=1024, de=16, L=12),   # maximum expert count
+    dict(d=4112, E=24, de=272, L=17),  # ragged tails in both projections; 3 up-projection blocks per expert
+    dict(d=384, E=40, de=320, L=24),   # up-projection blocks of 112, 112 and 96 rows
 ])
 def test_edge_shapes(bffn, cuda_device, shape):
     dl = _layer(11, shape["d"], shape["E"], shape["de"])
@@ -64,29 +70,32 @@ def test_edge_shapes(bffn, cuda_device, shape):
     _check_chunks(bffn, dl, xs)
 
 
-def test_no_active_expert(bffn, cuda_device):
+@pytest.mark.parametrize("L", [8, 24])
+def test_no_active_expert(bffn, cuda_device, L):
     from _parity import run_chunk
     dl = _layer(3, 256, 16, 64)
     dl.lay.br[:] = -50.0
     dl.br.fill_(-50.0)
-    x = gen.make_chunks(3, dl.lay, 1, 8, 0.3)[0]
+    x = gen.make_chunks(3, dl.lay, 1, L, 0.3)[0]
     got = run_chunk(bffn, dl, x)
     assert got["n_active"] == 0
-    assert got["counts"] == (8 * 16, 16)
+    assert got["counts"] == (L * 16, 16)
     assert np.all(got["y"] == 0.0) and np.all(got["r"] == 0.0)
 
 
-def test_every_expert_active(bffn, cuda_device):
+@pytest.mark.parametrize("L", [8, 32])
+def test_every_expert_active(bffn, cuda_device, L):
     dl = _layer(4, 256, 16, 64)
     dl.lay.br[:] = 50.0
     dl.br.fill_(50.0)
-    xs = gen.make_chunks(4, dl.lay, 1, 8, 0.3)
+    xs = gen.make_chunks(4, dl.lay, 1, L, 0.3)
     _check_chunks(bffn, dl, xs)
 
 
-def test_token_without_active_expert(bffn, cuda_device):
+@pytest.mark.parametrize("L", [8, 20])
+def test_token_without_active_expert(bffn, cuda_device, L):
     dl = _layer(5, 256, 16, 64)
-    x = gen.make_chunks(5, dl.lay, 1, 8, 0.3)[0]
+    x = gen.make_chunks(5, dl.lay, 1, L, 0.3)[0]
     x[3] = 0  # s = b < 0 for every expert: this token's row of y must be exactly zero
     _check_chunks(bffn, dl, [x])
 
@@ -103,11 +112,12 @@ def test_plain_entry_point_without_bias(bffn, cuda_device):
     _check_chunks(bffn, dl, xs, plain=True, bias=False)
 
 
-def test_caller_workspace_and_repeatability(bffn, cuda_device):
+@pytest.mark.parametrize("L", [8, 16])
+def test_caller_workspace_and_repeatability(bffn, cuda_device, L):
     from _parity import run_chunk
     dl = _layer(8, 1024, 64, 128, beta=1.0)
-    x = gen.make_chunks(8, dl.lay, 1, 8, 0.4)[0]
-    ws = bffn.new_workspace(8, 1024, 64, 128)
+    x = gen.make_chunks(8, dl.lay, 1, L, 0.4)[0]
+    ws = bffn.new_workspace(L, 1024, 64, 128)
     a = run_chunk(bffn, dl, x, workspace=ws)
     b = run_chunk(bffn, dl, x, workspace=ws)
     c = run_chunk(bffn, dl, x)
@@ -115,13 +125,13 @@ def test_caller_workspace_and_repeatability(bffn, cuda_device):
     assert np.array_equal(a["active_idx"], c["active_idx"])
 
 
-@pytest.mark.parametrize("share", [2, 4])
-def test_concurrency_hint_keeps_parity(bffn, cuda_device, share):
+@pytest.mark.parametrize("share,L", [(2, 8), (4, 8), (4, 16)])
+def test_concurrency_hint_keeps_parity(bffn, cuda_device, share, L):
     # flags bits 4-7 = k: the expert kernel takes 1/k of the SMs (a different work split); k calls on
     # k streams with their own workspaces run side by side, each still exact against the oracle
     import torch
     from _parity import assert_parity, bf16_tensor, reference
-    w = gen.workload("decode")
+    w = gen.workload("decode", L=L)
     from _parity import DeviceLayer
     dl = DeviceLayer(w.layer(0))
     xs = w.chunks(dl.lay, share)
