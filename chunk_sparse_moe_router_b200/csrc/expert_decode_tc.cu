@@ -594,7 +594,7 @@ __device__ void epilogue(const Params& p, const Smem& sm, const Work& w, uint32_
 // ------------------------------------------------------------------------------------- kernel
 template <int LC>
 __global__ void __launch_bounds__(kThreads, 1)
-    expert_decode_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps tm) {
+    expert_decode_tc_kernel(const __grid_constant__ Params p, const __grid_constant__ Maps tm) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Smem sm;
@@ -747,7 +747,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int LC>
 cudaError_t launch_lc(const Params& p, const Maps& tm, const Launch& plan, cudaStream_t st,
                       bool pdl) {
-  auto kfn = expert_decode_kernel<LC>;
+  auto kfn = expert_decode_tc_kernel<LC>;
   cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
@@ -832,7 +832,7 @@ bool plan(int L, int d, int E, int de, int grid, int max_smem, Params* p, Launch
 
 template <int LC>
 cudaError_t occupancy_lc(size_t smem, int* ctas) {
-  auto kfn = expert_decode_kernel<LC>;
+  auto kfn = expert_decode_tc_kernel<LC>;
   cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (err != cudaSuccess) return err;
   err = cudaFuncSetAttribute(kfn, cudaFuncAttributePreferredSharedMemoryCarveout, int(cudaSharedmemCarveoutMaxShared));
