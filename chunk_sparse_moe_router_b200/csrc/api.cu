@@ -125,7 +125,7 @@ bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* di
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Chunks of 9..32 tokens: the tcgen05 decode kernel (expert_decode_tc.cu).
+// Decode shapes decode_on_tc selects: the tcgen05 decode kernel (expert_decode_tc.cu).
 int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                       const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                       const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
@@ -391,7 +391,7 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
     return BFFN_ENOMEM;
   }
   if (decode) {
-    if (L > kTcSmallL)
+    if (decode_on_tc(L, d, de))
       return forward_decode_tc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
                                r_out, ws, di, share, st);
     return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,

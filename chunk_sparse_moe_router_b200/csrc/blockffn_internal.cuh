@@ -38,12 +38,17 @@ __host__ __device__ inline size_t align256(size_t v) { return (v + 255) & ~size_
 // lo rows) in the 128-byte-swizzled layout the down-projection loads.
 size_t decode_h_bytes(int L, int E, int de);
 
-// The tcgen05 decode path (8 < L <= 32; namespace tcdec): its h image has tiles of 2 LC rows
-// (LC = L rounded up to 16 or 32), and its stream-K scratch holds the partial accumulators of blocks
+// The tcgen05 decode path (decode_on_tc; namespace tcdec): its h image has tiles of 2 LC rows
+// (LC = L rounded up to 16 or 32, at least 16), and its stream-K scratch holds the partial accumulators of blocks
 // split between CTAs (two slots of 128 rows x LC fp32 per CTA) and one arrival counter per up- and
 // down-projection block.
-constexpr int kTcSmallL = 8;     // chunks of at most this many tokens take the mma.sync decode kernel
+constexpr int kTcSmallL = 8;     // the mma.sync decode kernel takes chunks of at most this many tokens
 constexpr int kTcMaxGrid = 160;  // CTAs of one tcgen05 decode launch
+// Which decode kernel a shape takes: the tcgen05 one for chunks of more than kTcSmallL tokens, and for
+// any chunk length once one expert's W1 and W2 hold 4 MiB or more (d de >= 2^20).  There its faster
+// streaming outweighs its larger fixed cost (the split-block reductions): measured 11-14 % faster at
+// d = 4096, de = 256 for L = 1..8, and 7 % slower at d = 2048, de = 256, L = 8.
+inline bool decode_on_tc(int L, int d, int de) { return L > kTcSmallL || 1ll * d * de >= (1ll << 20); }
 namespace tcdec {
 inline int lc_of(int L) { return L <= 16 ? 16 : 32; }
 inline size_t h_bytes(int L, int E, int de) { return size_t(E) * ((de + 63) / 64) * size_t(2 * lc_of(L)) * 128; }
@@ -98,7 +103,7 @@ inline WsLayout ws_layout(int L, int d, int E, int de) {
   w.s_off = sizeof(WsHeader);
   w.h_off = w.s_off + align256(parts * size_t(L) * E * sizeof(float));
   w.part_off = w.cnt_off = 0;
-  if (L <= kTcSmallL) {
+  if (L <= kDecodeMaxL && !decode_on_tc(L, d, de)) {
     w.total = w.h_off + align256(decode_h_bytes(L, E, de));
   } else if (L <= kDecodeMaxL) {
     w.part_off = w.h_off + align256(tcdec::h_bytes(L, E, de));
@@ -183,7 +188,7 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl);
 
-// ------------------------------------------------------------------------ decode on tcgen05 (8 < L <= 32)
+// ------------------------------------------------------------------------ decode on tcgen05 (decode_on_tc)
 namespace tcdec {
 struct Params {
   const __nv_bfloat16* x;     // [L,d]

@@ -1,5 +1,6 @@
-// Sparse expert kernel of the BlockFFN chunk layer for chunks of up to 8 tokens: one launch per chunk,
-// router included.  (Chunks of 9 to 32 tokens take the tcgen05 kernel of expert_decode_tc.cu.)
+// Sparse expert kernel of the BlockFFN chunk layer for chunks of up to 8 tokens of experts under 4 MiB
+// (decode_on_tc false): one launch per chunk, router included.  (Other decode shapes take the tcgen05
+// kernel of expert_decode_tc.cu.)
 //
 // Router (lsdiaocha.cn BlockFFN article, section 2: the router's linear map s = x Wr + b, before its
 // ReLU and RMSNorm): d is cut into parts of at most 256 rows and E into blocks of 32 experts; each

@@ -1,7 +1,9 @@
-// Sparse expert kernel of the BlockFFN chunk layer for chunks of 9 to 32 tokens, on the 5th-generation
-// tensor cores: one launch per chunk, router included.  (Chunks of up to 8 tokens take the mma.sync
-// kernel of expert_decode.cu, which is faster there; at 12 to 32 tokens that kernel's K split is
-// bound by its warp MMAs and this one streams the weights 1.2 to 3.7 times faster.)
+// Sparse expert kernel of the BlockFFN chunk layer for decode chunks (L <= 32) on the 5th-generation
+// tensor cores: one launch per chunk, router included.  It takes chunks of 9 to 32 tokens, where the
+// mma.sync kernel of expert_decode.cu is bound by its warp MMAs (this one streams the weights 1.2 to
+// 4.8 times faster), and chunks of any length when one expert's W1 and W2 hold 4 MiB or more
+// (decode_on_tc); the mma.sync kernel keeps small chunks of smaller experts, where its lower fixed
+// cost wins.
 //
 // Router and prologue (decode_router.cuh): s = x Wr + b split over the CTAs, a grid barrier, then in
 // every CTA the ReLU / RMSNorm statistics, the masks and the chunk's union of active experts
@@ -771,7 +773,7 @@ int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 
 bool plan(int L, int d, int E, int de, int grid, int max_smem, Params* p, Launch* out) {
-  if (L <= kTcSmallL || L > kDecodeMaxL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
+  if (L < 1 || L > kDecodeMaxL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
   const int G = grid;
   if (G < 1) return false;
   if ((E + G - 1) / G + 2 > kMaxSpan) return false;  // experts one CTA's up-projection rows touch
