@@ -1081,7 +1081,7 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
 
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl) {
-  // chunks of more than kTcSmallL tokens take the tcgen05 kernel (expert_decode_tc.cu)
+  // other decode shapes (decode_on_tc) take the tcgen05 kernel (expert_decode_tc.cu)
   if (plan.lclass != 8) return cudaErrorInvalidValue;
   return p.ksplit ? launch_lc<8, true>(p, tm, plan, st, pdl) : launch_lc<8, false>(p, tm, plan, st, pdl);
 }
