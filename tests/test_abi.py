@@ -90,3 +90,13 @@ def test_prefill_needs_a_16_byte_aligned_y(bffn):
 def test_plain_entry_point_validates(bffn):
     assert bffn.blockffn_chunk_forward(None, 8, 256, FAKE, FAKE, FAKE, FAKE, 16, 64, FAKE, FAKE, FAKE,
                                        None) == bffn.BFFN_EINVAL
+
+
+def test_workspace_holds_the_selected_decode_kernel_scratch(bffn):
+    # decode shapes of the tcgen05 kernel (more than 8 tokens, or d * de >= 2^20) need its stream-K
+    # scratch: 160 CTA slots x 2 partial accumulators x 128 rows x LC fp32, LC = 16 or 32
+    for L, d, E, de, lc in [(16, 1024, 64, 128, 16), (4, 4096, 128, 256, 16), (32, 2048, 64, 256, 32)]:
+        assert bffn.blockffn_workspace_size(L, d, E, de) >= 160 * 2 * 128 * lc * 4, (L, d, E, de)
+    # a chunk of 8 tokens of smaller experts takes the mma.sync kernel: header, router parts and h only
+    small = bffn.blockffn_workspace_size(8, 2048, 64, 256)
+    assert 64 * 4 * 2 * 8 * 128 <= small < 160 * 2 * 128 * 16 * 4
