@@ -24,10 +24,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(bffn):
 
 
 @pytest.mark.gpu
-def test_noalloc_matches_regular_entry_point_on_two_calls(bffn, cuda_device):
+@pytest.mark.parametrize("L", [8, 16])  # 16 tokens: the tcgen05 decode kernel and its stream-K scratch
+def test_noalloc_matches_regular_entry_point_on_two_calls(bffn, cuda_device, L):
     from _parity import DeviceLayer, bf16_tensor, y_violations
 
-    w = gen.workload("decode")
+    w = gen.workload("decode", L=L)
     dl = DeviceLayer(w.layer(0))
     xs = w.chunks(dl.lay, 2)
     L, d, E, de = w.L, w.d, w.E, w.de
