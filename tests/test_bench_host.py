@@ -71,3 +71,30 @@ def test_clock_summary_parses_samples(tmp_path):
     s = cs.summary()
     assert s["sm_mhz"] == 1950 and s["sm_max_mhz"] == 1965
     assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
+
+
+def test_reference_arm_prints_the_contract_line():
+    # bench.py --impl reference times the fp64 oracle on the host cores (no GPU) and prints one JSON
+    # line with the benchmark's keys, its own CPU-baseline record and a host-only end-to-end figure
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload", "tiny",
+                          "--steps", "2", "--warmup", "3"], capture_output=True, text=True, cwd=root, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["steps"] == 2 and j["warmup"] == 3 and j["value"] > 0
+    assert j["config"]["workload"].startswith("tiny")
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == j["value"]
+    e2e = j["e2e"]
+    assert e2e["value"] == j["value"] and e2e["unit"] == j["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
