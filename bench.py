@@ -456,6 +456,19 @@ def run_reference(args, w):
     print(json.dumps(out), flush=True)
 
 
+def launch_local_ranks(n: int, argv: list[str]) -> int:
+    """Run this script as n ranks on this node (one process per GPU, rendezvous on 127.0.0.1) when it
+    was started without a launcher; returns the launcher's exit status."""
+    import socket
+
+    with socket.socket() as sock:
+        sock.bind(("127.0.0.1", 0))
+        port = sock.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -476,6 +489,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_local_ranks(args.gpus, sys.argv[1:]))
+    if args.gpus != dist_env()[0]:
+        ap.error(f"--gpus {args.gpus} but the launcher started {dist_env()[0]} ranks")
 
     import gen
 

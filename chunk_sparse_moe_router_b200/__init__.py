@@ -18,6 +18,9 @@ BFFN_OK, BFFN_EINVAL, BFFN_ECUDA, BFFN_ENOMEM, BFFN_ETIMEOUT, BFFN_EUNSUPPORTED 
 BFFN_PATH_AUTO, BFFN_PATH_DECODE, BFFN_PATH_PREFILL = 0, 1, 2
 
 
+BFFN_FLAG_INJECT_ROUTER_TIMEOUT = 0x100  # fault injection for tests of the error path (decode path)
+
+
 def BFFN_FLAGS_SHARE(k: int) -> int:
     """Concurrency hint (decode path): the call takes 1/k of the SMs; k calls on k streams with k
     workspaces run side by side."""
@@ -30,6 +33,7 @@ SIGNATURES = {
     "blockffn_chunk_forward_ex": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P,
                                        _P, _I, _P, _S, _P]),
     "blockffn_chunk_forward_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P]),
+    "blockffn_noalloc_device_status": (_I, [_P]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_init": (_I, [_P, _S, _P]),
     "blockffn_device_status": (_I, [_P, _P]),
@@ -75,6 +79,10 @@ def blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_ac
 def blockffn_chunk_forward_noalloc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, stream):
     return _lib.blockffn_chunk_forward_noalloc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br,
                                                stream)
+
+
+def blockffn_noalloc_device_status(stream):
+    return _lib.blockffn_noalloc_device_status(stream)
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # BFFN_NOALLOC_SCRATCH_BYTES in include/blockffn.h

@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/blockffn.h: argument checks, workspace handling and
 // the kernel launches of one BlockFFN chunk-layer forward.
+#include <cstdlib>
 #include <mutex>
 
 #include "blockffn.h"
@@ -57,6 +58,11 @@ int device_info(DeviceInfo* out, int* dev_out) {
 
 // The library's per-device workspace, grown on demand (never during stream capture).
 int internal_workspace(int dev, size_t need, cudaStream_t st, void** ws) {
+  // BFFN_TEST_FAIL_ALLOC=1 makes every call that uses this workspace fail as its allocation would on a
+  // device without free memory (BFFN_ENOMEM, nothing enqueued): a host-side stand-in that lets tests
+  // reach that path without exhausting the GPU
+  const char* fake = getenv("BFFN_TEST_FAIL_ALLOC");
+  if (fake != nullptr && fake[0] == '1') return BFFN_ENOMEM;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceWorkspace& w = g_ws[dev];
   if (w.bytes < need) {
@@ -84,7 +90,7 @@ int internal_workspace(int dev, size_t need, cudaStream_t st, void** ws) {
 }
 
 bool shapes_ok(int L, int d, int E, int de) {
-  return L >= 1 && E >= 1 && E <= kMaxE && d >= 16 && d % 16 == 0 && de >= 16 && de % 16 == 0 &&
+  return L >= 1 && E >= 1 && E <= kMaxE && d >= 8 && d % 8 == 0 && de >= 8 && de % 8 == 0 &&
          (long long)L * d < (1ll << 31) && (long long)E * de * d < (1ll << 40);
 }
 
@@ -129,10 +135,11 @@ bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* di
 int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                       const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                       const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                      const DeviceInfo& di, int share, cudaStream_t st) {
+                      const DeviceInfo& di, int share, bool inject, cudaStream_t st) {
   const WsLayout lay = ws_layout(L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   tcdec::Params dp;
+  dp.inject_timeout = inject ? 1 : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.Wr = Wr;
   dp.br = br;
@@ -186,12 +193,13 @@ int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float*
 int forward_decode(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                   const DeviceInfo& di, int share, cudaStream_t st) {
+                   const DeviceInfo& di, int share, bool inject, cudaStream_t st) {
   const WsLayout lay = ws_layout(L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
 
   DecodeParams dp;
+  dp.inject_timeout = inject ? 1 : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.Wr = Wr;
   dp.br = br;
@@ -212,6 +220,13 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
   DecodeLaunch dl;
   const int grid = di.num_sms / share;  // one persistent CTA per SM of this call's share
   if (grid < 1 || !expert_decode_plan(L, d, E, de, grid, di.max_smem, &dp, &dl)) return BFFN_EUNSUPPORTED;
+  {
+    // the kernel's grid barriers need every CTA resident at once
+    int per_sm = 0;
+    const cudaError_t oe = expert_decode_occupancy(dp, dl.smem, &per_sm);
+    if (oe != cudaSuccess) return cuda_fail(oe);
+    if (per_sm < 1) return BFFN_EUNSUPPORTED;
+  }
 
   TensorMaps tm;
   {
@@ -300,9 +315,6 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
 
   PrefillMaps m;
   {
-    const uint64_t xd[2] = {uint64_t(d), uint64_t(L)}, xs[1] = {uint64_t(d) * 2};
-    const uint32_t xb[2] = {64, 1};
-    if (!encode_bf16(&m.xg, x, 2, xd, xs, xb)) return BFFN_ECUDA;
     const uint64_t w1d[2] = {uint64_t(d), uint64_t(E) * de}, w1s[1] = {uint64_t(d) * 2};
     const uint32_t w1b[2] = {64, uint32_t(p.N1)};
     if (!encode_bf16(&m.w1, W1, 2, w1d, w1s, w1b)) return BFFN_ECUDA;
@@ -370,9 +382,11 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   const int path = flags & 3;
   if (path == 3) return BFFN_EINVAL;
   const int share = ((flags >> 4) & 15) == 0 ? 1 : ((flags >> 4) & 15);
-  if ((flags & ~0xF3) != 0) return BFFN_EINVAL;
+  if ((flags & ~(0xF3 | BFFN_FLAG_INJECT_ROUTER_TIMEOUT)) != 0) return BFFN_EINVAL;
+  const bool inject = (flags & BFFN_FLAG_INJECT_ROUTER_TIMEOUT) != 0;
   const bool decode = (path == BFFN_PATH_DECODE) || (path == BFFN_PATH_AUTO && L <= kDecodeMaxL);
   if (decode && L > kDecodeMaxL) return BFFN_EUNSUPPORTED;
+  if (!decode && inject) return BFFN_EUNSUPPORTED;  // the injection exists on the decode path only
   if (!decode && L <= kDecodeMaxL) return BFFN_EUNSUPPORTED;  // the prefill path takes L > 32
   if (!decode && (d % 64 != 0 || de % 64 != 0 || de > 256)) return BFFN_EUNSUPPORTED;
   if (!decode && !aligned16(y)) return BFFN_EINVAL;  // the down-projection adds into y 16 bytes at a time
@@ -393,9 +407,9 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   if (decode) {
     if (decode_on_tc(L, d, de))
       return forward_decode_tc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                               r_out, ws, di, share, st);
+                               r_out, ws, di, share, inject, st);
     return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                          r_out, ws, di, share, st);
+                          r_out, ws, di, share, inject, st);
   }
   return forward_prefill(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts, r_out,
                          ws, di, st);

@@ -12,6 +12,10 @@ namespace bffn {
 constexpr int kMaxE = 1024;
 constexpr int kDecodeMaxL = 32;
 
+// A router barrier made unreachable on purpose (the fault-injection flag of blockffn_chunk_forward_ex)
+// gives up after this long; every other device wait gives up after about 2 s.
+constexpr uint64_t kInjectedWaitNs = 1000000ull;
+
 // Device error word bits (WsHeader::err).
 enum : uint32_t {
   kErrGridBarrier = 1u,   // expert kernel: waiting for every CTA to finish the up-projection
@@ -131,6 +135,7 @@ struct DecodeParams {
   uint8_t* h;                 // decode_h_bytes(L, E, de)
   WsHeader* hdr;
   int L, d, E, de;
+  int inject_timeout;  // 1: the router barrier waits for one arrival more than the grid has (1 ms limit)
   int S;            // ring slots
   int slot_bytes;   // bytes per slot (multiple of 1024)
   // up-projection: one stage = one W1 box of h (1, 2, 4 or 8 <= RSM) whole adjacent rows of one
@@ -185,6 +190,8 @@ struct DecodeLaunch {
 
 bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, DecodeParams* p,
                         DecodeLaunch* out);
+// CTAs of the kernel the plan selected that fit on one SM at once with `smem` bytes of dynamic shared memory.
+cudaError_t expert_decode_occupancy(const DecodeParams& p, size_t smem, int* ctas_per_sm);
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,
                                  cudaStream_t st, bool pdl);
 
@@ -208,6 +215,7 @@ struct Params {
   uint32_t* cntB;             // [nrb] down-projection block arrivals, right after cntA
   WsHeader* hdr;
   int L, d, E, de;
+  int inject_timeout;  // 1: the router barrier waits for one arrival more than the grid has (1 ms limit)
   int nck;          // 64-column chunks of d (the last may be ragged: the tensor maps read zeros past d)
   int nbpe, HA;     // up-projection blocks per expert and their height (multiple of 8, <= 128)
   int nrb, HB;      // down-projection blocks of y rows and their height (multiple of 8, <= 128)
@@ -280,7 +288,6 @@ struct PrefillParams {
 };
 
 struct PrefillMaps {
-  CUtensorMap xg;   // x [L rows, d] box 64 x 1 (gather4 of token rows)
   CUtensorMap w1;   // W1 [E*de rows, d] box 64 x N1
   CUtensorMap h;    // H [L*E rows, 2 de] box 64 x 128
   CUtensorMap w2;   // W2 [E*d rows, de] box 64 x N2

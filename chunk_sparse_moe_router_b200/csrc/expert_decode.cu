@@ -402,6 +402,17 @@ __device__ void produce_x_h(const DecodeParams& p, const TensorMaps& tm, const S
 }
 
 // ------------------------------------------------------------------------------------- consumers
+// Columns [de, 64 nJc) of an expert's last h tile face the zero columns the W2 boxes read past de, but
+// the workspace may hold any bytes there (another shape's data, possibly a NaN pattern, and 0 * NaN is
+// NaN): whoever writes the expert's last row of token t also zeroes that tail in rows t and L + t.  de
+// is a multiple of 8, so the tail is whole 16-byte pieces.  `img` is the start of the tile.
+__device__ __forceinline__ void zero_h_tail(const DecodeParams& p, uint8_t* img, int t) {
+  for (int c8 = (p.de & 63) >> 3; c8 != 0 && c8 < 8; ++c8) {
+    *reinterpret_cast<uint4*>(img + swz(t, c8)) = make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(img + swz(p.L + t, c8)) = make_uint4(0, 0, 0, 0);
+  }
+}
+
 // The epilogue of one up-projection value: h = r * Swish(u), stored as bf16 hi and lo parts in the
 // down-projection's tile layout.
 __device__ __forceinline__ void store_h(const DecodeParams& p, const Smem& sm, int a_first, int a, int j, int t,
@@ -416,11 +427,12 @@ __device__ __forceinline__ void store_h(const DecodeParams& p, const Smem& sm, i
   const int col = j & 63;
   *reinterpret_cast<__nv_bfloat16*>(himg + swz(t, col >> 3) + (col & 7) * 2) = hi;
   *reinterpret_cast<__nv_bfloat16*>(himg + swz(p.L + t, col >> 3) + (col & 7) * 2) = lo;
+  if (j == p.de - 1) zero_h_tail(p, himg, t);
 }
 
 // Epilogue of a block of the CTA's up-projection rows [r0, r1) (multiples of 8): h = r Swish(u) with
 // r = g relu(s) / rms, split into bf16 hi and lo parts and written to the global h image as 16-byte
-// pieces of 8 consecutive j (one expert each: row blocks are multiples of 8 and de of 16).  u of
+// pieces of 8 consecutive j (one expert each: row blocks and de are multiples of 8).  u of
 // row r0 + i waits in unit i / 8 of the staging buffer.
 __device__ void flush_u(const DecodeParams& p, const Smem& sm, int a_first, int r0, int r1) {
   const int units = (r1 - r0) >> 3;
@@ -447,6 +459,7 @@ __device__ void flush_u(const DecodeParams& p, const Smem& sm, int a_first, int 
     uint8_t* img = p.h + size_t(a) * p.h_expert_bytes + size_t(j >> 6) * p.HR * 128;
     *reinterpret_cast<uint4*>(img + swz(t, (j & 63) >> 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
     *reinterpret_cast<uint4*>(img + swz(p.L + t, (j & 63) >> 3)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    if (j + 8 == p.de) zero_h_tail(p, img, t);
   }
 }
 
@@ -909,8 +922,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       red_release_gpu_add(&p.hdr->router_bar, 1u);
       const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(&p.hdr->router_bar) < gridDim.x) {
-        if (globaltimer_ns() - t0 > kWaitNs) {
+      const uint32_t need = gridDim.x + (p.inject_timeout ? 1u : 0u);
+      const uint64_t limit = p.inject_timeout ? kInjectedWaitNs : kWaitNs;
+      while (ld_acquire_gpu(&p.hdr->router_bar) < need) {
+        if (globaltimer_ns() - t0 > limit) {
           set_error(p, sm, kErrRouterBarrier, uint32_t(blockIdx.x));
           break;
         }
@@ -983,7 +998,7 @@ size_t decode_h_bytes(int L, int E, int de) { return size_t(E) * ((de + 63) / 64
 
 bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, DecodeParams* p,
                         DecodeLaunch* out) {
-  if (L < 1 || L > kTcSmallL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
+  if (L < 1 || L > kTcSmallL || d % 8 != 0 || de % 8 != 0 || E < 1 || E > kMaxE) return false;
   const int lc = 8;
   const int mt = (2 * lc + 15) / 16;
   const int G = num_sms;
@@ -1077,6 +1092,13 @@ bool expert_decode_plan(int L, int d, int E, int de, int num_sms, int max_smem, 
   out->grid = G;
   out->lclass = lc;
   return true;
+}
+
+cudaError_t expert_decode_occupancy(const DecodeParams& p, size_t smem, int* ctas_per_sm) {
+  auto kfn = p.ksplit ? expert_decode_kernel<8, true> : expert_decode_kernel<8, false>;
+  cudaError_t err = cudaFuncSetAttribute(kfn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (err != cudaSuccess) return err;
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, kfn, kThreads, smem);
 }
 
 cudaError_t expert_decode_launch(const DecodeParams& p, const TensorMaps& tm, const DecodeLaunch& plan,

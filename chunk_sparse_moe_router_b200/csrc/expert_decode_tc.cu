@@ -552,6 +552,18 @@ __device__ void epilogue(const Params& p, const Smem& sm, const Work& w, uint32_
           *reinterpret_cast<__nv_bfloat16*>(himg + R1 * 128 + (((col >> 3) ^ (R1 & 7)) << 4)) = lo;
         }
       }
+      // Columns [de, 64 nJc) of the expert's last h tile face the zero columns the W2 boxes read past
+      // de, but the workspace may hold any bytes there (possibly a NaN pattern, and 0 * NaN is NaN):
+      // the thread of the expert's last row zeroes them (whole 16-byte pieces: de is a multiple of 8).
+      if (j == p.de - 1) {
+        uint8_t* tile = himg - (col & 7) * 2;
+        for (int t = 0; t < p.L; ++t)
+          for (int c8 = (p.de & 63) >> 3; c8 != 0 && c8 < 8; ++c8) {
+            const int R0 = t, R1 = LC + t;
+            *reinterpret_cast<uint4*>(tile + R0 * 128 + ((c8 ^ (R0 & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(tile + R1 * 128 + ((c8 ^ (R1 & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+          }
+      }
     }
   }
   // publish this CTA's h before any CTA reads it (every CTA arrives, also after an abort)
@@ -684,8 +696,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __threadfence();
       red_release_gpu_add(&p.hdr->router_bar, 1u);
       const uint64_t t0 = globaltimer_ns();
-      while (ld_acquire_gpu(&p.hdr->router_bar) < gridDim.x) {
-        if (globaltimer_ns() - t0 > kWaitNs) {
+      const uint32_t need = gridDim.x + (p.inject_timeout ? 1u : 0u);
+      const uint64_t limit = p.inject_timeout ? kInjectedWaitNs : kWaitNs;
+      while (ld_acquire_gpu(&p.hdr->router_bar) < need) {
+        if (globaltimer_ns() - t0 > limit) {
           set_error(p, sm, kErrRouterBarrier, uint32_t(blockIdx.x));
           break;
         }
@@ -773,7 +787,7 @@ int round_up(int v, int m) { return (v + m - 1) / m * m; }
 
 
 bool plan(int L, int d, int E, int de, int grid, int max_smem, Params* p, Launch* out) {
-  if (L < 1 || L > kDecodeMaxL || d % 16 != 0 || de % 16 != 0 || E < 1 || E > kMaxE) return false;
+  if (L < 1 || L > kDecodeMaxL || d % 8 != 0 || de % 8 != 0 || E < 1 || E > kMaxE) return false;
   const int G = grid;
   if (G < 1) return false;
   if ((E + G - 1) / G + 2 > kMaxSpan) return false;  // experts one CTA's up-projection rows touch

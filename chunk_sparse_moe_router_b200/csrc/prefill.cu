@@ -6,8 +6,8 @@
 //   P1 router       s = x Wr + b, fp32 FFMA tiles (the mask decisions need fp32 accuracy)
 //   P2 stats        per token: RMS of relu(s), active bits, optional r and masks
 //   P3 grouping     per expert: its tokens in ascending order with r_{t,e}, 128-row tiles
-//   P4 GEMM1        per (expert, 128-token tile): U = X[T_e] W1_e^T on tcgen05 (A rows gathered with
-//                   TMA gather4), h = r Swish(U) split into bf16 hi + lo parts
+//   P4 GEMM1        per (expert, 128-token tile): U = X[T_e] W1_e^T on tcgen05 (the A rows gathered by
+//                   four loader warps with coalesced cp.async), h = r Swish(U) split into bf16 hi + lo parts
 //   P5 GEMM2        per (expert tile, 256 columns of d): Y[T_e] += (H_hi + H_lo) W2_e^T on tcgen05,
 //                   added into y with vector reductions
 #include <cuda_bf16.h>

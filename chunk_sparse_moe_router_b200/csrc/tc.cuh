@@ -1,6 +1,6 @@
-// Inline-PTX wrappers for the 5th-generation tensor cores of sm_100a (tcgen05 + tensor memory) and the
-// TMA loads the tcgen05 GEMMs use.  One CTA per MMA (cta_group::1), bf16 operands (kind::f16), fp32
-// accumulators in tensor memory, operands K-major in shared memory with the 128-byte swizzle.
+// Inline-PTX wrappers for the 5th-generation tensor cores of sm_100a (tcgen05 + tensor memory).  One CTA
+// per MMA (cta_group::1), bf16 operands (kind::f16), fp32 accumulators in tensor memory, operands K-major
+// in shared memory with the 128-byte swizzle.
 #pragma once
 #include <cstdint>
 
@@ -97,18 +97,6 @@ __device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// ------------------------------------------------------------------------------ TMA
-// Four rows (row0..row3) of 64 bf16 starting at column `col` of a 2-D tensor whose map has a box of
-// 64 x 1, into 4 consecutive 128-byte rows at `dst` (no multicast).
-__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int col, int row0, int row1, int row2,
-                                            int row3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%2, "
-      "%3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
-      "l"(tmap), "r"(col), "r"(row0), "r"(row1), "r"(row2), "r"(row3), "r"(smem_u32(bar))
-      : "memory");
 }
 
 }  // namespace tc

@@ -28,7 +28,8 @@
  * n_active are unspecified. n_active stays on the device.
  *
  * Requirements, checked before anything is enqueued (BFFN_EINVAL otherwise):
- *   1 <= L, 1 <= E <= 1024, d >= 16 and d % 16 == 0, de >= 16 and de % 16 == 0;
+ *   1 <= L, 1 <= E <= 1024, d >= 8 and d % 8 == 0, de >= 8 and de % 8 == 0 (a row of x, W1 or W2
+ *   is then a whole number of 16-byte pieces, as the bulk copies need);
  *   x, Wr, W1, W2 16-byte aligned (they are read with bulk copies), a workspace 256-byte aligned,
  *   every other pointer 4-byte aligned; required pointers non-NULL.
  * Paths: L <= 32 runs the decode path (the union's weights streamed from HBM once for the whole chunk,
@@ -78,6 +79,13 @@ enum { BFFN_PATH_AUTO = 0, BFFN_PATH_DECODE = 1, BFFN_PATH_PREFILL = 2 };
  * the up-projection's grid barrier) overlap another chunk's weight streaming.  At most k such calls may
  * be in flight at once.  The results do not depend on k. */
 #define BFFN_FLAGS_SHARE(k) ((int)(k) << 4)
+
+/* Fault injection for tests of the error path (decode path only; off unless this bit is set): the
+ * call's router barrier waits for one CTA more than the launch has and gives up after 1 ms, as a wait
+ * whose peer never arrives would.  Every CTA then records the timeout, skips the rest of its work and
+ * exits; y, active_idx and the other outputs are left unspecified, blockffn_device_status reports
+ * BFFN_ETIMEOUT, and the next call on the same workspace runs normally.  Nothing faults or hangs. */
+#define BFFN_FLAG_INJECT_ROUTER_TIMEOUT 0x100
 
 /*
  * The layer forward over one chunk, with no router bias.  Uses a per-device workspace that the
@@ -136,8 +144,11 @@ BFFN_API int blockffn_device_status(void* workspace, void* stream);
  *   - Every call on a device shares the one array and leaves its contents behind: calls whose GPU
  *     work overlaps (different streams, or several host threads) race on it and must be ordered
  *     by the caller.
+ *   - It runs the decode path only: L > 32 returns BFFN_EUNSUPPORTED before anything is enqueued.
  *   - Device-side timeouts of this entry point are recorded in its own array, not in the
- *     workspace blockffn_device_status(NULL, ...) reads.
+ *     workspace blockffn_device_status(NULL, ...) reads: blockffn_noalloc_device_status reports them.
+ *   - The array's address is looked up once per device for the life of the process; resetting the
+ *     device (cudaDeviceReset) and then calling this entry point again is not supported.
  * Inputs and outputs are the caller's device buffers, as for blockffn_chunk_forward.
  */
 #define BFFN_NOALLOC_SCRATCH_BYTES (8u << 20)
@@ -145,6 +156,14 @@ BFFN_API int blockffn_chunk_forward_noalloc(const void* x, int L, int d, const f
                                             const float* g, const void* W1, const void* W2, int E,
                                             int de, float* y, int32_t* active_idx,
                                             int32_t* n_active, const float* br, void* stream);
+
+/*
+ * The error check of blockffn_chunk_forward_noalloc (no counterpart on the BlockFFN pages): synchronise
+ * `stream`, then read and clear the error word of the current device's compiled-in scratch array.
+ * Returns BFFN_OK, BFFN_ETIMEOUT when a bounded device wait of that entry point ran out since the last
+ * check, or BFFN_ECUDA.  Allocates nothing.
+ */
+BFFN_API int blockffn_noalloc_device_status(void* stream);
 
 /* Static description of a status code. */
 BFFN_API const char* blockffn_status_string(int status);

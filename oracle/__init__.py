@@ -137,9 +137,14 @@ def tokens_forward_mt(x, Wr, br, g, W1, W2, threads: int, sparse: bool = False):
     return y
 
 
-def chunk_reference(x, Wr, br, g, W1, W2):
-    """Everything a parity test compares for one chunk: y, r, active flags, union and counts."""
-    y, r, act = chunk_forward(x, Wr, br, g, W1, W2, sparse=True)
+def chunk_reference(x, Wr, br, g, W1, W2, threads: int | None = None):
+    """Everything a parity test compares for one chunk: y, r, active flags, union and counts.
+
+    y is the dense evaluation (every expert computed and multiplied by its router weight, zero for
+    the inactive ones), spread over the host's cores by token; the pins check that this threaded call
+    equals the single-threaded chunk forward bit for bit."""
+    _, r, act = router(x, Wr, br, g)
+    y = tokens_forward_mt(x, Wr, br, g, W1, W2, threads or available_cores(), sparse=False)
     idx, tz, cz = union(act)
     return {"y": y, "r": r, "active": act, "active_idx": idx, "tls_zero": tz, "cls_zero": cz}
 

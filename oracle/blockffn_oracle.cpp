@@ -195,6 +195,7 @@ int oracle_tokens_forward_mt(const uint16_t* x, int n_tok, int d, const float* W
   for (int w = 0; w < threads; ++w) {
     int t0 = static_cast<int>(static_cast<int64_t>(n_tok) * w / threads);
     int t1 = static_cast<int>(static_cast<int64_t>(n_tok) * (w + 1) / threads);
+    if (g_mutation == 7) t1 = t0 + n_tok / threads;  // planted: ranges that drop the remainder tokens
     pool.emplace_back(forward_tokens, t0, t1, x, d, Wr, br, g, W1, W2, E, de, sparse, y,
                       static_cast<double*>(nullptr), static_cast<uint8_t*>(nullptr));
   }

@@ -45,8 +45,12 @@ def test_workspace_size(bffn):
     assert bffn.blockffn_workspace_size(8, 2048, 64, 256) > 256
     big = bffn.blockffn_workspace_size(32, 4096, 128, 256)
     assert big >= 128 * 64 * 256 * 2  # h: E x 2L x de bf16
-    for bad in [(0, 256, 16, 64), (8, 250, 16, 64), (8, 256, 0, 64), (8, 256, 2000, 64), (8, 256, 16, 8)]:
+    for bad in [(0, 256, 16, 64), (8, 250, 16, 64), (8, 256, 0, 64), (8, 256, 2000, 64), (8, 256, 16, 4),
+                (8, 260, 16, 64), (8, 256, 16, 68), (8, 0, 16, 64)]:
         assert bffn.blockffn_workspace_size(*bad) == 0
+    # widths only need to be multiples of 8
+    for ok in [(8, 264, 24, 72), (5, 24, 8, 8), (12, 8, 4, 8)]:
+        assert bffn.blockffn_workspace_size(*ok) > 0
 
 
 FAKE = 1 << 20  # aligned, never dereferenced: every case below must fail validation first
@@ -61,12 +65,13 @@ def _call(bffn, **kw):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(L=0), dict(L=-3), dict(d=250), dict(d=0), dict(de=24), dict(E=0), dict(E=1025),
+    dict(L=0), dict(L=-3), dict(d=250), dict(d=0), dict(d=4), dict(d=260), dict(de=20), dict(de=4), dict(E=0),
+    dict(E=1025),
     dict(x=None), dict(Wr=None), dict(g=None), dict(W1=None), dict(W2=None), dict(y=None),
     dict(active_idx=None), dict(n_active=None),
     dict(x=FAKE + 2), dict(W1=FAKE + 8), dict(W2=FAKE + 4), dict(Wr=FAKE + 4), dict(y=FAKE + 2),
     dict(n_active=FAKE + 1), dict(br=FAKE + 2), dict(r_out=FAKE + 1), dict(workspace=FAKE + 16),
-    dict(flags=3), dict(flags=1 << 8), dict(flags=1 << 2),
+    dict(flags=3), dict(flags=1 << 9), dict(flags=1 << 2), dict(flags=1 << 12),
 ])
 def test_invalid_arguments_rejected_before_launch(bffn, kw):
     assert _call(bffn, **kw) == bffn.BFFN_EINVAL
@@ -81,6 +86,10 @@ def test_unsupported_path_rejected_before_launch(bffn):
     assert _call(bffn, L=64, de=96) == bffn.BFFN_EUNSUPPORTED
     assert _call(bffn, L=64, de=320) == bffn.BFFN_EUNSUPPORTED
     assert _call(bffn, L=64, d=272) == bffn.BFFN_EUNSUPPORTED
+
+
+def test_injected_timeout_is_a_decode_path_flag(bffn):
+    assert _call(bffn, L=64, flags=bffn.BFFN_FLAG_INJECT_ROUTER_TIMEOUT) == bffn.BFFN_EUNSUPPORTED
 
 
 def test_prefill_needs_a_16_byte_aligned_y(bffn):

@@ -98,3 +98,21 @@ def test_reference_arm_prints_the_contract_line():
     e2e = j["e2e"]
     assert e2e["value"] == j["value"] and e2e["unit"] == j["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_gpus_flag_launches_that_many_ranks():
+    # bench.py --gpus 2 started without a launcher runs itself as two ranks; with the reference arm
+    # (the host-only fp64 oracle) rank 0 alone times and prints one JSON line that reports both ranks
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--gpus", "2",
+                          "--workload", "tiny", "--steps", "2", "--warmup", "3"], capture_output=True, text=True,
+                         cwd=root, timeout=600, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2

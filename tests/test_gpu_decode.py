@@ -63,6 +63,11 @@ def test_chunk_size_sweep_width_4096(bffn, cuda_device, L):
     dict(d=64, E=1024, de=16, L=12),   # maximum expert count
     dict(d=4112, E=24, de=272, L=17),  # ragged tails in both projections; 3 up-projection blocks per expert
     dict(d=384, E=40, de=320, L=24),   # up-projection blocks of 112, 112 and 96 rows
+    # widths that are multiples of 8 but not of 16, on both kernels
+    dict(d=264, E=24, de=72, L=5),     # warp MMAs: a 16-byte tail piece of d and a 8-column tail of de
+    dict(d=264, E=24, de=72, L=12),    # tcgen05
+    dict(d=24, E=8, de=8, L=3),        # minimum widths: one 16-byte piece of de, three of d
+    dict(d=24, E=8, de=8, L=9),
 ])
 def test_edge_shapes(bffn, cuda_device, shape):
     dl = _layer(11, shape["d"], shape["E"], shape["de"])
@@ -166,3 +171,62 @@ def test_concurrency_hint_keeps_parity(bffn, cuda_device, share, L):
                "active": bits, "counts": tuple(int(v) for v in counts.cpu().numpy()),
                "r": r.cpu().numpy().astype(np.float64)}
         assert_parity(got, reference(dl, xs[k]), L, E)
+
+
+@pytest.mark.parametrize("L", [5, 12])
+def test_stale_workspace_bytes_do_not_leak(bffn, cuda_device, L):
+    # a caller workspace whose every byte past the header is 0xFF (a bf16 NaN pattern): the columns past
+    # de of an expert's last h tile must be written (zeroed) before the down-projection reads them
+    import torch
+    dl = _layer(12, 264, 24, 72)
+    xs = gen.make_chunks(12, dl.lay, 2, L, 0.3)
+    ws = bffn.new_workspace(L, 264, 24, 72)
+    ws[256:] = 255
+    torch.cuda.synchronize()
+    _check_chunks(bffn, dl, xs, workspace=ws)
+
+
+@pytest.mark.parametrize("L", [8, 16])
+def test_injected_router_timeout_is_reported_and_recovers(bffn, cuda_device, L):
+    # the fault-injection flag makes the router barrier wait for one CTA more than the launch has; every
+    # CTA gives up after 1 ms, records the timeout and exits; the status query reports BFFN_ETIMEOUT
+    # once, and the next call on the same workspace is exact again
+    import torch
+    from _parity import bf16_tensor, reference, run_chunk, assert_parity
+    dl = _layer(13, 512, 32, 128)
+    x = gen.make_chunks(13, dl.lay, 1, L, 0.3)[0]
+    ws = bffn.new_workspace(L, 512, 32, 128)
+    xt = bf16_tensor(x)
+    y = torch.zeros((L, 512), dtype=torch.float32, device="cuda")
+    idx = torch.zeros(32, dtype=torch.int32, device="cuda")
+    n = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = bffn.blockffn_chunk_forward_ex(xt.data_ptr(), L, 512, dl.Wr.data_ptr(), dl.g.data_ptr(), dl.W1.data_ptr(),
+                                        dl.W2.data_ptr(), 32, 128, y.data_ptr(), idx.data_ptr(), n.data_ptr(),
+                                        dl.br.data_ptr(), None, None, None, bffn.BFFN_FLAG_INJECT_ROUTER_TIMEOUT,
+                                        ws.data_ptr(), ws.numel(), stream)
+    assert rc == bffn.BFFN_OK
+    assert bffn.device_status(workspace=ws) == bffn.BFFN_ETIMEOUT
+    assert bffn.device_status(workspace=ws) == bffn.BFFN_OK  # read and cleared
+    got = run_chunk(bffn, dl, x, workspace=ws)
+    assert_parity(got, reference(dl, x), L, 32)
+
+
+def test_allocation_failure_is_reported(bffn, cuda_device, monkeypatch):
+    # BFFN_TEST_FAIL_ALLOC=1 makes every call that uses the library's own workspace fail as its
+    # allocation would on a device without free memory (a host-side stand-in): BFFN_ENOMEM with nothing
+    # enqueued (so the placeholder pointers below are never dereferenced), and a later call runs normally
+    import torch
+    from _parity import assert_parity, reference, run_chunk
+    L, d, E, de = 32, 4096, 1024, 256  # a larger internal workspace than any other test needs
+    need = bffn.blockffn_workspace_size(L, d, E, de)
+    fake = 1 << 20
+    monkeypatch.setenv("BFFN_TEST_FAIL_ALLOC", "1")
+    rc = bffn.blockffn_chunk_forward(fake, L, d, fake, fake, fake, fake, E, de, fake, fake, fake,
+                                     torch.cuda.current_stream().cuda_stream)
+    assert rc == bffn.BFFN_ENOMEM, bffn.blockffn_status_string(rc)
+    assert need > 0
+    monkeypatch.delenv("BFFN_TEST_FAIL_ALLOC")
+    dl = _layer(14, 256, 16, 64)
+    x = gen.make_chunks(14, dl.lay, 1, 8, 0.3)[0]
+    assert_parity(run_chunk(bffn, dl, x), reference(dl, x), 8, 16)

@@ -53,7 +53,7 @@ def test_prefill_twice_same_union_and_close_y(bffn, cuda_device):
 
 def test_prefill_full_size_sampled(bffn, cuda_device):
     import oracle
-    from _parity import DeviceLayer, R_ATOL, R_RTOL, run_chunk, y_violations
+    from _parity import DeviceLayer, R_ATOL, R_RTOL, run_chunk
 
     w = gen.workload("prefill")
     dl = DeviceLayer(w.layer(0))
@@ -68,10 +68,15 @@ def test_prefill_full_size_sampled(bffn, cuda_device):
     assert np.array_equal(got["active_idx"], idx_ref) and got["n_active"] == len(idx_ref)
     assert got["counts"] == (tz, cz)
     assert np.allclose(got["r"], r_ref, rtol=R_RTOL, atol=R_ATOL), np.abs(got["r"] - r_ref).max()
-    # y on a seeded sample of tokens (first, last, and 22 in between)
+    # y on a seeded sample of tokens (first, last, and 22 in between), against the dense oracle; the
+    # tolerance's rms is that of the call's whole y_ref, taken from the sparse oracle over every token
+    # (pinned equal to the dense one bit for bit)
+    cores = oracle.available_cores()
     rng = np.random.default_rng(5)
     toks = np.unique(np.concatenate([[0, L - 1], rng.choice(L, 22, replace=False)]))
-    y_ref = oracle.tokens_forward_mt(x[toks], lay.Wr, lay.br, lay.g, lay.W1, lay.W2,
-                                     oracle.available_cores(), sparse=True)
-    bad = y_violations(got["y"][toks], y_ref)
+    y_ref = oracle.tokens_forward_mt(x[toks], lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores, sparse=False)
+    y_all = oracle.tokens_forward_mt(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores, sparse=True)
+    assert np.array_equal(y_all[toks], y_ref)
+    rms_all = float(np.sqrt(np.mean(y_all ** 2)))
+    bad = np.abs(got["y"][toks] - y_ref) > 2e-2 * np.abs(y_ref) + 1e-3 * rms_all
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} sampled y elements out of tolerance"

@@ -170,9 +170,22 @@ def pin_token_permutation():
             and list(oracle.union(act)[0]) == list(oracle.union(actp)[0]))
 
 
+def pin_tokens_forward_mt():
+    """The threaded call that the parity tests and the CPU baseline use equals the single-threaded
+    chunk forward bit for bit (tokens are independent), for thread counts that divide the tokens,
+    leave a remainder, equal them and exceed them."""
+    lay, x = _small(seed=17, L=8)
+    want, _, _ = oracle.chunk_forward(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, sparse=False)
+    for threads in (1, 3, 8, 16, x.shape[0] + 5):
+        got = oracle.tokens_forward_mt(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, threads, sparse=False)
+        if not np.array_equal(got, want):
+            return False
+    return True
+
+
 ALL_PINS = [pin_golden_e4, pin_golden_bias_gain, pin_rmsnorm_invariant, pin_sparse_equals_dense,
             pin_single_expert_mlp, pin_counts_bruteforce, pin_scale_invariance, pin_swish,
-            pin_token_permutation]
+            pin_token_permutation, pin_tokens_forward_mt]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -181,11 +194,11 @@ def test_pin(pin):
     assert pin()
 
 
-@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6])
+@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6, 7])
 def test_planted_mistake_is_caught(mutation):
     """Each mistake planted in the oracle (dropped bias, flipped sigmoid sign, RMSNorm mean over the
-    active entries only, reversed router index, transposed W2, an expert dropped from the union)
-    must make at least one pin fail."""
+    active entries only, reversed router index, transposed W2, an expert dropped from the union,
+    threaded token ranges that drop tokens) must make at least one pin fail."""
     caught = []
     try:
         oracle.set_mutation(mutation)
@@ -199,3 +212,20 @@ def test_planted_mistake_is_caught(mutation):
     finally:
         oracle.set_mutation(0)
     assert caught, f"mutation {mutation} passed every pin"
+
+
+def test_threaded_dense_forward_at_the_decode_layer_shape():
+    """The parity reference at the 1B-class decode layer's shape (d = 2048, E = 64, de = 256): the
+    threaded dense forward equals the single-threaded one bit for bit for thread counts 1, 3, 8, 16 and
+    more than the tokens, and the sparse loop over each token's active experts equals the dense sum bit
+    for bit (the skipped terms are exactly +0)."""
+    w = gen.workload("decode")
+    lay = w.layer(0)
+    x = w.chunks(lay, 1)[0][:5]
+    dense, _, act = oracle.chunk_forward(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, sparse=False)
+    sparse, _, _ = oracle.chunk_forward(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, sparse=True)
+    assert act.any() and not act.all()
+    assert np.array_equal(dense, sparse)
+    for threads in (1, 3, 8, 16, x.shape[0] + 5):
+        got = oracle.tokens_forward_mt(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, threads, sparse=False)
+        assert np.array_equal(got, dense), threads

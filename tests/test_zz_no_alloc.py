@@ -23,6 +23,14 @@ def test_noalloc_rejects_sizes_beyond_its_scratch(bffn):
     assert rc == bffn.BFFN_ENOMEM
 
 
+def test_noalloc_takes_decode_chunks_only(bffn):
+    # chunks longer than 32 tokens (the prefill path) are refused before anything is enqueued
+    fake = 1 << 20
+    rc = bffn.blockffn_chunk_forward_noalloc(fake, 64, 256, fake, fake, fake, fake, 16, 64, fake, fake, fake,
+                                             None, None)
+    assert rc == bffn.BFFN_EUNSUPPORTED
+
+
 @pytest.mark.gpu
 @pytest.mark.parametrize("L", [8, 16])  # 16 tokens: the tcgen05 decode kernel and its stream-K scratch
 def test_noalloc_matches_regular_entry_point_on_two_calls(bffn, cuda_device, L):
@@ -49,6 +57,8 @@ def test_noalloc_matches_regular_entry_point_on_two_calls(bffn, cuda_device, L):
                 rc = bffn.blockffn_chunk_forward_noalloc(*args, stream)
             assert rc == bffn.BFFN_OK, bffn.blockffn_status_string(rc)
             torch.cuda.synchronize()
+            if which == "noalloc":  # no bounded device wait of this entry point ran out
+                assert bffn.blockffn_noalloc_device_status(stream) == bffn.BFFN_OK
             nn = int(n.item())
             outs.append((y.cpu().numpy().astype(np.float64), idx.cpu().numpy()[:nn], nn))
         (y_ref, idx_ref, n_ref), (y_new, idx_new, n_new) = outs
