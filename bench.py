@@ -1,11 +1,13 @@
 """Benchmark of the BlockFFN chunk-layer forward on B200.
 
 One step = one pass of the hot path over one batch of synthetic input: `chunks` chunk forwards
-(router + chunk union + sparse experts: one kernel per decode chunk, seven per prefill chunk) through
-the C ABI, chunk c using weight replica c % replicas.  The chunks are independent: chunk c is issued
-on stream c % K (--streams, default 8) with its own workspace and the concurrency hint, so K chunks
-run side by side, each on 1/K of the SMs, and one chunk's fixed latencies overlap the others' weight
-streaming.  The replicas stand for distinct layers of a stacked model and keep
+(router + chunk union + sparse experts) through the C ABI, chunk c using weight replica c % replicas.
+Decode chunks of up to 8 tokens go through one batched call per step (two launches: the router of
+every chunk, then a persistent expert kernel whose SMs form K = --streams teams, team k taking chunks
+k, k + K, ...).  With --mode streams (and for longer chunks) chunk c is issued on stream c % K with
+its own workspace and the concurrency hint, so K chunks run side by side, each on 1/K of the SMs.
+Decode lines also time one chunk at a time on the whole GPU (roofline.single_chunk).  The replicas
+stand for distinct layers of a stacked model and keep
 the weights (16 x 128 MiB for the default workload) well above the 126 MB L2, so every chunk streams
 its active experts from HBM ("inputs larger than L2").  A step is captured once into a CUDA graph
 and replayed; time is taken with CUDA events on the replay stream, with a barrier and a
@@ -178,29 +180,38 @@ def active_bytes(d, E, de, L, n_active):
 
 
 def build_inputs(w, rank, device, chunks):
+    """The workload's weight replicas stacked one after another on the device (W1 [R, E, de, d] and so
+    on, the layout the batched call takes; layers[r] holds views of replica r for the per-chunk call),
+    and the chunks on the host: chunk c uses replica c % R."""
     import numpy as np
     import torch
 
     import gen
 
-    def bf16(a):
-        return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(device).view(torch.bfloat16)
-
+    R, d, E, de = w.replicas, w.d, w.E, w.de
+    stack = {"Wr": torch.empty((R, d, E), dtype=torch.float32, device=device),
+             "br": torch.empty((R, E), dtype=torch.float32, device=device),
+             "g": torch.empty((R, E), dtype=torch.float32, device=device),
+             "W1": torch.empty((R, E, de, d), dtype=torch.bfloat16, device=device),
+             "W2": torch.empty((R, E, d, de), dtype=torch.bfloat16, device=device)}
     layers = []
     host_x = []
-    per = (chunks + w.replicas - 1) // w.replicas
-    for r in range(w.replicas):
+    per = (chunks + R - 1) // R
+    for r in range(R):
         lay = w.layer(r)
-        layers.append({
-            "lay": lay,
-            "Wr": torch.from_numpy(lay.Wr).to(device), "br": torch.from_numpy(lay.br).to(device),
-            "g": torch.from_numpy(lay.g).to(device), "W1": bf16(lay.W1), "W2": bf16(lay.W2)})
+        stack["Wr"][r].copy_(torch.from_numpy(lay.Wr))
+        stack["br"][r].copy_(torch.from_numpy(lay.br))
+        stack["g"][r].copy_(torch.from_numpy(lay.g))
+        stack["W1"][r].view(torch.int16).copy_(torch.from_numpy(lay.W1.view(np.int16)))
+        stack["W2"][r].view(torch.int16).copy_(torch.from_numpy(lay.W2.view(np.int16)))
+        layers.append({"lay": lay if r == 0 else None, **{k: v[r] for k, v in stack.items()}})
         host_x.append(gen.make_chunks(shard_seed(w.seed, rank), lay, per, w.L, w.noise, stream=r))
+        del lay
     # chunk c -> replica c % R, position c // R within that replica's stream
     x_all = np.empty((chunks, w.L, w.d), dtype=np.uint16)
     for c in range(chunks):
-        x_all[c] = host_x[c % w.replicas][c // w.replicas]
-    return layers, x_all
+        x_all[c] = host_x[c % R][c // R]
+    return layers, stack, x_all
 
 
 # ---------------------------------------------------------------------------------- our arm
@@ -220,24 +231,40 @@ def run_ours(args, w):
 
     chunks = args.chunks or w.n_chunks
     t_gen = time.time()
-    layers, x_host_np = build_inputs(w, rank, device, chunks)
+    layers, stack, x_host_np = build_inputs(w, rank, device, chunks)
     gen_s = time.time() - t_gen
     L, d, E, de = w.L, w.d, w.E, w.de
     x_dev = torch.from_numpy(x_host_np.view(np.int16)).to(device).view(torch.bfloat16)
     y = torch.empty((chunks, L, d), dtype=torch.float32, device=device)
     idx = torch.empty((chunks, E), dtype=torch.int32, device=device)
-    nact = torch.empty((chunks, 4), dtype=torch.int32, device=device)  # [c, 0] used
+    nact = torch.empty((chunks,), dtype=torch.int32, device=device)
     cnts = torch.empty((chunks, 2), dtype=torch.int32, device=device)  # TLS / CLS zero counts
 
-    # K streams, each with its own workspace: chunk c goes to stream c % K, and with K > 1 each call
-    # takes 1/K of the SMs (decode), so K independent chunks run side by side.
+    # Decode chunks of up to 8 tokens (default): the batched call, all chunks of a step in two launches,
+    # the SMs in K teams (--streams), team k taking chunks k, k + K, ...; chunk c uses replica c % R.
+    # Otherwise (--mode streams, longer chunks, prefill): K streams, each with its own workspace: chunk c
+    # goes to stream c % K, and with K > 1 each call takes 1/K of the SMs, so K chunks run side by side.
+    batched = args.mode == "batch" and L <= 8
     K = max(1, args.streams if L <= DECODE_MAX_L else 1)
     flags = bffn.BFFN_FLAGS_SHARE(K) if K > 1 else 0
-    ws_bytes = bffn.blockffn_workspace_size(L, d, E, de)
-    workspaces = [bffn.new_workspace(L, d, E, de, device) for _ in range(K)]  # zero-filled, 512-byte aligned
+    if batched:
+        ws_bytes = bffn.blockffn_batch_workspace_size(chunks, L, d, E, de, flags)
+        workspaces = [torch.zeros(ws_bytes, dtype=torch.uint8, device=device)]
+    else:
+        ws_bytes = bffn.blockffn_workspace_size(L, d, E, de)
+        workspaces = [bffn.new_workspace(L, d, E, de, device) for _ in range(K)]  # zero-filled
     ws_ptrs = [t.data_ptr() for t in workspaces]
 
     def step(streams):
+        if batched:
+            rc = bffn.blockffn_chunk_forward_batch(
+                x_dev.data_ptr(), chunks, L, d, None, w.replicas, stack["Wr"].data_ptr(), stack["g"].data_ptr(),
+                stack["br"].data_ptr(), stack["W1"].data_ptr(), stack["W2"].data_ptr(), E, de, y.data_ptr(),
+                idx.data_ptr(), nact.data_ptr(), cnts.data_ptr(), None, flags, ws_ptrs[0], ws_bytes,
+                streams[0].cuda_stream)
+            if rc != 0:
+                raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_batch")
+            return
         if K > 1:  # fork: the side streams start after everything queued on the main one
             ev = torch.cuda.Event()
             ev.record(streams[0])
@@ -248,7 +275,7 @@ def run_ours(args, w):
             k = c % K
             rc = bffn.blockffn_chunk_forward_ex(
                 x_dev[c].data_ptr(), L, d, lay["Wr"].data_ptr(), lay["g"].data_ptr(), lay["W1"].data_ptr(),
-                lay["W2"].data_ptr(), E, de, y[c].data_ptr(), idx[c].data_ptr(), nact[c].data_ptr(),
+                lay["W2"].data_ptr(), E, de, y[c].data_ptr(), idx[c].data_ptr(), nact[c:].data_ptr(),
                 lay["br"].data_ptr(), None, cnts[c].data_ptr(), None, flags, ws_ptrs[k], ws_bytes,
                 streams[k].cuda_stream)
             if rc != 0:
@@ -260,13 +287,13 @@ def run_ours(args, w):
                 streams[0].wait_event(ev)
 
     s = torch.cuda.Stream(device)
-    side = [torch.cuda.Stream(device) for _ in range(K - 1)]
+    side = [torch.cuda.Stream(device) for _ in range(0 if batched else K - 1)]
     streams = [s] + side
     with torch.cuda.stream(s):
         step(streams)
         s.synchronize()
-        for k in range(K):
-            if bffn.device_status(workspace=workspaces[k], stream=s.cuda_stream) != 0:
+        for ws in workspaces:
+            if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
                 raise RuntimeError("device-side wait ran out")
         graph = torch.cuda.CUDAGraph()
         graph.capture_begin()
@@ -289,8 +316,8 @@ def run_ours(args, w):
         torch.cuda.synchronize(device)
         barrier(device)
         t_ms = e0.elapsed_time(e1)
-        for k in range(K):
-            if bffn.device_status(workspace=workspaces[k], stream=s.cuda_stream) != 0:
+        for ws in workspaces:
+            if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
                 raise RuntimeError("device-side wait ran out during the timed region")
 
         # end to end: x from pinned host memory in, y and the active sets back, every step
@@ -322,9 +349,57 @@ def run_ours(args, w):
         barrier(device)
         e2e_ms = f0.elapsed_time(f1)
 
+        # one chunk at a time on the whole GPU (the latency a verification step sees per layer): the
+        # first n1 chunks through the per-chunk entry point on one stream, as one graph
+        single = None
+        if L <= DECODE_MAX_L:
+            n1 = min(chunks, 512)
+            ws1 = bffn.new_workspace(L, d, E, de, device)
+            ws1_bytes = bffn.blockffn_workspace_size(L, d, E, de)
+            y1 = torch.empty((n1, L, d), dtype=torch.float32, device=device)
+            i1 = torch.empty((n1, E), dtype=torch.int32, device=device)
+            c1 = torch.empty((n1, 2), dtype=torch.int32, device=device)
+            n1a = torch.empty((n1,), dtype=torch.int32, device=device)
+
+            def single_step():
+                for c in range(n1):
+                    lay = layers[c % w.replicas]
+                    rc = bffn.blockffn_chunk_forward_ex(
+                        x_dev[c].data_ptr(), L, d, lay["Wr"].data_ptr(), lay["g"].data_ptr(), lay["W1"].data_ptr(),
+                        lay["W2"].data_ptr(), E, de, y1[c].data_ptr(), i1[c].data_ptr(), n1a[c:].data_ptr(),
+                        lay["br"].data_ptr(), None, c1[c].data_ptr(), None, 0, ws1.data_ptr(), ws1_bytes,
+                        s.cuda_stream)
+                    if rc != 0:
+                        raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_ex")
+
+            single_step()
+            s.synchronize()
+            g1 = torch.cuda.CUDAGraph()
+            g1.capture_begin()
+            single_step()
+            g1.capture_end()
+            for _ in range(3):
+                g1.replay()
+            s.synchronize()
+            h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            reps = 5
+            h0.record(s)
+            for _ in range(reps):
+                g1.replay()
+            h1.record(s)
+            h1.synchronize()
+            if bffn.device_status(workspace=ws1, stream=s.cuda_stream) != 0:
+                raise RuntimeError("device-side wait ran out (single-chunk timing)")
+            us1 = h0.elapsed_time(h1) * 1e3 / (reps * n1)
+            b1 = float(sum(active_bytes(d, E, de, L, int(n)) for n in n1a.cpu().numpy())) / n1
+            single = {"us_per_chunk": round(us1, 3), "tokens_per_s": round(L / (us1 * 1e-6), 1),
+                      "achieved_gbs": round(b1 / (us1 * 1e-6) / 1e9, 1), "chunks": n1,
+                      "entry_point": "blockffn_chunk_forward_ex, whole GPU, one chunk at a time"}
+            del g1
+
     t_max = reduce_max(t_ms, device)
     e2e_max = reduce_max(e2e_ms, device)
-    n_act_host = nact[:, 0].cpu().numpy()
+    n_act_host = nact.cpu().numpy()
     pairs_host = L * E - cnts[:, 0].cpu().numpy().astype(np.int64)
     prefill = L > DECODE_MAX_L
     total_active = float(sum(active_bytes(d, E, de, L, int(n)) for n in n_act_host))
@@ -346,12 +421,16 @@ def run_ours(args, w):
                     "pairs_per_chunk": round(float(pairs_host.mean()), 1),
                     "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3), "traffic": None}
     else:
+        kname = ("batch_expert_kernel + batch_router_kernel: every chunk of the step in two launches (time "
+                 "of both counted)" if batched else "expert_decode_kernel: one chunk forward, router included")
         roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peak, "unit": "GB/s",
-                    "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind,
-                    "kernel": "expert_decode_kernel: one chunk forward, router included",
+                    "frac": round(achieved_gbs / peak, 4), "peak_kind": peak_kind, "kernel": kname,
                     "bytes_per_chunk": round(total_active / chunks, 1),
                     "us_per_chunk": round(ms_per_step * 1e3 / chunks, 3),
                     "traffic": None if traffic is None else round(traffic, 1)}
+        if single is not None:
+            single["frac"] = round(single["achieved_gbs"] / peak, 4)
+            roofline["single_chunk"] = single
     out = {
         "metric": METRIC_PREFILL if prefill else METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -363,13 +442,14 @@ def run_ours(args, w):
                    "mean_n_active": round(float(n_act_host.mean()), 3),
                    "cls": round(1.0 - float(n_act_host.mean()) / E, 4),
                    "parallelism": f"dp{world} (chunks sharded, no collective in the data path)",
+                   "mode": "batch" if batched else "streams",
                    "concurrent_chunks": K},
         "roofline": roofline,
         "e2e": {"value": round(tokens_step / (e2e_max / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host_np.nbytes),
                 "d2h_bytes_per_step": int(y.numel() * 4 + idx.numel() * 4 + nact.numel() * 4),
                 "steps": e2e_steps},
-        "gpu_launches": (7 if prefill else 1) * chunks * args.steps,
+        "gpu_launches": (2 if batched else (7 if prefill else 1) * chunks) * args.steps,
         "clocks": clk.summary(),
         "gen_seconds": round(gen_s, 1),
     }
@@ -381,6 +461,130 @@ def run_ours(args, w):
     del graph
     if world > 1:
         dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------------- sparsity sweep
+def run_tls_sweep(args):
+    """Config 4 of the measurement plan: a stacked model FFN of `--replicas` layers (default 32: d=4096,
+    E=128, de=256, 17.2 GB of bf16 expert weights), L=8 chunks, one batched call per step through all
+    layers (chunk c on layer c % layers).  The router bias is set per point for token-level sparsity
+    TLS in --tls-list, the chunk-level sparsity is measured, and a dense point forces every expert
+    active (bias +50) on the same layers, through the same kernels.  One JSON line per point; the
+    sparse points carry their speedup over the dense point next to the bound 1 / (1 - CLS)."""
+    import numpy as np
+    import torch
+
+    import chunk_sparse_moe_router_b200 as bffn
+    import gen
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    base = gen.workload("tls_sweep")
+    R = args.replicas or base.replicas
+    d, E, de, L = base.d, base.E, base.de, base.L
+    C = args.chunks or 8 * R
+    K = args.streams
+    t_gen = time.time()
+    W1 = torch.empty((R, E, de, d), dtype=torch.bfloat16, device=device)
+    W2 = torch.empty((R, E, d, de), dtype=torch.bfloat16, device=device)
+    Wr = torch.empty((R, d, E), dtype=torch.float32, device=device)
+    g = torch.empty((R, E), dtype=torch.float32, device=device)
+    host = []  # per layer: Wr (for the bias scale and the margin test)
+    for r in range(R):
+        lay = base.layer(r)
+        W1[r].view(torch.int16).copy_(torch.from_numpy(lay.W1.view(np.int16)))
+        W2[r].view(torch.int16).copy_(torch.from_numpy(lay.W2.view(np.int16)))
+        Wr[r].copy_(torch.from_numpy(lay.Wr))
+        g[r].copy_(torch.from_numpy(lay.g))
+        lay.W1 = lay.W2 = None
+        host.append(lay)
+    gen_s = time.time() - t_gen
+    peak, peak_kind = measured_peaks()
+    points = [p.strip() for p in args.tls_list.split(",")]
+    # the dense point first, so that every sparse line can quote its speedup over it
+    points = ["dense"] + [p for p in points if p != "dense"]
+    flags = bffn.BFFN_FLAGS_SHARE(K)
+    ws_bytes = bffn.blockffn_batch_workspace_size(C, L, d, E, de, flags)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=device)
+    y = torch.empty((C, L, d), dtype=torch.float32, device=device)
+    idx = torch.empty((C, E), dtype=torch.int32, device=device)
+    nact = torch.empty((C,), dtype=torch.int32, device=device)
+    cnts = torch.empty((C, 2), dtype=torch.int32, device=device)
+    dense_tps = None
+    s = torch.cuda.Stream(device)
+    for pt in points:
+        dense = pt == "dense"
+        tls = 0.5 if dense else float(pt)
+        beta = gen.beta_for_tls(tls)
+        br = torch.empty((R, E), dtype=torch.float32, device=device)
+        per = C // R
+        x_host = np.empty((C, L, d), dtype=np.uint16)
+        for r in range(R):
+            lay = host[r]
+            sigma = np.sqrt(lay.var_x * np.sum(lay.Wr.astype(np.float64) ** 2, axis=0))
+            lay.br = np.full(E, 50.0, np.float32) if dense else (-beta * sigma).astype(np.float32)
+            br[r].copy_(torch.from_numpy(lay.br))
+            xs = gen.make_chunks(base.seed, lay, per, L, base.noise, stream=r)
+            for q in range(per):
+                x_host[q * R + r] = xs[q]
+        x = torch.from_numpy(x_host.view(np.int16)).to(device).view(torch.bfloat16)
+
+        def step():
+            rc = bffn.blockffn_chunk_forward_batch(
+                x.data_ptr(), C, L, d, None, R, Wr.data_ptr(), g.data_ptr(), br.data_ptr(), W1.data_ptr(),
+                W2.data_ptr(), E, de, y.data_ptr(), idx.data_ptr(), nact.data_ptr(), cnts.data_ptr(), None, flags,
+                ws.data_ptr(), ws_bytes, s.cuda_stream)
+            if rc != 0:
+                raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_batch")
+
+        with torch.cuda.stream(s):
+            step()
+            s.synchronize()
+            if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
+                raise RuntimeError("device-side wait ran out")
+            graph = torch.cuda.CUDAGraph()
+            graph.capture_begin()
+            step()
+            graph.capture_end()
+            for _ in range(args.warmup):
+                graph.replay()
+            s.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(0) as clk:
+                e0.record(s)
+                for _ in range(args.steps):
+                    graph.replay()
+                e1.record(s)
+                e1.synchronize()
+            if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
+                raise RuntimeError("device-side wait ran out during the timed region")
+            del graph
+        ms = e0.elapsed_time(e1) / args.steps
+        n_host = nact.cpu().numpy()
+        zeros = cnts[:, 0].cpu().numpy().astype(np.float64)
+        total = float(sum(active_bytes(d, E, de, L, int(n)) for n in n_host))
+        tps = C * L / (ms * 1e-3)
+        gbs = total / (ms * 1e-3) / 1e9
+        cls = 1.0 - float(n_host.mean()) / E
+        line = {"metric": METRIC, "value": round(tps, 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"tls_sweep_{R}layers_d{d}_E{E}_de{de}_L{L}",
+                           "point": "dense (every expert active)" if dense else f"tls {tls}",
+                           "layers": R, "chunks_per_step": C, "teams": K,
+                           "weights_gb": round(R * E * 2 * d * de * 2 / 1e9, 2),
+                           "tls_measured": round(float(zeros.mean()) / (L * E), 4), "cls_measured": round(cls, 4),
+                           "mean_n_active": round(float(n_host.mean()), 3)},
+                "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                             "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                             "us_per_chunk": round(ms * 1e3 / C, 3)},
+                "gpu_launches": 2 * args.steps, "clocks": clk.summary(), "gen_seconds": round(gen_s, 1)}
+        if dense:
+            dense_tps = tps
+        else:
+            line["speedup_vs_dense"] = round(tps / dense_tps, 3)
+            line["speedup_bound"] = round(1.0 / max(1e-9, 1.0 - cls), 3)
+        print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------------------------- CPU oracle
@@ -479,10 +683,15 @@ def main():
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
     ap.add_argument("--tls", type=float, default=None, help="token-level sparsity for --workload tls_sweep")
     ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")
+    ap.add_argument("--tls-list", default="0.5,0.7,0.8,0.9,0.95",
+                    help="--workload tls_sweep: the token-level sparsity points (a dense point is always added)")
     ap.add_argument("--replicas", type=int, default=None,
                     help="weight replicas (default: the workload's; keep their weights above the 126 MB L2)")
     ap.add_argument("--streams", type=int, default=8,
-                    help="decode: independent chunks in flight at once, each on 1/streams of the SMs")
+                    help="decode: independent chunks in flight at once (teams of SMs), each on 1/streams of them")
+    ap.add_argument("--mode", choices=["batch", "streams"], default="batch",
+                    help="decode chunks of up to 8 tokens: one batched call per step (default), or one call per "
+                         "chunk on --streams streams")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-chunks", type=int, default=1)
@@ -503,6 +712,9 @@ def main():
         kw["tls"] = args.tls
     if args.replicas:
         kw["replicas"] = args.replicas
+    if args.workload == "tls_sweep" and args.impl == "ours" and not args.tls:
+        run_tls_sweep(args)
+        return
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":
         run_reference(args, w)

@@ -34,6 +34,9 @@ SIGNATURES = {
                                        _P, _I, _P, _S, _P]),
     "blockffn_chunk_forward_noalloc": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P]),
     "blockffn_noalloc_device_status": (_I, [_P]),
+    "blockffn_chunk_forward_batch": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P,
+                                         _I, _P, _S, _P]),
+    "blockffn_batch_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_init": (_I, [_P, _S, _P]),
     "blockffn_device_status": (_I, [_P, _P]),
@@ -74,6 +77,16 @@ def blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_ac
     return _lib.blockffn_chunk_forward_ex(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br,
                                           tok_mask, counts, r_out, flags, workspace, workspace_bytes,
                                           stream)
+
+
+def blockffn_chunk_forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx, n_active,
+                                 counts, tok_mask, flags, workspace, workspace_bytes, stream):
+    return _lib.blockffn_chunk_forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx,
+                                             n_active, counts, tok_mask, flags, workspace, workspace_bytes, stream)
+
+
+def blockffn_batch_workspace_size(C, L, d, E, de, flags):
+    return _lib.blockffn_batch_workspace_size(C, L, d, E, de, flags)
 
 
 def blockffn_chunk_forward_noalloc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, stream):
@@ -158,6 +171,54 @@ def chunk_forward(x, Wr, g, W1, W2, y, active_idx, n_active, br=None, tok_mask=N
                                    _ptr(counts), _ptr(r_out), int(path), ws_ptr, ws_bytes, stream)
     if rc != BFFN_OK:
         raise BlockFFNError(rc, "blockffn_chunk_forward_ex")
+
+
+def chunk_forward_batch(x, Wr, g, W1, W2, y, active_idx, n_active, layer=None, br=None, counts=None,
+                        tok_mask=None, teams=0, workspace=None, stream=None):
+    """C independent chunks in one call: x bf16 [C,L,d]; stacked weights Wr fp32 [n_layers,d,E],
+    g fp32 [n_layers,E], W1 bf16 [n_layers,E,de,d], W2 bf16 [n_layers,E,d,de] (br fp32 [n_layers,E]);
+    layer int32 [C] (None: chunk c uses layer c % n_layers); outputs y fp32 [C,L,d], active_idx int32
+    [C,E], n_active int32 [C] (+ counts int32 [C,2], tok_mask int32 [C,L,ceil(E/32)]).  teams = k of
+    BFFN_FLAGS_SHARE (0: the default).  Raises BlockFFNError."""
+    import torch
+
+    C, L, d = x.shape
+    nl, E, de = W1.shape[0], W1.shape[1], W1.shape[2]
+    dev = x.device
+    _check(x, "x", torch.bfloat16, (C, L, d), dev)
+    _check(Wr, "Wr", torch.float32, (nl, d, E), dev)
+    _check(g, "g", torch.float32, (nl, E), dev)
+    _check(W1, "W1", torch.bfloat16, (nl, E, de, d), dev)
+    _check(W2, "W2", torch.bfloat16, (nl, E, d, de), dev)
+    _check(y, "y", torch.float32, (C, L, d), dev)
+    _check(active_idx, "active_idx", torch.int32, (C, E), dev)
+    _check(n_active, "n_active", torch.int32, (C,), dev)
+    if layer is not None:
+        _check(layer, "layer", torch.int32, (C,), dev)
+    if br is not None:
+        _check(br, "br", torch.float32, (nl, E), dev)
+    if counts is not None:
+        _check(counts, "counts", torch.int32, (C, 2), dev)
+    if tok_mask is not None:
+        _check(tok_mask, "tok_mask", torch.int32, (C, L, (E + 31) // 32), dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    rc = blockffn_chunk_forward_batch(_ptr(x), C, L, d, _ptr(layer), nl, _ptr(Wr), _ptr(g), _ptr(br), _ptr(W1),
+                                      _ptr(W2), E, de, _ptr(y), _ptr(active_idx), _ptr(n_active), _ptr(counts),
+                                      _ptr(tok_mask), BFFN_FLAGS_SHARE(teams), ws_ptr, ws_bytes, stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_chunk_forward_batch")
+
+
+def new_batch_workspace(C, L, d, E, de, teams=0, device="cuda"):
+    """A zero-filled caller-owned workspace for blockffn_chunk_forward_batch."""
+    import torch
+
+    n = blockffn_batch_workspace_size(C, L, d, E, de, BFFN_FLAGS_SHARE(teams))
+    if n == 0:
+        raise BlockFFNError(BFFN_EINVAL, "blockffn_batch_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
 def device_status(workspace=None, stream=None):

@@ -330,6 +330,71 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
   return BFFN_OK;
 }
 
+int forward_batch(const void* x, int C, int L, int d, const int32_t* layer, int n_layers, const float* Wr,
+                  const float* g, const float* br, const void* W1, const void* W2, int E, int de, float* y,
+                  int32_t* active_idx, int32_t* n_active, int32_t* counts, uint32_t* tok_mask, int teams, void* ws,
+                  const DeviceInfo& di, cudaStream_t st) {
+  batch::Params p;
+  batch::Launch launch;
+  if (!batch::plan(C, L, d, E, de, teams, di.num_sms, di.max_smem, &p, &launch)) return BFFN_EUNSUPPORTED;
+  {
+    int per_sm = 0;  // the team barriers need every CTA of a team resident at once
+    const cudaError_t oe = batch::occupancy(launch.smem, &per_sm);
+    if (oe != cudaSuccess) return cuda_fail(oe);
+    if (per_sm < 1) return BFFN_EUNSUPPORTED;
+  }
+  const batch::Layout lay = batch::layout(C, L, E, de, teams);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  p.x = static_cast<const __nv_bfloat16*>(x);
+  p.layer = layer;
+  p.Wr = Wr;
+  p.g = g;
+  p.br = br;
+  p.y = y;
+  p.active_idx = active_idx;
+  p.n_active = n_active;
+  p.counts = counts;
+  p.tok_mask = tok_mask;
+  p.r = reinterpret_cast<float*>(base + lay.r_off);
+  p.h = base + lay.h_off;
+  p.chunk_bar = reinterpret_cast<uint32_t*>(base + lay.bar_off);
+  p.hdr = reinterpret_cast<WsHeader*>(base);
+  p.C = C;
+  p.L = L;
+  p.d = d;
+  p.E = E;
+  p.de = de;
+  p.n_layers = n_layers;
+  batch::Maps m;
+  {
+    const uint64_t NE = uint64_t(n_layers) * E;
+    const uint64_t w1d[3] = {uint64_t(d), uint64_t(de), NE}, w1s[2] = {uint64_t(d) * 2, uint64_t(d) * de * 2};
+    const uint64_t w2d[3] = {uint64_t(de), uint64_t(d), NE}, w2s[2] = {uint64_t(de) * 2, uint64_t(d) * de * 2};
+    for (int k = 0; k < 5; ++k) {
+      const uint32_t b[3] = {64, uint32_t(8u << k), 1};
+      if (!encode_bf16(&m.w1[k], W1, 3, w1d, w1s, b)) return BFFN_ECUDA;
+      if (!encode_bf16(&m.w2[k], W2, 3, w2d, w2s, b)) return BFFN_ECUDA;
+    }
+    const uint64_t xd[3] = {uint64_t(d), uint64_t(L), uint64_t(C)}, xs[2] = {uint64_t(d) * 2, uint64_t(L) * d * 2};
+    const uint32_t xb[3] = {64, 8, 1};
+    if (!encode_bf16(&m.x, x, 3, xd, xs, xb)) return BFFN_ECUDA;
+  }
+  const cudaError_t err = batch::launch(p, m, launch, st);
+  if (err != cudaSuccess) return cuda_fail(err);
+  return BFFN_OK;
+}
+
+bool batch_args_ok(int C, int L, int d, int n_layers, int E, int de) {
+  return C >= 1 && n_layers >= 1 && shapes_ok(L, d, E, de) && (long long)n_layers * E < (1ll << 31) &&
+         (long long)C * L * d < (1ll << 40) && (long long)n_layers * E * de * d < (1ll << 40);
+}
+
+int batch_teams(int flags, int C) {
+  const int k = (flags >> 4) & 15;
+  if (k != 0) return k;
+  return C < 8 ? C : 8;
+}
+
 }  // namespace
 }  // namespace bffn
 
@@ -422,6 +487,47 @@ int blockffn_chunk_forward(const void* x, int L, int d, const float* Wr, const f
                                    nullptr, nullptr, nullptr, BFFN_PATH_AUTO, nullptr, 0, stream);
 }
 
+size_t blockffn_batch_workspace_size(int C, int L, int d, int E, int de, int flags) {
+  if (!batch_args_ok(C, L, d, 1, E, de) || (flags & ~0xF0) != 0) return 0;
+  return batch::layout(C, L, E, de, batch_teams(flags, C)).total;
+}
+
+int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, const int32_t* layer, int n_layers,
+                                 const float* Wr, const float* g, const float* br, const void* W1, const void* W2,
+                                 int E, int de, float* y, int32_t* active_idx, int32_t* n_active, int32_t* counts,
+                                 uint32_t* tok_mask, int flags, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  if (!batch_args_ok(C, L, d, n_layers, E, de)) return BFFN_EINVAL;
+  if ((flags & ~0xF0) != 0) return BFFN_EINVAL;
+  const void* bulk[] = {x, Wr, W1, W2};
+  for (const void* p : bulk)
+    if (p == nullptr || !aligned16(p)) return BFFN_EINVAL;
+  const void* scalar[] = {g, y, active_idx, n_active};
+  for (const void* p : scalar)
+    if (p == nullptr || !aligned4(p)) return BFFN_EINVAL;
+  const void* optional[] = {layer, br, counts, tok_mask};
+  for (const void* p : optional)
+    if (p != nullptr && !aligned4(p)) return BFFN_EINVAL;
+  if (workspace != nullptr && !aligned256(workspace)) return BFFN_EINVAL;
+  if (L > batch::kMaxL) return BFFN_EUNSUPPORTED;
+  const int teams = batch_teams(flags, C);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DeviceInfo di;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != BFFN_OK) return rc;
+  const size_t need = batch::layout(C, L, E, de, teams).total;
+  void* ws = workspace;
+  if (ws == nullptr) {
+    rc = internal_workspace(dev, need, st, &ws);
+    if (rc != BFFN_OK) return rc;
+  } else if (workspace_bytes < need) {
+    return BFFN_ENOMEM;
+  }
+  return forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx, n_active, counts,
+                       tok_mask, teams, ws, di, st);
+}
+
 int blockffn_device_status(void* workspace, void* stream) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t err = cudaStreamSynchronize(st);
@@ -442,7 +548,8 @@ int blockffn_device_status(void* workspace, void* stream) {
   if ((err = cudaMemcpy(reinterpret_cast<uint8_t*>(ws) + offsetof(WsHeader, err), &zero, sizeof zero,
                         cudaMemcpyHostToDevice)) != cudaSuccess)
     return cuda_fail(err);
-  return BFFN_ETIMEOUT;
+  // a wait that ran out outranks a bad layer index (both may be recorded)
+  return (h.err & ~uint32_t(kErrBadLayer)) != 0 ? BFFN_ETIMEOUT : BFFN_EINVAL;
 }
 
 }  // extern "C"

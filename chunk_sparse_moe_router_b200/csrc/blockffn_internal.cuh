@@ -22,6 +22,8 @@ enum : uint32_t {
   kErrRingWait = 2u,      // expert kernel: waiting on a shared-memory ring barrier
   kErrPrefillWait = 4u,   // prefill GEMMs: waiting on a shared-memory barrier
   kErrRouterBarrier = 8u, // expert kernel: waiting for every CTA's router partial sums
+  kErrTeamBarrier = 16u,  // batched expert kernel: waiting for the team's up-projections
+  kErrBadLayer = 32u,     // batched router kernel: a chunk's layer index was outside [0, n_layers)
 };
 
 // First 256 bytes of every workspace.
@@ -254,6 +256,72 @@ cudaError_t launch(const Params& p, const Maps& tm, const Launch& plan, cudaStre
 // SM at once.
 cudaError_t occupancy(int L, size_t smem, int* ctas_per_sm);
 }  // namespace tcdec
+
+// ------------------------------------------------------------------------ batched decode (decode_batch.cu)
+// Many independent chunks of up to 8 tokens in two launches: a router kernel (one CTA per chunk: s,
+// the RMSNorm statistics, masks, union and counts of every chunk) and a persistent expert kernel whose
+// CTAs form `teams` teams of T; team k takes chunks k, k + teams, ... in order, and its CTAs split each
+// chunk's rows.  Weights of several layers are stacked: W1 [n_layers E, de, d], W2 [n_layers E, d, de].
+namespace batch {
+constexpr int kMaxL = 8;          // tokens per chunk (the MMA's N)
+constexpr int kHTile = 16 * 128;  // h tile of one 64-wide j chunk: 8 hi rows, then 8 lo rows, of 128 B
+constexpr int kMaxRowsB = 256;    // y rows per CTA (16 m-tiles of 16, two per consumer warp)
+constexpr int kMaxTeams = 15;
+constexpr int kHImagesPerTeam = 4;  // h images per team (the expert kernel's schedule keeps four in use)
+
+struct Params {
+  const __nv_bfloat16* x;   // [C, L, d]
+  const int32_t* layer;     // [C] weight set of each chunk, or null: chunk c uses c % n_layers
+  const float* Wr;          // [n_layers, d, E]
+  const float* g;           // [n_layers, E]
+  const float* br;          // [n_layers, E] or null
+  float* y;                 // [C, L, d]
+  int32_t* active_idx;      // [C, E]
+  int32_t* n_active;        // [C]
+  int32_t* counts;          // [C, 2] or null
+  uint32_t* tok_mask;       // [C, L, ceil(E/32)] or null
+  float* r;                 // [C, L, E] router outputs (workspace)
+  uint8_t* h;               // [teams][kHImagesPerTeam][E][nJc][kHTile] h images (workspace)
+  uint32_t* chunk_bar;      // [C] CTAs whose up-projection of the chunk is published (workspace; zeroed by
+                            // the router kernel)
+  WsHeader* hdr;
+  int C, L, d, E, de, n_layers;
+  int teams, T;             // teams, CTAs per team
+  int nKc, nJc;             // 64-wide chunks of d and of de
+  int S, slot_bytes;        // ring slots and their size (multiple of 1024)
+  int xbuf_bytes;           // x tile of a chunk: nKc x 8 rows x 128 B
+  int KWB;                  // 64-wide j chunks per down-projection stage
+  int router_smem;          // dynamic shared memory of the router kernel
+};
+
+struct Maps {
+  CUtensorMap w1[5];        // [d, de, n_layers E]   box {64, 8 << k, 1}
+  CUtensorMap w2[5];        // [de, d, n_layers E]   box {64, 8 << k, 1}
+  CUtensorMap x;            // [d, L, C]             box {64, 8, 1}
+};
+
+struct Launch {
+  int grid;
+  size_t smem;
+};
+
+// Workspace: header | r [C][L][E] | per-chunk counters | h images
+struct Layout {
+  size_t r_off, bar_off, h_off, total;
+};
+inline Layout layout(int C, int L, int E, int de, int teams) {
+  Layout l;
+  l.r_off = sizeof(WsHeader);
+  l.bar_off = l.r_off + align256(size_t(C) * L * E * 4);
+  l.h_off = l.bar_off + align256(size_t(C) * 4);
+  l.total = l.h_off + size_t(teams) * kHImagesPerTeam * size_t(E) * ((de + 63) / 64) * kHTile;
+  return l;
+}
+
+bool plan(int C, int L, int d, int E, int de, int teams, int num_sms, int max_smem, Params* p, Launch* out);
+cudaError_t launch(const Params& p, const Maps& m, const Launch& plan, cudaStream_t st);
+cudaError_t occupancy(size_t smem, int* ctas_per_sm);
+}  // namespace batch
 
 // ------------------------------------------------------------------------------------ prefill
 struct PrefillParams {

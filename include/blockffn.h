@@ -124,9 +124,44 @@ BFFN_API int blockffn_workspace_init(void* workspace, size_t workspace_bytes, vo
 /*
  * Synchronise `stream`, then read and clear the device error word of `workspace` (NULL = the
  * library's workspace of the current device).  Returns BFFN_OK, BFFN_ETIMEOUT when a bounded
- * device wait ran out since the last check, or BFFN_ECUDA.
+ * device wait ran out since the last check, BFFN_EINVAL when a batched call met a layer index outside
+ * [0, n_layers), or BFFN_ECUDA.
  */
 BFFN_API int blockffn_device_status(void* workspace, void* stream);
+
+/*
+ * Many independent chunks in one call: the batched decode path (lsdiaocha.cn BlockFFN article,
+ * sections 2, 4 and 7: per chunk the same router, union and sparse experts as blockffn_chunk_forward;
+ * the chunks may belong to different sequences of one serving step, or to different layers of a
+ * stacked model whose weights are stored one layer after another).
+ *   x           bf16 [C, L, d]            C chunks of L tokens (1 <= L <= 8)
+ *   layer       int32 [C] on the device: the weight set of each chunk, or NULL for chunk c -> c % n_layers.
+ *               An index outside [0, n_layers) leaves that chunk empty (n_active 0, y 0) and makes
+ *               blockffn_device_status report BFFN_EINVAL.
+ *   Wr          fp32 [n_layers, d, E]     g fp32 [n_layers, E]     br fp32 [n_layers, E] or NULL
+ *   W1          bf16 [n_layers, E, de, d] W2 bf16 [n_layers, E, d, de]
+ *   y           fp32 [C, L, d]            active_idx int32 [C, E]   n_active int32 [C]
+ *   counts      int32 [C, 2] or NULL      tok_mask uint32 [C, L, ceil(E/32)] or NULL
+ *   flags       BFFN_FLAGS_SHARE(k): the GPU's SMs form k teams (default min(8, C)); team i takes chunks
+ *               i, i + k, i + 2k, ... in order, and the next chunk's weights stream while the current
+ *               chunk finishes, so no SM idles between chunks.
+ *   workspace   at least blockffn_batch_workspace_size(C, L, d, E, de, flags) bytes, or NULL for the
+ *               library's per-device workspace (the same rules as blockffn_chunk_forward_ex).
+ * Two launches are enqueued: a router kernel (one CTA per chunk) and a persistent expert kernel.  The
+ * expert kernel needs the GPU's SMs to itself while it runs (its teams wait on one another with bounded
+ * waits).  Results equal blockffn_chunk_forward's within the layer's tolerance (the sums run in another
+ * order); the union, masks and counts are identical; y is bit-identical run to run.  L > 8, or shapes
+ * whose per-CTA tiles do not fit, return BFFN_EUNSUPPORTED before anything is enqueued.
+ */
+BFFN_API int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, const int32_t* layer,
+                                          int n_layers, const float* Wr, const float* g, const float* br,
+                                          const void* W1, const void* W2, int E, int de, float* y,
+                                          int32_t* active_idx, int32_t* n_active, int32_t* counts,
+                                          uint32_t* tok_mask, int flags, void* workspace,
+                                          size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace a blockffn_chunk_forward_batch call with these sizes and flags needs (0 if invalid). */
+BFFN_API size_t blockffn_batch_workspace_size(int C, int L, int d, int E, int de, int flags);
 
 /*
  * blockffn_chunk_forward_noalloc — no counterpart on the BlockFFN pages; this is a deployment aid.

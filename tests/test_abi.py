@@ -109,3 +109,32 @@ def test_workspace_holds_the_selected_decode_kernel_scratch(bffn):
     # a chunk of 8 tokens of smaller experts takes the mma.sync kernel: header, router parts and h only
     small = bffn.blockffn_workspace_size(8, 2048, 64, 256)
     assert 64 * 4 * 2 * 8 * 128 <= small < 160 * 2 * 128 * 16 * 4
+
+
+def _batch(bffn, **kw):
+    a = dict(x=FAKE, C=4, L=8, d=256, layer=None, n_layers=2, Wr=FAKE, g=FAKE, br=None, W1=FAKE, W2=FAKE, E=16,
+             de=64, y=FAKE, active_idx=FAKE, n_active=FAKE, counts=None, tok_mask=None, flags=0, workspace=None,
+             workspace_bytes=0, stream=None)
+    a.update(kw)
+    return bffn.blockffn_chunk_forward_batch(**a)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(C=0), dict(n_layers=0), dict(L=0), dict(d=250), dict(de=20), dict(E=0), dict(E=1025),
+    dict(x=None), dict(W1=FAKE + 8), dict(y=None), dict(n_active=FAKE + 2), dict(layer=FAKE + 1),
+    dict(flags=1), dict(flags=1 << 8), dict(workspace=FAKE + 16),
+])
+def test_batch_invalid_arguments_rejected_before_launch(bffn, kw):
+    assert _batch(bffn, **kw) == bffn.BFFN_EINVAL
+
+
+def test_batch_takes_chunks_of_up_to_8_tokens(bffn):
+    assert _batch(bffn, L=9) == bffn.BFFN_EUNSUPPORTED
+
+
+def test_batch_workspace_size(bffn):
+    # r [C, L, E] fp32 plus two h images per team of E x ceil(de / 64) tiles of 2 KB
+    n = bffn.blockffn_batch_workspace_size(4096, 8, 2048, 64, 256, bffn.BFFN_FLAGS_SHARE(8))
+    assert n >= 4096 * 8 * 64 * 4 + 8 * 2 * 64 * 4 * 2048
+    assert bffn.blockffn_batch_workspace_size(0, 8, 2048, 64, 256, 0) == 0
+    assert bffn.blockffn_batch_workspace_size(4, 8, 2050, 64, 256, 0) == 0
