@@ -375,6 +375,28 @@ int forward_batch(const void* x, int C, int L, int d, const int32_t* layer, int 
       if (!encode_bf16(&m.w1[k], W1, 3, w1d, w1s, b)) return BFFN_ECUDA;
       if (!encode_bf16(&m.w2[k], W2, 3, w2d, w2s, b)) return BFFN_ECUDA;
     }
+    // chunked views: one box is a whole stage (rows x consecutive 64-wide chunks)
+    if (p.nKf > 0) {
+      const uint64_t cd[4] = {64, uint64_t(de), uint64_t(p.nKf), NE};
+      const uint64_t cs[3] = {uint64_t(d) * 2, 128, uint64_t(d) * de * 2};
+      for (int k = 0; k < 16; ++k) {
+        const int h = 8 * (k + 1);
+        const uint32_t b[4] = {64, uint32_t(h), uint32_t(batch::chunks_per_stage_a(h, p.nKc)), 1};
+        if (!encode_bf16(&m.w1c[k], W1, 4, cd, cs, b)) return BFFN_ECUDA;
+      }
+    }
+    if (p.nJf > 0) {
+      const uint64_t cd[4] = {64, uint64_t(d), uint64_t(p.nJf), NE};
+      const uint64_t cs[3] = {uint64_t(de) * 2, 128, uint64_t(d) * de * 2};
+      for (int k = 0; k < 2; ++k) {
+        if (p.hB[k] < 8 || p.hB[k] > batch::kMaxRowsB) {
+          m.w2c[k] = m.w2[0];  // a height no CTA has
+          continue;
+        }
+        const uint32_t b[4] = {64, uint32_t(p.hB[k]), uint32_t(p.KWB), 1};
+        if (!encode_bf16(&m.w2c[k], W2, 4, cd, cs, b)) return BFFN_ECUDA;
+      }
+    }
     const uint64_t xd[3] = {uint64_t(d), uint64_t(L), uint64_t(C)}, xs[2] = {uint64_t(d) * 2, uint64_t(L) * d * 2};
     const uint32_t xb[3] = {64, 8, 1};
     if (!encode_bf16(&m.x, x, 3, xd, xs, xb)) return BFFN_ECUDA;

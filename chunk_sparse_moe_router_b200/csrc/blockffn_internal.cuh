@@ -291,10 +291,23 @@ struct Params {
   int S, slot_bytes;        // ring slots and their size (multiple of 1024)
   int xbuf_bytes;           // x tile of a chunk: nKc x 8 rows x 128 B
   int KWB;                  // 64-wide j chunks per down-projection stage
+  int nKf, nJf;             // full 64-wide chunks of d and de (the chunked views cover these)
+  int hB[2];                // the two heights of the CTAs' y-row ranges (8 floor(d / 8 / T), + 8)
   int router_smem;          // dynamic shared memory of the router kernel
 };
 
+// Stages are one tensor box each: W1 through its chunked view, with a box of h rows x KS(h) chunks for
+// every group height h = 8, 16, ..., 128; W2 likewise with a box of the CTA's y rows x KWB chunks.  A
+// stage that holds the ragged last chunk of d or de takes per-chunk boxes of the plain views instead.
+constexpr int kStageABytes = 32 * 1024;  // an up-projection stage holds at most this many bytes
+__host__ __device__ inline int chunks_per_stage_a(int rows, int nKc) {
+  const int r16 = (rows + 15) & ~15;
+  const int ks = kStageABytes / (r16 * 128);
+  return ks < 1 ? 1 : (ks > nKc ? nKc : ks);
+}
 struct Maps {
+  CUtensorMap w1c[16];      // [64, de, d / 64, n_layers E]   box {64, 8 (k + 1), KS, 1}   (d >= 64 only)
+  CUtensorMap w2c[2];       // [64, d, de / 64, n_layers E]   box {64, hB[k], KWB, 1}      (de >= 64 only)
   CUtensorMap w1[5];        // [d, de, n_layers E]   box {64, 8 << k, 1}
   CUtensorMap w2[5];        // [de, d, n_layers E]   box {64, 8 << k, 1}
   CUtensorMap x;            // [d, L, C]             box {64, 8, 1}

@@ -42,7 +42,7 @@ constexpr int kWarpH = NCW + 1;            // h copies of the down-projection
 constexpr int kWarpX = NCW + 2;            // x tiles of the up-projection
 constexpr int kThreads = (NCW + 3) * 32;
 constexpr int kGroupRows = 128;            // up-projection rows of one group (8 m-tiles)
-constexpr int kStageA = 32 * 1024;         // bytes of an up-projection stage (at most)
+constexpr int kStageA = kStageABytes;      // bytes of an up-projection stage (at most)
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kRouterThreads = 256;
 
@@ -286,10 +286,7 @@ __device__ __forceinline__ Group group_at(const Params& p, int r, int r_end) {
 // 64-column chunks of d per up-projection stage of a group of `rows` rows: about kStageA bytes, so that
 // a short group (a CTA's rows often start or end a few rows into an expert) still moves its weights in
 // a few large stages rather than many small ones.
-__device__ __forceinline__ int chunks_per_stage(const Params& p, int rows) {
-  const int ks = kStageA / (round16(rows) * 128);
-  return ks < 1 ? 1 : (ks > p.nKc ? p.nKc : ks);
-}
+__device__ __forceinline__ int chunks_per_stage(const Params& p, int rows) { return chunks_per_stage_a(rows, p.nKc); }
 __device__ __forceinline__ int stages_of_group(const Params& p, int rows) {
   const int ks = chunks_per_stage(p, rows);
   return (p.nKc + ks - 1) / ks;
@@ -360,19 +357,26 @@ __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, int te
       for (int r = w.rA0; r < w.rA1 && ok;) {
         const Group g = group_at(p, r, w.rA1);
         const int e = w.eb + __ldg(p.active_idx + size_t(c) * p.E + g.a);
-        const int nb = boxes_of(g.rows), rp16 = round16(g.rows);
+        const int nb = boxes_of(g.rows);
         const int KS = chunks_per_stage(p, g.rows), nsA = stages_of_group(p, g.rows);
         for (int ks = 0; ks < nsA; ++ks, rp.next(p.S)) {
           if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 1)) { ok = false; break; }
           const int nc = min(KS, p.nKc - ks * KS);
           uint8_t* st = sm.ring + size_t(rp.slot) * p.slot_bytes;
-          if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(nc * g.rows * 128));
-          __syncwarp();
-          int ro, k;
-          if (lane < nc * nb && box_of(g.rows, lane % nb, &ro, &k)) {
-            const int cc = lane / nb;
-            tma_load_3d(st + (cc * rp16 + ro) * 128, &tm.w1[k], (ks * KS + cc) * 64, g.j0 + ro, e,
-                        &sm.fullW[rp.slot], pol);
+          if (ks * KS + nc <= p.nKf) {  // one box of the chunked view (chunks past the last read as zeros)
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(KS * g.rows * 128));
+              tma_load_4d(st, &tm.w1c[(g.rows >> 3) - 1], 0, g.j0, ks * KS, e, &sm.fullW[rp.slot], pol);
+            }
+          } else {  // the stage holds the ragged last chunk of d: per-chunk boxes of the plain view
+            if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(nc * g.rows * 128));
+            __syncwarp();
+            int ro, k;
+            if (lane < nc * nb && box_of(g.rows, lane % nb, &ro, &k)) {
+              const int cc = lane / nb;
+              tma_load_3d(st + (cc * g.rows + ro) * 128, &tm.w1[k], (ks * KS + cc) * 64, g.j0 + ro, e,
+                          &sm.fullW[rp.slot], pol);
+            }
           }
           __syncwarp();
         }
@@ -383,20 +387,27 @@ __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, int te
       const int c = team + (st_i - 1) * p.teams;
       const Work w = make_work(p, c, gi);
       if (w.nB > 0) {
-        const int nb = boxes_of(w.nB), rp16 = round16(w.nB);
+        const int nb = boxes_of(w.nB);
         for (int a = 0; a < w.n_act && ok; ++a) {
           const int e = w.eb + __ldg(p.active_idx + size_t(c) * p.E + a);
           for (int jb = 0; jb < nsB; ++jb, rp.next(p.S)) {
             if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 2)) { ok = false; break; }
             const int nc = min(p.KWB, p.nJc - jb * p.KWB);
             uint8_t* st = sm.ring + size_t(rp.slot) * p.slot_bytes;
-            if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(nc * w.nB * 128));
-            __syncwarp();
-            int ro, k;
-            if (lane < nc * nb && box_of(w.nB, lane % nb, &ro, &k)) {
-              const int cc = lane / nb;
-              tma_load_3d(st + (cc * rp16 + ro) * 128, &tm.w2[k], (jb * p.KWB + cc) * 64, w.rB0 + ro, e,
-                          &sm.fullW[rp.slot], pol);
+            if (jb * p.KWB + nc <= p.nJf) {  // one box of the chunked view (chunks past the last read as zeros)
+              if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(p.KWB * w.nB * 128));
+                tma_load_4d(st, &tm.w2c[w.nB == p.hB[0] ? 0 : 1], 0, w.rB0, jb * p.KWB, e, &sm.fullW[rp.slot], pol);
+              }
+            } else {  // the stage holds the ragged last chunk of de: per-chunk boxes of the plain view
+              if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(nc * w.nB * 128));
+              __syncwarp();
+              int ro, k;
+              if (lane < nc * nb && box_of(w.nB, lane % nb, &ro, &k)) {
+                const int cc = lane / nb;
+                tma_load_3d(st + (cc * w.nB + ro) * 128, &tm.w2[k], (jb * p.KWB + cc) * 64, w.rB0 + ro, e,
+                            &sm.fullW[rp.slot], pol);
+              }
             }
             __syncwarp();
           }
@@ -504,6 +515,18 @@ __device__ __noinline__ bool team_passed(const Params& p, const Smem& sm, int c)
   return __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
 }
 
+__device__ __forceinline__ void prefetch_l1(const void* ptr) { asm volatile("prefetch.global.L1 [%0];" ::"l"(ptr)); }
+
+// The lines of chunk c's metadata that this CTA reads (n_active, the union list, r) into L1 ahead of use.
+__device__ __forceinline__ void prefetch_chunk(const Params& p, int c, int lane) {
+  if (c >= p.C) return;
+  const int act_lines = (p.E * 4 + 127) / 128, r_lines = (p.L * p.E * 4 + 127) / 128;
+  if (lane == 0) prefetch_l1(p.n_active + c);
+  for (int q = lane; q < act_lines + r_lines; q += 32)
+    prefetch_l1(q < act_lines ? reinterpret_cast<const char*>(p.active_idx + size_t(c) * p.E) + q * 128
+                              : reinterpret_cast<const char*>(p.r + size_t(c) * p.L * p.E) + (q - act_lines) * 128);
+}
+
 __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
   const int cw = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gid = lane >> 2, tig = lane & 3;
@@ -514,7 +537,9 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
   // ldmatrix lane addressing: A (x4) rows lane & 15, k half lane >> 4; B (x2) rows lane & 7, k half (lane >> 3) & 1
   const int arow = lane & 15, ahalf = lane >> 4, brow = lane & 7, bhalf = (lane >> 3) & 1;
   const int n = team_chunks(p, team);
+  if (cw == 0) prefetch_chunk(p, team, lane);
   for (int st_i = 0; st_i <= n; ++st_i) {
+    if (cw == 0) prefetch_chunk(p, team + (st_i + 1) * p.teams, lane);  // the next step's chunk
    if (st_i < n) {
     // ---------------- up-projection of chunk i = st_i
     const int i = st_i, c = team + i * p.teams;
@@ -523,24 +548,36 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
     const bool xok = wait(p, sm, sm.xfull, uint32_t(i) & 1u, 5);
     for (int r = w.rA0; r < w.rA1;) {
       const Group g = group_at(p, r, w.rA1);
-      const int rp16 = round16(g.rows);
       const int KS = chunks_per_stage(p, g.rows), nsA = stages_of_group(p, g.rows);
       const bool mine = 16 * cw < g.rows;
-      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      // the router outputs this lane's epilogue needs, loaded now so that their latency overlaps the stages
+      const int e = __ldg(p.active_idx + size_t(c) * p.E + g.a);
+      float rr[2] = {0.f, 0.f};
+      if (mine)
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          if (2 * tig + q < p.L) rr[q] = __ldg(p.r + (size_t(c) * p.L + 2 * tig + q) * p.E + e);
+      float acc[4][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[k][v] = 0.f;
       for (int ks = 0; ks < nsA; ++ks, rp.next(p.S)) {
         const int slot = rp.slot;
         if (wait(p, sm, &sm.fullW[slot], rp.ph, 6) && xok && mine) {
           const int nc = min(KS, p.nKc - ks * KS);
           const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
           for (int cc = 0; cc < nc; ++cc) {
-            const uint32_t wbase = sb + cc * rp16 * 128, xbase = xb + (ks * KS + cc) * 1024;
+            const uint32_t wbase = sb + cc * g.rows * 128, xbase = xb + (ks * KS + cc) * 1024;
+            // all fragments of the 64-column chunk, then its four MMAs into four accumulators
+            uint32_t a[4][4], b[4][2];
 #pragma unroll
             for (int k16 = 0; k16 < 4; ++k16) {
-              uint32_t a[4], b0, b1;
-              ldmatrix_x4(wbase + swz(16 * cw + arow, 2 * k16 + ahalf), a[0], a[1], a[2], a[3]);
-              ldmatrix_x2(xbase + swz(brow, 2 * k16 + bhalf), b0, b1);
-              mma_bf16_16816(acc[k16 & 1], a, b0, b1);
+              ldmatrix_x4(wbase + swz(16 * cw + arow, 2 * k16 + ahalf), a[k16][0], a[k16][1], a[k16][2], a[k16][3]);
+              ldmatrix_x2(xbase + swz(brow, 2 * k16 + bhalf), b[k16][0], b[k16][1]);
             }
+#pragma unroll
+            for (int k16 = 0; k16 < 4; ++k16) mma_bf16_16816(acc[k16], a[k16], b[k16][0], b[k16][1]);
           }
         }
         __syncwarp();
@@ -548,16 +585,14 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
       }
       if (mine && !aborted(sm)) {
         // h = r Swish(u) for rows 16 cw + gid (+ 8) and tokens 2 tig (+ 1), into the h image as bf16 hi / lo
-        const int e = __ldg(p.active_idx + size_t(c) * p.E + g.a);
         uint8_t* ex = himg + size_t(g.a) * p.nJc * kHTile;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int row = 16 * cw + gid + (v >> 1) * 8, t = 2 * tig + (v & 1);
           if (row < g.rows && t < p.L) {
             const int j = g.j0 + row, col = j & 63;
-            const float u = acc[0][v] + acc[1][v];
-            const float rr = __ldg(p.r + (size_t(c) * p.L + t) * p.E + e);
-            const float hv = rr * (u / (1.f + expf(-u)));
+            const float u = (acc[0][v] + acc[1][v]) + (acc[2][v] + acc[3][v]);
+            const float hv = rr[v & 1] * (u / (1.f + expf(-u)));
             const __nv_bfloat16 hi = __float2bfloat16_rn(hv);
             const __nv_bfloat16 lo = __float2bfloat16_rn(hv - __bfloat162float(hi));
             uint8_t* tile = ex + size_t(j >> 6) * kHTile;
@@ -591,16 +626,21 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
     // warp has left)
     const int i = st_i - 1, c = team + i * p.teams;
     const Work w = make_work(p, c, gi);
-    // every CTA of the team has published its h of chunk i: also a CTA with no down-projection stages
-    // waits, so that no CTA runs more than the schedule allows ahead of the h images others still read
-    const bool tok = team_passed(p, sm, c);
-    float acc[2][2][4];
+    const bool has_b = w.nB > 0 && w.n_act > 0;
+    // A CTA with down-projection stages learns that every CTA of the team published h of chunk i from
+    // the h tiles (the h copy warp waited for that); one without stages waits for the chunk's counter
+    // itself, so that no CTA runs further ahead of the h images others still read than the schedule
+    // allows.
+    const bool tok = has_b || team_passed(p, sm, c);
+    float acc[2][2][2][4];  // [m-tile][hi, lo][even, odd k16]
 #pragma unroll
     for (int m = 0; m < 2; ++m)
 #pragma unroll
       for (int q = 0; q < 2; ++q)
 #pragma unroll
-        for (int v = 0; v < 4; ++v) acc[m][q][v] = 0.f;
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int v = 0; v < 4; ++v) acc[m][q][k][v] = 0.f;
     const int MB = (w.nB + 15) >> 4, rp16 = round16(w.nB);
     const bool m0 = cw < MB, m1 = cw + 8 < MB;
     if (w.nB > 0) {
@@ -615,19 +655,31 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
             const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
             const uint32_t hb = sb + uint32_t(p.KWB * rp16 * 128);
             for (int cc = 0; cc < nc; ++cc) {
-              const uint32_t wbase = sb + cc * rp16 * 128, hbase = hb + cc * kHTile;
+              const uint32_t wbase = sb + cc * w.nB * 128, hbase = hb + cc * kHTile;
+              // all fragments of the 64-wide j chunk first, then the MMAs into the even / odd accumulators
+              uint32_t bh[4][2], bl[4][2], a0[4][4];
 #pragma unroll
               for (int k16 = 0; k16 < 4; ++k16) {
-                uint32_t bh0, bh1, bl0, bl1, a[4];
-                ldmatrix_x2(hbase + swz(brow, 2 * k16 + bhalf), bh0, bh1);
-                ldmatrix_x2(hbase + swz(8 + brow, 2 * k16 + bhalf), bl0, bl1);
-                ldmatrix_x4(wbase + swz(16 * cw + arow, 2 * k16 + ahalf), a[0], a[1], a[2], a[3]);
-                mma_bf16_16816(acc[0][0], a, bh0, bh1);
-                mma_bf16_16816(acc[0][1], a, bl0, bl1);
-                if (m1) {
-                  ldmatrix_x4(wbase + swz(16 * (cw + 8) + arow, 2 * k16 + ahalf), a[0], a[1], a[2], a[3]);
-                  mma_bf16_16816(acc[1][0], a, bh0, bh1);
-                  mma_bf16_16816(acc[1][1], a, bl0, bl1);
+                ldmatrix_x2(hbase + swz(brow, 2 * k16 + bhalf), bh[k16][0], bh[k16][1]);
+                ldmatrix_x2(hbase + swz(8 + brow, 2 * k16 + bhalf), bl[k16][0], bl[k16][1]);
+                ldmatrix_x4(wbase + swz(16 * cw + arow, 2 * k16 + ahalf), a0[k16][0], a0[k16][1], a0[k16][2],
+                            a0[k16][3]);
+              }
+#pragma unroll
+              for (int k16 = 0; k16 < 4; ++k16) {
+                mma_bf16_16816(acc[0][0][k16 & 1], a0[k16], bh[k16][0], bh[k16][1]);
+                mma_bf16_16816(acc[0][1][k16 & 1], a0[k16], bl[k16][0], bl[k16][1]);
+              }
+              if (m1) {
+                uint32_t a1[4][4];
+#pragma unroll
+                for (int k16 = 0; k16 < 4; ++k16)
+                  ldmatrix_x4(wbase + swz(16 * (cw + 8) + arow, 2 * k16 + ahalf), a1[k16][0], a1[k16][1], a1[k16][2],
+                              a1[k16][3]);
+#pragma unroll
+                for (int k16 = 0; k16 < 4; ++k16) {
+                  mma_bf16_16816(acc[1][0][k16 & 1], a1[k16], bh[k16][0], bh[k16][1]);
+                  mma_bf16_16816(acc[1][1][k16 & 1], a1[k16], bl[k16][0], bl[k16][1]);
                 }
               }
             }
@@ -644,7 +696,8 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int row = 16 * (cw + 8 * m) + gid + (v >> 1) * 8, t = 2 * tig + (v & 1);
-          if (row < w.nB && t < p.L) yc[size_t(t) * p.d + row] = acc[m][0][v] + acc[m][1][v];
+          if (row < w.nB && t < p.L)
+            yc[size_t(t) * p.d + row] = (acc[m][0][0][v] + acc[m][0][1][v]) + (acc[m][1][0][v] + acc[m][1][1][v]);
         }
       }
     }
@@ -728,6 +781,10 @@ bool plan(int C, int L, int d, int E, int de, int teams, int num_sms, int max_sm
   p->T = T;
   p->nKc = (d + 63) / 64;
   p->nJc = (de + 63) / 64;
+  p->nKf = d / 64;
+  p->nJf = de / 64;
+  p->hB[0] = 8 * ((d / 8) / T);
+  p->hB[1] = p->hB[0] + 8;
   p->xbuf_bytes = p->nKc * 1024;
   if (p->xbuf_bytes > 96 * 1024) return false;
   const int rp16 = (nB_max + 15) & ~15;
