@@ -21,9 +21,13 @@
 //    (article, section 2), goes to the team's h image as bf16 hi + lo parts (about 16 mantissa bits).
 //  * a team barrier (one arrival counter per chunk) publishes h.  Each role walks the schedule A(0),
 //    A(1), B(0), A(2), B(1), ...: a chunk's down-projection follows the next chunk's up-projection, so
-//    the barrier has a whole phase of slack and the weight stream never waits on it.
+//    the barrier has a whole phase of slack and the weight stream practically never waits on it.
+//  * one warp issues every copy into the ring in stage order (W1 boxes, W2 boxes with the stage's h
+//    tiles on the same barrier), another the x tiles; eight consumer warps run the MMAs.  Each ring
+//    barrier keeps one parity bit, so every waiter on it stays within one pass of the ring: the copy
+//    warp waits for each slot's release in turn and the consumers for each stage in turn.
 //  * down-projection: y rows are split over the team's CTAs in 8-row units; a stage holds one active
-//    expert's W2 rows of this CTA for one or two 64-wide j chunks, plus the matching h tiles.  Warp w
+//    expert's W2 rows of this CTA for one or more 64-wide j chunks, plus the matching h tiles.  Warp w
 //    owns m-tiles w and w + 8 of the CTA's rows for the whole chunk (output-stationary: no cross-warp
 //    reduction), with separate accumulators for the hi and lo parts of h, added once at the end.
 //    Every y element has one writer and a fixed summation order: y is bit-reproducible.
@@ -37,10 +41,9 @@ namespace batch {
 namespace {
 
 constexpr int NCW = 8;                     // consumer warps
-constexpr int kWarpW = NCW;                // weight copies (W1, W2)
-constexpr int kWarpH = NCW + 1;            // h copies of the down-projection
-constexpr int kWarpX = NCW + 2;            // x tiles of the up-projection
-constexpr int kThreads = (NCW + 3) * 32;
+constexpr int kWarpW = NCW;                // copies into the ring: W1, W2 and the h tiles
+constexpr int kWarpX = NCW + 1;            // x tiles of the up-projection
+constexpr int kThreads = (NCW + 2) * 32;
 constexpr int kGroupRows = 128;            // up-projection rows of one group (8 m-tiles)
 constexpr int kStageA = kStageABytes;      // bytes of an up-projection stage (at most)
 constexpr uint64_t kWaitNs = 2000000000ull;
@@ -202,8 +205,7 @@ __global__ void __launch_bounds__(kRouterThreads) batch_router_kernel(const Para
 struct Smem {
   uint8_t* xbuf;        // x of the current chunk: [nKc][8 rows][128 B], 128-byte swizzled
   uint8_t* ring;        // S slots
-  uint64_t* fullW;      // [S] weight tiles landed
-  uint64_t* fullH;      // [S] h tiles landed (down-projection stages)
+  uint64_t* fullW;      // [S] the stage's tiles landed (weights; and h for down-projection stages)
   uint64_t* empty;      // [S] every consumer warp is done with the slot (NCW arrivals)
   uint64_t* xfull;      // x of the chunk landed
   uint64_t* xfree;      // every consumer warp is done with x (NCW arrivals)
@@ -218,10 +220,14 @@ __device__ __forceinline__ bool aborted(const Smem& sm) {
 __device__ __forceinline__ void set_abort(const Smem& sm) {
   asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(smem_u32((const void*)sm.abort_flag)), "r"(1u) : "memory");
 }
+// The first error of a launch keeps its record: err_info = where (bits 0-7) | CTA (bits 8-15) | ring
+// stage index, low 16 bits (bits 16-31).
 __device__ __forceinline__ void set_error(const Params& p, const Smem& sm, uint32_t bit, uint32_t info) {
-  atomicOr(&p.hdr->err, bit);
-  p.hdr->err_info = info;
+  if (atomicOr(&p.hdr->err, bit) == 0u) p.hdr->err_info = info;
   set_abort(sm);
+}
+__device__ __forceinline__ uint32_t site(uint32_t where, int stage) {
+  return where | (uint32_t(blockIdx.x & 255) << 8) | (uint32_t(stage) << 16);
 }
 
 // A bounded wait: on timeout it records the error and marks the CTA aborted; once the CTA is aborted,
@@ -360,7 +366,7 @@ __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, int te
         const int nb = boxes_of(g.rows);
         const int KS = chunks_per_stage(p, g.rows), nsA = stages_of_group(p, g.rows);
         for (int ks = 0; ks < nsA; ++ks, rp.next(p.S)) {
-          if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 1)) { ok = false; break; }
+          if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, site(1, rp.i))) { ok = false; break; }
           const int nc = min(KS, p.nKc - ks * KS);
           uint8_t* st = sm.ring + size_t(rp.slot) * p.slot_bytes;
           if (ks * KS + nc <= p.nKf) {  // one box of the chunked view (chunks past the last read as zeros)
@@ -384,30 +390,48 @@ __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, int te
       }
     }
     if (st_i >= 1 && ok) {  // B(st_i - 1)
-      const int c = team + (st_i - 1) * p.teams;
+      const int i = st_i - 1, c = team + i * p.teams;
       const Work w = make_work(p, c, gi);
-      if (w.nB > 0) {
-        const int nb = boxes_of(w.nB);
+      if (w.nB > 0 && w.n_act > 0) {
+        {  // every CTA of the team has published its h of chunk i (normally long since: a phase of slack)
+          const uint64_t t0 = globaltimer_ns();
+          bool passed = true;
+          while (ld_acquire_gpu(&p.chunk_bar[c]) < uint32_t(p.T)) {
+            if (aborted(sm) || globaltimer_ns() - t0 > kWaitNs) { passed = false; break; }
+            __nanosleep(64);
+          }
+          passed = __all_sync(0xffffffffu, passed);
+          if (!passed) {
+            if (lane == 0 && !aborted(sm)) set_error(p, sm, kErrTeamBarrier, site(11, i));
+            return rp.i;
+          }
+          fence_proxy_async_global();  // h was written with generic stores; the bulk copies read it
+        }
+        const uint8_t* himg = h_image(p, team, i);
+        const int nb = boxes_of(w.nB), rp16 = round16(w.nB);
         for (int a = 0; a < w.n_act && ok; ++a) {
           const int e = w.eb + __ldg(p.active_idx + size_t(c) * p.E + a);
           for (int jb = 0; jb < nsB; ++jb, rp.next(p.S)) {
-            if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 2)) { ok = false; break; }
+            if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, site(2, rp.i))) { ok = false; break; }
             const int nc = min(p.KWB, p.nJc - jb * p.KWB);
             uint8_t* st = sm.ring + size_t(rp.slot) * p.slot_bytes;
-            if (jb * p.KWB + nc <= p.nJf) {  // one box of the chunked view (chunks past the last read as zeros)
-              if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(p.KWB * w.nB * 128));
+            const uint32_t hbytes = uint32_t(nc * kHTile);
+            const bool chunked = jb * p.KWB + nc <= p.nJf;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t((chunked ? p.KWB : nc) * w.nB * 128) + hbytes);
+              // the h tiles of the stage: one bulk copy of nc tiles after the W2 rows
+              bulk_g2s(st + size_t(p.KWB) * rp16 * 128, himg + (size_t(a) * p.nJc + jb * p.KWB) * kHTile, hbytes,
+                       &sm.fullW[rp.slot], pol);
+              // one box of the chunked view (chunks past the last read as zeros)
+              if (chunked)
                 tma_load_4d(st, &tm.w2c[w.nB == p.hB[0] ? 0 : 1], 0, w.rB0, jb * p.KWB, e, &sm.fullW[rp.slot], pol);
-              }
-            } else {  // the stage holds the ragged last chunk of de: per-chunk boxes of the plain view
-              if (lane == 0) mbar_arrive_expect_tx(&sm.fullW[rp.slot], uint32_t(nc * w.nB * 128));
-              __syncwarp();
-              int ro, k;
-              if (lane < nc * nb && box_of(w.nB, lane % nb, &ro, &k)) {
-                const int cc = lane / nb;
-                tma_load_3d(st + (cc * w.nB + ro) * 128, &tm.w2[k], (jb * p.KWB + cc) * 64, w.rB0 + ro, e,
-                            &sm.fullW[rp.slot], pol);
-              }
+            }
+            __syncwarp();
+            int ro, k;  // the stage holds the ragged last chunk of de: per-chunk boxes of the plain view
+            if (!chunked && lane < nc * nb && box_of(w.nB, lane % nb, &ro, &k)) {
+              const int cc = lane / nb;
+              tma_load_3d(st + (cc * w.nB + ro) * 128, &tm.w2[k], (jb * p.KWB + cc) * 64, w.rB0 + ro, e,
+                          &sm.fullW[rp.slot], pol);
             }
             __syncwarp();
           }
@@ -418,66 +442,6 @@ __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, int te
   return rp.i;
 }
 
-// h copy warp: for each B(i) of the schedule, after the team barrier of chunk i, the h tiles of its
-// down-projection stages (one bulk copy of up to KWB tiles per stage).  Returns the per-slot parity
-// bits of the next h phase; `used` gets the slots it filled.
-__device__ uint32_t produce_h(const Params& p, const Smem& sm, int team, int gi, uint32_t* used) {
-  const int lane = threadIdx.x & 31;
-  const uint64_t pol = policy_evict_first();  // each h tile is read once per CTA
-  RingPos rp;
-  uint32_t hph = 0;
-  *used = 0;
-  const int nsB = stages_b_per_expert(p), n = team_chunks(p, team);
-  for (int st_i = 0; st_i <= n; ++st_i) {
-    if (st_i < n) {
-      // A(st_i): not this warp's stages, but it still waits for each one's slot to be released in turn,
-      // like every user of the ring: a waiter that skipped ahead by more than one pass of the ring
-      // could take a phase two passes old for the one it waits for (the barriers keep one parity bit)
-      const int nA = stages_a(p, make_work(p, team + st_i * p.teams, gi));
-      for (int k = 0; k < nA; ++k, rp.next(p.S))
-        if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 10)) return hph;
-    }
-    if (st_i == 0) continue;
-    const int i = st_i - 1, c = team + i * p.teams;
-    const Work w = make_work(p, c, gi);
-    {  // every CTA of the team has published its h of chunk i (a counter per chunk: with this schedule a
-       // CTA may already count its next chunk's up-projection before another has counted this one)
-      const uint32_t need = uint32_t(p.T);
-      const uint64_t t0 = globaltimer_ns();
-      bool ok = true;
-      while (ld_acquire_gpu(&p.chunk_bar[c]) < need) {
-        if (aborted(sm) || globaltimer_ns() - t0 > kWaitNs) { ok = false; break; }
-        __nanosleep(64);
-      }
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) {
-        if (lane == 0 && !aborted(sm)) set_error(p, sm, kErrTeamBarrier, uint32_t(blockIdx.x));
-        return hph;
-      }
-      fence_proxy_async_global();  // h was written with generic stores; bulk copies read it
-    }
-    if (w.nB == 0) continue;
-    const uint8_t* himg = h_image(p, team, i);
-    const int rp16 = round16(w.nB);
-    for (int a = 0; a < w.n_act; ++a) {
-      for (int jb = 0; jb < nsB; ++jb, rp.next(p.S)) {
-        if (rp.i >= p.S && !wait(p, sm, &sm.empty[rp.slot], rp.ph ^ 1u, 3)) return hph;
-        const int nc = min(p.KWB, p.nJc - jb * p.KWB);
-        uint8_t* st = sm.ring + size_t(rp.slot) * p.slot_bytes + size_t(p.KWB) * rp16 * 128;
-        if (lane == 0) {
-          mbar_arrive_expect_tx(&sm.fullH[rp.slot], uint32_t(nc * kHTile));
-          bulk_g2s(st, himg + (size_t(a) * p.nJc + jb * p.KWB) * kHTile, uint32_t(nc * kHTile), &sm.fullH[rp.slot],
-                   pol);
-        }
-        __syncwarp();
-        hph ^= 1u << rp.slot;
-        *used |= 1u << rp.slot;
-      }
-    }
-  }
-  return hph;
-}
-
 // x copy warp: x of each chunk into xbuf once the consumers are done with the previous chunk's.
 // Returns the number of x loads issued.
 __device__ int produce_x(const Params& p, const Maps& tm, const Smem& sm, int team) {
@@ -485,7 +449,7 @@ __device__ int produce_x(const Params& p, const Maps& tm, const Smem& sm, int te
   const uint64_t pol = policy_evict_first();
   int i = 0;
   for (int c = team; c < p.C; ++i, c += p.teams) {
-    if (i > 0 && !wait(p, sm, sm.xfree, uint32_t(i - 1) & 1u, 4)) break;
+    if (i > 0 && !wait(p, sm, sm.xfree, uint32_t(i - 1) & 1u, site(4, i))) break;
     if (lane == 0) mbar_arrive_expect_tx(sm.xfull, uint32_t(p.nKc) * 1024);
     __syncwarp();
     for (int k = lane; k < p.nKc; k += 32) tma_load_3d(sm.xbuf + k * 1024, &tm.x, k * 64, 0, c, sm.xfull, pol);
@@ -505,7 +469,7 @@ __device__ __noinline__ bool team_passed(const Params& p, const Smem& sm, int c)
     while (ld_acquire_gpu(&p.chunk_bar[c]) < uint32_t(p.T)) {
       if (aborted(sm)) { ok = false; break; }
       if (globaltimer_ns() - t0 > kWaitNs) {
-        set_error(p, sm, kErrTeamBarrier, uint32_t(blockIdx.x));
+        set_error(p, sm, kErrTeamBarrier, site(12, c));
         ok = false;
         break;
       }
@@ -533,7 +497,6 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
   const uint32_t xb = smem_u32(sm.xbuf);
   const int nsB = stages_b_per_expert(p);
   RingPos rp;
-  uint32_t hph = 0;
   // ldmatrix lane addressing: A (x4) rows lane & 15, k half lane >> 4; B (x2) rows lane & 7, k half (lane >> 3) & 1
   const int arow = lane & 15, ahalf = lane >> 4, brow = lane & 7, bhalf = (lane >> 3) & 1;
   const int n = team_chunks(p, team);
@@ -545,7 +508,7 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
     const int i = st_i, c = team + i * p.teams;
     const Work w = make_work(p, c, gi);
     uint8_t* himg = h_image(p, team, i);
-    const bool xok = wait(p, sm, sm.xfull, uint32_t(i) & 1u, 5);
+    const bool xok = wait(p, sm, sm.xfull, uint32_t(i) & 1u, site(5, i));
     for (int r = w.rA0; r < w.rA1;) {
       const Group g = group_at(p, r, w.rA1);
       const int KS = chunks_per_stage(p, g.rows), nsA = stages_of_group(p, g.rows);
@@ -564,7 +527,7 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
         for (int v = 0; v < 4; ++v) acc[k][v] = 0.f;
       for (int ks = 0; ks < nsA; ++ks, rp.next(p.S)) {
         const int slot = rp.slot;
-        if (wait(p, sm, &sm.fullW[slot], rp.ph, 6) && xok && mine) {
+        if (wait(p, sm, &sm.fullW[slot], rp.ph, site(6, rp.i)) && xok && mine) {
           const int nc = min(KS, p.nKc - ks * KS);
           const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
           for (int cc = 0; cc < nc; ++cc) {
@@ -628,9 +591,9 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
     const Work w = make_work(p, c, gi);
     const bool has_b = w.nB > 0 && w.n_act > 0;
     // A CTA with down-projection stages learns that every CTA of the team published h of chunk i from
-    // the h tiles (the h copy warp waited for that); one without stages waits for the chunk's counter
-    // itself, so that no CTA runs further ahead of the h images others still read than the schedule
-    // allows.
+    // the h tiles (the copy warp waited for that before copying them); one without stages waits for the
+    // chunk's counter itself, so that no CTA runs further ahead of the h images others still read than
+    // the schedule allows.
     const bool tok = has_b || team_passed(p, sm, c);
     float acc[2][2][2][4];  // [m-tile][hi, lo][even, odd k16]
 #pragma unroll
@@ -647,10 +610,8 @@ __device__ void consume(const Params& p, const Smem& sm, int team, int gi) {
       for (int a = 0; a < w.n_act; ++a) {
         for (int jb = 0; jb < nsB; ++jb, rp.next(p.S)) {
           const int slot = rp.slot;
-          const bool okW = tok && wait(p, sm, &sm.fullW[slot], rp.ph, 8);
-          const bool okH = okW && wait(p, sm, &sm.fullH[slot], (hph >> slot) & 1u, 9);
-          hph ^= 1u << slot;
-          if (okH && m0) {
+          const bool okW = tok && wait(p, sm, &sm.fullW[slot], rp.ph, site(8, rp.i));
+          if (okW && m0) {
             const int nc = min(p.KWB, p.nJc - jb * p.KWB);
             const uint32_t sb = smem_u32(sm.ring + size_t(slot) * p.slot_bytes);
             const uint32_t hb = sb + uint32_t(p.KWB * rp16 * 128);
@@ -714,9 +675,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm.ring = base + p.xbuf_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm.ring + size_t(p.S) * p.slot_bytes);
   sm.fullW = bars;
-  sm.fullH = bars + p.S;
-  sm.empty = bars + 2 * p.S;
-  sm.xfull = bars + 3 * p.S;
+  sm.empty = bars + p.S;
+  sm.xfull = bars + 2 * p.S;
   sm.xfree = sm.xfull + 1;
   sm.abort_flag = reinterpret_cast<volatile int*>(sm.xfull + 2);
 
@@ -724,7 +684,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0) {
     for (int s = 0; s < p.S; ++s) {
       mbar_init(&sm.fullW[s], 1);
-      mbar_init(&sm.fullH[s], 1);
       mbar_init(&sm.empty[s], NCW);
     }
     mbar_init(sm.xfull, 1);
@@ -744,13 +703,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();
   const int team = blockIdx.x / p.T, gi = blockIdx.x - team * p.T;
   int issuedW = 0, issuedX = 0;
-  uint32_t hph = 0, hused = 0;
   if (warp < NCW) {
     consume(p, sm, team, gi);
   } else if (warp == kWarpW) {
     issuedW = produce_w(p, tm, sm, team, gi);
-  } else if (warp == kWarpH) {
-    hph = produce_h(p, sm, team, gi, &hused);
   } else {
     issuedX = produce_x(p, tm, sm, team);
   }
@@ -759,11 +715,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpW)
       for (int k = max(0, issuedW - p.S); k < issuedW; ++k)
         mbar_wait_bounded(&sm.fullW[k % p.S], uint32_t(k / p.S) & 1u, kWaitNs / 10);
-    if (warp == kWarpH) {
-      // the last h phase of every slot it filled: its parity bit was flipped after the copy was issued
-      for (int s = 0; s < p.S; ++s)
-        if ((hused >> s) & 1u) mbar_wait_bounded(&sm.fullH[s], ((hph >> s) & 1u) ^ 1u, kWaitNs / 10);
-    }
     if (warp == kWarpX && issuedX > 0) mbar_wait_bounded(sm.xfull, uint32_t(issuedX - 1) & 1u, kWaitNs / 10);
   }
 }

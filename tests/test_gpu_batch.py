@@ -182,3 +182,31 @@ def test_bad_layer_index_is_reported(bffn, cuda_device):
     assert tuple(got["counts"][1]) == (8 * 16, 16)
     check_chunk(got, 0, lays[0], xs[0])
     check_chunk(got, 2, lays[0], xs[2])
+
+
+@pytest.mark.parametrize("tls", [0.50, 0.95])
+def test_sparsity_sweep_points_width_4096(bffn, cuda_device, tls):
+    # the stacked-model sweep's layer (d=4096, E=128, de=256, L=8) at its extreme token-level sparsity
+    # points, two layers, 8 teams of SMs, three chunks per team; oracle on the first two chunks
+    lays = [gen.make_layer(41 + k, 4096, 128, 256, gen.beta_for_tls(tls), 1.09) for k in range(2)]
+    sl = StackedLayers(lays)
+    C = 24
+    xs = np.stack([gen.make_chunks(41, lays[c % 2], 1, 8, 0.3, stream=c)[0] for c in range(C)])
+    got = run_batch(bffn, sl, xs, teams=8)
+    assert got["status"] == bffn.BFFN_OK
+    for c in (0, 1):
+        check_chunk(got, c, lays[c % 2], xs[c])
+
+
+def test_every_expert_active_long_phases(bffn, cuda_device):
+    # every one of 128 experts active at d=4096: up-projection phases of several hundred stages per CTA
+    # and several chunks per team (the copy warp and the consumers stay within one pass of the ring)
+    lay = gen.make_layer(51, 4096, 128, 256, 0.0, 1.09)
+    lay.br[:] = 50.0
+    sl = StackedLayers([lay])
+    C = 32
+    xs = gen.make_chunks(51, lay, C, 8, 0.3)
+    got = run_batch(bffn, sl, xs, teams=8)
+    assert got["status"] == bffn.BFFN_OK
+    assert np.all(got["n"] == 128)
+    check_chunk(got, C - 1, lay, xs[C - 1])
