@@ -293,7 +293,6 @@ struct Params {
   int KWB;                  // 64-wide j chunks per down-projection stage
   int nKf, nJf;             // full 64-wide chunks of d and de (the chunked views cover these)
   int hB[2];                // the two heights of the CTAs' y-row ranges (8 floor(d / 8 / T), + 8)
-  int router_smem;          // dynamic shared memory of the router kernel
 };
 
 // Stages are one tensor box each: W1 through its chunked view, with a box of h rows x KS(h) chunks for

@@ -1,7 +1,8 @@
 // Batched decode path of the BlockFFN chunk layer: many independent chunks of up to 8 tokens (one per
 // sequence of a serving step, or one per layer of a stacked model) in two launches.
 //
-// Router kernel (one CTA per chunk): s = x Wr + b in fp32, then ReLU, the RMSNorm statistics over the
+// Router kernel (one CTA per group of up to 64 tokens of one layer): s = x Wr + b in fp32, then ReLU, the
+// RMSNorm statistics over the
 // E router entries, the per-token active bits with __ballot_sync, the chunk's union of active experts
 // as an ascending list built with __popc and a warp scan, the sparsity counts, and
 // r = g relu(s) / rms for the expert kernel (lsdiaocha.cn BlockFFN article, sections 2 and 4; BlockFFN
@@ -58,110 +59,151 @@ __device__ __forceinline__ int layer_of(const Params& p, int c) { return p.layer
 __device__ __forceinline__ bool layer_ok(const Params& p, int l) { return l >= 0 && l < p.n_layers; }
 
 // ===================================================================================== router kernel
-// Shared memory: x [L][d] bf16 | warp partial sums [8 warps][8 tokens][32] | s [L][E] | masks [L][32] |
-// rms [8] | union list [E] | n_act.
-__global__ void __launch_bounds__(kRouterThreads) batch_router_kernel(const Params p) {
-  extern __shared__ __align__(16) uint8_t rsm[];
-  const int c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int L = p.L, d = p.d, E = p.E, nW = (E + 31) >> 5;
-  __nv_bfloat162* xs = reinterpret_cast<__nv_bfloat162*>(rsm);
-  float* red = reinterpret_cast<float*>(rsm + size_t(L) * d * 2);
-  float* s = red + 8 * 8 * 32;
-  uint32_t* maskw = reinterpret_cast<uint32_t*>(s + size_t(L) * E);
-  float* rms = reinterpret_cast<float*>(maskw + 8 * 32);
-  int32_t* act = reinterpret_cast<int32_t*>(rms + 8);
-  int32_t* n_act_s = act + E;
+// One CTA routes a group of up to 64 tokens (kRouterTokens): G = 64 / L chunks that use the same layer
+// (chunks l, l + n_layers, l + 2 n_layers, ... when there is no layer array; one chunk per CTA when
+// there is one).  s = x Wr (+ b) is a small GEMM of the group's tokens against the layer's Wr: tiles of
+// 32 rows of d x 64 experts staged in shared memory, each thread a 4 x 4 register tile of (token,
+// expert) sums accumulated over d in increasing order, so s does not depend on timing.  s goes to
+// r's place in the workspace; then one warp per token takes the RMS of relu(s) over the E experts and
+// the active bits (__ballot_sync), one warp per chunk the union (__popc and a warp scan) and counts, and
+// r = g relu(s) / rms overwrites s.
+constexpr int kRouterTokens = 64;
+constexpr int kRtK = 32;   // rows of d per tile
+constexpr int kRtE = 64;   // experts per tile
 
-  if (tid == 0) p.chunk_bar[c] = 0u;  // the expert kernel's counter of this chunk starts at 0 (it runs after this grid)
-  const int layer = layer_of(p, c);
+__device__ __forceinline__ int router_group_size(const Params& p) {
+  return p.layer ? 1 : max(1, kRouterTokens / p.L);
+}
+// Chunk of slot j of router CTA b (or -1): without a layer array, CTA b takes layer b % n_layers and
+// that layer's chunks [G (b / n_layers), + G) in its own order.
+__device__ __forceinline__ int router_chunk(const Params& p, int b, int j) {
+  if (p.layer) return j == 0 ? b : -1;
+  const int G = router_group_size(p), l = b % p.n_layers, q = b / p.n_layers;
+  const long long c = (long long)l + (long long)p.n_layers * (G * q + j);
+  return c < p.C ? int(c) : -1;
+}
+
+__global__ void __launch_bounds__(kRouterThreads) batch_router_kernel(const Params p) {
+  __shared__ __align__(16) float Xs[kRtK][kRouterTokens];
+  __shared__ __align__(16) float Ws[kRtK][kRtE];
+  __shared__ uint32_t maskw[kRouterTokens][32];
+  __shared__ float rms[kRouterTokens];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L = p.L, d = p.d, E = p.E, nW = (E + 31) >> 5;
+  const int G = router_group_size(p);
+  const int c0 = router_chunk(p, blockIdx.x, 0);
+  if (c0 < 0) return;
+  const int layer = layer_of(p, c0);
+  int nchunks = 0;
+  while (nchunks < G && router_chunk(p, blockIdx.x, nchunks) >= 0) ++nchunks;
+  const int M = nchunks * L;  // tokens of the group
+  if (tid < nchunks) p.chunk_bar[router_chunk(p, blockIdx.x, tid)] = 0u;  // the expert kernel's counters
   if (!layer_ok(p, layer)) {  // an invalid layer index: the chunk is left empty and the error recorded
     if (tid == 0) {
       atomicOr(&p.hdr->err, kErrBadLayer);
-      p.hdr->err_info = uint32_t(c);
-      p.n_active[c] = 0;
-      if (p.counts) p.counts[2 * c] = L * E, p.counts[2 * c + 1] = E;
+      p.hdr->err_info = uint32_t(c0);
+      p.n_active[c0] = 0;
+      if (p.counts) p.counts[2 * c0] = L * E, p.counts[2 * c0 + 1] = E;
     }
     if (p.tok_mask)
-      for (int o = tid; o < L * nW; o += kRouterThreads) p.tok_mask[size_t(c) * L * nW + o] = 0u;
+      for (int o = tid; o < L * nW; o += kRouterThreads) p.tok_mask[size_t(c0) * L * nW + o] = 0u;
     return;
   }
   const float* Wr = p.Wr + size_t(layer) * d * E;
   const float* g = p.g + size_t(layer) * E;
   const float* br = p.br ? p.br + size_t(layer) * E : nullptr;
+  // token m of the group: chunk router_chunk(m / L), row m % L
+  auto token_row = [&](int m) -> const __nv_bfloat16* {
+    return p.x + (size_t(router_chunk(p, blockIdx.x, m / L)) * L + (m % L)) * d;
+  };
+  auto s_row = [&](int m) -> float* {  // s (then r) of token m, in r's place in the workspace
+    return p.r + (size_t(router_chunk(p, blockIdx.x, m / L)) * L + (m % L)) * E;
+  };
 
-  {  // x [L][d] bf16 into shared memory, 16 bytes at a time (d is a multiple of 8)
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + size_t(c) * L * d);
-    uint4* dst = reinterpret_cast<uint4*>(rsm);
-    for (int o = tid; o < L * d / 8; o += kRouterThreads) dst[o] = src[o];
-  }
-  __syncthreads();
-
-  // s = x Wr (+ b): experts in blocks of 32 (lane = expert), d split over the 8 warps in even-sized
-  // parts; each warp's sum runs over its columns in increasing order, then the warps' sums are added
-  // in warp order, so s does not depend on timing.
-  const int kper = (((d + 7) / 8) + 1) & ~1;
-  const int k0 = min(d, warp * kper), k1 = min(d, k0 + kper);
-  const int dh = d / 2;
-  for (int eb = 0; eb < E; eb += 32) {
-    const int e = eb + lane;
-    const bool have = e < E;
-    float acc[kMaxL];
+  // ---- s = x Wr + b
+  const int ty = tid >> 4, tx = tid & 15;  // tokens 4 ty .. 4 ty + 3, experts 4 tx .. 4 tx + 3 of the tile
+  for (int eb = 0; eb < E; eb += kRtE) {
+    float acc[4][4] = {};
+    for (int k0 = 0; k0 < d; k0 += kRtK) {
+      {  // x: 64 tokens x 32 columns (bf16 -> fp32, transposed), 8 columns per thread
+        const int m = tid >> 2, k8 = (tid & 3) * 8;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (m < M && k0 + k8 < d) v = *reinterpret_cast<const uint4*>(token_row(m) + k0 + k8);
+        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&v);
 #pragma unroll
-    for (int t = 0; t < kMaxL; ++t) acc[t] = 0.f;
-#pragma unroll 4
-    for (int k = k0; k < k1; k += 2) {
-      const float w0 = have ? __ldg(Wr + size_t(k) * E + e) : 0.f;
-      const float w1 = have ? __ldg(Wr + size_t(k + 1) * E + e) : 0.f;
+        for (int i = 0; i < 8; ++i) Xs[k8 + i][m] = __bfloat162float(hv[i]);
+      }
 #pragma unroll
-      for (int t = 0; t < kMaxL; ++t) {
-        if (t < L) {
-          const float2 xv = __bfloat1622float2(xs[t * dh + (k >> 1)]);
-          acc[t] = fmaf(xv.x, w0, acc[t]);
-          acc[t] = fmaf(xv.y, w1, acc[t]);
+      for (int h = 0; h < 2; ++h) {  // Wr: 32 rows x 64 experts, 4 per thread and pass
+        const int o = tid + h * kRouterThreads, k = o >> 4, e4 = (o & 15) * 4;
+        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (k0 + k < d) {
+          const float* src = Wr + size_t(k0 + k) * E + eb + e4;
+          if ((E & 3) == 0 && eb + e4 + 3 < E) {
+            w = *reinterpret_cast<const float4*>(src);
+          } else {
+            if (eb + e4 + 0 < E) w.x = src[0];
+            if (eb + e4 + 1 < E) w.y = src[1];
+            if (eb + e4 + 2 < E) w.z = src[2];
+            if (eb + e4 + 3 < E) w.w = src[3];
+          }
         }
+        *reinterpret_cast<float4*>(&Ws[k][e4]) = w;
       }
+      __syncthreads();
+#pragma unroll 8
+      for (int k = 0; k < kRtK; ++k) {
+        const float4 a = *reinterpret_cast<const float4*>(&Xs[k][ty * 4]);
+        const float4 b = *reinterpret_cast<const float4*>(&Ws[k][tx * 4]);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
+      __syncthreads();
     }
 #pragma unroll
-    for (int t = 0; t < kMaxL; ++t) red[(warp * 8 + t) * 32 + lane] = acc[t];
-    __syncthreads();
-    for (int o = tid; o < L * 32; o += kRouterThreads) {
-      const int t = o >> 5, ln = o & 31, ee = eb + ln;
-      if (ee < E) {
-        float v = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      const int m = ty * 4 + i;
+      if (m >= M) continue;
+      float* sr = s_row(m);
 #pragma unroll
-        for (int w = 0; w < 8; ++w) v += red[(w * 8 + t) * 32 + ln];
-        if (br) v += br[ee];
-        s[t * E + ee] = v;
+      for (int j = 0; j < 4; ++j) {
+        const int e = eb + tx * 4 + j;
+        if (e < E) sr[e] = acc[i][j] + (br ? br[e] : 0.f);
       }
     }
-    __syncthreads();
   }
+  __syncthreads();  // s of every token is written (global memory, this CTA)
 
-  // per token (one warp each): the RMS of relu(s) over the E experts and the active bits
-  for (int t = warp; t < L; t += kRouterThreads / 32) {
+  // ---- per token (one warp each): the RMS of relu(s) over the E experts and the active bits
+  for (int m = warp; m < M; m += kRouterThreads / 32) {
+    const float* sr = s_row(m);
     float sumsq = 0.f;
     for (int ww = 0; ww < nW; ++ww) {
       const int e = ww * 32 + lane;
-      const float sv = e < E ? s[t * E + e] : -1.f;
+      const float sv = e < E ? sr[e] : -1.f;
       const float a = fmaxf(sv, 0.f);
       sumsq = fmaf(a, a, sumsq);
       const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
-      if (lane == 0) maskw[t * 32 + ww] = bits;
+      if (lane == 0) maskw[m][ww] = bits;
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-    if (lane == 0) rms[t] = sqrtf(sumsq / float(E));
+    if (lane == 0) rms[m] = sqrtf(sumsq / float(E));
   }
   __syncthreads();
-  // the chunk's union, ascending (warp 0: lane w holds word w of the OR of the masks), and the counts
-  if (warp == 0) {
+  // ---- per chunk (one warp each): the union, ascending (lane w holds word w of the OR of the masks)
+  for (int j = warp; j < nchunks; j += kRouterThreads / 32) {
+    const int c = router_chunk(p, blockIdx.x, j);
     uint32_t u = 0;
     int tok_active = 0;
     if (lane < nW)
       for (int t = 0; t < L; ++t) {
-        const uint32_t m = maskw[t * 32 + lane];
-        u |= m;
-        tok_active += __popc(m);
+        const uint32_t mw = maskw[j * L + t][lane];
+        u |= mw;
+        tok_active += __popc(mw);
       }
     const int cnt = __popc(u);
     int incl = cnt;
@@ -173,31 +215,31 @@ __global__ void __launch_bounds__(kRouterThreads) batch_router_kernel(const Para
     const int total = __shfl_sync(0xffffffffu, incl, 31);
     int pos = incl - cnt;
     uint32_t rest = u;
+    int32_t* out = p.active_idx + size_t(c) * E;
     while (rest) {
       const int b = __ffs(rest) - 1;
       rest &= rest - 1;
-      act[pos++] = lane * 32 + b;
+      out[pos++] = lane * 32 + b;
     }
     int act_sum = tok_active;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) act_sum += __shfl_xor_sync(0xffffffffu, act_sum, o);
     if (lane == 0) {
-      *n_act_s = total;
       p.n_active[c] = total;
       if (p.counts) {
         p.counts[2 * c] = L * E - act_sum;
         p.counts[2 * c + 1] = E - total;
       }
     }
+    if (p.tok_mask)
+      for (int o = lane; o < L * nW; o += 32) p.tok_mask[size_t(c) * L * nW + o] = maskw[j * L + o / nW][o % nW];
   }
-  __syncthreads();
-  for (int a = tid; a < *n_act_s; a += kRouterThreads) p.active_idx[size_t(c) * E + a] = act[a];
-  if (p.tok_mask)
-    for (int o = tid; o < L * nW; o += kRouterThreads) p.tok_mask[size_t(c) * L * nW + o] = maskw[(o / nW) * 32 + (o % nW)];
-  for (int o = tid; o < L * E; o += kRouterThreads) {  // r = g relu(s) / rms (0 for a token with no active expert)
-    const int t = o / E, e = o - t * E;
-    const float rm = rms[t];
-    p.r[size_t(c) * L * E + o] = rm > 0.f ? (g[e] * fmaxf(s[o], 0.f)) / rm : 0.f;
+  // ---- r = g relu(s) / rms over s (0 for a token with no active expert); each thread its own elements
+  for (int o = tid; o < M * E; o += kRouterThreads) {
+    const int m = o / E, e = o - m * E;
+    float* sr = s_row(m);
+    const float rm = rms[m];
+    sr[e] = rm > 0.f ? (g[e] * fmaxf(sr[e], 0.f)) / rm : 0.f;
   }
 }
 
@@ -753,10 +795,6 @@ bool plan(int C, int L, int d, int E, int de, int teams, int num_sms, int max_sm
   if (S > 8) S = 8;
   if (S < 2) return false;
   p->S = int(S);
-  // router kernel: x [L][d] bf16, warp sums, s [L][E], masks, rms, union list, n_act
-  const size_t rs = size_t(L) * d * 2 + 8 * 8 * 32 * 4 + size_t(L) * E * 4 + 8 * 32 * 4 + 8 * 4 + size_t(E) * 4 + 16;
-  if (rs > size_t(max_smem)) return false;
-  p->router_smem = int(rs);
   out->grid = teams * T;
   out->smem = fixed + size_t(p->xbuf_bytes) + size_t(p->S) * slot;
   return true;
@@ -770,11 +808,16 @@ cudaError_t occupancy(size_t smem, int* ctas_per_sm) {
 
 cudaError_t launch(const Params& p, const Maps& m, const Launch& plan, cudaStream_t st) {
   cudaError_t err;
-  if (p.router_smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(batch_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, p.router_smem);
-    if (err != cudaSuccess) return err;
+  {
+    // router CTAs: one per chunk with a layer array, else ceil(chunks of a layer / G) per layer
+    int ctas = p.C;
+    if (!p.layer) {
+      const int G = kRouterTokens / p.L < 1 ? 1 : kRouterTokens / p.L;
+      const int per_layer = (p.C + p.n_layers - 1) / p.n_layers;
+      ctas = p.n_layers * ((per_layer + G - 1) / G);
+    }
+    batch_router_kernel<<<ctas, kRouterThreads, 0, st>>>(p);
   }
-  batch_router_kernel<<<p.C, kRouterThreads, p.router_smem, st>>>(p);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   err = cudaFuncSetAttribute(batch_expert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
