@@ -408,7 +408,7 @@ def run_ours(args, w):
     value = tokens_step / (ms_per_step * 1e-3)
     achieved_gbs = total_active / (ms_per_step * 1e-3) / 1e9  # per GPU: every rank streams its own
     peak, peak_kind = measured_peaks()
-    ratio = recorded_traffic_ratio(w.name)
+    ratio = recorded_traffic_ratio(w.name + ("/batch" if batched else "/streams"))
     traffic = None if ratio is None else ratio * total_active / chunks
     if prefill:
         flops = float(sum(prefill_flops(d, E, de, L, int(p)) for p in pairs_host))
