@@ -587,6 +587,117 @@ def run_tls_sweep(args):
         print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------------- cross-chunk reuse
+def run_reuse(args):
+    """Cross-chunk expert reuse on the per-chunk path (one chunk at a time on the whole GPU): the
+    consecutive verification chunks of one sequence, as a drifting sequence of chunk bases (gen's
+    make_sequence_chunks, --drift list).  For each drift: the mean reuse rate |U_k ∩ U_(k-1)| / |U_k|
+    (blockffn_union_overlap on the device), and tokens/s with the experts' weights read evict-first
+    (default) and evict-last (BFFN_FLAG_KEEP_EXPERTS_IN_L2), (a) one layer, steps back to back, and
+    (b) the sequence through a stack of --replicas layers, step k visiting every layer before step k+1,
+    as autoregressive decoding does.  One JSON line per drift and case."""
+    import numpy as np
+    import torch
+
+    import chunk_sparse_moe_router_b200 as bffn
+    import gen
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = gen.workload("decode")
+    R = args.replicas or 16
+    d, E, de, L = w.d, w.E, w.de, w.L
+    n_steps = args.chunks or 256
+    lays = [w.layer(r) for r in range(R)]
+    dev = {k: [] for k in ("Wr", "br", "g", "W1", "W2")}
+    for lay in lays:
+        dev["Wr"].append(torch.from_numpy(lay.Wr).to(device))
+        dev["br"].append(torch.from_numpy(lay.br).to(device))
+        dev["g"].append(torch.from_numpy(lay.g).to(device))
+        dev["W1"].append(torch.from_numpy(lay.W1.view(np.int16)).to(device))
+        dev["W2"].append(torch.from_numpy(lay.W2.view(np.int16)).to(device))
+    peak, peak_kind = measured_peaks()
+    ws = bffn.new_workspace(L, d, E, de, device)
+    ws_bytes = bffn.blockffn_workspace_size(L, d, E, de)
+    s = torch.cuda.Stream(device)
+    for drift in [float(v) for v in args.drift.split(",")]:
+        for case, layers in (("one layer, steps back to back", 1), (f"{R} layers per step", R)):
+            # x[k, l]: step k's chunk at layer l (each layer sees its own drifting sequence)
+            xs = np.stack([gen.make_sequence_chunks(w.seed, lays[l], n_steps, L, w.noise, drift, stream=l)
+                           for l in range(layers)], axis=1)
+            x = torch.from_numpy(xs.view(np.int16)).to(device)
+            y = torch.empty((n_steps, layers, L, d), dtype=torch.float32, device=device)
+            idx = torch.full((n_steps, layers, E), -1, dtype=torch.int32, device=device)
+            nact = torch.zeros((n_steps, layers), dtype=torch.int32, device=device)
+            line_base = None
+            for keep in (False, True):
+                flags = bffn.BFFN_FLAG_KEEP_EXPERTS_IN_L2 if keep else 0
+
+                def step():
+                    for k in range(n_steps):
+                        for l in range(layers):
+                            rc = bffn.blockffn_chunk_forward_ex(
+                                x[k, l].data_ptr(), L, d, dev["Wr"][l].data_ptr(), dev["g"][l].data_ptr(),
+                                dev["W1"][l].data_ptr(), dev["W2"][l].data_ptr(), E, de, y[k, l].data_ptr(),
+                                idx[k, l].data_ptr(), nact[k, l:].data_ptr(), dev["br"][l].data_ptr(), None, None,
+                                None, flags, ws.data_ptr(), ws_bytes, s.cuda_stream)
+                            if rc != 0:
+                                raise bffn.BlockFFNError(rc, "blockffn_chunk_forward_ex")
+
+                with torch.cuda.stream(s):
+                    step()
+                    s.synchronize()
+                    graph = torch.cuda.CUDAGraph()
+                    graph.capture_begin()
+                    step()
+                    graph.capture_end()
+                    for _ in range(args.warmup):
+                        graph.replay()
+                    s.synchronize()
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(s)
+                    for _ in range(args.steps):
+                        graph.replay()
+                    e1.record(s)
+                    e1.synchronize()
+                    if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
+                        raise RuntimeError("device-side wait ran out")
+                    del graph
+                ms = e0.elapsed_time(e1) / args.steps
+                calls = n_steps * layers
+                # reuse rate of consecutive steps at each layer
+                ov = torch.empty(((n_steps - 1) * layers,), dtype=torch.int32, device=device)
+                ia = idx[:-1].reshape(-1, E).contiguous()
+                ib = idx[1:].reshape(-1, E).contiguous()
+                na = nact[:-1].reshape(-1).contiguous()
+                nb = nact[1:].reshape(-1).contiguous()
+                rc = bffn.blockffn_union_overlap(ia.data_ptr(), na.data_ptr(), ib.data_ptr(), nb.data_ptr(),
+                                                 ov.numel(), E, ov.data_ptr(), s.cuda_stream)
+                if rc != 0:
+                    raise bffn.BlockFFNError(rc, "blockffn_union_overlap")
+                s.synchronize()
+                reuse = float((ov.float() / nb.float().clamp(min=1)).mean().item())
+                n_host = nact.cpu().numpy()
+                total = float(sum(active_bytes(d, E, de, L, int(v)) for v in n_host.reshape(-1)))
+                tps = calls * L / (ms * 1e-3)
+                line = {"metric": METRIC, "value": round(tps, 1), "unit": "tokens/s", "n_gpus": 1,
+                        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 4),
+                        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+                        "data": "synthetic",
+                        "config": {"workload": "reuse_decode_d2048_E64_de256_L8", "case": case, "drift": drift,
+                                   "steps_per_sequence": n_steps, "layers": layers,
+                                   "keep_experts_in_l2": keep, "mean_n_active": round(float(n_host.mean()), 3),
+                                   "reuse_rate": round(reuse, 4)},
+                        "roofline": {"bound": "hbm", "achieved": round(total / (ms * 1e-3) / 1e9, 1), "peak": peak,
+                                     "unit": "GB/s", "frac": round(total / (ms * 1e-3) / 1e9 / peak, 4),
+                                     "peak_kind": peak_kind, "us_per_chunk": round(ms * 1e3 / calls, 3)},
+                        "gpu_launches": calls * args.steps}
+                if keep and line_base:
+                    line["speedup_vs_evict_first"] = round(tps / line_base, 3)
+                line_base = tps
+                print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
     """The fp64 dense oracle timed on this host's cores on a bounded sample of the workload (tokens
@@ -679,7 +790,10 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="decode", choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse"])
+    ap.add_argument("--drift", default="0.0,0.9,0.97",
+                    help="--workload reuse: drift of the chunk bases of a sequence (0: independent chunks)")
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
     ap.add_argument("--tls", type=float, default=None, help="token-level sparsity for --workload tls_sweep")
     ap.add_argument("--chunks", type=int, default=None, help="chunks per step (default: the workload's)")
@@ -714,6 +828,9 @@ def main():
         kw["replicas"] = args.replicas
     if args.workload == "tls_sweep" and args.impl == "ours" and not args.tls:
         run_tls_sweep(args)
+        return
+    if args.workload == "reuse":
+        run_reuse(args)
         return
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":

@@ -19,6 +19,8 @@ BFFN_PATH_AUTO, BFFN_PATH_DECODE, BFFN_PATH_PREFILL = 0, 1, 2
 
 
 BFFN_FLAG_INJECT_ROUTER_TIMEOUT = 0x100  # fault injection for tests of the error path (decode path)
+BFFN_FLAG_ROUTER_SUM_NORM = 0x200  # the ReMoE router: r = g relu(s) / sum relu(s) instead of the RMS
+BFFN_FLAG_KEEP_EXPERTS_IN_L2 = 0x400  # per-chunk decode: expert weights read with the L2 evict-last policy
 
 
 def BFFN_FLAGS_SHARE(k: int) -> int:
@@ -37,6 +39,7 @@ SIGNATURES = {
     "blockffn_chunk_forward_batch": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P,
                                          _I, _P, _S, _P]),
     "blockffn_batch_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
+    "blockffn_union_overlap": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_init": (_I, [_P, _S, _P]),
     "blockffn_device_status": (_I, [_P, _P]),
@@ -83,6 +86,10 @@ def blockffn_chunk_forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2,
                                  counts, tok_mask, flags, workspace, workspace_bytes, stream):
     return _lib.blockffn_chunk_forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx,
                                              n_active, counts, tok_mask, flags, workspace, workspace_bytes, stream)
+
+
+def blockffn_union_overlap(active_idx_a, n_active_a, active_idx_b, n_active_b, C, E, overlap, stream):
+    return _lib.blockffn_union_overlap(active_idx_a, n_active_a, active_idx_b, n_active_b, C, E, overlap, stream)
 
 
 def blockffn_batch_workspace_size(C, L, d, E, de, flags):
@@ -138,10 +145,11 @@ def _check(t, name, dtype, shape, device):
 
 
 def chunk_forward(x, Wr, g, W1, W2, y, active_idx, n_active, br=None, tok_mask=None, counts=None,
-                  r_out=None, path=BFFN_PATH_AUTO, workspace=None, stream=None):
+                  r_out=None, path=BFFN_PATH_AUTO, workspace=None, stream=None, flags=0):
     """One chunk: x bf16 [L,d], Wr fp32 [d,E], g fp32 [E], W1 bf16 [E,de,d], W2 bf16 [E,d,de];
     outputs y fp32 [L,d], active_idx int32 [E], n_active int32 [1] (+ optional tok_mask int32
-    [L,ceil(E/32)] (bit patterns), counts int32 [2], r_out fp32 [L,E]).  Raises BlockFFNError."""
+    [L,ceil(E/32)] (bit patterns), counts int32 [2], r_out fp32 [L,E]).  `flags` adds BFFN_FLAG_* bits to the
+    path.  Raises BlockFFNError."""
     import torch
 
     L, d = x.shape
@@ -168,13 +176,13 @@ def chunk_forward(x, Wr, g, W1, W2, y, active_idx, n_active, br=None, tok_mask=N
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
     rc = blockffn_chunk_forward_ex(_ptr(x), L, d, _ptr(Wr), _ptr(g), _ptr(W1), _ptr(W2), E, de, _ptr(y),
                                    _ptr(active_idx), _ptr(n_active), _ptr(br), _ptr(tok_mask),
-                                   _ptr(counts), _ptr(r_out), int(path), ws_ptr, ws_bytes, stream)
+                                   _ptr(counts), _ptr(r_out), int(path) | int(flags), ws_ptr, ws_bytes, stream)
     if rc != BFFN_OK:
         raise BlockFFNError(rc, "blockffn_chunk_forward_ex")
 
 
 def chunk_forward_batch(x, Wr, g, W1, W2, y, active_idx, n_active, layer=None, br=None, counts=None,
-                        tok_mask=None, teams=0, workspace=None, stream=None):
+                        tok_mask=None, teams=0, workspace=None, stream=None, flags=0):
     """C independent chunks in one call: x bf16 [C,L,d]; stacked weights Wr fp32 [n_layers,d,E],
     g fp32 [n_layers,E], W1 bf16 [n_layers,E,de,d], W2 bf16 [n_layers,E,d,de] (br fp32 [n_layers,E]);
     layer int32 [C] (None: chunk c uses layer c % n_layers); outputs y fp32 [C,L,d], active_idx int32
@@ -206,7 +214,7 @@ def chunk_forward_batch(x, Wr, g, W1, W2, y, active_idx, n_active, layer=None, b
     ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
     rc = blockffn_chunk_forward_batch(_ptr(x), C, L, d, _ptr(layer), nl, _ptr(Wr), _ptr(g), _ptr(br), _ptr(W1),
                                       _ptr(W2), E, de, _ptr(y), _ptr(active_idx), _ptr(n_active), _ptr(counts),
-                                      _ptr(tok_mask), BFFN_FLAGS_SHARE(teams), ws_ptr, ws_bytes, stream)
+                                      _ptr(tok_mask), BFFN_FLAGS_SHARE(teams) | int(flags), ws_ptr, ws_bytes, stream)
     if rc != BFFN_OK:
         raise BlockFFNError(rc, "blockffn_chunk_forward_batch")
 

@@ -135,11 +135,14 @@ bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* di
 int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                       const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                       const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                      const DeviceInfo& di, int share, bool inject, cudaStream_t st) {
+                      const DeviceInfo& di, int share, bool inject, bool sum_norm, bool keep_l2,
+                      cudaStream_t st) {
   const WsLayout lay = ws_layout(L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   tcdec::Params dp;
   dp.inject_timeout = inject ? 1 : 0;
+  dp.sum_norm = sum_norm ? 1 : 0;
+  dp.keep_l2 = keep_l2 ? 1 : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.Wr = Wr;
   dp.br = br;
@@ -193,13 +196,15 @@ int forward_decode_tc(const void* x, int L, int d, const float* Wr, const float*
 int forward_decode(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                    const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                    const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                   const DeviceInfo& di, int share, bool inject, cudaStream_t st) {
+                   const DeviceInfo& di, int share, bool inject, bool sum_norm, bool keep_l2, cudaStream_t st) {
   const WsLayout lay = ws_layout(L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   WsHeader* hdr = reinterpret_cast<WsHeader*>(base);
 
   DecodeParams dp;
   dp.inject_timeout = inject ? 1 : 0;
+  dp.sum_norm = sum_norm ? 1 : 0;
+  dp.keep_l2 = keep_l2 ? 1 : 0;
   dp.x = static_cast<const __nv_bfloat16*>(x);
   dp.Wr = Wr;
   dp.br = br;
@@ -276,12 +281,13 @@ int forward_decode(const void* x, int L, int d, const float* Wr, const float* g,
 int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g, const void* W1,
                     const void* W2, int E, int de, float* y, int32_t* active_idx, int32_t* n_active,
                     const float* br, uint32_t* tok_mask, int32_t* counts, float* r_out, void* ws,
-                    const DeviceInfo& di, cudaStream_t st) {
+                    const DeviceInfo& di, bool sum_norm, cudaStream_t st) {
   if (!aligned16(y)) return BFFN_EINVAL;  // the down-projection adds into y 16 bytes at a time
   const WsLayout lay = ws_layout(L, d, E, de);
   const PrefillLayout pl = prefill_layout(lay.h_off, L, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   PrefillParams p;
+  p.sum_norm = sum_norm ? 1 : 0;
   p.x = static_cast<const __nv_bfloat16*>(x);
   p.Wr = Wr;
   p.br = br;
@@ -332,8 +338,8 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
 
 int forward_batch(const void* x, int C, int L, int d, const int32_t* layer, int n_layers, const float* Wr,
                   const float* g, const float* br, const void* W1, const void* W2, int E, int de, float* y,
-                  int32_t* active_idx, int32_t* n_active, int32_t* counts, uint32_t* tok_mask, int teams, void* ws,
-                  const DeviceInfo& di, cudaStream_t st) {
+                  int32_t* active_idx, int32_t* n_active, int32_t* counts, uint32_t* tok_mask, int teams,
+                  bool sum_norm, void* ws, const DeviceInfo& di, cudaStream_t st) {
   batch::Params p;
   batch::Launch launch;
   if (!batch::plan(C, L, d, E, de, teams, di.num_sms, di.max_smem, &p, &launch)) return BFFN_EUNSUPPORTED;
@@ -365,6 +371,7 @@ int forward_batch(const void* x, int C, int L, int d, const int32_t* layer, int 
   p.E = E;
   p.de = de;
   p.n_layers = n_layers;
+  p.sum_norm = sum_norm ? 1 : 0;
   batch::Maps m;
   {
     const uint64_t NE = uint64_t(n_layers) * E;
@@ -469,8 +476,11 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   const int path = flags & 3;
   if (path == 3) return BFFN_EINVAL;
   const int share = ((flags >> 4) & 15) == 0 ? 1 : ((flags >> 4) & 15);
-  if ((flags & ~(0xF3 | BFFN_FLAG_INJECT_ROUTER_TIMEOUT)) != 0) return BFFN_EINVAL;
+  if ((flags & ~(0xF3 | BFFN_FLAG_INJECT_ROUTER_TIMEOUT | BFFN_FLAG_ROUTER_SUM_NORM | BFFN_FLAG_KEEP_EXPERTS_IN_L2)) != 0)
+    return BFFN_EINVAL;
   const bool inject = (flags & BFFN_FLAG_INJECT_ROUTER_TIMEOUT) != 0;
+  const bool sum_norm = (flags & BFFN_FLAG_ROUTER_SUM_NORM) != 0;
+  const bool keep_l2 = (flags & BFFN_FLAG_KEEP_EXPERTS_IN_L2) != 0;
   const bool decode = (path == BFFN_PATH_DECODE) || (path == BFFN_PATH_AUTO && L <= kDecodeMaxL);
   if (decode && L > kDecodeMaxL) return BFFN_EUNSUPPORTED;
   if (!decode && inject) return BFFN_EUNSUPPORTED;  // the injection exists on the decode path only
@@ -494,12 +504,12 @@ int blockffn_chunk_forward_ex(const void* x, int L, int d, const float* Wr, cons
   if (decode) {
     if (decode_on_tc(L, d, de))
       return forward_decode_tc(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                               r_out, ws, di, share, inject, st);
+                               r_out, ws, di, share, inject, sum_norm, keep_l2, st);
     return forward_decode(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts,
-                          r_out, ws, di, share, inject, st);
+                          r_out, ws, di, share, inject, sum_norm, keep_l2, st);
   }
   return forward_prefill(x, L, d, Wr, g, W1, W2, E, de, y, active_idx, n_active, br, tok_mask, counts, r_out,
-                         ws, di, st);
+                         ws, di, sum_norm, st);
 }
 
 int blockffn_chunk_forward(const void* x, int L, int d, const float* Wr, const float* g,
@@ -510,7 +520,7 @@ int blockffn_chunk_forward(const void* x, int L, int d, const float* Wr, const f
 }
 
 size_t blockffn_batch_workspace_size(int C, int L, int d, int E, int de, int flags) {
-  if (!batch_args_ok(C, L, d, 1, E, de) || (flags & ~0xF0) != 0) return 0;
+  if (!batch_args_ok(C, L, d, 1, E, de) || (flags & ~(0xF0 | BFFN_FLAG_ROUTER_SUM_NORM)) != 0) return 0;
   return batch::layout(C, L, E, de, batch_teams(flags, C)).total;
 }
 
@@ -520,7 +530,7 @@ int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, const int32
                                  uint32_t* tok_mask, int flags, void* workspace, size_t workspace_bytes,
                                  void* stream) {
   if (!batch_args_ok(C, L, d, n_layers, E, de)) return BFFN_EINVAL;
-  if ((flags & ~0xF0) != 0) return BFFN_EINVAL;
+  if ((flags & ~(0xF0 | BFFN_FLAG_ROUTER_SUM_NORM)) != 0) return BFFN_EINVAL;
   const void* bulk[] = {x, Wr, W1, W2};
   for (const void* p : bulk)
     if (p == nullptr || !aligned16(p)) return BFFN_EINVAL;
@@ -547,7 +557,19 @@ int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, const int32
     return BFFN_ENOMEM;
   }
   return forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx, n_active, counts,
-                       tok_mask, teams, ws, di, st);
+                       tok_mask, teams, (flags & BFFN_FLAG_ROUTER_SUM_NORM) != 0, ws, di, st);
+}
+
+int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* n_active_a, const int32_t* active_idx_b,
+                           const int32_t* n_active_b, int C, int E, int32_t* overlap, void* stream) {
+  if (C < 1 || E < 1 || E > kMaxE) return BFFN_EINVAL;
+  const void* ptrs[] = {active_idx_a, n_active_a, active_idx_b, n_active_b, overlap};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned4(p)) return BFFN_EINVAL;
+  const cudaError_t err =
+      union_overlap_launch(active_idx_a, n_active_a, active_idx_b, n_active_b, C, E, overlap,
+                           static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
 }
 
 int blockffn_device_status(void* workspace, void* stream) {

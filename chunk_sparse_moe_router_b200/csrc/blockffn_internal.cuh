@@ -16,6 +16,12 @@ constexpr int kDecodeMaxL = 32;
 // gives up after this long; every other device wait gives up after about 2 s.
 constexpr uint64_t kInjectedWaitNs = 1000000ull;
 
+// The per-token normaliser of the router's ReLU outputs a: their RMS over the E experts (BlockFFN's
+// RMSNorm), or their sum (the ReMoE router).  r = g a / normaliser, and r = 0 when it is 0.
+__device__ __forceinline__ float router_norm(int sum_norm, float sum, float sumsq, int E) {
+  return sum_norm ? sum : sqrtf(sumsq / float(E));
+}
+
 // Device error word bits (WsHeader::err).
 enum : uint32_t {
   kErrGridBarrier = 1u,   // expert kernel: waiting for every CTA to finish the up-projection
@@ -138,6 +144,8 @@ struct DecodeParams {
   WsHeader* hdr;
   int L, d, E, de;
   int inject_timeout;  // 1: the router barrier waits for one arrival more than the grid has (1 ms limit)
+  int sum_norm;        // 1: r = g relu(s) / sum relu(s) (the ReMoE router) instead of the RMS
+  int keep_l2;         // 1: expert weights are read with the L2 evict-last policy (BFFN_FLAG_KEEP_EXPERTS_IN_L2)
   int S;            // ring slots
   int slot_bytes;   // bytes per slot (multiple of 1024)
   // up-projection: one stage = one W1 box of h (1, 2, 4 or 8 <= RSM) whole adjacent rows of one
@@ -218,6 +226,8 @@ struct Params {
   WsHeader* hdr;
   int L, d, E, de;
   int inject_timeout;  // 1: the router barrier waits for one arrival more than the grid has (1 ms limit)
+  int sum_norm;        // 1: r = g relu(s) / sum relu(s) (the ReMoE router) instead of the RMS
+  int keep_l2;         // 1: expert weights are read with the L2 evict-last policy (BFFN_FLAG_KEEP_EXPERTS_IN_L2)
   int nck;          // 64-column chunks of d (the last may be ragged: the tensor maps read zeros past d)
   int nbpe, HA;     // up-projection blocks per expert and their height (multiple of 8, <= 128)
   int nrb, HB;      // down-projection blocks of y rows and their height (multiple of 8, <= 128)
@@ -286,6 +296,7 @@ struct Params {
                             // the router kernel)
   WsHeader* hdr;
   int C, L, d, E, de, n_layers;
+  int sum_norm;             // 1: r = g relu(s) / sum relu(s) (the ReMoE router) instead of the RMS
   int teams, T;             // teams, CTAs per team
   int nKc, nJc;             // 64-wide chunks of d and of de
   int S, slot_bytes;        // ring slots and their size (multiple of 1024)
@@ -335,6 +346,10 @@ cudaError_t launch(const Params& p, const Maps& m, const Launch& plan, cudaStrea
 cudaError_t occupancy(size_t smem, int* ctas_per_sm);
 }  // namespace batch
 
+// Cross-chunk expert reuse (union_overlap.cu): overlap[c] = |U_a(c) ∩ U_b(c)| from two calls' active lists.
+cudaError_t union_overlap_launch(const int32_t* idx_a, const int32_t* n_a, const int32_t* idx_b, const int32_t* n_b,
+                                 int C, int E, int32_t* overlap, cudaStream_t st);
+
 // ------------------------------------------------------------------------------------ prefill
 struct PrefillParams {
   const __nv_bfloat16* x;   // [L,d]
@@ -350,6 +365,7 @@ struct PrefillParams {
   int32_t* counts;          // optional
   float* r_out;             // optional
   int L, d, E, de, W;       // W = ceil(E / 32)
+  int sum_norm;             // 1: r = g relu(s) / sum relu(s) (the ReMoE router) instead of the RMS
   float* s;                 // [L,E]
   float* s_part;            // [ksplit][L,E] partial router projections
   int ksplit;               // K parts of the router projection (d / ksplit a multiple of 32)

@@ -66,7 +66,7 @@ __device__ __forceinline__ bool layer_ok(const Params& p, int l) { return l >= 0
 // expert) sums accumulated over d in increasing order, so s does not depend on timing.  s goes to
 // r's place in the workspace; then one warp per token takes the RMS of relu(s) over the E experts and
 // the active bits (__ballot_sync), one warp per chunk the union (__popc and a warp scan) and counts, and
-// r = g relu(s) / rms overwrites s.
+// r = g relu(s) / rms overwrites s (rms: the RMS of the ReLU outputs, or their sum for the ReMoE router).
 constexpr int kRouterTokens = 64;
 constexpr int kRtK = 32;   // rows of d per tile
 constexpr int kRtE = 64;   // experts per tile
@@ -180,18 +180,22 @@ __global__ void __launch_bounds__(kRouterThreads) batch_router_kernel(const Para
   // ---- per token (one warp each): the RMS of relu(s) over the E experts and the active bits
   for (int m = warp; m < M; m += kRouterThreads / 32) {
     const float* sr = s_row(m);
-    float sumsq = 0.f;
+    float sumsq = 0.f, sum = 0.f;
     for (int ww = 0; ww < nW; ++ww) {
       const int e = ww * 32 + lane;
       const float sv = e < E ? sr[e] : -1.f;
       const float a = fmaxf(sv, 0.f);
       sumsq = fmaf(a, a, sumsq);
+      sum += a;
       const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
       if (lane == 0) maskw[m][ww] = bits;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-    if (lane == 0) rms[m] = sqrtf(sumsq / float(E));
+    for (int o = 16; o > 0; o >>= 1) {
+      sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    if (lane == 0) rms[m] = router_norm(p.sum_norm, sum, sumsq, E);  // the normaliser: RMS or sum
   }
   __syncthreads();
   // ---- per chunk (one warp each): the union, ascending (lane w holds word w of the OR of the masks)

@@ -160,18 +160,22 @@ __device__ void prologue_router_stats(const P& p, const SM& sm, const RouterStag
   __syncthreads();
   for (int t = warp; t < p.L; t += NT / 32) {
     const float* st = sbuf + size_t(t) * p.E;
-    float sumsq = 0.f;
+    float sumsq = 0.f, sum = 0.f;
     for (int ww = 0; ww < nW; ++ww) {
       const int e = ww * 32 + lane;
       const float sv = e < p.E ? st[e] : -1.f;
       const float a = fmaxf(sv, 0.f);
       sumsq = fmaf(a, a, sumsq);
+      sum += a;
       const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
       if (lane == 0) sm.maskw[t * 32 + ww] = bits;
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-    if (lane == 0) sm.rms[t] = sqrtf(sumsq / float(p.E));
+    for (int o = 16; o > 0; o >>= 1) {
+      sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+      sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    }
+    if (lane == 0) sm.rms[t] = router_norm(p.sum_norm, sum, sumsq, p.E);  // the normaliser: RMS or sum
   }
   __syncthreads();
   if (warp == 0) {

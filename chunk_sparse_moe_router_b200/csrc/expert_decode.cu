@@ -210,7 +210,8 @@ struct RingPos {
 template <bool KSPLIT>
 __device__ void produce_weights(const DecodeParams& p, const TensorMaps& tm, const Smem& sm, const Work& w) {
   const int lane = threadIdx.x & 31;
-  const uint64_t pol_w = policy_evict_first();
+  // weights stream through once (evict first), unless the caller expects the next call to reuse them
+  const uint64_t pol_w = p.keep_l2 ? policy_evict_last() : policy_evict_first();
   RingPos rp;
   bool ok = true;
   // ---- phase A: stage = one box of a group's whole rows over the pass's columns

@@ -262,7 +262,8 @@ __device__ __forceinline__ void load_rows(uint8_t* dst, const CUtensorMap* maps,
 // Weight copy warp (lane 0): W1 rows with the matching x columns, then W2 rows, in stage order.
 // Returns the number of stages issued.
 __device__ int produce_w(const Params& p, const Maps& tm, const Smem& sm, const Work& w) {
-  const uint64_t pol_w = policy_evict_first(), pol_x = policy_evict_last();
+  // weights stream through once (evict first), unless the caller expects the next call to reuse them
+  const uint64_t pol_w = p.keep_l2 ? policy_evict_last() : policy_evict_first(), pol_x = policy_evict_last();
   RingPos rp;
   Seg sg;
   for (SegIter it(cta_range(w.CA, w.nKA)); it.next(sg);) {

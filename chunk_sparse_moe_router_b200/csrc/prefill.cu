@@ -105,13 +105,14 @@ __global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
     st[e] = v + (p.br ? p.br[e] : 0.f);
   }
   __syncwarp();
-  float sumsq = 0.f;
+  float sumsq = 0.f, sum = 0.f;
   int n_pos = 0;
   for (int w = 0; w < p.W; ++w) {
     const int e = w * 32 + lane;
     const float sv = e < p.E ? st[e] : -1.f;
     const float a = fmaxf(sv, 0.f);
     sumsq = fmaf(a, a, sumsq);
+    sum += a;
     const uint32_t bits = __ballot_sync(0xffffffffu, sv > 0.f);
     if (lane == 0) {
       p.mask[size_t(t) * p.W + w] = bits;
@@ -120,8 +121,11 @@ __global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
     n_pos += __popc(bits);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
-  const float rms = sqrtf(sumsq / float(p.E));
+  for (int o = 16; o > 0; o >>= 1) {
+    sumsq += __shfl_xor_sync(0xffffffffu, sumsq, o);
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  const float rms = router_norm(p.sum_norm, sum, sumsq, p.E);  // the normaliser: RMS or sum
   if (lane == 0) {
     p.rms[t] = rms;
     atomicAdd(p.n_pos, n_pos);  // an integer sum: the same in any order

@@ -29,7 +29,7 @@ import numpy as np
 
 __all__ = [
     "f32_to_bf16_bits", "bf16_bits_to_f32", "Layer", "make_layer", "make_chunks",
-    "expected_cls", "solve_noise_for_cls", "beta_for_tls", "Workload", "workload",
+    "expected_cls", "solve_noise_for_cls", "beta_for_tls", "Workload", "workload", "make_sequence_chunks",
     "WORKLOADS",
 ]
 
@@ -156,6 +156,32 @@ def make_chunks(seed: int, layer: Layer, n_chunks: int, L: int, noise: float | N
             s_b = _pre_activation(cand, layer)
             bad = bad[np.any(np.abs(s_b) < margin, axis=1)]
         out[c0:c0 + nb] = xb
+    return out
+
+
+def make_sequence_chunks(seed: int, layer: Layer, n_steps: int, L: int, noise: float, drift: float,
+                         margin: float = MARGIN, stream: int = 0) -> np.ndarray:
+    """Consecutive chunks of one sequence as bf16 bits [n_steps, L, d]: the chunk bases follow
+    z_k = drift z_{k-1} + sqrt(1 - drift^2) e_k (z_0, e_k ~ N(0, I)), so consecutive chunks share experts
+    more as drift -> 1; tokens are x_t = z_k + noise n_t.  The margin rule of make_chunks applies (a
+    token within `margin` of a zero pre-activation gets a fresh noise draw)."""
+    d = layer.d
+    rng = _rng(seed, stream, 0x5E9C4A)
+    out = np.empty((n_steps, L, d), dtype=np.uint16)
+    z = rng.standard_normal(d, dtype=np.float32)
+    keep = np.float32(drift)
+    fresh_w = np.float32(math.sqrt(max(0.0, 1.0 - drift * drift)))
+    for k in range(n_steps):
+        if k > 0:
+            z = keep * z + fresh_w * rng.standard_normal(d, dtype=np.float32)
+        xb = f32_to_bf16_bits(z[None, :] + np.float32(noise) * rng.standard_normal((L, d), dtype=np.float32))
+        bad = np.flatnonzero(np.any(np.abs(_pre_activation(xb, layer)) < margin, axis=1))
+        while bad.size:
+            cand = f32_to_bf16_bits(z[None, :] + np.float32(noise) * rng.standard_normal((bad.size, d),
+                                                                                         dtype=np.float32))
+            xb[bad] = cand
+            bad = bad[np.any(np.abs(_pre_activation(cand, layer)) < margin, axis=1)]
+        out[k] = xb
     return out
 
 

@@ -87,6 +87,22 @@ enum { BFFN_PATH_AUTO = 0, BFFN_PATH_DECODE = 1, BFFN_PATH_PREFILL = 2 };
  * BFFN_ETIMEOUT, and the next call on the same workspace runs normally.  Nothing faults or hangs. */
 #define BFFN_FLAG_INJECT_ROUTER_TIMEOUT 0x100
 
+/* Router variant (every path; blockffn_chunk_forward_ex and blockffn_chunk_forward_batch): the ReMoE
+ * router, with the sum of the ReLU outputs as the normaliser instead of their RMS (intelliparadigm survey,
+ * section 5.1: gate G = ReLU(x W_g), output sum_i G_i Expert_i(x) / sum_i G_i; the BlockFFN article, section
+ * 2, compares BlockFFN's RMSNorm router against it):
+ *   r_{t,i} = g_i relu(s_{t,i}) / sum_i relu(s_{t,i})      (r_t = 0 when no s_{t,i} is positive)
+ * The active sets, union and counts are those of the RMSNorm router; only r, and so y, change. */
+#define BFFN_FLAG_ROUTER_SUM_NORM 0x200
+
+/* Cache policy for cross-chunk expert reuse (per-chunk decode path, blockffn_chunk_forward_ex): the
+ * active experts' weights are read with the L2 evict-last policy instead of evict-first, so that a next
+ * call that activates the same experts (the next chunk of the same sequence at the same layer; the
+ * BlockFFN article, section 5, finds most experts shared by consecutive tokens) can find them in L2.  It
+ * pays only when that next call comes before other traffic has pushed them out (an L2 of 126 MB; one
+ * layer's union of 20-40 experts of 2-4 MiB fits).  Results do not depend on it. */
+#define BFFN_FLAG_KEEP_EXPERTS_IN_L2 0x400
+
 /*
  * The layer forward over one chunk, with no router bias.  Uses a per-device workspace that the
  * library allocates on the first call (and grows when a later call needs more); make that first
@@ -162,6 +178,19 @@ BFFN_API int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, co
 
 /* Bytes of workspace a blockffn_chunk_forward_batch call with these sizes and flags needs (0 if invalid). */
 BFFN_API size_t blockffn_batch_workspace_size(int C, int L, int d, int E, int de, int flags);
+
+/*
+ * Cross-chunk expert reuse (the BlockFFN article, section 5: most experts a token activates are active for
+ * the next one as well).  For c < C: overlap[c] = |U_a(c) ∩ U_b(c)|, the experts in both chunk c's union
+ * of call a and chunk c's union of call b, given as the active lists and counts those calls wrote
+ * (active_idx [C, E] with the first n_active[c] entries of row c ascending, n_active [C]; all device
+ * memory).  The reuse rate of chunk c is overlap[c] / n_active_b[c].  One small kernel on `stream`;
+ * BFFN_EINVAL for bad sizes or pointers (4-byte alignment, non-NULL), BFFN_ECUDA for a launch failure.
+ * Entries outside [0, E) are ignored.
+ */
+BFFN_API int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* n_active_a,
+                                    const int32_t* active_idx_b, const int32_t* n_active_b, int C, int E,
+                                    int32_t* overlap, void* stream);
 
 /*
  * blockffn_chunk_forward_noalloc — no counterpart on the BlockFFN pages; this is a deployment aid.

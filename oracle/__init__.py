@@ -42,13 +42,14 @@ def _load():
             lib.oracle_get_mutation.restype = i
             lib.oracle_swish.argtypes = [C.c_double]
             lib.oracle_swish.restype = C.c_double
-            lib.oracle_router.argtypes = [p, i, i, p, p, p, i, dptr, dptr, p]
+            lib.oracle_router.argtypes = [p, i, i, p, p, p, i, i, dptr, dptr, p]
             lib.oracle_union.argtypes = [p, i, i, p, p, p, p]
             lib.oracle_expert.argtypes = [p, i, p, p, i, i, dptr]
-            lib.oracle_chunk_forward.argtypes = [p, i, i, p, p, p, p, p, i, i, i, dptr, dptr, p]
-            lib.oracle_tokens_forward_mt.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, dptr]
+            lib.oracle_chunk_forward.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, dptr, dptr, p]
+            lib.oracle_tokens_forward_mt.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, i, dptr]
+            lib.oracle_union_overlap.argtypes = [p, i, p, i, i, p]
             for f in ("oracle_router", "oracle_union", "oracle_expert", "oracle_chunk_forward",
-                      "oracle_tokens_forward_mt"):
+                      "oracle_tokens_forward_mt", "oracle_union_overlap"):
                 getattr(lib, f).restype = i
             _lib = lib
     return _lib
@@ -71,7 +72,11 @@ def swish(u: float) -> float:
     return float(_load().oracle_swish(float(u)))
 
 
-def router(x, Wr, br, g):
+# router normalisation: the RMS of the ReLU outputs (BlockFFN) or their sum (the ReMoE variant)
+NORMS = {"rms": 0, "sum": 1}
+
+
+def router(x, Wr, br, g, norm: str = "rms"):
     """x bf16 bits [L,d]; returns s fp64 [L,E], r fp64 [L,E], active bool [L,E]."""
     lib = _load()
     x = _c(x, np.uint16)
@@ -80,7 +85,7 @@ def router(x, Wr, br, g):
     L, d = x.shape
     E = Wr.shape[1]
     s = np.zeros((L, E)); r = np.zeros((L, E)); act = np.zeros((L, E), np.uint8)
-    rc = lib.oracle_router(_ptr(x), L, d, _ptr(Wr), _ptr(br), _ptr(g), E, _ptr(s), _ptr(r), _ptr(act))
+    rc = lib.oracle_router(_ptr(x), L, d, _ptr(Wr), _ptr(br), _ptr(g), E, NORMS[norm], _ptr(s), _ptr(r), _ptr(act))
     assert rc == 0
     return s, r, act.astype(bool)
 
@@ -97,6 +102,17 @@ def union(active):
     return idx[: n[0]].copy(), int(tz[0]), int(cz[0])
 
 
+def union_overlap(a, b, E) -> int:
+    """|a ∩ b| for two lists of expert indices (the reuse of one union by the next)."""
+    lib = _load()
+    a = np.ascontiguousarray(a, dtype=np.int32)
+    b = np.ascontiguousarray(b, dtype=np.int32)
+    out = np.zeros(1, np.int32)
+    rc = lib.oracle_union_overlap(_ptr(a), a.size, _ptr(b), b.size, int(E), _ptr(out))
+    assert rc == 0
+    return int(out[0])
+
+
 def expert(xt, W1, W2, i):
     lib = _load()
     xt = _c(xt, np.uint16); W1 = _c(W1, np.uint16); W2 = _c(W2, np.uint16)
@@ -107,7 +123,7 @@ def expert(xt, W1, W2, i):
     return out
 
 
-def chunk_forward(x, Wr, br, g, W1, W2, sparse: bool = False):
+def chunk_forward(x, Wr, br, g, W1, W2, sparse: bool = False, norm: str = "rms"):
     """Full layer over one chunk -> (y fp64 [L,d], r fp64 [L,E], active bool [L,E])."""
     lib = _load()
     x = _c(x, np.uint16)
@@ -117,12 +133,12 @@ def chunk_forward(x, Wr, br, g, W1, W2, sparse: bool = False):
     E, de, _ = W1.shape
     y = np.zeros((L, d)); r = np.zeros((L, E)); act = np.zeros((L, E), np.uint8)
     rc = lib.oracle_chunk_forward(_ptr(x), L, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1), _ptr(W2),
-                                  E, de, int(bool(sparse)), _ptr(y), _ptr(r), _ptr(act))
+                                  E, de, int(bool(sparse)), NORMS[norm], _ptr(y), _ptr(r), _ptr(act))
     assert rc == 0
     return y, r, act.astype(bool)
 
 
-def tokens_forward_mt(x, Wr, br, g, W1, W2, threads: int, sparse: bool = False):
+def tokens_forward_mt(x, Wr, br, g, W1, W2, threads: int, sparse: bool = False, norm: str = "rms"):
     """Layer over n tokens [n,d] on `threads` host threads -> y fp64 [n,d]."""
     lib = _load()
     x = _c(x, np.uint16)
@@ -132,19 +148,19 @@ def tokens_forward_mt(x, Wr, br, g, W1, W2, threads: int, sparse: bool = False):
     E, de, _ = W1.shape
     y = np.zeros((n, d))
     rc = lib.oracle_tokens_forward_mt(_ptr(x), n, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1),
-                                      _ptr(W2), E, de, int(bool(sparse)), int(threads), _ptr(y))
+                                      _ptr(W2), E, de, int(bool(sparse)), NORMS[norm], int(threads), _ptr(y))
     assert rc == 0
     return y
 
 
-def chunk_reference(x, Wr, br, g, W1, W2, threads: int | None = None):
+def chunk_reference(x, Wr, br, g, W1, W2, threads: int | None = None, norm: str = "rms"):
     """Everything a parity test compares for one chunk: y, r, active flags, union and counts.
 
     y is the dense evaluation (every expert computed and multiplied by its router weight, zero for
     the inactive ones), spread over the host's cores by token; the pins check that this threaded call
     equals the single-threaded chunk forward bit for bit."""
-    _, r, act = router(x, Wr, br, g)
-    y = tokens_forward_mt(x, Wr, br, g, W1, W2, threads or available_cores(), sparse=False)
+    _, r, act = router(x, Wr, br, g, norm=norm)
+    y = tokens_forward_mt(x, Wr, br, g, W1, W2, threads or available_cores(), sparse=False, norm=norm)
     idx, tz, cz = union(act)
     return {"y": y, "r": r, "active": act, "active_idx": idx, "tls_zero": tz, "cls_zero": cz}
 

@@ -24,6 +24,11 @@
 // r = 0 and y = 0); Swish has beta = 1; the RMSNorm mean runs over all E entries, zeros included;
 // the union is listed in ascending expert order.
 //
+// The ReMoE router variant (intelliparadigm survey, section 5.1: the gate G = ReLU(x W_g) and the layer's
+// output the sum of G_i times expert i, divided by the sum of G): norm = 1 replaces the RMS by the sum of
+// the ReLU outputs, r_{t,i} = g_i a_{t,i} / sum_i a_{t,i} (r_t = 0 when every a is 0); the gain g is kept
+// (g = 1 gives the survey's formula).
+//
 // Storage: x is bf16 bit patterns [L,d]; Wr fp32 [d,E]; br fp32 [E] (may be null = no bias);
 // g fp32 [E]; W1 bf16 bits [E,de,d]; W2 bf16 bits [E,d,de]; everything row-major.
 
@@ -52,7 +57,7 @@ double swish(double u) {
 
 // Router for one token: s (pre-activation), r (normalised weights), active flags.
 void router_token(const uint16_t* xt, int d, const float* Wr, const float* br, const float* g,
-                  int E, double* s, double* r, uint8_t* act) {
+                  int E, int norm, double* s, double* r, uint8_t* act) {
   for (int i = 0; i < E; ++i) {
     double acc = 0.0;
     for (int k = 0; k < d; ++k) {
@@ -62,20 +67,24 @@ void router_token(const uint16_t* xt, int d, const float* Wr, const float* br, c
     if (br != nullptr && g_mutation != 1) acc += static_cast<double>(br[i]);  // planted 1: bias dropped
     s[i] = acc;
   }
-  double sumsq = 0.0;
+  double sumsq = 0.0, sum = 0.0;
   int n_pos = 0;
   for (int i = 0; i < E; ++i) {
     double a = s[i] > 0.0 ? s[i] : 0.0;
     sumsq += a * a;
+    sum += a;
     if (a > 0.0) ++n_pos;
   }
   // planted 3: mean over the active entries only instead of over all E
   double denom = (g_mutation == 3) ? static_cast<double>(n_pos > 0 ? n_pos : 1) : static_cast<double>(E);
   double ms = sumsq / denom;
+  // the normaliser: the RMS of the ReLU outputs (BlockFFN), or their sum (ReMoE)
+  double nrm = std::sqrt(ms);
+  if (norm == 1) nrm = (g_mutation == 8) ? sum / static_cast<double>(E) : sum;  // planted 8: the mean, not the sum
   for (int i = 0; i < E; ++i) {
     double a = s[i] > 0.0 ? s[i] : 0.0;
     act[i] = s[i] > 0.0 ? 1 : 0;
-    r[i] = (ms > 0.0) ? static_cast<double>(g[i]) * a / std::sqrt(ms) : 0.0;
+    r[i] = (nrm > 0.0) ? static_cast<double>(g[i]) * a / nrm : 0.0;
   }
 }
 
@@ -102,13 +111,13 @@ void expert_token(const uint16_t* xt, int d, const uint16_t* W1, const uint16_t*
 }
 
 void forward_tokens(int t0, int t1, const uint16_t* x, int d, const float* Wr, const float* br,
-                    const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de, int sparse,
+                    const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de, int sparse, int norm,
                     double* y, double* r_out, uint8_t* act_out) {
   std::vector<double> s(E), r(E), e(d);
   std::vector<uint8_t> act(E);
   for (int t = t0; t < t1; ++t) {
     const uint16_t* xt = x + static_cast<size_t>(t) * d;
-    router_token(xt, d, Wr, br, g, E, s.data(), r.data(), act.data());
+    router_token(xt, d, Wr, br, g, E, norm, s.data(), r.data(), act.data());
     double* yt = y + static_cast<size_t>(t) * d;
     for (int k = 0; k < d; ++k) yt[k] = 0.0;
     for (int i = 0; i < E; ++i) {
@@ -134,10 +143,10 @@ double oracle_swish(double u) { return swish(u); }
 
 // Router over a chunk: s, r as fp64 [L,E]; act as 0/1 bytes [L,E].
 int oracle_router(const uint16_t* x, int L, int d, const float* Wr, const float* br, const float* g,
-                  int E, double* s, double* r, uint8_t* act) {
-  if (bad_dims(L, d, E, 1)) return 1;
+                  int E, int norm, double* s, double* r, uint8_t* act) {
+  if (bad_dims(L, d, E, 1) || norm < 0 || norm > 1) return 1;
   for (int t = 0; t < L; ++t)
-    router_token(x + static_cast<size_t>(t) * d, d, Wr, br, g, E, s + static_cast<size_t>(t) * E,
+    router_token(x + static_cast<size_t>(t) * d, d, Wr, br, g, E, norm, s + static_cast<size_t>(t) * E,
                  r + static_cast<size_t>(t) * E, act + static_cast<size_t>(t) * E);
   return 0;
 }
@@ -166,6 +175,20 @@ int oracle_union(const uint8_t* act, int L, int E, int32_t* active_idx, int32_t*
   return 0;
 }
 
+// Cross-chunk expert reuse (the BlockFFN article, section 5): the number of experts in both of two unions,
+// each given as a list of expert indices, counted by marking one list and scanning the other.
+int oracle_union_overlap(const int32_t* a, int na, const int32_t* b, int nb, int E, int32_t* overlap) {
+  if (E <= 0 || na < 0 || nb < 0) return 1;
+  std::vector<uint8_t> in_b(static_cast<size_t>(E), 0);
+  for (int q = 0; q < nb; ++q)
+    if (b[q] >= 0 && b[q] < E) in_b[b[q]] = 1;
+  int hits = 0;
+  for (int q = 0; q < na; ++q)
+    if (a[q] >= 0 && a[q] < E && in_b[a[q]]) ++hits;
+  *overlap = hits;
+  return 0;
+}
+
 // One expert on one token (exposed for the special-case pins).
 int oracle_expert(const uint16_t* xt, int d, const uint16_t* W1, const uint16_t* W2, int de, int i,
                   double* out) {
@@ -179,9 +202,9 @@ int oracle_expert(const uint16_t* xt, int d, const uint16_t* W1, const uint16_t*
 // y fp64 [L,d]; r_out fp64 [L,E] and act_out [L,E] may be null.
 int oracle_chunk_forward(const uint16_t* x, int L, int d, const float* Wr, const float* br,
                          const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de,
-                         int sparse, double* y, double* r_out, uint8_t* act_out) {
-  if (bad_dims(L, d, E, de)) return 1;
-  forward_tokens(0, L, x, d, Wr, br, g, W1, W2, E, de, sparse, y, r_out, act_out);
+                         int sparse, int norm, double* y, double* r_out, uint8_t* act_out) {
+  if (bad_dims(L, d, E, de) || norm < 0 || norm > 1) return 1;
+  forward_tokens(0, L, x, d, Wr, br, g, W1, W2, E, de, sparse, norm, y, r_out, act_out);
   return 0;
 }
 
@@ -189,14 +212,14 @@ int oracle_chunk_forward(const uint16_t* x, int L, int d, const float* Wr, const
 // result is identical to the single-threaded call). Used for the timed CPU baseline.
 int oracle_tokens_forward_mt(const uint16_t* x, int n_tok, int d, const float* Wr, const float* br,
                              const float* g, const uint16_t* W1, const uint16_t* W2, int E, int de,
-                             int sparse, int threads, double* y) {
-  if (bad_dims(n_tok, d, E, de) || threads < 1) return 1;
+                             int sparse, int norm, int threads, double* y) {
+  if (bad_dims(n_tok, d, E, de) || threads < 1 || norm < 0 || norm > 1) return 1;
   std::vector<std::thread> pool;
   for (int w = 0; w < threads; ++w) {
     int t0 = static_cast<int>(static_cast<int64_t>(n_tok) * w / threads);
     int t1 = static_cast<int>(static_cast<int64_t>(n_tok) * (w + 1) / threads);
     if (g_mutation == 7) t1 = t0 + n_tok / threads;  // planted: ranges that drop the remainder tokens
-    pool.emplace_back(forward_tokens, t0, t1, x, d, Wr, br, g, W1, W2, E, de, sparse, y,
+    pool.emplace_back(forward_tokens, t0, t1, x, d, Wr, br, g, W1, W2, E, de, sparse, norm, y,
                       static_cast<double*>(nullptr), static_cast<uint8_t*>(nullptr));
   }
   for (auto& th : pool) th.join();

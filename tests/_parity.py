@@ -31,7 +31,7 @@ def bf16_tensor(bits: np.ndarray, device="cuda"):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(device).view(torch.bfloat16)
 
 
-def run_chunk(bffn, dl: DeviceLayer, x_bits: np.ndarray, bias=True, path=0, workspace=None, plain=False):
+def run_chunk(bffn, dl: DeviceLayer, x_bits: np.ndarray, bias=True, path=0, workspace=None, plain=False, flags=0):
     L, d = x_bits.shape
     E = dl.E
     dev = dl.Wr.device
@@ -52,7 +52,7 @@ def run_chunk(bffn, dl: DeviceLayer, x_bits: np.ndarray, bias=True, path=0, work
         counts = torch.full((2,), -7, dtype=torch.int32, device=dev)
         r = torch.full((L, E), float("nan"), dtype=torch.float32, device=dev)
         bffn.chunk_forward(x, dl.Wr, dl.g, dl.W1, dl.W2, y, idx, n, br=dl.br if bias else None,
-                           tok_mask=mask, counts=counts, r_out=r, path=path, workspace=workspace)
+                           tok_mask=mask, counts=counts, r_out=r, path=path, workspace=workspace, flags=flags)
     torch.cuda.synchronize()
     assert bffn.device_status(workspace) == 0
     n_act = int(n.item())
@@ -66,9 +66,9 @@ def run_chunk(bffn, dl: DeviceLayer, x_bits: np.ndarray, bias=True, path=0, work
     return out
 
 
-def reference(dl: DeviceLayer, x_bits, bias=True):
+def reference(dl: DeviceLayer, x_bits, bias=True, norm="rms"):
     lay = dl.lay
-    return oracle.chunk_reference(x_bits, lay.Wr, lay.br if bias else None, lay.g, lay.W1, lay.W2)
+    return oracle.chunk_reference(x_bits, lay.Wr, lay.br if bias else None, lay.g, lay.W1, lay.W2, norm=norm)
 
 
 def y_violations(y, y_ref):

@@ -71,7 +71,7 @@ def _call(bffn, **kw):
     dict(active_idx=None), dict(n_active=None),
     dict(x=FAKE + 2), dict(W1=FAKE + 8), dict(W2=FAKE + 4), dict(Wr=FAKE + 4), dict(y=FAKE + 2),
     dict(n_active=FAKE + 1), dict(br=FAKE + 2), dict(r_out=FAKE + 1), dict(workspace=FAKE + 16),
-    dict(flags=3), dict(flags=1 << 9), dict(flags=1 << 2), dict(flags=1 << 12),
+    dict(flags=3), dict(flags=1 << 11), dict(flags=1 << 2), dict(flags=1 << 12),
 ])
 def test_invalid_arguments_rejected_before_launch(bffn, kw):
     assert _call(bffn, **kw) == bffn.BFFN_EINVAL
@@ -138,3 +138,20 @@ def test_batch_workspace_size(bffn):
     assert n >= 4096 * 8 * 64 * 4 + 8 * 2 * 64 * 4 * 2048
     assert bffn.blockffn_batch_workspace_size(0, 8, 2048, 64, 256, 0) == 0
     assert bffn.blockffn_batch_workspace_size(4, 8, 2050, 64, 256, 0) == 0
+
+
+def test_router_variant_flag_is_accepted_by_validation(bffn):
+    # the flag passes argument checking (nothing is launched here: the placeholder x is misaligned, so the
+    # call still stops at validation) and unknown bits next to it do not
+    assert _call(bffn, x=FAKE + 2, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM) == bffn.BFFN_EINVAL
+    assert _call(bffn, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM | (1 << 11)) == bffn.BFFN_EINVAL
+    assert bffn.blockffn_batch_workspace_size(4, 8, 256, 16, 64, bffn.BFFN_FLAG_ROUTER_SUM_NORM) > 0
+    assert bffn.blockffn_batch_workspace_size(4, 8, 256, 16, 64, 1 << 11) == 0
+
+
+@pytest.mark.parametrize("kw", [dict(C=0), dict(E=0), dict(E=1025), dict(a=None), dict(overlap=FAKE + 2)])
+def test_union_overlap_validates(bffn, kw):
+    a = dict(a=FAKE, na=FAKE, b=FAKE, nb=FAKE, C=4, E=16, overlap=FAKE)
+    a.update(kw)
+    assert bffn.blockffn_union_overlap(a["a"], a["na"], a["b"], a["nb"], a["C"], a["E"], a["overlap"],
+                                       None) == bffn.BFFN_EINVAL

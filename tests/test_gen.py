@@ -78,3 +78,21 @@ def test_tiny_workload_sparsity():
     cls = cz / (w.n_chunks * w.E)
     assert abs(tls - 0.788) < 0.04
     assert abs(cls - gen.expected_cls(0.3, 8, 0.8)) < 0.06
+
+
+def test_sequence_chunks_share_more_experts_as_drift_grows():
+    # consecutive chunks of a drifting sequence: the mean overlap of consecutive unions (counted with
+    # Python sets from the fp64 pre-activations on the bf16 tokens) rises with the drift, and drift 0
+    # behaves like independent chunks
+    lay = gen.make_layer(3, 256, 32, 16, 1.0, 1.09)
+    rates = []
+    for drift in (0.0, 0.9, 0.99):
+        xs = gen.make_sequence_chunks(5, lay, 24, 8, 0.3, drift)
+        assert xs.shape == (24, 8, 256) and xs.dtype == np.uint16
+        unions = []
+        for x in xs:
+            s = gen.bf16_bits_to_f32(x).astype(np.float64) @ lay.Wr.astype(np.float64) + lay.br
+            assert np.abs(s).min() >= gen.MARGIN
+            unions.append(set(np.nonzero((s > 0).any(axis=0))[0].tolist()))
+        rates.append(np.mean([len(unions[k] & unions[k - 1]) / max(1, len(unions[k])) for k in range(1, 24)]))
+    assert rates[0] < rates[1] < rates[2]

@@ -27,7 +27,7 @@ class StackedLayers:
         self.W2 = torch.from_numpy(st(lambda l: l.W2).view(np.int16)).to(device).view(torch.bfloat16)
 
 
-def run_batch(bffn, sl, xs, layer=None, teams=0, workspace=None, bias=True):
+def run_batch(bffn, sl, xs, layer=None, teams=0, workspace=None, bias=True, flags=0):
     import torch
     C, L, d = xs.shape
     E = sl.E
@@ -39,7 +39,7 @@ def run_batch(bffn, sl, xs, layer=None, teams=0, workspace=None, bias=True):
     mask = torch.zeros((C, L, (E + 31) // 32), dtype=torch.int32, device="cuda")
     lt = None if layer is None else torch.from_numpy(np.asarray(layer, np.int32)).cuda()
     bffn.chunk_forward_batch(x, sl.Wr, sl.g, sl.W1, sl.W2, y, idx, n, layer=lt, br=sl.br if bias else None,
-                             counts=counts, tok_mask=mask, teams=teams, workspace=workspace)
+                             counts=counts, tok_mask=mask, teams=teams, workspace=workspace, flags=flags)
     torch.cuda.synchronize()
     status = bffn.device_status(workspace)
     words = mask.cpu().numpy().view(np.uint32)
@@ -48,10 +48,10 @@ def run_batch(bffn, sl, xs, layer=None, teams=0, workspace=None, bias=True):
             "counts": counts.cpu().numpy(), "active": bits, "status": status}
 
 
-def check_chunk(got, c, lay, x, bias=True):
+def check_chunk(got, c, lay, x, bias=True, norm="rms"):
     import oracle
     from _parity import y_violations
-    ref = oracle.chunk_reference(x, lay.Wr, lay.br if bias else None, lay.g, lay.W1, lay.W2)
+    ref = oracle.chunk_reference(x, lay.Wr, lay.br if bias else None, lay.g, lay.W1, lay.W2, norm=norm)
     n = int(got["n"][c])
     assert n == len(ref["active_idx"]), (c, n, len(ref["active_idx"]))
     assert np.array_equal(got["idx"][c][:n], ref["active_idx"]), c
@@ -210,3 +210,16 @@ def test_every_expert_active_long_phases(bffn, cuda_device):
     assert got["status"] == bffn.BFFN_OK
     assert np.all(got["n"] == 128)
     check_chunk(got, C - 1, lay, xs[C - 1])
+
+
+def test_remoe_router_variant(bffn, cuda_device):
+    # the sum-normalised (ReMoE) router through the batched call: two layers with unequal gains
+    lays = [gen.make_layer(61 + k, 512, 32, 128, 1.0, 1.09) for k in range(2)]
+    for lay in lays:
+        lay.g[:] = np.linspace(0.5, 2.0, 32, dtype=np.float32)
+    sl = StackedLayers(lays)
+    xs = np.stack([gen.make_chunks(61, lays[c % 2], 1, 8, 0.3, stream=c)[0] for c in range(6)])
+    got = run_batch(bffn, sl, xs, teams=2, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM)
+    assert got["status"] == bffn.BFFN_OK
+    for c in range(6):
+        check_chunk(got, c, lays[c % 2], xs[c], norm="sum")

@@ -230,3 +230,48 @@ def test_allocation_failure_is_reported(bffn, cuda_device, monkeypatch):
     dl = _layer(14, 256, 16, 64)
     x = gen.make_chunks(14, dl.lay, 1, 8, 0.3)[0]
     assert_parity(run_chunk(bffn, dl, x), reference(dl, x), 8, 16)
+
+
+@pytest.mark.parametrize("L", [5, 8, 16])
+def test_remoe_router_variant(bffn, cuda_device, L):
+    # BFFN_FLAG_ROUTER_SUM_NORM: r = g relu(s) / sum relu(s) (the ReMoE router) on both per-chunk kernels;
+    # masks, union and counts as for RMSNorm, r and y against the oracle's sum-normalised router
+    from _parity import assert_parity, reference, run_chunk
+    dl = _layer(15, 512, 32, 128)
+    dl.lay.g[:] = np.linspace(0.5, 2.0, 32, dtype=np.float32)
+    dl.g.copy_(__import__("torch").from_numpy(dl.lay.g))
+    for x in gen.make_chunks(15, dl.lay, 2, L, 0.3):
+        got = run_chunk(bffn, dl, x, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM)
+        assert_parity(got, reference(dl, x, norm="sum"), L, 32)
+
+
+def test_union_overlap_of_consecutive_chunks(bffn, cuda_device):
+    # a drifting sequence's consecutive chunks through the per-chunk path; blockffn_union_overlap of step
+    # k's and step k-1's active lists equals the overlap of the oracle's unions (an integer, bit-exact);
+    # calls made with BFFN_FLAG_KEEP_EXPERTS_IN_L2 return the same bits as calls without it
+    import oracle
+    import torch
+    from _parity import bf16_tensor, run_chunk, assert_parity, reference
+    dl = _layer(16, 512, 32, 128, beta=1.0)
+    xs = gen.make_sequence_chunks(16, dl.lay, 6, 8, 0.3, 0.95)
+    idx = torch.full((6, 32), -1, dtype=torch.int32, device="cuda")
+    n = torch.zeros(6, dtype=torch.int32, device="cuda")
+    unions = []
+    for k, x in enumerate(xs):
+        got = run_chunk(bffn, dl, x, flags=bffn.BFFN_FLAG_KEEP_EXPERTS_IN_L2 if k % 2 else 0)
+        ref = reference(dl, x)
+        assert_parity(got, ref, 8, 32)
+        if k % 2:  # the cache policy changes no arithmetic
+            again = run_chunk(bffn, dl, x)
+            assert np.array_equal(again["y"], got["y"])
+        idx[k, :got["n_active"]] = torch.from_numpy(got["active_idx"].astype(np.int32)).cuda()
+        n[k] = got["n_active"]
+        unions.append(ref["active_idx"])
+    overlap = torch.full((5,), -1, dtype=torch.int32, device="cuda")
+    rc = bffn.blockffn_union_overlap(idx[:5].data_ptr(), n[:5].data_ptr(), idx[1:].data_ptr(), n[1:].data_ptr(), 5, 32,
+                                     overlap.data_ptr(), torch.cuda.current_stream().cuda_stream)
+    assert rc == bffn.BFFN_OK
+    torch.cuda.synchronize()
+    want = [oracle.union_overlap(unions[k], unions[k + 1], 32) for k in range(5)]
+    assert overlap.cpu().numpy().tolist() == want
+    assert max(want) > 0

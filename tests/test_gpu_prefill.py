@@ -80,3 +80,12 @@ def test_prefill_full_size_sampled(bffn, cuda_device):
     rms_all = float(np.sqrt(np.mean(y_all ** 2)))
     bad = np.abs(got["y"][toks] - y_ref) > 2e-2 * np.abs(y_ref) + 1e-3 * rms_all
     assert not bad.any(), f"{int(bad.sum())} of {bad.size} sampled y elements out of tolerance"
+
+
+def test_prefill_remoe_router_variant(bffn, cuda_device):
+    # the sum-normalised (ReMoE) router on the prefill path
+    from _parity import assert_parity, reference, run_chunk
+    dl = _layer(17, 256, 24, 128, 0.6)
+    x = _tokens(dl, 18, 100)
+    got = run_chunk(bffn, dl, x, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM)
+    assert_parity(got, reference(dl, x, norm="sum"), 100, 24)

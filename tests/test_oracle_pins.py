@@ -60,8 +60,9 @@ def _small(seed=3, d=48, E=12, de=16, L=6, gain=None):
 def pin_golden(name):
     spec, x, Wr, br, g, W1, W2 = _golden_inputs(name)
     exp = spec["expected"]
-    s, r, act = oracle.router(x, Wr, br, g)
-    y, r2, act2 = oracle.chunk_forward(x, Wr, br, g, W1, W2, sparse=False)
+    norm = spec.get("norm", "rms")
+    s, r, act = oracle.router(x, Wr, br, g, norm=norm)
+    y, r2, act2 = oracle.chunk_forward(x, Wr, br, g, W1, W2, sparse=False, norm=norm)
     idx, tz, cz = oracle.union(act)
     want_s = np.vectorize(_closed_form)(np.array(exp["s"], dtype=object)).astype(float)
     want_r = np.vectorize(_closed_form)(np.array(exp["r"], dtype=object)).astype(float)
@@ -79,6 +80,43 @@ def pin_golden_e4():
 
 def pin_golden_bias_gain():
     return pin_golden("worked_example_bias_gain.json")
+
+
+def pin_golden_e4_sum_norm():
+    return pin_golden("worked_example_e4_sum.json")
+
+
+def pin_sum_norm_invariant():
+    """ReMoE router: sum_i r_{t,i} / g_i = 1 for every token with an active expert (r = 0 otherwise), the
+    active sets are those of the RMSNorm router, and r is the RMSNorm router's r rescaled per token by
+    rms / sum (the two normalisers of the same ReLU outputs)."""
+    rng = np.random.default_rng(12)
+    gain = rng.uniform(0.5, 2.0, 12)
+    lay, x = _small(seed=19, gain=gain)
+    s, r, act = oracle.router(x, lay.Wr, lay.br, lay.g, norm="sum")
+    _, r_rms, act_rms = oracle.router(x, lay.Wr, lay.br, lay.g, norm="rms")
+    ok = np.array_equal(act, act_rms) and bool(act.any()) and not bool(act.all())
+    gg = lay.g.astype(np.float64)
+    for t in range(x.shape[0]):
+        a = np.maximum(s[t], 0.0)
+        if act[t].any():
+            ok &= abs(np.sum(r[t] / gg) - 1.0) < 1e-14
+            ok &= np.allclose(r[t] * a.sum(), r_rms[t] * math.sqrt(np.mean(a ** 2)), rtol=1e-13, atol=1e-15)
+        else:
+            ok &= bool(np.all(r[t] == 0.0))
+    return bool(ok)
+
+
+def pin_sum_norm_layer_equals_weighted_experts():
+    """ReMoE layer: y_t = sum_i r_{t,i} E_i(x_t) with r from the sum-normalised router, every expert
+    evaluated on its own (oracle_expert) and weighted here."""
+    lay, x = _small(seed=23, L=3)
+    y, r, act = oracle.chunk_forward(x, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, norm="sum")
+    want = np.zeros_like(y)
+    for t in range(x.shape[0]):
+        for i in range(lay.E):
+            want[t] += r[t, i] * oracle.expert(x[t], lay.W1, lay.W2, i)
+    return bool(np.allclose(y, want, rtol=1e-12, atol=1e-14))
 
 
 def pin_rmsnorm_invariant():
@@ -183,9 +221,25 @@ def pin_tokens_forward_mt():
     return True
 
 
+def pin_union_overlap():
+    """The overlap of two unions against Python sets on random lists (including duplicates across lists,
+    disjoint and identical lists), and |A ∩ A| = |A|."""
+    rng = np.random.default_rng(31)
+    for E in (1, 7, 40, 1024):
+        for _ in range(20):
+            a = np.sort(rng.choice(E, rng.integers(0, E + 1), replace=False))
+            b = np.sort(rng.choice(E, rng.integers(0, E + 1), replace=False))
+            if oracle.union_overlap(a, b, E) != len(set(a.tolist()) & set(b.tolist())):
+                return False
+            if oracle.union_overlap(a, a, E) != len(a):
+                return False
+    return oracle.union_overlap([0, 5], [1, 2], 8) == 0 and oracle.union_overlap([3], [3], 4) == 1
+
+
 ALL_PINS = [pin_golden_e4, pin_golden_bias_gain, pin_rmsnorm_invariant, pin_sparse_equals_dense,
             pin_single_expert_mlp, pin_counts_bruteforce, pin_scale_invariance, pin_swish,
-            pin_token_permutation, pin_tokens_forward_mt]
+            pin_token_permutation, pin_tokens_forward_mt, pin_golden_e4_sum_norm, pin_sum_norm_invariant,
+            pin_sum_norm_layer_equals_weighted_experts, pin_union_overlap]
 
 
 @pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
@@ -194,11 +248,12 @@ def test_pin(pin):
     assert pin()
 
 
-@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6, 7])
+@pytest.mark.parametrize("mutation", [1, 2, 3, 4, 5, 6, 7, 8])
 def test_planted_mistake_is_caught(mutation):
     """Each mistake planted in the oracle (dropped bias, flipped sigmoid sign, RMSNorm mean over the
     active entries only, reversed router index, transposed W2, an expert dropped from the union,
-    threaded token ranges that drop tokens) must make at least one pin fail."""
+    threaded token ranges that drop tokens, the ReMoE normaliser taken as the mean instead of the sum)
+    must make at least one pin fail."""
     caught = []
     try:
         oracle.set_mutation(mutation)
