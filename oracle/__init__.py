@@ -48,6 +48,9 @@ def _load():
             lib.oracle_chunk_forward.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, dptr, dptr, p]
             lib.oracle_tokens_forward_mt.argtypes = [p, i, i, p, p, p, p, p, i, i, i, i, i, dptr]
             lib.oracle_union_overlap.argtypes = [p, i, p, i, i, p]
+            dbl = C.c_double
+            lib.oracle_cls_losses.argtypes = [p, i, i, i, p, p, i, dbl, dbl, dbl, dptr, dptr, dptr, dptr, dptr]
+            lib.oracle_cls_losses.restype = i
             for f in ("oracle_router", "oracle_union", "oracle_expert", "oracle_chunk_forward",
                       "oracle_tokens_forward_mt", "oracle_union_overlap"):
                 getattr(lib, f).restype = i
@@ -111,6 +114,22 @@ def union_overlap(a, b, E) -> int:
     rc = lib.oracle_union_overlap(_ptr(a), a.size, _ptr(b), b.size, int(E), _ptr(out))
     assert rc == 0
     return int(out[0])
+
+
+def cls_losses(x, C, L, Wr, br, alpha, w_al=1.0, w_cs=1.0):
+    """The CLS-aware objectives over C chunks of L tokens (x bf16 bits [C*L, d]) and their backward through
+    the router: returns (L_AL, L_CS, dS [C*L,E], dWr [d,E], db [E], dx [C*L,d]) for J = w_al L_AL + w_cs L_CS."""
+    lib = _load()
+    x = _c(x, np.uint16)
+    Wr, br = _c(Wr, np.float32), _c(br, np.float32)
+    T, d = x.shape
+    E = Wr.shape[1]
+    assert T == C * L
+    loss = np.zeros(2); dS = np.zeros((T, E)); dWr = np.zeros((d, E)); db = np.zeros(E); dx = np.zeros((T, d))
+    rc = lib.oracle_cls_losses(_ptr(x), int(C), int(L), d, _ptr(Wr), _ptr(br), E, float(alpha), float(w_al),
+                               float(w_cs), _ptr(loss), _ptr(dS), _ptr(dWr), _ptr(db), _ptr(dx))
+    assert rc == 0
+    return loss[0], loss[1], dS, dWr, db, dx
 
 
 def expert(xt, W1, W2, i):

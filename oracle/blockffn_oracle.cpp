@@ -29,6 +29,9 @@
 // the ReLU outputs, r_{t,i} = g_i a_{t,i} / sum_i a_{t,i} (r_t = 0 when every a is 0); the gain g is kept
 // (g = 1 gives the survey's formula).
 //
+// The CLS-aware training objectives (activation locality, chunk sparsification; article, section 3) and
+// their backward through the router are at the end of this file, with the readings they take.
+//
 // Storage: x is bf16 bit patterns [L,d]; Wr fp32 [d,E]; br fp32 [E] (may be null = no bias);
 // g fp32 [E]; W1 bf16 bits [E,de,d]; W2 bf16 bits [E,d,de]; everything row-major.
 
@@ -223,6 +226,102 @@ int oracle_tokens_forward_mt(const uint16_t* x, int n_tok, int d, const float* W
                       static_cast<double*>(nullptr), static_cast<uint8_t*>(nullptr));
   }
   for (auto& th : pool) th.join();
+  return 0;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------------------
+// CLS-aware training objectives (lsdiaocha.cn BlockFFN article, section 3) and their backward through the
+// router, in fp64.  The pages describe both objectives in words only; the readings taken here:
+//   p_{t,i} = sigmoid(alpha s_{t,i})              the "sharp sigmoid" that approximates the activation
+//                                                 pattern 1[s > 0] (alpha large)
+//   activation locality: the binary cross-entropy between each token's approximate pattern and the next
+//     token's (the LeftShift of p along the chunk), both soft and both carrying gradient, averaged over
+//     the chunks' (L - 1) E adjacent pairs:  L_AL = mean_{c, t < L-1, i} BCE(p_{c,t,i}; q = p_{c,t+1,i})
+//     with BCE(p; q) = -(q log p + (1 - q) log(1 - p))
+//   chunk sparsification: the probability that at least one token of the chunk activates expert i,
+//     averaged over chunks and experts:  L_CS = mean_{c,i} (1 - prod_t (1 - p_{c,t,i}))
+// and the combined objective J = w_al L_AL + w_cs L_CS.  Gradients (the plain chain rule):
+//   dJ/ds_{c,t,i} = w_al alpha (p_t - p_{t+1}) / N_AL [t < L-1]            (through the predicted side)
+//                 - w_al alpha^2 s_{t-1} p_t (1 - p_t) / N_AL [t > 0]      (through the LeftShift target:
+//                                                   d BCE / d q = -logit(p_{t-1}) = -alpha s_{t-1})
+//                 + w_cs alpha p_t (1 - p_t) prod_{t' != t} (1 - p_{c,t',i}) / N_CS
+//   dJ/dWr[k,i] = sum_{c,t} x_{c,t,k} dJ/ds_{c,t,i};  dJ/db_i = sum_{c,t} dJ/ds_{c,t,i};
+//   dJ/dx_{c,t,k} = sum_i dJ/ds_{c,t,i} Wr[k,i].
+namespace {
+double log_sigmoid(double z) { return z >= 0.0 ? -std::log1p(std::exp(-z)) : z - std::log1p(std::exp(z)); }
+}  // namespace
+
+extern "C" {
+
+// x bf16 bits [C*L, d]; Wr [d, E]; br [E] or null.  Out: loss[2] = {L_AL, L_CS} (the unweighted objectives),
+// dS [C*L, E], dWr [d, E], db [E] (may be null), dx [C*L, d] (may be null), all for J = w_al L_AL + w_cs L_CS.
+int oracle_cls_losses(const uint16_t* x, int C, int L, int d, const float* Wr, const float* br, int E,
+                      double alpha, double w_al, double w_cs, double* loss, double* dS, double* dWr, double* db,
+                      double* dx) {
+  if (C < 1 || L < 1 || d < 1 || E < 1) return 1;
+  const int T = C * L;
+  std::vector<double> s(static_cast<size_t>(T) * E), p(s.size());
+  for (int t = 0; t < T; ++t)
+    for (int i = 0; i < E; ++i) {
+      double acc = 0.0;
+      for (int k = 0; k < d; ++k)
+        acc += widen_bf16(x[static_cast<size_t>(t) * d + k]) * static_cast<double>(Wr[static_cast<size_t>(k) * E + i]);
+      if (br) acc += static_cast<double>(br[i]);
+      s[static_cast<size_t>(t) * E + i] = acc;
+      p[static_cast<size_t>(t) * E + i] = 1.0 / (1.0 + std::exp(-alpha * acc));
+    }
+  const double n_al = static_cast<double>(C) * (L - 1) * E, n_cs = static_cast<double>(C) * E;
+  double l_al = 0.0, l_cs = 0.0;
+  for (size_t q = 0; q < s.size(); ++q) dS[q] = 0.0;
+  for (int c = 0; c < C; ++c)
+    for (int i = 0; i < E; ++i) {
+      double keep_all = 1.0;  // prod_t (1 - p)
+      for (int t = 0; t < L; ++t) {
+        const size_t q = (static_cast<size_t>(c) * L + t) * E + i;
+        keep_all *= 1.0 - p[q];
+        if (t + 1 < L) {
+          // planted 11: the shift taken the other way (token t+1 predicts token t's pattern)
+          const size_t pred = (g_mutation == 11) ? q + E : q, targ = (g_mutation == 11) ? q : q + E;
+          const double y = p[targ];  // the next token's pattern
+          const double z = alpha * s[pred];
+          l_al += -(y * log_sigmoid(z) + (1.0 - y) * log_sigmoid(-z));
+          dS[pred] += w_al * alpha * (p[pred] - y) / n_al;
+          if (g_mutation != 9)  // planted 9: no gradient through the shifted target
+            dS[targ] += -w_al * alpha * z * y * (1.0 - y) / n_al;
+        }
+      }
+      l_cs += 1.0 - keep_all;
+      for (int t = 0; t < L; ++t) {
+        const size_t q = (static_cast<size_t>(c) * L + t) * E + i;
+        double others = 1.0;  // prod_{t' != t} (1 - p)
+        for (int u = 0; u < L; ++u)
+          if (u != t || g_mutation == 10) others *= 1.0 - p[(static_cast<size_t>(c) * L + u) * E + i];  // planted 10
+        dS[q] += w_cs * alpha * p[q] * (1.0 - p[q]) * others / n_cs;
+      }
+    }
+  loss[0] = L > 1 ? l_al / n_al : 0.0;
+  loss[1] = l_cs / n_cs;
+  for (int k = 0; k < d; ++k)
+    for (int i = 0; i < E; ++i) {
+      double acc = 0.0;
+      for (int t = 0; t < T; ++t) acc += widen_bf16(x[static_cast<size_t>(t) * d + k]) * dS[static_cast<size_t>(t) * E + i];
+      dWr[static_cast<size_t>(k) * E + i] = acc;
+    }
+  if (db)
+    for (int i = 0; i < E; ++i) {
+      double acc = 0.0;
+      for (int t = 0; t < T; ++t) acc += dS[static_cast<size_t>(t) * E + i];
+      db[i] = acc;
+    }
+  if (dx)
+    for (int t = 0; t < T; ++t)
+      for (int k = 0; k < d; ++k) {
+        double acc = 0.0;
+        for (int i = 0; i < E; ++i) acc += dS[static_cast<size_t>(t) * E + i] * static_cast<double>(Wr[static_cast<size_t>(k) * E + i]);
+        dx[static_cast<size_t>(t) * d + k] = acc;
+      }
   return 0;
 }
 
