@@ -698,6 +698,86 @@ def run_reuse(args):
                 print(json.dumps(line), flush=True)
 
 
+def run_cls_losses(args):
+    """The CLS-aware losses and their backward through the router (blockffn_cls_losses): one step = the
+    activation-locality and chunk-sparsification losses of a training batch of --chunks chunks of 8 tokens
+    (default 4096: 32768 tokens, x 128 MiB, above the 126 MB L2) with dS, dWr, db and dx, at the decode
+    layer's router shape (d = 2048, E = 64).  Roofline: the step's algorithmic bytes (x read once, Wr, dS
+    and dx written once) over its CUDA-event time; the kernels' shares come from the ncu launch list.
+    The oracle is timed beside it on a bounded sample of whole chunks."""
+    import numpy as np
+    import torch
+
+    import chunk_sparse_moe_router_b200 as bffn
+    import gen
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    C, L, d, E, alpha = args.chunks or 4096, 8, 2048, 64, 4.0
+    T = C * L
+    lay = gen.make_layer(0, d, E, 8, beta=1.04, var_x=1.09)
+    x_np = gen.make_chunks(0, lay, C, L, 0.3).reshape(T, d)
+    x = torch.from_numpy(x_np.view(np.int16)).view(torch.bfloat16).to(device)
+    Wr, br = torch.from_numpy(lay.Wr).to(device), torch.from_numpy(lay.br).to(device)
+    f32 = dict(dtype=torch.float32, device=device)
+    loss, dS, dWr, db, dx = (torch.empty(2, **f32), torch.empty(T, E, **f32), torch.empty(d, E, **f32),
+                             torch.empty(E, **f32), torch.empty(T, d, **f32))
+    ws = torch.empty(bffn.blockffn_cls_losses_workspace_size(C, L, d, E), dtype=torch.uint8, device=device)
+    s = torch.cuda.Stream(device)
+
+    def step():
+        bffn.cls_losses(x, C, L, Wr, br, alpha, 1.0, 1.0, loss, dS, dWr, db, dx, workspace=ws,
+                        stream=s.cuda_stream)
+
+    with torch.cuda.stream(s):
+        step()
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()  # one step per replay: no host work between steps
+        graph.capture_begin()
+        step()
+        graph.capture_end()
+        for _ in range(args.warmup):
+            graph.replay()
+        s.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(0) as clocks:
+            e0.record(s)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(s)
+            e1.synchronize()
+        clk = clocks.summary()
+        del graph
+    ms = e0.elapsed_time(e1) / args.steps
+    alg = T * d * 2 + d * E * 4 + E * 4 + T * E * 4 + d * E * 4 + E * 4 + T * d * 4 + 8
+    peak, peak_kind = measured_peaks()
+    gbs = alg / (ms * 1e-3) / 1e9
+    line = {"metric": "CLS-aware losses + router backward tokens/s and achieved HBM GB/s over the step's I/O",
+            "value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp32 (bf16 x; fp32 operands as bf16 hi+lo pairs on the tensor cores)",
+            "data": "synthetic",
+            "config": {"workload": f"cls_losses_C{C}_L{L}_d{d}_E{E}", "tokens": T, "alpha": alpha,
+                       "l2": "inputs larger than L2 (x 128 MiB, dx 256 MiB written per step)"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                         "algorithmic_bytes_per_step": alg},
+            "losses": [round(float(v), 6) for v in loss.cpu()],
+            "gpu_launches": 6 * args.steps, "clocks": clk}
+    if not args.no_cpu_baseline:
+        import oracle
+        n = 0
+        t0 = time.time()
+        while time.time() - t0 < args.cpu_seconds and n < C:
+            m = min(64, C - n)
+            oracle.cls_losses(x_np[n * L:(n + m) * L], m, L, lay.Wr, lay.br, alpha)
+            n += m
+        dt = time.time() - t0
+        line["cpu_baseline"] = {"value": round(n * L / dt, 1), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} chunks ({n * L} tokens) in groups of 64 chunks, {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 # ---------------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(w, lay0, x_host_np, seconds, y_gpu=None, n_gpu=None):
     """The fp64 dense oracle timed on this host's cores on a bounded sample of the workload (tokens
@@ -791,7 +871,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse"])
+                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses"])
     ap.add_argument("--drift", default="0.0,0.9,0.97",
                     help="--workload reuse: drift of the chunk bases of a sequence (0: independent chunks)")
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
@@ -831,6 +911,9 @@ def main():
         return
     if args.workload == "reuse":
         run_reuse(args)
+        return
+    if args.workload == "cls_losses":
+        run_cls_losses(args)
         return
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":

@@ -29,7 +29,7 @@ def BFFN_FLAGS_SHARE(k: int) -> int:
     return int(k) << 4
 
 # Every symbol include/blockffn.h declares: name -> (restype, argtypes)
-_P, _I, _S = C.c_void_p, C.c_int, C.c_size_t
+_P, _I, _S, _F = C.c_void_p, C.c_int, C.c_size_t, C.c_float
 SIGNATURES = {
     "blockffn_chunk_forward": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P]),
     "blockffn_chunk_forward_ex": (_I, [_P, _I, _I, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P,
@@ -40,6 +40,8 @@ SIGNATURES = {
                                          _I, _P, _S, _P]),
     "blockffn_batch_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
     "blockffn_union_overlap": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
+    "blockffn_cls_losses": (_I, [_P, _I, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "blockffn_cls_losses_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_init": (_I, [_P, _S, _P]),
     "blockffn_device_status": (_I, [_P, _P]),
@@ -106,6 +108,16 @@ def blockffn_noalloc_device_status(stream):
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # BFFN_NOALLOC_SCRATCH_BYTES in include/blockffn.h
+
+
+def blockffn_cls_losses(x, C, L, d, Wr, br, E, alpha, w_al, w_cs, loss, dS, dWr, db, dx, workspace,
+                        workspace_bytes, stream):
+    return _lib.blockffn_cls_losses(x, C, L, d, Wr, br, E, alpha, w_al, w_cs, loss, dS, dWr, db, dx, workspace,
+                                    workspace_bytes, stream)
+
+
+def blockffn_cls_losses_workspace_size(C, L, d, E):
+    return _lib.blockffn_cls_losses_workspace_size(C, L, d, E)
 
 
 def blockffn_workspace_size(L, d, E, de):
@@ -227,6 +239,49 @@ def new_batch_workspace(C, L, d, E, de, teams=0, device="cuda"):
     if n == 0:
         raise BlockFFNError(BFFN_EINVAL, "blockffn_batch_workspace_size")
     return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def cls_losses(x, C, L, Wr, br=None, alpha=1.0, w_al=1.0, w_cs=1.0, loss=None, dS=None, dWr=None, db=None,
+               dx=None, want_dWr=True, want_db=True, want_dx=True, workspace=None, stream=None):
+    """The CLS-aware objectives over C chunks of L tokens (x bf16 [C*L, d], Wr fp32 [d, E], br fp32 [E])
+    and the backward of J = w_al L_AL + w_cs L_CS through the router.  Returns (loss fp32 [2] = {L_AL,
+    L_CS}, dS fp32 [C*L, E], dWr fp32 [d, E] or None, db fp32 [E] or None, dx fp32 [C*L, d] or None); the
+    outputs are allocated unless given.  Raises BlockFFNError."""
+    import torch
+
+    T, d = x.shape
+    E = Wr.shape[1]
+    dev = x.device
+    if T != C * L:
+        raise ValueError(f"x has {T} rows, expected C * L = {C * L}")
+    _check(x, "x", torch.bfloat16, (T, d), dev)
+    _check(Wr, "Wr", torch.float32, (d, E), dev)
+    if br is not None:
+        _check(br, "br", torch.float32, (E,), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    loss = torch.empty(2, **f32) if loss is None else loss
+    dS = torch.empty(T, E, **f32) if dS is None else dS
+    dWr = (torch.empty(d, E, **f32) if want_dWr else None) if dWr is None else dWr
+    db = (torch.empty(E, **f32) if want_db else None) if db is None else db
+    dx = (torch.empty(T, d, **f32) if want_dx else None) if dx is None else dx
+    _check(loss, "loss", torch.float32, (2,), dev)
+    _check(dS, "dS", torch.float32, (T, E), dev)
+    for t, name, shape in ((dWr, "dWr", (d, E)), (db, "db", (E,)), (dx, "dx", (T, d))):
+        if t is not None:
+            _check(t, name, torch.float32, shape, dev)
+    need = blockffn_cls_losses_workspace_size(C, L, d, E)
+    if need == 0:
+        raise BlockFFNError(BFFN_EINVAL, "blockffn_cls_losses_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = blockffn_cls_losses(_ptr(x), C, L, d, _ptr(Wr), _ptr(br), E, float(alpha), float(w_al), float(w_cs),
+                             _ptr(loss), _ptr(dS), _ptr(dWr), _ptr(db), _ptr(dx), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_cls_losses")
+    return loss, dS, dWr, db, dx
 
 
 def device_status(workspace=None, stream=None):

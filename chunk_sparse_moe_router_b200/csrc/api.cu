@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/blockffn.h: argument checks, workspace handling and
 // the kernel launches of one BlockFFN chunk-layer forward.
+#include <cmath>
 #include <cstdlib>
 #include <mutex>
 
@@ -569,6 +570,34 @@ int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* n_active_
   const cudaError_t err =
       union_overlap_launch(active_idx_a, n_active_a, active_idx_b, n_active_b, C, E, overlap,
                            static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
+}
+
+size_t blockffn_cls_losses_workspace_size(int C, int L, int d, int E) {
+  if (C < 1 || L < 1 || d < 8 || d % 8 != 0 || E < 1 || E > kMaxE || 1ll * C * L > (1ll << 30)) return 0;
+  return cls::plan(C, L, d, E).total;
+}
+
+int blockffn_cls_losses(const void* x, int C, int L, int d, const float* Wr, const float* br, int E, float alpha,
+                        float w_al, float w_cs, float* loss, float* dS, float* dWr, float* db, float* dx,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  const size_t need = blockffn_cls_losses_workspace_size(C, L, d, E);
+  if (need == 0) return BFFN_EINVAL;
+  if (!(alpha > 0.f) || !std::isfinite(alpha) || !std::isfinite(w_al) || !std::isfinite(w_cs)) return BFFN_EINVAL;
+  if (x == nullptr || !aligned16(x) || Wr == nullptr || !aligned4(Wr) || loss == nullptr || !aligned4(loss) ||
+      dS == nullptr || !aligned4(dS) || workspace == nullptr || !aligned256(workspace))
+    return BFFN_EINVAL;
+  if ((br != nullptr && !aligned4(br)) || (dWr != nullptr && !aligned4(dWr)) || (db != nullptr && !aligned4(db)) ||
+      (dx != nullptr && !aligned16(dx)))
+    return BFFN_EINVAL;
+  if (!cls::chunk_fits(L)) return BFFN_EUNSUPPORTED;
+  if (workspace_bytes < need) return BFFN_ENOMEM;
+  DeviceInfo di;
+  int dev = 0;
+  const int rc = device_info(&di, &dev);
+  if (rc != BFFN_OK) return rc;
+  const cudaError_t err = cls::launch(x, C, L, d, Wr, br, E, alpha, w_al, w_cs, loss, dS, dWr, db, dx, workspace,
+                                      di.num_sms, static_cast<cudaStream_t>(stream));
   return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
 }
 

@@ -397,4 +397,20 @@ struct PrefillLaunch {
 bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, PrefillParams* p, PrefillLaunch* out);
 cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st);
 
+// ---------------------------------------------------------------- CLS-aware losses (cls_losses.cu)
+namespace cls {
+constexpr int kTargetCtas = 296;               // dWr grid: two CTAs on each SM of a B200
+constexpr int kTargetCtasTerms = 1184;         // chunk_terms grid: eight CTAs on each SM
+constexpr int kMaxChunkTileBytes = 128 << 10;  // s tile of 4 chunks x 64 experts: L <= 128
+struct Plan {
+  int T, Ep, dtiles, tok_per_split, splits, b_rows;
+  size_t wr_off, ds_off, part_off, loss_off, db_off, total;
+};
+Plan plan(int C, int L, int d, int E);
+bool chunk_fits(int L);
+cudaError_t launch(const void* x, int C, int L, int d, const float* Wr, const float* br, int E, float alpha,
+                   float w_al, float w_cs, float* loss, float* dS, float* dWr, float* db, float* dx, void* ws,
+                   int num_sms, cudaStream_t st);
+}  // namespace cls
+
 }  // namespace bffn

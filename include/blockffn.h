@@ -193,6 +193,39 @@ BFFN_API int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* 
                                     int32_t* overlap, void* stream);
 
 /*
+ * The CLS-aware training objectives and their backward through the router (lsdiaocha.cn BlockFFN article,
+ * section 3: an activation-locality loss, a binary cross-entropy between adjacent tokens' activation
+ * patterns compared through LeftShift, the patterns approximated by a sharp sigmoid; and a
+ * chunk-sparsification loss, the probability that an expert is activated by at least one token of a
+ * chunk of L consecutive tokens, minimised).  With s = x Wr + br and p = sigmoid(alpha s):
+ *   L_AL = mean over chunks c, adjacent pairs (t, t+1) of the chunk and experts i of
+ *          BCE(p_{c,t,i}; q = p_{c,t+1,i}) = -(q log p + (1 - q) log(1 - p))   (0 when L = 1)
+ *   L_CS = mean over chunks c and experts i of 1 - prod_t (1 - p_{c,t,i})
+ *   J    = w_al L_AL + w_cs L_CS;  the gradient flows through both sides of each pair.
+ *   x     bf16 [C * L, d], the chunks one after another       Wr fp32 [d, E]    br fp32 [E] or NULL
+ *   loss  fp32 [2] out: { L_AL, L_CS } (unweighted)
+ *   dS    fp32 [C * L, E] out: dJ/ds (also the call's scratch for s)
+ *   dWr   fp32 [d, E] out: x^T dS, or NULL     db fp32 [E] out: sum_t dS, or NULL
+ *   dx    fp32 [C * L, d] out: dS Wr^T (this term of the input gradient, overwritten), or NULL
+ *   workspace  device memory of at least blockffn_cls_losses_workspace_size(C, L, d, E) bytes, 256-byte
+ *              aligned, owned by the caller; its contents need not be initialised.
+ * All pointers are DEVICE pointers; work is enqueued on `stream` (six kernel launches, fewer without
+ * dx or dWr) and the call returns without synchronising.  Results are bit-identical run to run (every
+ * sum runs in a fixed order).  The products run on the bf16 tensor cores with fp32 operands carried as
+ * hi + lo bf16 pairs (about 2^-17 relative), accumulated in fp32.
+ * Requirements (BFFN_EINVAL otherwise, nothing enqueued): C, L >= 1, C * L <= 2^30, d >= 8, d % 8 == 0,
+ * 1 <= E <= 1024, alpha > 0 and finite, w_al and w_cs finite; x and dx 16-byte aligned, every other
+ * array 4-byte aligned; x, Wr, loss, dS and workspace non-NULL.  L > 128 returns BFFN_EUNSUPPORTED;
+ * a workspace smaller than needed BFFN_ENOMEM; a failed launch BFFN_ECUDA.
+ */
+BFFN_API int blockffn_cls_losses(const void* x, int C, int L, int d, const float* Wr, const float* br, int E,
+                                 float alpha, float w_al, float w_cs, float* loss, float* dS, float* dWr,
+                                 float* db, float* dx, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace blockffn_cls_losses needs for these sizes (0 if the sizes are invalid). */
+BFFN_API size_t blockffn_cls_losses_workspace_size(int C, int L, int d, int E);
+
+/*
  * blockffn_chunk_forward_noalloc — no counterpart on the BlockFFN pages; this is a deployment aid.
  *
  * The same forward as blockffn_chunk_forward (plus the optional router bias `br`, may be NULL) for

@@ -303,11 +303,12 @@ int oracle_cls_losses(const uint16_t* x, int C, int L, int d, const float* Wr, c
     }
   loss[0] = L > 1 ? l_al / n_al : 0.0;
   loss[1] = l_cs / n_cs;
-  for (int k = 0; k < d; ++k)
-    for (int i = 0; i < E; ++i) {
-      double acc = 0.0;
-      for (int t = 0; t < T; ++t) acc += widen_bf16(x[static_cast<size_t>(t) * d + k]) * dS[static_cast<size_t>(t) * E + i];
-      dWr[static_cast<size_t>(k) * E + i] = acc;
+  // dWr[k,i] = sum over t in ascending order (the loops run t outermost only to read x row by row)
+  for (size_t q = 0; q < static_cast<size_t>(d) * E; ++q) dWr[q] = 0.0;
+  for (int t = 0; t < T; ++t)
+    for (int k = 0; k < d; ++k) {
+      const double xv = widen_bf16(x[static_cast<size_t>(t) * d + k]);
+      for (int i = 0; i < E; ++i) dWr[static_cast<size_t>(k) * E + i] += xv * dS[static_cast<size_t>(t) * E + i];
     }
   if (db)
     for (int i = 0; i < E; ++i) {

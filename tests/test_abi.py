@@ -155,3 +155,41 @@ def test_union_overlap_validates(bffn, kw):
     a.update(kw)
     assert bffn.blockffn_union_overlap(a["a"], a["na"], a["b"], a["nb"], a["C"], a["E"], a["overlap"],
                                        None) == bffn.BFFN_EINVAL
+
+
+def _cls_call(bffn, **kw):
+    a = dict(x=FAKE, C=4, L=8, d=256, Wr=FAKE, br=None, E=64, alpha=4.0, w_al=1.0, w_cs=1.0, loss=FAKE, dS=FAKE,
+             dWr=FAKE, db=FAKE, dx=FAKE, workspace=FAKE, workspace_bytes=1 << 40)
+    a.update(kw)
+    return bffn.blockffn_cls_losses(a["x"], a["C"], a["L"], a["d"], a["Wr"], a["br"], a["E"], a["alpha"], a["w_al"],
+                                    a["w_cs"], a["loss"], a["dS"], a["dWr"], a["db"], a["dx"], a["workspace"],
+                                    a["workspace_bytes"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(C=0), dict(L=0), dict(d=0), dict(d=12), dict(E=0), dict(E=1025), dict(C=1 << 16, L=1 << 15),
+    dict(alpha=0.0), dict(alpha=-1.0), dict(alpha=float("inf")), dict(alpha=float("nan")), dict(w_al=float("nan")),
+    dict(w_cs=float("inf")), dict(x=None), dict(x=FAKE + 8), dict(Wr=None), dict(Wr=FAKE + 2), dict(br=FAKE + 1),
+    dict(loss=None), dict(dS=None), dict(dS=FAKE + 2), dict(dWr=FAKE + 2), dict(db=FAKE + 1), dict(dx=FAKE + 4),
+    dict(workspace=None), dict(workspace=FAKE + 16),
+])
+def test_cls_losses_invalid_arguments_rejected_before_launch(bffn, kw):
+    assert _cls_call(bffn, **kw) == bffn.BFFN_EINVAL
+
+
+def test_cls_losses_unsupported_and_small_workspace(bffn):
+    assert _cls_call(bffn, L=129) == bffn.BFFN_EUNSUPPORTED
+    need = bffn.blockffn_cls_losses_workspace_size(4, 8, 256, 64)
+    assert _cls_call(bffn, workspace_bytes=need - 1) == bffn.BFFN_ENOMEM
+
+
+def test_cls_losses_workspace_size(bffn):
+    T, d, E = 4096 * 8, 2048, 64
+    n = bffn.blockffn_cls_losses_workspace_size(4096, 8, d, E)
+    assert n >= 2 * d * E * 2 + 2 * T * E * 2  # the hi/lo pairs of Wr and of dS
+    for bad in [(0, 8, 256, 64), (4, 0, 256, 64), (4, 8, 250, 64), (4, 8, 0, 64), (4, 8, 256, 0),
+                (4, 8, 256, 1025)]:
+        assert bffn.blockffn_cls_losses_workspace_size(*bad) == 0
+    # experts are padded to 64 in the split copies: E = 1 and E = 64 need the same
+    assert (bffn.blockffn_cls_losses_workspace_size(4, 8, 256, 1)
+            == bffn.blockffn_cls_losses_workspace_size(4, 8, 256, 64))
