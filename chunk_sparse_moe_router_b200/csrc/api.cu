@@ -285,7 +285,7 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
                     const DeviceInfo& di, bool sum_norm, cudaStream_t st) {
   if (!aligned16(y)) return BFFN_EINVAL;  // the down-projection adds into y 16 bytes at a time
   const WsLayout lay = ws_layout(L, d, E, de);
-  const PrefillLayout pl = prefill_layout(lay.h_off, L, E, de);
+  const PrefillLayout pl = prefill_layout(lay.h_off, L, d, E, de);
   uint8_t* base = static_cast<uint8_t*>(ws);
   PrefillParams p;
   p.sum_norm = sum_norm ? 1 : 0;
@@ -307,6 +307,7 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
   p.de = de;
   p.s = reinterpret_cast<float*>(base + lay.s_off);
   p.s_part = reinterpret_cast<float*>(base + pl.spart_off);
+  p.wsplit = reinterpret_cast<__nv_bfloat16*>(base + pl.wsplit_off);
   p.mask = reinterpret_cast<uint32_t*>(base + pl.mask_off);
   p.rms = reinterpret_cast<float*>(base + pl.rms_off);
   p.cnt = reinterpret_cast<int32_t*>(base + pl.cnt_off);
@@ -332,7 +333,7 @@ int forward_prefill(const void* x, int L, int d, const float* Wr, const float* g
     const uint32_t w2b[2] = {64, uint32_t(p.N2)};
     if (!encode_bf16(&m.w2, W2, 2, w2d, w2s, w2b)) return BFFN_ECUDA;
   }
-  const cudaError_t err = prefill_launch(p, m, launch, st);
+  const cudaError_t err = prefill_launch(p, m, launch, di.num_sms, st);
   if (err != cudaSuccess) return cuda_fail(err);
   return BFFN_OK;
 }

@@ -68,20 +68,20 @@ inline size_t part_bytes(int L) { return size_t(kTcMaxGrid) * 2 * 128 * lc_of(L)
 inline size_t cnt_words(int d, int E, int de) { return size_t(E) * ((de + 127) / 128) + (d + 127) / 128; }
 }  // namespace tcdec
 
-// Prefill workspace regions (L > 32), after s: the router's K-split partial projections, per-token
-// masks and RMS, per-expert counts and
-// offsets, the pair lists (token, r) in expert-major order, and H = [pairs][2 de] bf16 (hi | lo).
-constexpr int kPrefillRouterSplit = 4;  // K parts of the prefill router projection
-
+// Prefill workspace regions (L > 32), after s: Wr as bf16 hi + lo pairs [2][d][E rounded up to 64], the
+// router projection, per-token masks and RMS, per-expert counts and offsets, the pair lists (token, r)
+// in expert-major order, and H = [pairs][2 de] bf16 (hi | lo).
 struct PrefillLayout {
-  size_t spart_off, mask_off, rms_off, cnt_off, off_off, toff_off, npos_off, tok_off, rv_off, h_off, end;
+  size_t wsplit_off, spart_off, mask_off, rms_off, cnt_off, off_off, toff_off, npos_off, tok_off, rv_off, h_off,
+      end;
 };
 
-inline PrefillLayout prefill_layout(size_t start, int L, int E, int de) {
+inline PrefillLayout prefill_layout(size_t start, int L, int d, int E, int de) {
   PrefillLayout p;
-  const size_t W = size_t(E + 31) / 32, P = size_t(L) * E;
-  p.spart_off = start;
-  p.mask_off = p.spart_off + align256(size_t(kPrefillRouterSplit) * L * E * 4);
+  const size_t W = size_t(E + 31) / 32, P = size_t(L) * E, Ep = size_t(E + 63) / 64 * 64;
+  p.wsplit_off = start;
+  p.spart_off = p.wsplit_off + align256(2 * size_t(d) * Ep * 2);
+  p.mask_off = p.spart_off + align256(size_t(4) * L * E * 4);  // up to 4 router parts (cls::kMaxRouterParts)
   p.rms_off = p.mask_off + align256(size_t(L) * W * 4);
   p.cnt_off = p.rms_off + align256(size_t(L) * 4);
   p.off_off = p.cnt_off + align256(size_t(E) * 4);
@@ -122,7 +122,7 @@ inline WsLayout ws_layout(int L, int d, int E, int de) {
     w.cnt_off = w.part_off + align256(tcdec::part_bytes(L));
     w.total = w.cnt_off + align256(tcdec::cnt_words(d, E, de) * 4);
   } else {
-    w.total = prefill_layout(w.h_off, L, E, de).end;
+    w.total = prefill_layout(w.h_off, L, d, E, de).end;
   }
   return w;
 }
@@ -367,8 +367,9 @@ struct PrefillParams {
   int L, d, E, de, W;       // W = ceil(E / 32)
   int sum_norm;             // 1: r = g relu(s) / sum relu(s) (the ReMoE router) instead of the RMS
   float* s;                 // [L,E]
-  float* s_part;            // [ksplit][L,E] partial router projections
-  int ksplit;               // K parts of the router projection (d / ksplit a multiple of 32)
+  float* s_part;            // [ksplit][L,E] partial router projections x Wr over ranges of d (without b)
+  int ksplit;               // their count
+  __nv_bfloat16* wsplit;    // [2][d][Ep] Wr as bf16 hi + lo pairs, Ep = E rounded up to 64
   uint32_t* mask;           // [L,W]
   float* rms;               // [L]
   int32_t* cnt;             // [E] tokens per expert
@@ -395,7 +396,8 @@ struct PrefillLaunch {
 };
 
 bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, PrefillParams* p, PrefillLaunch* out);
-cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st);
+cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, int num_sms,
+                           cudaStream_t st);
 
 // ---------------------------------------------------------------- CLS-aware losses (cls_losses.cu)
 namespace cls {
@@ -411,6 +413,15 @@ bool chunk_fits(int L);
 cudaError_t launch(const void* x, int C, int L, int d, const float* Wr, const float* br, int E, float alpha,
                    float w_al, float w_cs, float* loss, float* dS, float* dWr, float* db, float* dx, void* ws,
                    int num_sms, cudaStream_t st);
+// s = x [T, d] Wr [d, E] (no bias) on the warp tensor cores with Wr carried as bf16 hi + lo pairs
+// (|error| <= 2^-18 sum_k |x_k Wr_k| from the pairs, plus fp32 accumulation), as `parts` partial
+// products over consecutive ranges of d: s holds parts x [T, E] fp32, to be added in part order; wsplit
+// holds 2 d (E rounded up to 64) bf16.  Two launches.  router_projection_parts picks the part count
+// (1 .. kMaxRouterParts) that gives the GPU about two CTAs per SM.
+constexpr int kMaxRouterParts = 4;
+int router_projection_parts(int T, int d, int E, int num_sms);
+cudaError_t router_projection(const __nv_bfloat16* x, int T, int d, const float* Wr, int E, __nv_bfloat16* wsplit,
+                              float* s, int parts, int num_sms, cudaStream_t st);
 }  // namespace cls
 
 }  // namespace bffn

@@ -89,34 +89,39 @@ __global__ void __launch_bounds__(kThreads) split_wr_kernel(const float* __restr
 }
 
 // s[t0 .. t0+128, e0 .. e0+64] = x W + b.  Warp w owns tokens 64 (w & 1) .. +63 and experts
-// 32 (w >> 1) .. +31: each operand fragment it loads from shared memory feeds four MMAs.
+// 32 (w >> 1) .. +31: each operand fragment it loads from shared memory feeds four MMAs.  With a K split
+// (gridDim.z > 1) CTA z takes columns [z kper, (z+1) kper) of x and writes its partial product to
+// s + z T E (b, if any, goes to part 0).
 __global__ void __launch_bounds__(kGemmThreads) router_gemm_kernel(const __nv_bfloat16* __restrict__ x, int T,
                                                                    int d, const __nv_bfloat16* __restrict__ wh,
                                                                    const __nv_bfloat16* __restrict__ wl, int Ep,
                                                                    const float* __restrict__ br, int E,
-                                                                   float* __restrict__ s) {
+                                                                   float* __restrict__ s, int kper) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kXBytes = kTokTile * kPitch * 2, kWBytes = kKTile * kPitch * 2;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, wm = warp & 1, wn = warp >> 1;
   const int t0 = blockIdx.x * kTokTile, e0 = blockIdx.y * kNTile;
-  const int nk = (d + kKTile - 1) / kKTile;
+  const int kbeg = blockIdx.z * kper, kend = min(d, kbeg + kper);
+  const int nk = (kend - kbeg + kKTile - 1) / kKTile;
   const uint32_t sbase = smem_u32(smem);
+  if (blockIdx.z > 0) br = nullptr;
+  s += size_t(blockIdx.z) * T * E;
 
   auto load = [&](int kt) {
     const uint32_t st = sbase + (kt % kStages) * kRouterStage;
-    const int k0 = kt * kKTile;
+    const int k0 = kbeg + kt * kKTile;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {  // x: 128 rows x 8 pieces of 16 B
       const int idx = tid + j * kGemmThreads, row = idx >> 3, ch = idx & 7;
       const int gt = t0 + row, gk = k0 + ch * 8;
-      const bool ok = gt < T && gk < d;
+      const bool ok = gt < T && gk < kend;
       cp_async16(st + (row * kPitch + ch * 8) * 2, ok ? x + size_t(gt) * d + gk : x, ok ? 16 : 0);
     }
 #pragma unroll
     for (int j = 0; j < 4; ++j) {  // Wr hi and lo: 64 rows x 8 pieces each
       const int idx = tid + j * kGemmThreads, row = idx >> 3, ch = idx & 7;
       const int gk = k0 + row;
-      const bool ok = gk < d;
+      const bool ok = gk < kend;
       const size_t off = ok ? size_t(gk) * Ep + e0 + ch * 8 : 0;
       cp_async16(st + kXBytes + (row * kPitch + ch * 8) * 2, wh + off, ok ? 16 : 0);
       cp_async16(st + kXBytes + kWBytes + (row * kPitch + ch * 8) * 2, wl + off, ok ? 16 : 0);
@@ -663,7 +668,8 @@ cudaError_t launch(const void* x, int C, int L, int d, const float* Wr, const fl
   const size_t nw = size_t(d) * p.Ep;
   split_wr_kernel<<<unsigned(std::min<size_t>((nw + kThreads - 1) / kThreads, size_t(num_sms) * 8)), kThreads, 0,
                     st>>>(Wr, d, E, p.Ep, wh, wl);
-  router_gemm_kernel<<<dim3(tok_tiles, n_eg), kGemmThreads, kRouterSmem, st>>>(xb, p.T, d, wh, wl, p.Ep, br, E, dS);
+  router_gemm_kernel<<<dim3(tok_tiles, n_eg), kGemmThreads, kRouterSmem, st>>>(xb, p.T, d, wh, wl, p.Ep, br, E, dS,
+                                                                             d);
   const double n_al = double(C) * (L - 1) * E, n_cs = double(C) * E;
   const float f_al = L > 1 ? float(double(w_al) * alpha / n_al) : 0.f;
   const float f_cs = float(double(w_cs) * alpha / n_cs);
@@ -684,6 +690,33 @@ cudaError_t launch(const void* x, int C, int L, int d, const float* Wr, const fl
   reduce_kernel<<<grid_r, kReduceThreads, 0, st>>>(part, p.splits, d, E, p.Ep, dWr, db_part, p.splits * p.dtiles, db,
                                                     loss_part, p.b_rows * n_eg, L > 1 ? 1.0 / n_al : 0.0,
                                                     1.0 / n_cs, loss);
+  return cudaGetLastError();
+}
+
+int router_projection_parts(int T, int d, int E, int num_sms) {
+  const long long tiles = 1ll * ((T + kTokTile - 1) / kTokTile) * ((E + 63) / 64);
+  const int kt = (d + kKTile - 1) / kKTile;  // 64-column slices of x
+  long long parts = (2ll * num_sms + tiles - 1) / tiles;
+  if (parts > kMaxRouterParts) parts = kMaxRouterParts;
+  if (parts > kt) parts = kt;
+  const int per = (kt + int(parts) - 1) / int(parts);  // slices per part
+  return (kt + per - 1) / per;
+}
+
+cudaError_t router_projection(const __nv_bfloat16* x, int T, int d, const float* Wr, int E, __nv_bfloat16* wsplit,
+                              float* s, int parts, int num_sms, cudaStream_t st) {
+  cudaError_t err =
+      cudaFuncSetAttribute(router_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kRouterSmem);
+  if (err != cudaSuccess) return err;
+  const int Ep = (E + 63) / 64 * 64;
+  const size_t nw = size_t(d) * Ep;
+  __nv_bfloat16* wh = wsplit;
+  __nv_bfloat16* wl = wsplit + nw;
+  const int kt = (d + kKTile - 1) / kKTile, kper = (kt + parts - 1) / parts * kKTile;
+  split_wr_kernel<<<unsigned(std::min<size_t>((nw + kThreads - 1) / kThreads, size_t(num_sms) * 8)), kThreads, 0,
+                    st>>>(Wr, d, E, Ep, wh, wl);
+  router_gemm_kernel<<<dim3(unsigned((T + kTokTile - 1) / kTokTile), Ep / 64, parts), kGemmThreads, kRouterSmem,
+                       st>>>(x, T, d, wh, wl, Ep, nullptr, E, s, kper);
   return cudaGetLastError();
 }
 

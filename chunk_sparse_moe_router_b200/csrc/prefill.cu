@@ -3,7 +3,9 @@
 // At this size the layer is a dense contraction per expert, so it runs as grouped GEMMs on the
 // tcgen05 tensor cores (lsdiaocha.cn BlockFFN article, sections 2 and 4: the same router and experts;
 // the tokens of the chunk are grouped per active expert instead of evaluated as one batch):
-//   P1 router       s = x Wr + b, fp32 FFMA tiles (the mask decisions need fp32 accuracy)
+//   P1 router       x Wr on the warp tensor cores with Wr as bf16 hi + lo pairs (cls_losses.cu): the
+//                   error, at most 2^-18 sum_k |x_k Wr_k| plus fp32 rounding, stays below the 1e-3 margin
+//                   of the workloads' pre-activations, so the mask decisions match fp32 and fp64
 //   P2 stats        per token: RMS of relu(s), active bits, optional r and masks
 //   P3 grouping     per expert: its tokens in ascending order with r_{t,e}, 128-row tiles
 //   P4 GEMM1        per (expert, 128-token tile): U = X[T_e] W1_e^T on tcgen05 (the A rows gathered by
@@ -21,77 +23,6 @@ namespace {
 
 constexpr uint64_t kPWaitNs = 2000000000ull;
 
-// ---------------------------------------------------------------------------------- P1 router
-// Tile: 64 tokens x 64 experts x (d / ksplit) of K per CTA, 256 threads with 4 x 4 outputs each.
-// The ksplit partial projections go to the workspace; the stats kernel adds them in fixed order.
-constexpr int kRtT = 64, kRtE = 64, kRtK = 32;
-
-__global__ void __launch_bounds__(256) prefill_router_kernel(PrefillParams p) {
-  __shared__ __align__(16) float Xs[kRtK][kRtT];
-  __shared__ __align__(16) float Ws[kRtK][kRtE];
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
-  const int t0 = blockIdx.x * kRtT, e0 = blockIdx.y * kRtE;
-  const int kper = p.d / p.ksplit, kbeg = blockIdx.z * kper;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && tid == 0) *p.n_pos = 0;
-  const bool e_vec = (p.E & 3) == 0;
-  float acc[4][4] = {};
-  for (int k0 = kbeg; k0 < kbeg + kper; k0 += kRtK) {
-    {  // x: 64 tokens x 32 columns of bf16, one 16-byte load per thread, stored transposed as fp32
-      const int t = tid >> 2, k8 = (tid & 3) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t0 + t < p.L) v = *reinterpret_cast<const uint4*>(p.x + size_t(t0 + t) * p.d + k0 + k8);
-      const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) Xs[k8 + i][t] = __bfloat162float(hv[i]);
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {  // Wr: 32 rows x 64 experts of fp32, two 16-byte loads per thread
-      const int o = tid + h * 256, k = o >> 4, e4 = (o & 15) * 4;
-      float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-      const float* src = p.Wr + size_t(k0 + k) * p.E + e0 + e4;
-      if (e_vec && e0 + e4 + 3 < p.E) {
-        w = *reinterpret_cast<const float4*>(src);
-      } else {
-        if (e0 + e4 + 0 < p.E) w.x = src[0];
-        if (e0 + e4 + 1 < p.E) w.y = src[1];
-        if (e0 + e4 + 2 < p.E) w.z = src[2];
-        if (e0 + e4 + 3 < p.E) w.w = src[3];
-      }
-      *reinterpret_cast<float4*>(&Ws[k][e4]) = w;
-    }
-    __syncthreads();
-    // a partial sum per K tile, added to the running total: a two-level sum keeps the rounding of a
-    // d-term dot product near that of its shorter levels rather than of one long chain
-    float part[4][4] = {};
-#pragma unroll 8
-    for (int k = 0; k < kRtK; ++k) {
-      const float4 a = *reinterpret_cast<const float4*>(&Xs[k][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&Ws[k][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) part[i][j] = fmaf(av[i], bv[j], part[i][j]);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) acc[i][j] += part[i][j];
-    __syncthreads();
-  }
-  float* out = p.s_part + size_t(blockIdx.z) * p.L * p.E;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= p.L) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < p.E) out[size_t(t) * p.E + e] = acc[i][j];
-    }
-  }
-}
-
 // ---------------------------------------------------------------------------------- P2 stats
 // One warp per token: RMS over the E router entries of relu(s), the active bits, r if asked for.
 __global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
@@ -99,7 +30,7 @@ __global__ void __launch_bounds__(256) prefill_stats_kernel(PrefillParams p) {
   const int t = warp;
   if (t >= p.L) return;
   float* st = p.s + size_t(t) * p.E;
-  for (int e = lane; e < p.E; e += 32) {  // s = the split-K parts in order, plus the bias
+  for (int e = lane; e < p.E; e += 32) {  // s = the projection's parts in order, plus the bias
     float v = 0.f;
     for (int k = 0; k < p.ksplit; ++k) v += p.s_part[(size_t(k) * p.L + t) * p.E + e];
     st[e] = v + (p.br ? p.br[e] : 0.f);
@@ -234,6 +165,7 @@ constexpr int kGThreads = 192;   // warp 0: TMA producer, warp 1: MMA issuer (ow
 constexpr int kG1Threads = 320;  // GEMM1 adds warps 6-9: the gathered A rows, one token row per thread
 constexpr int kTileM = 128;
 constexpr int kPf1 = 12;  // GEMM1: W1 rows are prefetched into L2 this many stages ahead
+constexpr int kEpPitch = 36;  // GEMM2 epilogue block: 144-byte rows, so 8 lanes' 16-byte stores hit 32 banks
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -259,6 +191,7 @@ struct GemmSmem {
   int* toff;        // [E+1] copies of the per-expert tile offsets, pair offsets and token counts
   int* off;         // [E+1]
   int* cnt;         // [E]
+  float* ep_buf;    // GEMM2: per epilogue warp a 32 x 32 fp32 block (row pitch kEpPitch)
 };
 
 __device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_bytes, int E) {
@@ -274,7 +207,7 @@ __device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_by
   g.toff = reinterpret_cast<int*>(g.tmem_slot + 4);
   g.off = g.toff + (E + 1);
   g.cnt = g.off + (E + 1);
-  (void)E;
+  g.ep_buf = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(g.cnt + E) + 15) & ~uintptr_t(15));
   return g;
 }
 
@@ -609,8 +542,12 @@ __global__ void __launch_bounds__(kGThreads, 1)
       __syncwarp();
     }
   } else {
+    // Each 32-row x 32-column block leaves tensor memory one row per lane, goes through this warp's
+    // shared block, and is added into y by rows: 8 lanes cover one row's 128 bytes, so a reduction
+    // instruction writes 4 whole lines of y instead of 32 pieces of 32 different lines.
     const int q = warp & 3;
     const uint64_t pol_y = policy_evict_last();
+    float* blk = g.ep_buf + q * 32 * kEpPitch;
     int tcount = 0;
     for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++tcount) {
       const int ab = tcount & 1;
@@ -619,17 +556,23 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const Tile2 tl = tile2_at(g, p.E, NT, tile);
       const int e = tl.e, jn = tl.jn, m0 = tl.m0, ne = g.cnt[e];
       const int row = q * 32 + lane;
-      const bool valid = m0 + row < ne;
-      const int tok = valid ? p.tok[g.off[e] + m0 + row] : 0;
-      float* yrow = p.y + size_t(tok) * p.d + size_t(jn) * N;
+      const int tok = m0 + row < ne ? p.tok[g.off[e] + m0 + row] : -1;  // this lane's row's token
+      float* ycols = p.y + size_t(jn) * N + (lane & 7) * 4;
       for (int c0 = 0; c0 < N; c0 += 32) {
         float v[32];
         tc::ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * N + c0), v);
-        if (valid) {
+        float4* mine = reinterpret_cast<float4*>(blk + lane * kEpPitch);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            red_add_v4(yrow + c0 + 4 * k, v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3], pol_y);
+        for (int k = 0; k < 8; ++k) mine[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const int r = 4 * i + (lane >> 3);
+          const int tok_r = __shfl_sync(0xffffffffu, tok, r);
+          const float4 a = *reinterpret_cast<const float4*>(blk + r * kEpPitch + (lane & 7) * 4);
+          if (tok_r >= 0) red_add_v4(ycols + size_t(tok_r) * p.d + c0, a.x, a.y, a.z, a.w, pol_y);
         }
+        __syncwarp();  // the block is read before the next one overwrites it
       }
       tc::fence_before_sync();
       __syncwarp();
@@ -645,28 +588,33 @@ bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, Prefil
   if (L <= kDecodeMaxL || d % 64 != 0 || de % 64 != 0 || de > 256 || E < 1 || E > kMaxE) return false;
   if ((long long)L * E >= (1ll << 31) / 2) return false;  // pair indices, and H rows as TMA coordinates
   p->W = (E + 31) / 32;
-  p->ksplit = d % (kPrefillRouterSplit * 32) == 0 ? kPrefillRouterSplit : 2;  // d / ksplit: whole K tiles
+  p->ksplit = cls::router_projection_parts(L, d, E, num_sms);
   p->N1 = de;
   p->N2 = d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
   // alignment slack, barriers, tensor-memory slot, abort flag, the three per-expert tables
   const size_t fixed = 1024 + 256 + (3 * size_t(E) + 2) * 4;
+  const size_t fixed2 = fixed + 16 + 4 * 32 * kEpPitch * sizeof(float);  // + the epilogue blocks
   const size_t st1 = size_t(kTileM) * 128 + size_t(p->N1) * 128;
   const size_t st2 = 2 * size_t(kTileM) * 128 + size_t(p->N2) * 128;
   p->S1 = int((size_t(max_smem) - fixed) / st1);
-  p->S2 = int((size_t(max_smem) - fixed) / st2);
+  p->S2 = int((size_t(max_smem) - fixed2) / st2);
   if (p->S1 > 6) p->S1 = 6;
   if (p->S2 > 6) p->S2 = 6;
   if (p->S1 < 2 || p->S2 < 2) return false;
   out->grid = num_sms;
   out->smem1 = fixed + size_t(p->S1) * st1;
-  out->smem2 = fixed + size_t(p->S2) * st2;
+  out->smem2 = fixed2 + size_t(p->S2) * st2;
   return true;
 }
 
-cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, cudaStream_t st) {
+cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, int num_sms,
+                           cudaStream_t st) {
   cudaError_t err = cudaMemsetAsync(p.y, 0, size_t(p.L) * p.d * sizeof(float), st);
   if (err != cudaSuccess) return err;
-  prefill_router_kernel<<<dim3((p.L + kRtT - 1) / kRtT, (p.E + kRtE - 1) / kRtE, p.ksplit), 256, 0, st>>>(p);
+  if ((err = cudaMemsetAsync(p.n_pos, 0, sizeof(int32_t), st)) != cudaSuccess) return err;
+  if ((err = cls::router_projection(p.x, p.L, p.d, p.Wr, p.E, p.wsplit, p.s_part, p.ksplit, num_sms, st)) !=
+      cudaSuccess)
+    return err;
   prefill_stats_kernel<<<(p.L + 7) / 8, 256, 0, st>>>(p);
   prefill_count_kernel<<<p.E, 256, 0, st>>>(p);
   prefill_scan_kernel<<<1, 32, 0, st>>>(p);

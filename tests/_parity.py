@@ -77,15 +77,38 @@ def y_violations(y, y_ref):
     return np.abs(y - y_ref) > bound
 
 
-def assert_parity(got, ref, L, E, check_r=True):
-    """Bit-exact: active flags, union list, n_active, counts. Tolerance: r, y."""
+def pair_router_r_bound(dl: DeviceLayer, x_bits, bias=True, norm="rms"):
+    """Extra allowance on r where the router projection carries Wr as bf16 hi + lo pairs (the prefill
+    path): hi = bf16(w), lo = bf16(w - hi) leave |w - hi - lo| <= 2^-18 |w|, so the pairs move s_{t,i} by
+    at most 2^-18 sum_k |x_tk Wr_ki|; the fp32 accumulation of the products is allowed three times that
+    again, |ds| <= 2^-16 sum_k |x_tk Wr_ki|.  With a = relu(s) and r_i = g_i a_i / n(a), n the RMS (or
+    the sum for the ReMoE router), n moves by at most max_j |ds_j| (the sum by sum_j |ds_j|), so
+    |dr_i| <= (g_i |ds_i| + |r_i| dn) / n(a)."""
+    lay = dl.lay
+    s, r, _ = oracle.router(x_bits, lay.Wr, lay.br if bias else None, lay.g, norm=norm)
+    xa = np.abs(gen.bf16_bits_to_f32(x_bits).astype(np.float64))
+    ds = 2.0 ** -16 * (xa @ np.abs(lay.Wr.astype(np.float64)))
+    a = np.maximum(s, 0.0)
+    if norm == "sum":
+        n, dn = a.sum(axis=1, keepdims=True), ds.sum(axis=1, keepdims=True)
+    else:
+        n, dn = np.sqrt(np.mean(a * a, axis=1, keepdims=True)), ds.max(axis=1, keepdims=True)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        bound = (lay.g.astype(np.float64)[None, :] * ds + np.abs(r) * dn) / n
+    return np.where(n > 0, bound, 0.0)
+
+
+def assert_parity(got, ref, L, E, check_r=True, r_bound=None):
+    """Bit-exact: active flags, union list, n_active, counts. Tolerance: r (plus r_bound where given), y."""
     assert got["n_active"] == len(ref["active_idx"]), (got["n_active"], len(ref["active_idx"]))
     assert np.array_equal(got["active_idx"], ref["active_idx"])
     if "active" in got:
         assert np.array_equal(got["active"], ref["active"])
         assert got["counts"] == (ref["tls_zero"], ref["cls_zero"])
         if check_r:
-            assert np.allclose(got["r"], ref["r"], rtol=R_RTOL, atol=R_ATOL), np.abs(got["r"] - ref["r"]).max()
+            err = np.abs(got["r"] - ref["r"])
+            tol = R_ATOL + R_RTOL * np.abs(ref["r"]) + (0.0 if r_bound is None else r_bound)
+            assert np.all(err <= tol), err.max()
     bad = y_violations(got["y"], ref["y"])
     assert not bad.any(), (f"{int(bad.sum())} of {bad.size} y elements out of tolerance; "
                            f"max abs err {np.abs(got['y'] - ref['y']).max():.3e}")

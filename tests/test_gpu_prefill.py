@@ -2,7 +2,9 @@
 oracle, through the C ABI.
 
 Bit-exact: per-token active flags, the union list, n_active, the sparsity counts.
-Within tolerance: r (fp32 vs fp64) and y (|y - y_ref| <= 2e-2 |y_ref| + 1e-3 rms(y_ref)).
+Within tolerance: y (|y - y_ref| <= 2e-2 |y_ref| + 1e-3 rms(y_ref)) and r: the prefill router carries Wr
+as bf16 hi + lo pairs on the tensor cores, so r gets the fp32 allowance plus the bound that error
+propagates to (_parity.pair_router_r_bound).
 At the full prefill size (L = 4096, d = 4096, E = 128, de = 256) the flags, union and counts are
 compared for every token, y and r on a seeded sample of tokens (the dense fp64 oracle costs about
 0.5 GFLOP per token).
@@ -31,12 +33,12 @@ def _tokens(dl, seed, L):
     dict(L=257, d=384, E=8, de=192, beta=-0.5),   # most experts on for most tokens, N2 = 128
 ])
 def test_prefill_shapes(bffn, cuda_device, shape):
-    from _parity import assert_parity, reference, run_chunk
+    from _parity import assert_parity, pair_router_r_bound, reference, run_chunk
     dl = _layer(11, shape["d"], shape["E"], shape["de"], shape["beta"])
     x = _tokens(dl, 12, shape["L"])
     got = run_chunk(bffn, dl, x)
     ref = reference(dl, x)
-    assert_parity(got, ref, shape["L"], shape["E"])
+    assert_parity(got, ref, shape["L"], shape["E"], r_bound=pair_router_r_bound(dl, x))
 
 
 def test_prefill_twice_same_union_and_close_y(bffn, cuda_device):
@@ -53,7 +55,7 @@ def test_prefill_twice_same_union_and_close_y(bffn, cuda_device):
 
 def test_prefill_full_size_sampled(bffn, cuda_device):
     import oracle
-    from _parity import DeviceLayer, R_ATOL, R_RTOL, run_chunk
+    from _parity import DeviceLayer, R_ATOL, R_RTOL, pair_router_r_bound, run_chunk
 
     w = gen.workload("prefill")
     dl = DeviceLayer(w.layer(0))
@@ -67,7 +69,8 @@ def test_prefill_full_size_sampled(bffn, cuda_device):
     assert np.array_equal(got["active"], act_ref)
     assert np.array_equal(got["active_idx"], idx_ref) and got["n_active"] == len(idx_ref)
     assert got["counts"] == (tz, cz)
-    assert np.allclose(got["r"], r_ref, rtol=R_RTOL, atol=R_ATOL), np.abs(got["r"] - r_ref).max()
+    err = np.abs(got["r"] - r_ref)
+    assert np.all(err <= R_ATOL + R_RTOL * np.abs(r_ref) + pair_router_r_bound(dl, x)), err.max()
     # y on a seeded sample of tokens (first, last, and 22 in between), against the dense oracle; the
     # tolerance's rms is that of the call's whole y_ref, taken from the sparse oracle over every token
     # (pinned equal to the dense one bit for bit)
@@ -84,8 +87,8 @@ def test_prefill_full_size_sampled(bffn, cuda_device):
 
 def test_prefill_remoe_router_variant(bffn, cuda_device):
     # the sum-normalised (ReMoE) router on the prefill path
-    from _parity import assert_parity, reference, run_chunk
+    from _parity import assert_parity, pair_router_r_bound, reference, run_chunk
     dl = _layer(17, 256, 24, 128, 0.6)
     x = _tokens(dl, 18, 100)
     got = run_chunk(bffn, dl, x, flags=bffn.BFFN_FLAG_ROUTER_SUM_NORM)
-    assert_parity(got, reference(dl, x, norm="sum"), 100, 24)
+    assert_parity(got, reference(dl, x, norm="sum"), 100, 24, r_bound=pair_router_r_bound(dl, x, norm="sum"))
