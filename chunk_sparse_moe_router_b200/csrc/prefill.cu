@@ -256,19 +256,30 @@ __device__ __forceinline__ int tile_expert(const int32_t* toff, int E, int tile)
   return lo;
 }
 
-// GEMM2 tile -> (expert e, N tile jn, 128-row tile of the expert): the tiles of one expert are
-// contiguous, N-tile-major, so the CTAs working on one W2_e slice at a time read it once from HBM
-// and the expert's (few) rows of H repeat from L2.
+// GEMM2 tile -> (N tile jn, expert e, 128-row tile of the expert).  The d / N column slices of y form
+// groups of G; a group's tiles come before the next group's, expert-major inside it, and an expert's
+// tiles in a group are N-tile-major.  So the CTAs working on one W2_e slice at a time share it in L2
+// and it comes from HBM once; an expert's H rows repeat from L2 over the group's G slices; and the y
+// elements the tiles add into are those of one group's columns (L x G N fp32, 32 MiB at L = 4096,
+// G N = 2048), which stay in L2 through the ~E_t additions each takes.  H is read from HBM once per
+// group.
 struct Tile2 {
   int e, jn, m0;
 };
+__device__ __forceinline__ int slice_group(int NT) {
+  int G = NT < 8 ? NT : 8;
+  while (NT % G != 0) --G;
+  return G;
+}
 __device__ __forceinline__ Tile2 tile2_at(const GemmSmem& g, int E, int NT, int tile) {
+  const int G = slice_group(NT), T1 = g.toff[E];
+  const int grp = tile / (T1 * G), rem = tile - grp * (T1 * G);
   Tile2 t;
-  t.e = tile_expert(g.toff, E, tile / NT);  // the expert's tiles are [toff[e] NT, toff[e+1] NT)
+  t.e = tile_expert(g.toff, E, rem / G);  // the expert's tiles in the group are [toff[e] G, toff[e+1] G)
   const int nm = g.toff[t.e + 1] - g.toff[t.e];
-  const int li = tile - g.toff[t.e] * NT;
-  t.jn = li / nm;
-  t.m0 = (li - t.jn * nm) * kTileM;
+  const int li = rem - g.toff[t.e] * G;
+  t.jn = grp * G + li / nm;
+  t.m0 = (li - (li / nm) * nm) * kTileM;
   return t;
 }
 
@@ -492,7 +503,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
 
   if (warp == 0) {
     const uint64_t pol_h = policy_evict_normal();  // an expert's H rows repeat over its N tiles, soon
-    const uint64_t pol_w = policy_evict_first();  // W2 streams through (y stays in L2 for the adds)
+    const uint64_t pol_w = policy_evict_normal();  // W2_e[jn] is read by every row tile of e, close together
     Ring rp;
     bool ok = true;
     for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
