@@ -51,6 +51,12 @@ def _load():
             dbl = C.c_double
             lib.oracle_cls_losses.argtypes = [p, i, i, i, p, p, i, dbl, dbl, dbl, dptr, dptr, dptr, dptr, dptr]
             lib.oracle_cls_losses.restype = i
+            lib.oracle_e4m3_value.argtypes = [i]
+            lib.oracle_e4m3_value.restype = dbl
+            lib.oracle_e4m3_nearest.argtypes = [dbl]
+            lib.oracle_e4m3_nearest.restype = i
+            lib.oracle_quantize_fp8.argtypes = [p, p, i, i, i, i, p, p, p, p, p]
+            lib.oracle_quantize_fp8.restype = i
             for f in ("oracle_router", "oracle_union", "oracle_expert", "oracle_chunk_forward",
                       "oracle_tokens_forward_mt", "oracle_union_overlap"):
                 getattr(lib, f).restype = i
@@ -130,6 +136,44 @@ def cls_losses(x, C, L, Wr, br, alpha, w_al=1.0, w_cs=1.0):
                                float(w_cs), _ptr(loss), _ptr(dS), _ptr(dWr), _ptr(db), _ptr(dx))
     assert rc == 0
     return loss[0], loss[1], dS, dWr, db, dx
+
+
+def e4m3_value(code):
+    return _load().oracle_e4m3_value(int(code))
+
+
+def e4m3_nearest(v):
+    return _load().oracle_e4m3_nearest(float(v))
+
+
+def quantize_fp8(W1, W2, n_layers):
+    """fp8 (e4m3) expert weights with power-of-two scales: W1 bf16 bits [n_layers*E, de, d] and W2 bf16 bits
+    [n_layers*E, d, de] -> (q1 uint8, q2 uint8, s1 fp32 [NE, de], s2 fp32 [NE, de], t2 fp32 [n_layers])."""
+    lib = _load()
+    W1, W2 = _c(W1, np.uint16), _c(W2, np.uint16)
+    NE, de, d = W1.shape
+    assert W2.shape == (NE, d, de) and NE % n_layers == 0
+    q1 = np.zeros(W1.shape, np.uint8); q2 = np.zeros(W2.shape, np.uint8)
+    s1 = np.zeros((NE, de), np.float32); s2 = np.zeros((NE, de), np.float32); t2 = np.zeros(n_layers, np.float32)
+    rc = lib.oracle_quantize_fp8(_ptr(W1), _ptr(W2), int(n_layers), NE // n_layers, d, de, _ptr(q1), _ptr(q2),
+                                 _ptr(s1), _ptr(s2), _ptr(t2))
+    assert rc == 0
+    return q1, q2, s1, s2, t2
+
+
+def dequantize_fp8(q1, q2, s1, s2, t2):
+    """The weights the quantised format stands for, as bf16 bits (every one is exactly a bf16 value):
+    W1 = s1 q1 (per row), W2 = t2[layer] s2 q2 (per column)."""
+    table = np.array([e4m3_value(c) for c in range(256)], np.float64)
+    NE = q1.shape[0]
+    L = t2.shape[0]
+    W1 = table[q1] * s1.astype(np.float64)[:, :, None]
+    lay = np.repeat(np.arange(L), NE // L)
+    W2 = table[q2] * (s2.astype(np.float64) * t2.astype(np.float64)[lay][:, None])[:, None, :]
+    b1 = W1.astype(np.float32).view(np.uint32)
+    b2 = W2.astype(np.float32).view(np.uint32)
+    assert np.all(b1 & 0xFFFF == 0) and np.all(b2 & 0xFFFF == 0), "dequantised weights must be bf16-exact"
+    return (b1 >> 16).astype(np.uint16), (b2 >> 16).astype(np.uint16)
 
 
 def expert(xt, W1, W2, i):

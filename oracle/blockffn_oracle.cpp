@@ -327,3 +327,91 @@ int oracle_cls_losses(const uint16_t* x, int C, int L, int d, const float* Wr, c
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------------
+// Low-bit expert weights (the survey's low-bit quantisation of MoE weights, intelliparadigm survey, section
+// 4.1; not a BlockFFN claim).  The format this build reads:
+//   W1[e][j][k] = s1[e][j] * q1[e][j][k]          one power-of-two scale per row of W1 (over d)
+//   W2[e][k][j] = t2[l] * s2[e][j] * q2[e][k][j]  one power-of-two scale per column of W2 (over d), written
+//                                                  as a per-layer power of two t2 times a ratio s2 <= 1
+// with q an fp8 e4m3 code (1 sign, 4 exponent bits with bias 7, 3 mantissa bits; no infinity; the
+// largest finite value 448).  The scale of a row (column) is the smallest 2^m with 448 * 2^m >= its largest
+// |w|; the code is w / 2^m rounded to the nearest e4m3 value, ties to the even code.  Every dequantised
+// weight is then exactly a bf16 value.
+namespace {
+double e4m3_value(uint8_t code) {  // the value an e4m3 code stands for (NaN codes are never produced)
+  const int sgn = code >> 7, ex = (code >> 3) & 15, man = code & 7;
+  const double mag = ex == 0 ? std::ldexp(double(man), -9) : std::ldexp(1.0 + man / 8.0, ex - 7);
+  return sgn ? -mag : mag;
+}
+// nearest e4m3 code to v (|v| <= 448), ties to the even code; the sign is kept (-0 for a negative input
+// that rounds to zero)
+uint8_t e4m3_nearest(double v) {
+  const uint8_t sgn = (std::signbit(v) ? 0x80 : 0x00);
+  const double a = std::fabs(v);
+  int best = 0;
+  double best_d = a;  // distance to code 0
+  for (int c = 1; c < 127; ++c) {  // 0x7F is NaN
+    const double dd = std::fabs(e4m3_value(uint8_t(c)) - a);
+    if (dd < best_d || (dd == best_d && (c & 1) == 0 && (best & 1) == 1)) {
+      best = c;
+      best_d = dd;
+    }
+  }
+  if (g_mutation == 12) best = best > 0 ? best - 1 : 0;  // planted: rounds one code toward zero
+  return uint8_t(sgn | best);
+}
+int pow2_exponent_for(double amax) {  // the smallest m with 448 * 2^m >= amax (0 for amax == 0)
+  if (amax == 0.0) return 0;
+  int m = -200;
+  while (448.0 * std::ldexp(1.0, m) < amax) ++m;
+  if (g_mutation == 13) ++m;  // planted: a scale twice too large
+  return m;
+}
+}  // namespace
+
+extern "C" {
+
+double oracle_e4m3_value(int code) { return e4m3_value(uint8_t(code)); }
+int oracle_e4m3_nearest(double v) { return e4m3_nearest(v); }
+
+// W1 bf16 bits [NE, de, d], W2 bf16 bits [NE, d, de] for NE = n_layers * E experts (layer l owns experts
+// l E .. l E + E - 1).  Out: q1 [NE, de, d], q2 [NE, d, de] codes, s1 [NE, de], s2 [NE, de], t2 [n_layers].
+int oracle_quantize_fp8(const uint16_t* W1, const uint16_t* W2, int n_layers, int E, int d, int de, uint8_t* q1,
+                        uint8_t* q2, float* s1, float* s2, float* t2) {
+  if (n_layers < 1 || E < 1 || d < 1 || de < 1) return 1;
+  const int NE = n_layers * E;
+  std::vector<int> m2(static_cast<size_t>(NE) * de);
+  for (int e = 0; e < NE; ++e)
+    for (int j = 0; j < de; ++j) {
+      const uint16_t* row = W1 + (static_cast<size_t>(e) * de + j) * d;
+      double amax = 0.0;
+      for (int k = 0; k < d; ++k) amax = std::max(amax, std::fabs(widen_bf16(row[k])));
+      const int m = pow2_exponent_for(amax);
+      s1[static_cast<size_t>(e) * de + j] = static_cast<float>(std::ldexp(1.0, m));
+      for (int k = 0; k < d; ++k)
+        q1[(static_cast<size_t>(e) * de + j) * d + k] = e4m3_nearest(std::ldexp(widen_bf16(row[k]), -m));
+      double cmax = 0.0;
+      for (int k = 0; k < d; ++k)
+        cmax = std::max(cmax, std::fabs(widen_bf16(W2[(static_cast<size_t>(e) * d + k) * de + j])));
+      m2[static_cast<size_t>(e) * de + j] = pow2_exponent_for(cmax);
+    }
+  for (int l = 0; l < n_layers; ++l) {
+    int M = -100000;
+    for (int e = l * E; e < (l + 1) * E; ++e)
+      for (int j = 0; j < de; ++j) M = std::max(M, m2[static_cast<size_t>(e) * de + j]);
+    t2[l] = static_cast<float>(std::ldexp(1.0, M));
+    for (int e = l * E; e < (l + 1) * E; ++e)
+      for (int j = 0; j < de; ++j) {
+        const int m = m2[static_cast<size_t>(e) * de + j];
+        s2[static_cast<size_t>(e) * de + j] = static_cast<float>(std::ldexp(1.0, m - M));
+        for (int k = 0; k < d; ++k) {
+          const size_t q = (static_cast<size_t>(e) * d + k) * de + j;
+          q2[q] = e4m3_nearest(std::ldexp(widen_bf16(W2[q]), -m));
+        }
+      }
+  }
+  return 0;
+}
+
+}  // extern "C"
