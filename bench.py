@@ -698,6 +698,96 @@ def run_reuse(args):
                 print(json.dumps(line), flush=True)
 
 
+def run_fp8(args):
+    """The batched decode step on fp8 (e4m3) expert weights (blockffn_quantize_fp8 once, then
+    blockffn_chunk_forward_batch_fp8 per step) on the decode workload's inputs, next to the bf16 batched
+    call on the same inputs.  Roofline: the step's active bytes with one byte per expert weight (plus the
+    per-(expert, j) scales) over its CUDA-event time."""
+    import copy
+
+    import numpy as np
+    import torch
+
+    import chunk_sparse_moe_router_b200 as bffn
+    import gen
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    w = gen.workload("decode")
+    chunks = args.chunks or w.n_chunks
+    layers, stack, x_host_np = build_inputs(w, 0, device, chunks)
+    L, d, E, de, R = w.L, w.d, w.E, w.de, w.replicas
+    x_dev = torch.from_numpy(x_host_np.view(np.int16)).to(device).view(torch.bfloat16)
+    y = torch.empty((chunks, L, d), dtype=torch.float32, device=device)
+    y16 = torch.empty_like(y)
+    idx = torch.empty((chunks, E), dtype=torch.int32, device=device)
+    nact = torch.empty((chunks,), dtype=torch.int32, device=device)
+    q = bffn.quantize_fp8(stack["W1"].view(R * E, de, d), stack["W2"].view(R * E, d, de), R)
+    ws = torch.zeros(bffn.blockffn_batch_fp8_workspace_size(chunks, L, d, E, de), dtype=torch.uint8, device=device)
+    ws16 = torch.zeros(bffn.blockffn_batch_workspace_size(chunks, L, d, E, de, bffn.BFFN_FLAGS_SHARE(8)),
+                       dtype=torch.uint8, device=device)
+    s = torch.cuda.Stream(device)
+
+    def step_fp8():
+        bffn.chunk_forward_batch_fp8(x_dev, stack["Wr"], stack["g"], q, y, idx, nact, br=stack["br"], workspace=ws,
+                                     stream=s.cuda_stream)
+
+    def step_bf16():
+        bffn.chunk_forward_batch(x_dev, stack["Wr"], stack["g"], stack["W1"], stack["W2"], y16, idx, nact,
+                                 br=stack["br"], teams=8, workspace=ws16, stream=s.cuda_stream)
+
+    def timed(step, clocks=False):
+        with torch.cuda.stream(s):
+            step()
+            s.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            graph.capture_begin()
+            step()
+            graph.capture_end()
+            for _ in range(args.warmup):
+                graph.replay()
+            s.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with ClockSampler(0) as clk:
+                e0.record(s)
+                for _ in range(args.steps):
+                    graph.replay()
+                e1.record(s)
+                e1.synchronize()
+            del graph
+        return e0.elapsed_time(e1) / args.steps, clk.summary()
+
+    ms16, _ = timed(step_bf16)
+    ms, clk = timed(step_fp8)
+    n_host = nact.cpu().numpy()
+    fixed = 4 * d * E + 8 * E + 2 * L * d + 4 * L * d
+    bytes_fp8 = float(sum(fixed + int(n) * (2 * d * de + 8 * de) for n in n_host)) + 4 * R
+    bytes_bf16 = float(sum(active_bytes(d, E, de, L, int(n)) for n in n_host))
+    peak, peak_kind = measured_peaks()
+    gbs = bytes_fp8 / (ms * 1e-3) / 1e9
+    line = {"metric": METRIC + " (fp8 e4m3 expert weights)", "value": round(chunks * L / (ms * 1e-3), 1),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "fp8 e4m3 weights (power-of-two scales), f16 MMA, fp32 accumulate", "data": "synthetic",
+            "config": {**w.describe(), "chunks_per_step": chunks, "mean_n_active": round(float(n_host.mean()), 3),
+                       "l2": f"inputs larger than L2: {R} weight replicas, "
+                             f"{R * E * 2 * d * de / 1e9:.2f} GB of fp8 expert weights"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                         "bytes_per_chunk": round(bytes_fp8 / chunks, 1), "us_per_chunk": round(ms * 1e3 / chunks, 3)},
+            "bf16_same_inputs": {"ms_per_step": round(ms16, 4), "tokens_per_s": round(chunks * L / (ms16 * 1e-3), 1),
+                                 "frac": round(bytes_bf16 / (ms16 * 1e-3) / 1e9 / peak, 4)},
+            "speedup_vs_bf16": round(ms16 / ms, 3),
+            "gpu_launches": (3 + 2 * ((chunks + 511) // 512)) * args.steps, "clocks": clk}
+    if not args.no_cpu_baseline:
+        import oracle
+        lay0 = copy.copy(w.layer(0))
+        q1, q2, s1, s2, t2 = oracle.quantize_fp8(lay0.W1, lay0.W2, 1)
+        lay0.W1, lay0.W2 = oracle.dequantize_fp8(q1, q2, s1, s2, t2)
+        line["cpu_baseline"] = cpu_baseline(w, lay0, x_host_np, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
 def run_cls_losses(args):
     """The CLS-aware losses and their backward through the router (blockffn_cls_losses): one step = the
     activation-locality and chunk-sparsification losses of a training batch of --chunks chunks of 8 tokens
@@ -871,7 +961,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses"])
+                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses", "fp8"])
     ap.add_argument("--drift", default="0.0,0.9,0.97",
                     help="--workload reuse: drift of the chunk bases of a sequence (0: independent chunks)")
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
@@ -914,6 +1004,9 @@ def main():
         return
     if args.workload == "cls_losses":
         run_cls_losses(args)
+        return
+    if args.workload == "fp8":
+        run_fp8(args)
         return
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":

@@ -40,6 +40,10 @@ SIGNATURES = {
                                          _I, _P, _S, _P]),
     "blockffn_batch_workspace_size": (_S, [_I, _I, _I, _I, _I, _I]),
     "blockffn_union_overlap": (_I, [_P, _P, _P, _P, _I, _I, _P, _P]),
+    "blockffn_quantize_fp8": (_I, [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P]),
+    "blockffn_chunk_forward_batch_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P,
+                                             _P, _P, _P, _I, _P, _S, _P]),
+    "blockffn_batch_fp8_workspace_size": (_S, [_I, _I, _I, _I, _I]),
     "blockffn_cls_losses": (_I, [_P, _I, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _P, _P, _P, _S, _P]),
     "blockffn_cls_losses_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
@@ -108,6 +112,22 @@ def blockffn_noalloc_device_status(stream):
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20  # BFFN_NOALLOC_SCRATCH_BYTES in include/blockffn.h
+
+
+def blockffn_quantize_fp8(W1, W2, n_layers, E, d, de, W1q, W2q, s1, s2, t2, stream):
+    return _lib.blockffn_quantize_fp8(W1, W2, n_layers, E, d, de, W1q, W2q, s1, s2, t2, stream)
+
+
+def blockffn_chunk_forward_batch_fp8(x, C, L, d, layer, n_layers, Wr, g, br, W1q, s1, W2q, s2, t2, E, de, y,
+                                     active_idx, n_active, counts, tok_mask, flags, workspace, workspace_bytes,
+                                     stream):
+    return _lib.blockffn_chunk_forward_batch_fp8(x, C, L, d, layer, n_layers, Wr, g, br, W1q, s1, W2q, s2, t2, E,
+                                                 de, y, active_idx, n_active, counts, tok_mask, flags, workspace,
+                                                 workspace_bytes, stream)
+
+
+def blockffn_batch_fp8_workspace_size(C, L, d, E, de):
+    return _lib.blockffn_batch_fp8_workspace_size(C, L, d, E, de)
 
 
 def blockffn_cls_losses(x, C, L, d, Wr, br, E, alpha, w_al, w_cs, loss, dS, dWr, db, dx, workspace,
@@ -282,6 +302,73 @@ def cls_losses(x, C, L, Wr, br=None, alpha=1.0, w_al=1.0, w_cs=1.0, loss=None, d
     if rc != BFFN_OK:
         raise BlockFFNError(rc, "blockffn_cls_losses")
     return loss, dS, dWr, db, dx
+
+
+def quantize_fp8(W1, W2, n_layers, stream=None):
+    """fp8 (e4m3) expert weights with power-of-two scales from bf16 W1 [n_layers*E, de, d] and W2
+    [n_layers*E, d, de]: returns (W1q uint8, W2q uint8, s1 fp32 [NE, de], s2 fp32 [NE, de], t2 fp32
+    [n_layers]).  Raises BlockFFNError."""
+    import torch
+
+    NE, de, d = W1.shape
+    dev = W1.device
+    _check(W1, "W1", torch.bfloat16, (NE, de, d), dev)
+    _check(W2, "W2", torch.bfloat16, (NE, d, de), dev)
+    if NE % n_layers != 0:
+        raise ValueError("the expert count must be a multiple of n_layers")
+    E = NE // n_layers
+    W1q = torch.empty((NE, de, d), dtype=torch.uint8, device=dev)
+    W2q = torch.empty((NE, d, de), dtype=torch.uint8, device=dev)
+    s1 = torch.empty((NE, de), dtype=torch.float32, device=dev)
+    s2 = torch.empty((NE, de), dtype=torch.float32, device=dev)
+    t2 = torch.empty((n_layers,), dtype=torch.float32, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = blockffn_quantize_fp8(_ptr(W1), _ptr(W2), n_layers, E, d, de, _ptr(W1q), _ptr(W2q), _ptr(s1), _ptr(s2),
+                               _ptr(t2), stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_quantize_fp8")
+    return W1q, W2q, s1, s2, t2
+
+
+def chunk_forward_batch_fp8(x, Wr, g, q, y, active_idx, n_active, layer=None, br=None, counts=None, tok_mask=None,
+                            workspace=None, stream=None, flags=0):
+    """The batched decode forward on fp8 expert weights: q = (W1q, W2q, s1, s2, t2) from quantize_fp8; the
+    other arguments as chunk_forward_batch.  Raises BlockFFNError."""
+    import torch
+
+    W1q, W2q, s1, s2, t2 = q
+    C, L, d = x.shape
+    nl = t2.shape[0]
+    NE, de = s1.shape
+    E = NE // nl
+    dev = x.device
+    _check(x, "x", torch.bfloat16, (C, L, d), dev)
+    _check(Wr, "Wr", torch.float32, (nl, d, E), dev)
+    _check(g, "g", torch.float32, (nl, E), dev)
+    _check(W1q, "W1q", torch.uint8, (NE, de, d), dev)
+    _check(W2q, "W2q", torch.uint8, (NE, d, de), dev)
+    _check(s2, "s2", torch.float32, (NE, de), dev)
+    _check(y, "y", torch.float32, (C, L, d), dev)
+    _check(active_idx, "active_idx", torch.int32, (C, E), dev)
+    _check(n_active, "n_active", torch.int32, (C,), dev)
+    if layer is not None:
+        _check(layer, "layer", torch.int32, (C,), dev)
+    if br is not None:
+        _check(br, "br", torch.float32, (nl, E), dev)
+    if counts is not None:
+        _check(counts, "counts", torch.int32, (C, 2), dev)
+    if tok_mask is not None:
+        _check(tok_mask, "tok_mask", torch.int32, (C, L, (E + 31) // 32), dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    ws_ptr, ws_bytes = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel() * workspace.element_size())
+    rc = blockffn_chunk_forward_batch_fp8(_ptr(x), C, L, d, _ptr(layer), nl, _ptr(Wr), _ptr(g), _ptr(br), _ptr(W1q),
+                                          _ptr(s1), _ptr(W2q), _ptr(s2), _ptr(t2), E, de, _ptr(y), _ptr(active_idx),
+                                          _ptr(n_active), _ptr(counts), _ptr(tok_mask), int(flags), ws_ptr, ws_bytes,
+                                          stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_chunk_forward_batch_fp8")
 
 
 def device_status(workspace=None, stream=None):

@@ -115,6 +115,23 @@ EncodeTiledFn encode_fn() {
 }
 
 // bf16 tensor of `rank` dims (innermost first), 128-byte swizzle, out-of-bounds elements read as 0.
+bool encode_tiled(CUtensorMap* tm, CUtensorMapDataType type, const void* base, int rank, const uint64_t* dims,
+                  const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[5], gstride[4];
+  cuuint32_t bdim[5], estride[5];
+  for (int i = 0; i < rank; ++i) {
+    gdim[i] = dims[i];
+    bdim[i] = box[i];
+    estride[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gstride[i] = strides_bytes[i];
+  return fn(tm, type, cuuint32_t(rank), const_cast<void*>(base), gdim, gstride, bdim, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool encode_bf16(CUtensorMap* tm, const void* base, int rank, const uint64_t* dims, const uint64_t* strides_bytes,
                  const uint32_t* box) {
   EncodeTiledFn fn = encode_fn();
@@ -560,6 +577,123 @@ int blockffn_chunk_forward_batch(const void* x, int C, int L, int d, const int32
   }
   return forward_batch(x, C, L, d, layer, n_layers, Wr, g, br, W1, W2, E, de, y, active_idx, n_active, counts,
                        tok_mask, teams, (flags & BFFN_FLAG_ROUTER_SUM_NORM) != 0, ws, di, st);
+}
+
+bool fp8_args_ok(int C, int L, int d, int n_layers, int E, int de) {
+  return batch_args_ok(C, L, d, n_layers, E, de) && d % 16 == 0 && de % 16 == 0 && L <= batch::kMaxL &&
+         1ll * C * 8 * d < (1ll << 40);
+}
+
+int blockffn_quantize_fp8(const void* W1, const void* W2, int n_layers, int E, int d, int de, uint8_t* W1q,
+                          uint8_t* W2q, float* s1, float* s2, float* t2, void* stream) {
+  if (n_layers < 1 || E < 1 || E > kMaxE || d < 16 || d % 16 != 0 || de < 16 || de % 16 != 0 ||
+      1ll * n_layers * E * de * d >= (1ll << 40))
+    return BFFN_EINVAL;
+  const void* bulk[] = {W1, W2, W1q, W2q};
+  for (const void* p : bulk)
+    if (p == nullptr || !aligned16(p)) return BFFN_EINVAL;
+  const void* scal[] = {s1, s2, t2};
+  for (const void* p : scal)
+    if (p == nullptr || !aligned4(p)) return BFFN_EINVAL;
+  const cudaError_t err =
+      fp8::quantize(static_cast<const __nv_bfloat16*>(W1), static_cast<const __nv_bfloat16*>(W2), n_layers, E, d, de,
+                    W1q, W2q, s1, s2, t2, static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
+}
+
+size_t blockffn_batch_fp8_workspace_size(int C, int L, int d, int E, int de) {
+  if (!fp8_args_ok(C, L, d, 1, E, de)) return 0;
+  return fp8::workspace_bytes(C, L, d, E, de);
+}
+
+int blockffn_chunk_forward_batch_fp8(const void* x, int C, int L, int d, const int32_t* layer, int n_layers,
+                                     const float* Wr, const float* g, const float* br, const uint8_t* W1q,
+                                     const float* s1, const uint8_t* W2q, const float* s2, const float* t2, int E,
+                                     int de, float* y, int32_t* active_idx, int32_t* n_active, int32_t* counts,
+                                     uint32_t* tok_mask, int flags, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  if (!fp8_args_ok(C, L, d, n_layers, E, de)) return BFFN_EINVAL;
+  if ((flags & ~BFFN_FLAG_ROUTER_SUM_NORM) != 0) return BFFN_EINVAL;
+  const void* bulk[] = {x, W1q, W2q};
+  for (const void* p : bulk)
+    if (p == nullptr || !aligned16(p)) return BFFN_EINVAL;
+  const void* scalar[] = {Wr, g, s1, s2, t2, y, active_idx, n_active};
+  for (const void* p : scalar)
+    if (p == nullptr || !aligned4(p)) return BFFN_EINVAL;
+  const void* optional[] = {layer, br, counts, tok_mask};
+  for (const void* p : optional)
+    if (p != nullptr && !aligned4(p)) return BFFN_EINVAL;
+  if (workspace != nullptr && !aligned256(workspace)) return BFFN_EINVAL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  DeviceInfo di;
+  int dev = 0;
+  int rc = device_info(&di, &dev);
+  if (rc != BFFN_OK) return rc;
+  const fp8::Fp8Layout lay = fp8::layout(C, L, d, E, de);
+  void* ws = workspace;
+  if (ws == nullptr) {
+    rc = internal_workspace(dev, lay.total, st, &ws);
+    if (rc != BFFN_OK) return rc;
+  } else if (workspace_bytes < lay.total) {
+    return BFFN_ENOMEM;
+  }
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  batch::Params rp{};
+  rp.x = static_cast<const __nv_bfloat16*>(x);
+  rp.layer = layer;
+  rp.Wr = Wr;
+  rp.g = g;
+  rp.br = br;
+  rp.y = y;
+  rp.active_idx = active_idx;
+  rp.n_active = n_active;
+  rp.counts = counts;
+  rp.tok_mask = tok_mask;
+  rp.r = reinterpret_cast<float*>(base + lay.r_off);
+  rp.chunk_bar = reinterpret_cast<uint32_t*>(base + lay.bar_off);
+  rp.hdr = reinterpret_cast<WsHeader*>(base);
+  rp.C = C;
+  rp.L = L;
+  rp.d = d;
+  rp.E = E;
+  rp.de = de;
+  rp.n_layers = n_layers;
+  rp.sum_norm = (flags & BFFN_FLAG_ROUTER_SUM_NORM) != 0 ? 1 : 0;
+  Fp8Params p{};
+  p.layer = layer;
+  p.active_idx = active_idx;
+  p.n_active = n_active;
+  p.r = rp.r;
+  p.W1q = W1q;
+  p.W2q = W2q;
+  p.s1 = s1;
+  p.s2 = s2;
+  p.t2 = t2;
+  p.xh = reinterpret_cast<__half*>(base + lay.xh_off);
+  p.offs = reinterpret_cast<int32_t*>(base + lay.offs_off);
+  p.h = reinterpret_cast<__half*>(base + lay.h_off);
+  p.desc = reinterpret_cast<int4*>(base + lay.desc_off);
+  p.y = y;
+  p.C = C;
+  p.L = L;
+  p.d = d;
+  p.E = E;
+  p.de = de;
+  p.n_layers = n_layers;
+  p.JB = (de + 63) / 64;
+  p.wave = lay.wave;
+  p.hdr = rp.hdr;
+  fp8::Maps maps;
+  {  // the code matrices as 2D byte tensors, boxes of 128 bytes x 64 rows in the 128-byte swizzle
+    const uint64_t NE = uint64_t(n_layers) * E;
+    const uint64_t d1[2] = {uint64_t(d), NE * de}, s1b[1] = {uint64_t(d)};
+    const uint64_t d2[2] = {uint64_t(de), NE * d}, s2b[1] = {uint64_t(de)};
+    const uint32_t box[2] = {128, 64};
+    if (!encode_tiled(&maps.w1, CU_TENSOR_MAP_DATA_TYPE_UINT8, W1q, 2, d1, s1b, box)) return BFFN_ECUDA;
+    if (!encode_tiled(&maps.w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, W2q, 2, d2, s2b, box)) return BFFN_ECUDA;
+  }
+  const cudaError_t err = fp8::forward(p, maps, rp, di.num_sms, st);
+  return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
 }
 
 int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* n_active_a, const int32_t* active_idx_b,

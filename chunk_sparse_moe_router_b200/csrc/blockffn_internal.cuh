@@ -2,6 +2,7 @@
 #pragma once
 #include <cuda.h>  // CUtensorMap (header only; driver entry points are looked up at run time)
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstddef>
@@ -343,6 +344,9 @@ inline Layout layout(int C, int L, int E, int de, int teams) {
 
 bool plan(int C, int L, int d, int E, int de, int teams, int num_sms, int max_smem, Params* p, Launch* out);
 cudaError_t launch(const Params& p, const Maps& m, const Launch& plan, cudaStream_t st);
+// The router kernel alone (it reads x, layer, Wr, g, br and writes r, active_idx, n_active, counts,
+// tok_mask, chunk_bar and the header's error word).
+cudaError_t launch_router(const Params& p, cudaStream_t st);
 cudaError_t occupancy(size_t smem, int* ctas_per_sm);
 }  // namespace batch
 
@@ -398,6 +402,42 @@ struct PrefillLaunch {
 bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, PrefillParams* p, PrefillLaunch* out);
 cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const PrefillLaunch& pl, int num_sms,
                            cudaStream_t st);
+
+// ---------------------------------------------------------------- fp8 expert weights (fp8_decode.cu)
+struct Fp8Params {
+  const int32_t* layer;     // [C] or null
+  const int32_t* active_idx;  // [C, E] (router output)
+  const int32_t* n_active;  // [C]
+  const float* r;           // [C, L, E] (router output)
+  const uint8_t* W1q;       // [NE, de, d] e4m3 codes
+  const uint8_t* W2q;       // [NE, d, de]
+  const float* s1;          // [NE, de]
+  const float* s2;          // [NE, de]
+  const float* t2;          // [n_layers]
+  __half* xh;               // [C, 8, d] x in f16, rows past L zero (workspace)
+  int32_t* offs;            // [C + 1] up-projection items before each chunk (workspace)
+  __half* h;                // [wave, E, 2, 8, de] h'' hi and lo planes (workspace)
+  int4* desc;               // [wave * E * ceil(de / 64)] up-projection item descriptors (workspace)
+  float* y;                 // [C, L, d]
+  WsHeader* hdr;             // error word (a bounded wait that ran out)
+  int C, L, d, E, de, n_layers, JB, wave;
+};
+namespace fp8 {
+struct Maps {
+  CUtensorMap w1;  // W1q as [NE de rows][d bytes], box 128 B x 64 rows, 128-byte swizzle
+  CUtensorMap w2;  // W2q as [NE d rows][de bytes], the same box
+};
+constexpr size_t kHBufBytes = size_t(256) << 20;  // the h buffer: chunks per wave = this / (E 2 8 de 2)
+struct Fp8Layout {
+  size_t r_off, bar_off, offs_off, xh_off, h_off, desc_off, total;
+  int wave;
+};
+Fp8Layout layout(int C, int L, int d, int E, int de);
+size_t workspace_bytes(int C, int L, int d, int E, int de);
+cudaError_t quantize(const __nv_bfloat16* W1, const __nv_bfloat16* W2, int n_layers, int E, int d, int de,
+                     uint8_t* q1, uint8_t* q2, float* s1, float* s2, float* t2, cudaStream_t st);
+cudaError_t forward(const Fp8Params& p, const Maps& m, const batch::Params& rp, int num_sms, cudaStream_t st);
+}  // namespace fp8
 
 // ---------------------------------------------------------------- CLS-aware losses (cls_losses.cu)
 namespace cls {

@@ -810,19 +810,21 @@ cudaError_t occupancy(size_t smem, int* ctas_per_sm) {
   return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, batch_expert_kernel, kThreads, smem);
 }
 
+cudaError_t launch_router(const Params& p, cudaStream_t st) {
+  // router CTAs: one per chunk with a layer array, else ceil(chunks of a layer / G) per layer
+  int ctas = p.C;
+  if (!p.layer) {
+    const int G = kRouterTokens / p.L < 1 ? 1 : kRouterTokens / p.L;
+    const int per_layer = (p.C + p.n_layers - 1) / p.n_layers;
+    ctas = p.n_layers * ((per_layer + G - 1) / G);
+  }
+  batch_router_kernel<<<ctas, kRouterThreads, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch(const Params& p, const Maps& m, const Launch& plan, cudaStream_t st) {
   cudaError_t err;
-  {
-    // router CTAs: one per chunk with a layer array, else ceil(chunks of a layer / G) per layer
-    int ctas = p.C;
-    if (!p.layer) {
-      const int G = kRouterTokens / p.L < 1 ? 1 : kRouterTokens / p.L;
-      const int per_layer = (p.C + p.n_layers - 1) / p.n_layers;
-      ctas = p.n_layers * ((per_layer + G - 1) / G);
-    }
-    batch_router_kernel<<<ctas, kRouterThreads, 0, st>>>(p);
-  }
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  if ((err = launch_router(p, st)) != cudaSuccess) return err;
   err = cudaFuncSetAttribute(batch_expert_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, int(plan.smem));
   if (err != cudaSuccess) return err;
   // programmatic dependent launch: the expert kernel's set-up overlaps the router kernel's tail; it

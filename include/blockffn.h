@@ -193,6 +193,46 @@ BFFN_API int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* 
                                     int32_t* overlap, void* stream);
 
 /*
+ * Low-bit expert weights (not a BlockFFN claim: the intelliparadigm survey, section 4.1, lists low-bit
+ * quantisation of MoE expert weights; the layer computed is unchanged, lsdiaocha.cn BlockFFN article,
+ * sections 2 and 4).  Format, for NE = n_layers * E experts (layer l owns experts l E .. l E + E - 1):
+ *   W1[e][j][k] = s1[e][j] * e4m3(q1[e][j][k])            one power-of-two scale per row of W1
+ *   W2[e][k][j] = t2[l] * s2[e][j] * e4m3(q2[e][k][j])    one per column of W2, as the layer's largest
+ *                                                         power of two t2[l] times a ratio s2 <= 1
+ * e4m3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, largest finite value 448.  A row's (column's)
+ * scale is the smallest 2^m with 448 * 2^m >= its largest |w|; a code is w / 2^m rounded to the nearest
+ * e4m3 value, ties to even.  Every dequantised weight is exactly a bf16 value.
+ *
+ * blockffn_quantize_fp8: W1 bf16 [NE, de, d], W2 bf16 [NE, d, de] -> W1q uint8 [NE, de, d], W2q uint8
+ * [NE, d, de], s1 fp32 [NE, de], s2 fp32 [NE, de], t2 fp32 [n_layers].  Device pointers; W1, W2, W1q, W2q
+ * 16-byte aligned, the rest 4-byte aligned; d, de multiples of 16.  Six kernels on `stream`.
+ */
+BFFN_API int blockffn_quantize_fp8(const void* W1, const void* W2, int n_layers, int E, int d, int de,
+                                   uint8_t* W1q, uint8_t* W2q, float* s1, float* s2, float* t2, void* stream);
+
+/*
+ * The batched decode forward (as blockffn_chunk_forward_batch: C chunks of up to 8 tokens, the same router,
+ * union, r, y, masks and counts) on fp8 expert weights in the format above.  The expert weights stream at
+ * one byte each: an up-projection kernel per 64 rows of an active expert's W1 and an output-stationary
+ * down-projection kernel per 64 rows of y, both converting the codes to f16 for the warp tensor cores
+ * (x is converted to f16 too: |x| must stay below 65504).  y is bit-reproducible.
+ *   flags: BFFN_FLAG_ROUTER_SUM_NORM or 0.
+ *   workspace: at least blockffn_batch_fp8_workspace_size(C, L, d, E, de) bytes (256-byte aligned), or
+ *   NULL for the library's per-device workspace.
+ * Requirements as blockffn_chunk_forward_batch, plus d and de multiples of 16 (BFFN_EINVAL otherwise).
+ */
+BFFN_API int blockffn_chunk_forward_batch_fp8(const void* x, int C, int L, int d, const int32_t* layer,
+                                              int n_layers, const float* Wr, const float* g, const float* br,
+                                              const uint8_t* W1q, const float* s1, const uint8_t* W2q,
+                                              const float* s2, const float* t2, int E, int de, float* y,
+                                              int32_t* active_idx, int32_t* n_active, int32_t* counts,
+                                              uint32_t* tok_mask, int flags, void* workspace,
+                                              size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace blockffn_chunk_forward_batch_fp8 needs (0 if the sizes are invalid). */
+BFFN_API size_t blockffn_batch_fp8_workspace_size(int C, int L, int d, int E, int de);
+
+/*
  * The CLS-aware training objectives and their backward through the router (lsdiaocha.cn BlockFFN article,
  * section 3: an activation-locality loss, a binary cross-entropy between adjacent tokens' activation
  * patterns compared through LeftShift, the patterns approximated by a sharp sigmoid; and a

@@ -193,3 +193,40 @@ def test_cls_losses_workspace_size(bffn):
     # experts are padded to 64 in the split copies: E = 1 and E = 64 need the same
     assert (bffn.blockffn_cls_losses_workspace_size(4, 8, 256, 1)
             == bffn.blockffn_cls_losses_workspace_size(4, 8, 256, 64))
+
+
+@pytest.mark.parametrize("kw", [
+    dict(n_layers=0), dict(E=0), dict(E=1025), dict(d=24), dict(de=8), dict(W1=None), dict(W1=FAKE + 8),
+    dict(W2q=FAKE + 4), dict(s1=None), dict(t2=FAKE + 2),
+])
+def test_quantize_fp8_validates(bffn, kw):
+    a = dict(W1=FAKE, W2=FAKE, n_layers=2, E=16, d=256, de=64, W1q=FAKE, W2q=FAKE, s1=FAKE, s2=FAKE, t2=FAKE)
+    a.update(kw)
+    assert bffn.blockffn_quantize_fp8(a["W1"], a["W2"], a["n_layers"], a["E"], a["d"], a["de"], a["W1q"], a["W2q"],
+                                      a["s1"], a["s2"], a["t2"], None) == bffn.BFFN_EINVAL
+
+
+@pytest.mark.parametrize("kw", [
+    dict(C=0), dict(L=9), dict(d=24), dict(de=40), dict(x=None), dict(x=FAKE + 8), dict(W1q=FAKE + 4),
+    dict(s2=None), dict(y=FAKE + 2), dict(layer=FAKE + 1), dict(flags=1 << 4), dict(flags=1 << 11),
+    dict(workspace=FAKE + 16),
+])
+def test_batch_fp8_validates(bffn, kw):
+    a = dict(x=FAKE, C=4, L=8, d=256, layer=None, n_layers=2, Wr=FAKE, g=FAKE, br=None, W1q=FAKE, s1=FAKE, W2q=FAKE,
+             s2=FAKE, t2=FAKE, E=16, de=64, y=FAKE, active_idx=FAKE, n_active=FAKE, counts=None, tok_mask=None,
+             flags=0, workspace=None, workspace_bytes=0)
+    a.update(kw)
+    assert bffn.blockffn_chunk_forward_batch_fp8(
+        a["x"], a["C"], a["L"], a["d"], a["layer"], a["n_layers"], a["Wr"], a["g"], a["br"], a["W1q"], a["s1"],
+        a["W2q"], a["s2"], a["t2"], a["E"], a["de"], a["y"], a["active_idx"], a["n_active"], a["counts"],
+        a["tok_mask"], a["flags"], a["workspace"], a["workspace_bytes"], None) == bffn.BFFN_EINVAL
+
+
+def test_batch_fp8_workspace_size(bffn):
+    assert bffn.blockffn_batch_fp8_workspace_size(4096, 8, 2048, 64, 256) > 0
+    for bad in [(0, 8, 256, 16, 64), (4, 9, 256, 16, 64), (4, 8, 24, 16, 64), (4, 8, 256, 16, 40)]:
+        assert bffn.blockffn_batch_fp8_workspace_size(*bad) == 0
+    # the workspace does not grow past the h buffer of one wave of chunks
+    a = bffn.blockffn_batch_fp8_workspace_size(4096, 8, 2048, 64, 256)
+    b = bffn.blockffn_batch_fp8_workspace_size(8192, 8, 2048, 64, 256)
+    assert b - a < 8192 * 8 * 2048 * 2 + 4096 * 8 * 64 * 4 + (1 << 20)
