@@ -57,6 +57,9 @@ def _load():
             lib.oracle_e4m3_nearest.restype = i
             lib.oracle_quantize_fp8.argtypes = [p, p, i, i, i, i, p, p, p, p, p]
             lib.oracle_quantize_fp8.restype = i
+            lib.oracle_layer_backward.argtypes = [dptr, i, i, dptr, dptr, dptr, dptr, dptr, i, i, dptr, dptr, dptr,
+                                                  dptr, dptr, dptr, dptr, dptr]
+            lib.oracle_layer_backward.restype = i
             for f in ("oracle_router", "oracle_union", "oracle_expert", "oracle_chunk_forward",
                       "oracle_tokens_forward_mt", "oracle_union_overlap"):
                 getattr(lib, f).restype = i
@@ -174,6 +177,23 @@ def dequantize_fp8(q1, q2, s1, s2, t2):
     b2 = W2.astype(np.float32).view(np.uint32)
     assert np.all(b1 & 0xFFFF == 0) and np.all(b2 & 0xFFFF == 0), "dequantised weights must be bf16-exact"
     return (b1 >> 16).astype(np.uint16), (b2 >> 16).astype(np.uint16)
+
+
+def layer_backward(x, Wr, br, g, W1, W2, dy):
+    """The layer's backward for upstream gradient dy, every argument fp64 (widen bf16 inputs first): x [T,d],
+    Wr [d,E], br [E] or None, g [E], W1 [E,de,d], W2 [E,d,de], dy [T,d].  Returns a dict with y (the
+    forward), dx, dWr, db, dg, dW1, dW2."""
+    lib = _load()
+    f = lambda a: None if a is None else np.ascontiguousarray(a, dtype=np.float64)
+    x, Wr, br, g, W1, W2, dy = map(f, (x, Wr, br, g, W1, W2, dy))
+    T, d = x.shape
+    E, de = W1.shape[0], W1.shape[1]
+    out = {"y": np.zeros((T, d)), "dx": np.zeros((T, d)), "dWr": np.zeros((d, E)), "db": np.zeros(E),
+           "dg": np.zeros(E), "dW1": np.zeros((E, de, d)), "dW2": np.zeros((E, d, de))}
+    rc = lib.oracle_layer_backward(_ptr(x), T, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1), _ptr(W2), E, de, _ptr(dy),
+                                   *[_ptr(out[k]) for k in ("y", "dx", "dWr", "db", "dg", "dW1", "dW2")])
+    assert rc == 0
+    return out
 
 
 def expert(xt, W1, W2, i):

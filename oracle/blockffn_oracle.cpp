@@ -30,7 +30,8 @@
 // (g = 1 gives the survey's formula).
 //
 // The CLS-aware training objectives (activation locality, chunk sparsification; article, section 3) and
-// their backward through the router are at the end of this file, with the readings they take.
+// their backward through the router, the fp8 weight quantiser, and the layer's own backward are at the end
+// of this file, with the readings they take.
 //
 // Storage: x is bf16 bit patterns [L,d]; Wr fp32 [d,E]; br fp32 [E] (may be null = no bias);
 // g fp32 [E]; W1 bf16 bits [E,de,d]; W2 bf16 bits [E,d,de]; everything row-major.
@@ -345,19 +346,28 @@ double e4m3_value(uint8_t code) {  // the value an e4m3 code stands for (NaN cod
   return sgn ? -mag : mag;
 }
 // nearest e4m3 code to v (|v| <= 448), ties to the even code; the sign is kept (-0 for a negative input
-// that rounds to zero)
+// that rounds to zero).  The non-negative finite codes 0 .. 126 have increasing values, so the nearest is
+// one of the two codes around |v|, found by bisection.
 uint8_t e4m3_nearest(double v) {
+  static const std::vector<double> values = [] {
+    std::vector<double> t(127);
+    for (int c = 0; c < 127; ++c) t[c] = e4m3_value(uint8_t(c));  // 0x7F is NaN
+    return t;
+  }();
   const uint8_t sgn = (std::signbit(v) ? 0x80 : 0x00);
   const double a = std::fabs(v);
-  int best = 0;
-  double best_d = a;  // distance to code 0
-  for (int c = 1; c < 127; ++c) {  // 0x7F is NaN
-    const double dd = std::fabs(e4m3_value(uint8_t(c)) - a);
-    if (dd < best_d || (dd == best_d && (c & 1) == 0 && (best & 1) == 1)) {
-      best = c;
-      best_d = dd;
+  int lo = 0, hi = 126;  // values[lo] <= a < values[hi], or a at an end
+  if (a >= values[126]) {
+    lo = hi = 126;
+  } else {
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) / 2;
+      if (values[mid] <= a) lo = mid;
+      else hi = mid;
     }
   }
+  const double dlo = a - values[lo], dhi = values[hi] - a;
+  int best = (dlo < dhi || (dlo == dhi && (lo & 1) == 0)) ? lo : hi;
   if (g_mutation == 12) best = best > 0 ? best - 1 : 0;  // planted: rounds one code toward zero
   return uint8_t(sgn | best);
 }
@@ -410,6 +420,100 @@ int oracle_quantize_fp8(const uint16_t* W1, const uint16_t* W2, int n_layers, in
           q2[q] = e4m3_nearest(std::ldexp(widen_bf16(W2[q]), -m));
         }
       }
+  }
+  return 0;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------------------------------------------
+// The layer's backward (the training side of the same layer, lsdiaocha.cn BlockFFN article, section 2; the
+// pages print no backward, so it is the chain rule through the forward above, RMSNorm router only).  For
+// upstream gradient dy [T, d] of y:
+//   q_{t,e} = W2_e^T dy_t                       (de)
+//   dr_{t,e} = h_{t,e} . q_{t,e},  h = Swish(u), u = W1_e x_t
+//   du_{t,e} = r_{t,e} q_{t,e} * Swish'(u),  Swish'(u) = sig(u) (1 + u (1 - sig(u)))
+//   dW2_e += r_{t,e} dy_t h_{t,e}^T,  dW1_e += du_{t,e} x_t^T,  dx_t += W1_e^T du_{t,e}
+//   r_i = g_i a_i / rho, a = relu(s), rho = sqrt(mean_i a_i^2):
+//   dg_i += dr_i a_i / rho;  da_j = g_j dr_j / rho - a_j sum_i(dr_i g_i a_i) / (E rho^3);  ds = da [s > 0]
+//   dWr += x_t ds_t^T,  db += ds_t,  dx_t += Wr ds_t
+// A token with no positive s has r = 0 for every expert and gets no router gradient.  Every expert is
+// evaluated (dense); an inactive one contributes exact zeros through r = 0.  Weights and x are fp64 here
+// (the caller widens bf16), so finite differences can perturb any of them.
+extern "C" {
+
+// x [T,d], Wr [d,E], br [E] or null, g [E], W1 [E,de,d], W2 [E,d,de], dy [T,d]: all fp64.  Out (fp64): y
+// [T,d] (the forward, for finite differences of J = sum dy . y), dx [T,d], dWr [d,E], db [E], dg [E],
+// dW1 [E,de,d], dW2 [E,d,de].
+int oracle_layer_backward(const double* x, int T, int d, const double* Wr, const double* br, const double* g,
+                          const double* W1, const double* W2, int E, int de, const double* dy, double* y,
+                          double* dx, double* dWr, double* db, double* dg, double* dW1, double* dW2) {
+  if (T < 1 || d < 1 || E < 1 || de < 1) return 1;
+  for (size_t q = 0; q < static_cast<size_t>(T) * d; ++q) y[q] = dx[q] = 0.0;
+  for (size_t q = 0; q < static_cast<size_t>(d) * E; ++q) dWr[q] = 0.0;
+  for (int i = 0; i < E; ++i) db[i] = dg[i] = 0.0;
+  for (size_t q = 0; q < static_cast<size_t>(E) * de * d; ++q) dW1[q] = dW2[q] = 0.0;
+  std::vector<double> s(E), a(E), r(E), dr(E), u(de), h(de), q(de);
+  for (int t = 0; t < T; ++t) {
+    const double* xt = x + static_cast<size_t>(t) * d;
+    const double* dyt = dy + static_cast<size_t>(t) * d;
+    double sumsq = 0.0;
+    for (int i = 0; i < E; ++i) {
+      double acc = br ? br[i] : 0.0;
+      for (int k = 0; k < d; ++k) acc += xt[k] * Wr[static_cast<size_t>(k) * E + i];
+      s[i] = acc;
+      a[i] = acc > 0.0 ? acc : 0.0;
+      sumsq += a[i] * a[i];
+    }
+    const double rho = std::sqrt(sumsq / E);
+    for (int i = 0; i < E; ++i) r[i] = rho > 0.0 ? g[i] * a[i] / rho : 0.0;
+    for (int e = 0; e < E; ++e) {
+      const double* W1e = W1 + static_cast<size_t>(e) * de * d;
+      const double* W2e = W2 + static_cast<size_t>(e) * d * de;
+      for (int j = 0; j < de; ++j) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += W1e[static_cast<size_t>(j) * d + k] * xt[k];
+        u[j] = acc;
+        h[j] = acc / (1.0 + std::exp(-acc));
+      }
+      for (int k = 0; k < d; ++k) {
+        double acc = 0.0;
+        for (int j = 0; j < de; ++j) acc += W2e[static_cast<size_t>(k) * de + j] * h[j];
+        y[static_cast<size_t>(t) * d + k] += r[e] * acc;
+      }
+      for (int j = 0; j < de; ++j) {
+        double acc = 0.0;
+        for (int k = 0; k < d; ++k) acc += W2e[static_cast<size_t>(k) * de + j] * dyt[k];
+        q[j] = acc;
+      }
+      double dre = 0.0;
+      for (int j = 0; j < de; ++j) dre += h[j] * q[j];
+      dr[e] = dre;
+      for (int k = 0; k < d; ++k)
+        for (int j = 0; j < de; ++j) dW2[(static_cast<size_t>(e) * d + k) * de + j] += r[e] * dyt[k] * h[j];
+      for (int j = 0; j < de; ++j) {
+        const double sg = 1.0 / (1.0 + std::exp(-u[j]));
+        const double du = r[e] * q[j] * (g_mutation == 14 ? sg : sg * (1.0 + u[j] * (1.0 - sg)));  // planted 14
+        for (int k = 0; k < d; ++k) {
+          dW1[(static_cast<size_t>(e) * de + j) * d + k] += du * xt[k];
+          dx[static_cast<size_t>(t) * d + k] += W1e[static_cast<size_t>(j) * d + k] * du;
+        }
+      }
+    }
+    if (rho > 0.0) {
+      double c = 0.0;  // sum_i dr_i g_i a_i
+      for (int i = 0; i < E; ++i) c += dr[i] * g[i] * a[i];
+      for (int i = 0; i < E; ++i) {
+        dg[i] += dr[i] * a[i] / rho;
+        const double da = g[i] * dr[i] / rho - (g_mutation == 15 ? 0.0 : a[i] * c / (E * rho * rho * rho));  // planted 15
+        const double ds = s[i] > 0.0 ? da : 0.0;
+        db[i] += ds;
+        for (int k = 0; k < d; ++k) {
+          dWr[static_cast<size_t>(k) * E + i] += xt[k] * ds;
+          dx[static_cast<size_t>(t) * d + k] += Wr[static_cast<size_t>(k) * E + i] * ds;
+        }
+      }
+    }
   }
   return 0;
 }
