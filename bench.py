@@ -788,6 +788,82 @@ def run_fp8(args):
     print(json.dumps(line), flush=True)
 
 
+def run_backward(args):
+    """The layer's backward (blockffn_layer_backward) for --chunks chunks of 8 tokens (default 512: 4096
+    tokens) at the decode layer's shape (d = 2048, E = 64, de = 256) with a random upstream gradient.
+    Roofline: the dense contraction flops of the step (5 products of 2 T d E de: U, Q, dW2, dW1, dX; the
+    router's are 4 T d E) over its CUDA-event time, against the measured bf16 tensor peak; the MMAs
+    issued are about twice that (fp32 operands as bf16 hi + lo pairs)."""
+    import numpy as np
+    import torch
+
+    import chunk_sparse_moe_router_b200 as bffn
+    import gen
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    C, L, d, E, de = args.chunks or 512, 8, 2048, 64, 256
+    T = C * L
+    lay = gen.make_layer(0, d, E, de, beta=0.84, var_x=1.09)
+    x_np = gen.make_chunks(0, lay, C, L, 0.3).reshape(T, d)
+    dy_np = np.random.default_rng(1).standard_normal((T, d)).astype(np.float32)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    bf = lambda bits: t(bits.view(np.int16)).view(torch.bfloat16)
+    x, W1, W2 = bf(x_np), bf(lay.W1), bf(lay.W2)
+    Wr, br, g, dy = t(lay.Wr), t(lay.br), t(lay.g), t(dy_np)
+    ws = torch.empty(bffn.blockffn_layer_backward_workspace_size(T, d, E, de), dtype=torch.uint8, device=device)
+    s = torch.cuda.Stream(device)
+
+    def step():
+        bffn.layer_backward(x, Wr, g, W1, W2, dy, br=br, workspace=ws, stream=s.cuda_stream)
+
+    with torch.cuda.stream(s):
+        step()
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        graph.capture_begin()
+        step()
+        graph.capture_end()
+        for _ in range(args.warmup):
+            graph.replay()
+        s.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(0) as clocks:
+            e0.record(s)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(s)
+            e1.synchronize()
+        del graph
+    ms = e0.elapsed_time(e1) / args.steps
+    flops = 5 * 2.0 * T * d * E * de + 4.0 * T * d * E
+    peak, peak_kind = measured_peaks("bf16_tflops")
+    tf = flops / (ms * 1e-3) / 1e12
+    line = {"metric": "BlockFFN layer backward tokens/s and achieved TFLOP/s (dense over experts)",
+            "value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16 x and weights; fp32 dy and gradients (hi + lo bf16 pairs on warp MMAs)",
+            "data": "synthetic",
+            "config": {"workload": f"backward_T{T}_d{d}_E{E}_de{de}", "tokens": T,
+                       "l2": "inputs larger than L2 (U, Q and the pairs: 1.1 GB of intermediates per step)"},
+            "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(tf / peak, 4), "peak_kind": peak_kind, "traffic": None,
+                         "flops_per_step": flops},
+            "gpu_launches": 14 * args.steps, "clocks": clocks.summary()}
+    if not args.no_cpu_baseline:
+        import oracle
+        w = lambda b: gen.bf16_bits_to_f32(b).astype(np.float64)
+        W1f, W2f = w(lay.W1), w(lay.W2)
+        n, t0 = 0, time.time()
+        while time.time() - t0 < args.cpu_seconds and n < T:
+            oracle.layer_backward(w(x_np[n:n + 1]), lay.Wr, lay.br, lay.g, W1f, W2f, dy_np[n:n + 1])
+            n += 1
+        dt = time.time() - t0
+        line["cpu_baseline"] = {"value": round(n / dt, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{n} tokens, one at a time (dense fp64), {dt:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
 def run_cls_losses(args):
     """The CLS-aware losses and their backward through the router (blockffn_cls_losses): one step = the
     activation-locality and chunk-sparsification losses of a training batch of --chunks chunks of 8 tokens
@@ -961,7 +1037,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses", "fp8"])
+                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses", "fp8", "backward"])
     ap.add_argument("--drift", default="0.0,0.9,0.97",
                     help="--workload reuse: drift of the chunk bases of a sequence (0: independent chunks)")
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
@@ -1007,6 +1083,9 @@ def main():
         return
     if args.workload == "fp8":
         run_fp8(args)
+        return
+    if args.workload == "backward":
+        run_backward(args)
         return
     w = gen.workload(args.workload, **kw)
     if args.impl == "reference":

@@ -44,6 +44,8 @@ SIGNATURES = {
     "blockffn_chunk_forward_batch_fp8": (_I, [_P, _I, _I, _I, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _P, _P,
                                              _P, _P, _P, _I, _P, _S, _P]),
     "blockffn_batch_fp8_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "blockffn_layer_backward": (_I, [_P, _I, _I, _P, _P, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P]),
+    "blockffn_layer_backward_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_cls_losses": (_I, [_P, _I, _I, _I, _P, _P, _I, _F, _F, _F, _P, _P, _P, _P, _P, _P, _S, _P]),
     "blockffn_cls_losses_workspace_size": (_S, [_I, _I, _I, _I]),
     "blockffn_workspace_size": (_S, [_I, _I, _I, _I]),
@@ -128,6 +130,16 @@ def blockffn_chunk_forward_batch_fp8(x, C, L, d, layer, n_layers, Wr, g, br, W1q
 
 def blockffn_batch_fp8_workspace_size(C, L, d, E, de):
     return _lib.blockffn_batch_fp8_workspace_size(C, L, d, E, de)
+
+
+def blockffn_layer_backward(x, T, d, Wr, br, g, W1, W2, E, de, dy, dx, dWr, db, dg, dW1, dW2, workspace,
+                            workspace_bytes, stream):
+    return _lib.blockffn_layer_backward(x, T, d, Wr, br, g, W1, W2, E, de, dy, dx, dWr, db, dg, dW1, dW2, workspace,
+                                        workspace_bytes, stream)
+
+
+def blockffn_layer_backward_workspace_size(T, d, E, de):
+    return _lib.blockffn_layer_backward_workspace_size(T, d, E, de)
 
 
 def blockffn_cls_losses(x, C, L, d, Wr, br, E, alpha, w_al, w_cs, loss, dS, dWr, db, dx, workspace,
@@ -302,6 +314,41 @@ def cls_losses(x, C, L, Wr, br=None, alpha=1.0, w_al=1.0, w_cs=1.0, loss=None, d
     if rc != BFFN_OK:
         raise BlockFFNError(rc, "blockffn_cls_losses")
     return loss, dS, dWr, db, dx
+
+
+def layer_backward(x, Wr, g, W1, W2, dy, br=None, workspace=None, stream=None):
+    """The layer's backward: x bf16 [T, d], Wr fp32 [d, E], g fp32 [E], W1 bf16 [E, de, d], W2 bf16 [E, d, de],
+    dy fp32 [T, d] (br fp32 [E] or None).  Returns a dict of fp32 tensors dx, dWr, db, dg, dW1, dW2.
+    Raises BlockFFNError."""
+    import torch
+
+    T, d = x.shape
+    E, de = W1.shape[0], W1.shape[1]
+    dev = x.device
+    _check(x, "x", torch.bfloat16, (T, d), dev)
+    _check(Wr, "Wr", torch.float32, (d, E), dev)
+    _check(g, "g", torch.float32, (E,), dev)
+    _check(W1, "W1", torch.bfloat16, (E, de, d), dev)
+    _check(W2, "W2", torch.bfloat16, (E, d, de), dev)
+    _check(dy, "dy", torch.float32, (T, d), dev)
+    if br is not None:
+        _check(br, "br", torch.float32, (E,), dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    out = {"dx": torch.empty((T, d), **f32), "dWr": torch.empty((d, E), **f32), "db": torch.empty(E, **f32),
+           "dg": torch.empty(E, **f32), "dW1": torch.empty((E, de, d), **f32), "dW2": torch.empty((E, d, de), **f32)}
+    need = blockffn_layer_backward_workspace_size(T, d, E, de)
+    if need == 0:
+        raise BlockFFNError(BFFN_EINVAL, "blockffn_layer_backward_workspace_size")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if stream is None:
+        stream = torch.cuda.current_stream(dev).cuda_stream
+    rc = blockffn_layer_backward(_ptr(x), T, d, _ptr(Wr), _ptr(br), _ptr(g), _ptr(W1), _ptr(W2), E, de, _ptr(dy),
+                                 *[_ptr(out[k]) for k in ("dx", "dWr", "db", "dg", "dW1", "dW2")],
+                                 workspace.data_ptr(), workspace.numel() * workspace.element_size(), stream)
+    if rc != BFFN_OK:
+        raise BlockFFNError(rc, "blockffn_layer_backward")
+    return out
 
 
 def quantize_fp8(W1, W2, n_layers, stream=None):

@@ -14,7 +14,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libblockffn.so")
 SOURCES = ["api.cu", "expert_decode.cu", "expert_decode_tc.cu", "decode_batch.cu", "prefill.cu", "noalloc.cu",
-           "union_overlap.cu", "cls_losses.cu", "fp8_decode.cu"]
+           "union_overlap.cu", "cls_losses.cu", "fp8_decode.cu",
+           "layer_backward.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

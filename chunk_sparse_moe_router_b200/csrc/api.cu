@@ -696,6 +696,44 @@ int blockffn_chunk_forward_batch_fp8(const void* x, int C, int L, int d, const i
   return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
 }
 
+size_t blockffn_layer_backward_workspace_size(int T, int d, int E, int de) {
+  if (T < 1 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
+      1ll * T * E * de >= (1ll << 31) || 1ll * T * d >= (1ll << 31))
+    return 0;
+  DeviceInfo di;
+  int dev = 0;
+  const int sms = device_info(&di, &dev) == BFFN_OK ? di.num_sms : 148;
+  return bwd::layout(T, d, E, de, sms).total;
+}
+
+int blockffn_layer_backward(const void* x, int T, int d, const float* Wr, const float* br, const float* g,
+                            const void* W1, const void* W2, int E, int de, const float* dy, float* dx, float* dWr,
+                            float* db, float* dg, float* dW1, float* dW2, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (T < 1 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
+      1ll * T * E * de >= (1ll << 31) || 1ll * T * d >= (1ll << 31))
+    return BFFN_EINVAL;
+  const void* bulk[] = {x, W1, W2};
+  for (const void* p : bulk)
+    if (p == nullptr || !aligned16(p)) return BFFN_EINVAL;
+  const void* req[] = {Wr, g, dy, dx, dWr, db, dg, dW1, dW2};
+  for (const void* p : req)
+    if (p == nullptr || !aligned4(p)) return BFFN_EINVAL;
+  if (!aligned16(dy)) return BFFN_EINVAL;
+  if (br != nullptr && !aligned4(br)) return BFFN_EINVAL;
+  if (workspace == nullptr || !aligned256(workspace)) return BFFN_EINVAL;
+  DeviceInfo di;
+  int dev = 0;
+  const int rc = device_info(&di, &dev);
+  if (rc != BFFN_OK) return rc;
+  if (workspace_bytes < bwd::layout(T, d, E, de, di.num_sms).total) return BFFN_ENOMEM;
+  const cudaError_t err =
+      bwd::launch(static_cast<const __nv_bfloat16*>(x), T, d, Wr, br, g, static_cast<const __nv_bfloat16*>(W1),
+                  static_cast<const __nv_bfloat16*>(W2), E, de, dy, dx, dWr, db, dg, dW1, dW2, workspace, di.num_sms,
+                  static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? BFFN_OK : cuda_fail(err);
+}
+
 int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* n_active_a, const int32_t* active_idx_b,
                            const int32_t* n_active_b, int C, int E, int32_t* overlap, void* stream) {
   if (C < 1 || E < 1 || E > kMaxE) return BFFN_EINVAL;

@@ -439,6 +439,18 @@ cudaError_t quantize(const __nv_bfloat16* W1, const __nv_bfloat16* W2, int n_lay
 cudaError_t forward(const Fp8Params& p, const Maps& m, const batch::Params& rp, int num_sms, cudaStream_t st);
 }  // namespace fp8
 
+// ---------------------------------------------------------------- layer backward (layer_backward.cu)
+namespace bwd {
+struct Layout {  // byte offsets into the workspace
+  size_t wsplit, sparts, s, r, rho, dyhl, U, Q, rhhl, duhl, dr, ds, dgc, dshl, total;
+  int parts;
+};
+Layout layout(int T, int d, int E, int de, int num_sms);
+cudaError_t launch(const __nv_bfloat16* x, int T, int d, const float* Wr, const float* br, const float* g,
+                   const __nv_bfloat16* W1, const __nv_bfloat16* W2, int E, int de, const float* dy, float* dx,
+                   float* dWr, float* db, float* dg, float* dW1, float* dW2, void* ws, int num_sms, cudaStream_t st);
+}  // namespace bwd
+
 // ---------------------------------------------------------------- CLS-aware losses (cls_losses.cu)
 namespace cls {
 constexpr int kTargetCtas = 296;               // dWr grid: two CTAs on each SM of a B200

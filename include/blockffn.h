@@ -193,6 +193,30 @@ BFFN_API int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* 
                                     int32_t* overlap, void* stream);
 
 /*
+ * The layer's backward (the training side of the layer computed by blockffn_chunk_forward, RMSNorm router;
+ * lsdiaocha.cn BlockFFN article, section 2 gives the forward; the backward is its chain rule).  For T tokens
+ * x (bf16 [T, d]) and upstream gradient dy (fp32 [T, d], 16-byte aligned) of y:
+ *   dx fp32 [T, d], dWr fp32 [d, E], db fp32 [E], dg fp32 [E], dW1 fp32 [E, de, d], dW2 fp32 [E, d, de]
+ * are written (overwritten), with Wr fp32 [d, E], br fp32 [E] or NULL, g fp32 [E], W1 bf16 [E, de, d],
+ * W2 bf16 [E, d, de] as in the forward.  A token whose router outputs are all zero has r = 0 and passes no
+ * gradient to the router.  The experts are evaluated densely (an inactive expert's terms are exact zeros
+ * through r = 0); every contraction runs on the warp tensor cores, fp32 operands carried as bf16 hi + lo
+ * pairs, with fp32 accumulation in a fixed order (bit-identical reruns).
+ * workspace: device memory of at least blockffn_layer_backward_workspace_size(T, d, E, de) bytes, 256-byte
+ * aligned (about 12 T E de bytes; its contents need not be initialised).
+ * Requirements (BFFN_EINVAL otherwise): T >= 1, d and de multiples of 8, 1 <= E <= 1024, T E de < 2^31;
+ * x, W1, W2, dy 16-byte aligned, the rest 4-byte aligned, non-NULL except br.  A smaller workspace returns
+ * BFFN_ENOMEM, a failed launch BFFN_ECUDA.
+ */
+BFFN_API int blockffn_layer_backward(const void* x, int T, int d, const float* Wr, const float* br, const float* g,
+                                     const void* W1, const void* W2, int E, int de, const float* dy, float* dx,
+                                     float* dWr, float* db, float* dg, float* dW1, float* dW2, void* workspace,
+                                     size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace blockffn_layer_backward needs (0 if the sizes are invalid). */
+BFFN_API size_t blockffn_layer_backward_workspace_size(int T, int d, int E, int de);
+
+/*
  * Low-bit expert weights (not a BlockFFN claim: the intelliparadigm survey, section 4.1, lists low-bit
  * quantisation of MoE expert weights; the layer computed is unchanged, lsdiaocha.cn BlockFFN article,
  * sections 2 and 4).  Format, for NE = n_layers * E experts (layer l owns experts l E .. l E + E - 1):

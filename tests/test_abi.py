@@ -230,3 +230,23 @@ def test_batch_fp8_workspace_size(bffn):
     a = bffn.blockffn_batch_fp8_workspace_size(4096, 8, 2048, 64, 256)
     b = bffn.blockffn_batch_fp8_workspace_size(8192, 8, 2048, 64, 256)
     assert b - a < 8192 * 8 * 2048 * 2 + 4096 * 8 * 64 * 4 + (1 << 20)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=0), dict(d=12), dict(de=4), dict(E=0), dict(E=1025), dict(x=None), dict(x=FAKE + 8), dict(W1=FAKE + 2),
+    dict(dy=FAKE + 4), dict(dx=None), dict(dW2=FAKE + 2), dict(br=FAKE + 1), dict(workspace=None),
+    dict(workspace=FAKE + 16),
+])
+def test_layer_backward_validates(bffn, kw):
+    a = dict(x=FAKE, T=64, d=256, Wr=FAKE, br=None, g=FAKE, W1=FAKE, W2=FAKE, E=16, de=64, dy=FAKE, dx=FAKE,
+             dWr=FAKE, db=FAKE, dg=FAKE, dW1=FAKE, dW2=FAKE, workspace=FAKE, workspace_bytes=1 << 40)
+    a.update(kw)
+    assert bffn.blockffn_layer_backward(
+        a["x"], a["T"], a["d"], a["Wr"], a["br"], a["g"], a["W1"], a["W2"], a["E"], a["de"], a["dy"], a["dx"],
+        a["dWr"], a["db"], a["dg"], a["dW1"], a["dW2"], a["workspace"], a["workspace_bytes"], None) == bffn.BFFN_EINVAL
+
+
+def test_layer_backward_workspace_size(bffn):
+    assert bffn.blockffn_layer_backward_workspace_size(4096, 2048, 64, 256) > 4096 * 64 * 256 * 12
+    for bad in [(0, 256, 16, 64), (64, 250, 16, 64), (64, 256, 0, 64), (64, 256, 16, 60)]:
+        assert bffn.blockffn_layer_backward_workspace_size(*bad) == 0
