@@ -84,10 +84,15 @@ def measured_peaks(key="hbm_gbs"):
         return (FALLBACK_HBM_GBS if key == "hbm_gbs" else 1590.0), "fallback"
 
 
+# the sources the batched decode kernels are compiled from (the kernels, the headers they include, the
+# host code that sizes their launches); a change to any of them makes recorded counters stale
+BATCH_KERNEL_SOURCES = ("api.cu", "decode_batch.cu", "blockffn_internal.cuh", "ptx.cuh")
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "chunk_sparse_moe_router_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in BATCH_KERNEL_SOURCES:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode())
             h.update(f.read())
@@ -254,8 +259,10 @@ def run_ours(args, w):
         ws_bytes = bffn.blockffn_workspace_size(L, d, E, de)
         workspaces = [bffn.new_workspace(L, d, E, de, device) for _ in range(K)]  # zero-filled
     ws_ptrs = [t.data_ptr() for t in workspaces]
+    bufs = [(x_dev, y, idx, nact, cnts)]  # a second set is added for the end-to-end pipeline
 
-    def step(streams):
+    def step(streams, buf=None):
+        x_dev, y, idx, nact, cnts = buf if buf is not None else bufs[0]
         if batched:
             rc = bffn.blockffn_chunk_forward_batch(
                 x_dev.data_ptr(), chunks, L, d, None, w.replicas, stack["Wr"].data_ptr(), stack["g"].data_ptr(),
@@ -320,34 +327,70 @@ def run_ours(args, w):
             if bffn.device_status(workspace=ws, stream=s.cuda_stream) != 0:
                 raise RuntimeError("device-side wait ran out during the timed region")
 
-        # end to end: x from pinned host memory in, y and the active sets back, every step
+        # end to end, as a serving loop runs it: every step copies its x in from pinned host memory and its
+        # y and active sets back out, double-buffered on two copy streams, so that step k+1's input and step
+        # k-1's results cross PCIe while step k computes
         x_pin = torch.from_numpy(x_host_np.view(np.int16)).pin_memory()
-        y_pin = torch.empty(y.shape, dtype=y.dtype).pin_memory()
-        idx_pin = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-        n_pin = torch.empty(nact.shape, dtype=nact.dtype).pin_memory()
-        x_dev_i16 = x_dev.view(torch.int16)
-
-        def e2e_step():
-            x_dev_i16.copy_(x_pin, non_blocking=True)
-            graph.replay()
-            y_pin.copy_(y, non_blocking=True)
-            idx_pin.copy_(idx, non_blocking=True)
-            n_pin.copy_(nact, non_blocking=True)
-
-        for _ in range(2):
-            e2e_step()
+        bufs.append((torch.empty_like(x_dev), torch.empty_like(y), torch.empty_like(idx), torch.empty_like(nact),
+                     torch.empty_like(cnts)))
+        graphs = [graph, torch.cuda.CUDAGraph()]
+        step(streams, bufs[1])
         s.synchronize()
+        graphs[1].capture_begin()
+        step(streams, bufs[1])
+        graphs[1].capture_end()
+        pins = [(torch.empty(y.shape, dtype=y.dtype).pin_memory(), torch.empty(idx.shape, dtype=idx.dtype).pin_memory(),
+                 torch.empty(nact.shape, dtype=nact.dtype).pin_memory()) for _ in range(2)]
+        s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(k):
+            b = k % 2
+            xb, yb, ib, nb, _ = bufs[b]
+            if k >= 2:  # buffer b's previous input has been consumed
+                s_in.wait_event(ev_done[b])
+            with torch.cuda.stream(s_in):
+                xb.view(torch.int16).copy_(x_pin, non_blocking=True)
+            ev_in[b].record(s_in)
+            s.wait_event(ev_in[b])
+            if k >= 2:  # buffer b's previous results have left the device
+                s.wait_event(ev_out[b])
+            graphs[b].replay()
+            ev_done[b].record(s)
+            s_out.wait_event(ev_done[b])
+            with torch.cuda.stream(s_out):
+                pins[b][0].copy_(yb, non_blocking=True)
+                pins[b][1].copy_(ib, non_blocking=True)
+                pins[b][2].copy_(nb, non_blocking=True)
+            ev_out[b].record(s_out)
+
+        def run(n):  # n pipelined steps between events on s (the copy streams start after the first)
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record(s)
+            s_in.wait_event(start)
+            s_out.wait_event(start)
+            for k in range(n):
+                e2e_step(k)
+            for b in range(2):
+                s.wait_event(ev_out[b])
+            end.record(s)
+            end.synchronize()
+            return start, end
+
+        run(2)
+        torch.cuda.synchronize(device)
         barrier(device)
         torch.cuda.synchronize(device)
-        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e2e_steps = max(3, args.steps // 2)
-        f0.record(s)
-        for _ in range(e2e_steps):
-            e2e_step()
-        f1.record(s)
-        f1.synchronize()
+        f0, f1 = run(e2e_steps)
         barrier(device)
         e2e_ms = f0.elapsed_time(f1)
+        last = pins[(e2e_steps - 1) % 2]
+        if not (torch.equal(last[0], y.cpu()) and torch.equal(last[2], nact.cpu())):
+            raise RuntimeError("the pipelined end-to-end results differ from the device-timed step's")
+        del graphs
 
         # one chunk at a time on the whole GPU (the latency a verification step sees per layer): the
         # first n1 chunks through the per-chunk entry point on one stream, as one graph
@@ -448,7 +491,8 @@ def run_ours(args, w):
         "e2e": {"value": round(tokens_step / (e2e_max / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": int(x_host_np.nbytes),
                 "d2h_bytes_per_step": int(y.numel() * 4 + idx.numel() * 4 + nact.numel() * 4),
-                "steps": e2e_steps},
+                "steps": e2e_steps,
+                "pipeline": "double-buffered: step k+1's x in and step k-1's results out overlap step k"},
         "gpu_launches": (2 if batched else (7 if prefill else 1) * chunks) * args.steps,
         "clocks": clk.summary(),
         "gen_seconds": round(gen_s, 1),
