@@ -15,11 +15,13 @@
 // Kernels of a forward call: the batched router (decode_batch.cu), x to f16, a scan of the per-chunk
 // up-projection items, then per wave of chunks an up-projection and a down-projection kernel.  Both
 // stream kernels take 64 weight rows per item through a ring of stages (64 rows x 256 bytes of codes as
-// two TMA boxes, plus the matching activations by cp.async); warps own 16 rows and half of a stage's k:
-// ldmatrix brings four fp8 codes per thread, integer ops turn them into f16 pairs, and mma.sync f16
-// (fp32 accumulate) contracts them with the activations in f16, read in the same order of k (a thread's
-// pair of A slots 2c, 2c+1 holds codes 4c, 4c+1 and slots 2c+8, 2c+9 codes 4c+2, 4c+3, so its B fragment
-// is the activations at 4c .. 4c+3).  cvt turns a pair of codes into their exact f16 values.
+// two TMA boxes, plus the matching f16 activations by cp.async), filled by one producer warp; eight
+// consumer warps own 16 rows and half of a stage's k each: ldmatrix brings four fp8 codes per thread, cvt
+// turns each pair into its exact f16 values, and mma.sync f16 (fp32 accumulate) contracts them with the
+// activations in f16, read in the same order of k (a thread's pair of A slots 2c, 2c+1 holds codes 4c,
+// 4c+1 and slots 2c+8, 2c+9 codes 4c+2, 4c+3, so its B fragment is the activations at 4c .. 4c+3).  The
+// activations are x (bf16 values, exact in f16 in the normal range) and h'' rounded once to f16 (a
+// relative 2^-11 per element, the one rounding the fp8 path adds beyond fp32 accumulation).
 // Every sum runs in a fixed order: y is bit-reproducible.
 #include <algorithm>
 #include <cuda_fp16.h>
@@ -31,21 +33,33 @@ namespace bffn {
 namespace fp8 {
 namespace {
 
-constexpr int kT = 256;             // stream kernels: 8 warps = 4 groups of 16 weight rows x 2 halves of k
+constexpr int kCT = 256;            // consumer threads: 8 warps = 4 groups of 16 weight rows x 2 halves of k
+constexpr int kT = kCT + 32;        // + one producer warp: the code boxes (TMA) and activations (cp.async)
 constexpr int kRows = 64;           // weight rows per item
 constexpr int kKB = 256;            // code bytes (k values) of a row per stage
 constexpr int kWSub = kRows * 128;  // one tensor box: 64 rows x 128 codes, 128-byte swizzle (8 KB)
 constexpr int kWBytes = 2 * kWSub;  // a stage's codes: two boxes side by side along k
 constexpr int kAPitch = 2 * kKB + 32;  // 544 B rows of 256 f16 activations: conflict-free 8-byte loads
 constexpr int kStages = 4;
-constexpr int kXBytes = 8 * kAPitch;              // 4352 (8 token rows)
-constexpr int kUpStage = (kWBytes + kXBytes + 1023) / 1024 * 1024;       // 21504: boxes stay 1024-aligned
-constexpr int kDownStage = (kWBytes + 2 * kXBytes + 1023) / 1024 * 1024;  // 25600 (h hi and lo planes)
-constexpr int kUpSmem = kStages * kUpStage + 1024;  // + alignment slack
-constexpr int kDownSmem = kStages * kDownStage + 1024;
+constexpr int kXBytes = 8 * kAPitch;                                // 4352 (8 token rows)
+constexpr int kStage = (kWBytes + kXBytes + 1023) / 1024 * 1024;  // 21504: boxes stay 1024-aligned
+constexpr int kSmem = kStages * kStage + 1024;                    // + alignment slack
 constexpr uint64_t kFp8WaitNs = 2000000000ull;
 
 __device__ __forceinline__ int layer_of(const Fp8Params& p, int c) { return p.layer ? p.layer[c] : c % p.n_layers; }
+
+// The mbarrier receives one arrival once every cp.async this thread issued before has landed (its
+// expected count includes these arrivals).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Barrier `id` (1 .. 15) among `n` threads (whole warps).
+__device__ __forceinline__ void named_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 
 // The smallest m with 448 2^m >= amax (0 for amax == 0), in exact fp32 comparisons.
@@ -229,17 +243,18 @@ __global__ void __launch_bounds__(256) decode_items_kernel(const Fp8Params p, in
 // ------------------------------------------------------------------------------------ up-projection
 // Items of chunks [c0, c1): (chunk, active expert, 64-row block of de), described by desc[].  A CTA walks
 // items blockIdx.x, + gridDim.x, ...; each item is ns = ceil(d / 256) stages of 64 rows x 256 codes of W1
-// and 8 x 256 f16 of x.  The copies of stage i + 3 are issued while stage i is contracted; the next item's
-// descriptor and the epilogue's r and scales are fetched into registers stages before they are used, so
-// no global load sits between a stage and the issue of its copies.  The epilogue writes
-// h'' = s2 r Swish(s1 u) as f16 hi + lo into h[chunk - c0][a][plane][t][j].
+// and 8 x 256 f16 of x.  Warp 8 produces: it waits until the 8 consumer warps have released a ring slot
+// (empty[s]), then issues the slot's two code boxes (TMA, transaction bytes on full[s]) and the x rows
+// (cp.async, one arrival per lane on full[s] once its copies land).  The consumers wait on full[s] only,
+// so no CTA-wide barrier sits between stages.  At an item's end the two k-halves of a row group meet at a
+// barrier of their own; the epilogue writes h'' = s2 r Swish(s1 u) as f16 into h[chunk - c0][a][t][j].
 __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_constant__ Maps mp, int c0, int c1,
                                                const int4* __restrict__ desc) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ float4 xchg[4 * 32];  // the k-half 1 warps' partial sums at an item's end
-  __shared__ __align__(8) uint64_t full[kStages];  // a stage's code boxes landed
-  const int tid = threadIdx.x, lane = tid & 31, g = lane >> 2, cq = lane & 3;
-  const int warp = (tid >> 5) & 3, wk = tid >> 7;  // row group, half of the stage's k
+  __shared__ float4 xchg[2][4 * 32];  // the k-half 1 warps' partial sums at an item's end (by item parity)
+  __shared__ __align__(8) uint64_t full[kStages];   // a stage's code boxes and x rows landed
+  __shared__ __align__(8) uint64_t empty[kStages];  // the 8 consumer warps are done reading a stage
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int n_items = p.offs[c1] - p.offs[c0];
   const int G = int(gridDim.x), b = int(blockIdx.x);
   const int mine = n_items > b ? (n_items - b + G - 1) / G : 0;
@@ -249,46 +264,54 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
   uint8_t* const sgen = smem_raw + (sbase - smem_u32(smem_raw));
   if (tid == 0) {
     prefetch_tensormap(&mp.w1);
-    for (int q = 0; q < kStages; ++q) mbar_init(&full[q], 1);
+    for (int q = 0; q < kStages; ++q) {
+      mbar_init(&full[q], 1 + 32);
+      mbar_init(&empty[q], kCT / 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
-  const uint64_t pol = policy_evict_first();  // the codes stream through once
 
-  // loader: the descriptor of the item being loaded, and the next one's (in flight)
-  int4 dl = make_int4(0, 0, 0, 0), dn = make_int4(0, 0, 0, 0);
-  if (mine > 0) dl = desc[b];
-  if (mine > 1) dn = desc[b + G];
-  int ml = 0;
-  auto load = [&](int i) {
-    const int m = i / ns, ks = i - m * ns;
-    if (m != ml) {  // next item: its descriptor arrived long ago; fetch the one after
-      ml = m;
-      dl = dn;
-      if (m + 1 < mine) dn = desc[b + (m + 1) * G];
-    }
-    const int slot = i % kStages;
-    const uint32_t st = sbase + slot * kUpStage;
-    const int k0 = ks * kKB;
-    if (tid == 0) {  // W1 codes: two boxes (rows past de belong to the next expert: their u is never stored;
-                     // columns past d and rows past the last expert read as zeros)
-      fence_proxy_async_smem();
-      mbar_arrive_expect_tx(&full[slot], kWBytes);
-      uint8_t* dst = sgen + slot * kUpStage;
-      tma_load_2d(dst, &mp.w1, k0, dl.w * p.de + dl.z * kRows, &full[slot], pol);
-      tma_load_2d(dst + kWSub, &mp.w1, k0 + 128, dl.w * p.de + dl.z * kRows, &full[slot], pol);
-    }
-    {  // x in f16: 8 rows x 32 pieces
-      const int idx = tid, t = idx >> 5, ch = idx & 31;
-      const int k = k0 + ch * 8;
+  if (wid == kCT / 32) {  // producer
+    const uint64_t pol = policy_evict_first();  // the codes stream through once
+    int4 dl = make_int4(0, 0, 0, 0), dn = make_int4(0, 0, 0, 0);  // the item being loaded, the next one
+    if (mine > 0) dl = desc[b];
+    if (mine > 1) dn = desc[b + G];
+    int ml = 0;
+    for (int i = 0; i < total; ++i) {
+      const int m = i / ns, ks = i - m * ns;
+      if (m != ml) {  // next item: its descriptor arrived long ago; fetch the one after
+        ml = m;
+        dl = dn;
+        if (m + 1 < mine) dn = desc[b + (m + 1) * G];
+      }
+      const int slot = i % kStages;
+      if (i >= kStages && !mbar_wait_bounded(&empty[slot], uint32_t(i / kStages - 1) & 1u, kFp8WaitNs))
+        atomicOr(&p.hdr->err, uint32_t(kErrRingWait));  // recorded; the CTA goes on without hanging
+      const int k0 = ks * kKB;
+      if (lane == 0) {  // W1 codes: two boxes (rows past de belong to the next expert: their u is never
+                        // stored; columns past d and rows past the last expert read as zeros)
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&full[slot], kWBytes);
+        uint8_t* dst = sgen + slot * kStage;
+        tma_load_2d(dst, &mp.w1, k0, dl.w * p.de + dl.z * kRows, &full[slot], pol);
+        tma_load_2d(dst + kWSub, &mp.w1, k0 + 128, dl.w * p.de + dl.z * kRows, &full[slot], pol);
+      }
+      const int k = k0 + lane * 8;  // x in f16: 8 rows, this lane's 16-byte piece of each
       const bool ok = k < p.d;
-      const __half* src = ok ? p.xh + (size_t(dl.x) * 8 + t) * p.d + k : p.xh;
-      cp_async16(st + kWBytes + t * kAPitch + ch * 16, src, ok ? 16 : 0);
+      const uint32_t xs = sbase + slot * kStage + kWBytes + lane * 16;
+#pragma unroll
+      for (int t = 0; t < 8; ++t)
+        cp_async16(xs + t * kAPitch, ok ? p.xh + (size_t(dl.x) * 8 + t) * p.d + k : p.xh, ok ? 16 : 0);
+      cp_async_arrive_noinc(&full[slot]);
     }
-  };
+    cp_async_wait_all();
+    return;
+  }
 
-  // consumer: the current item's descriptor and the epilogue's inputs, fetched at its first stages
-  int4 dc = make_int4(0, 0, 0, 0);
+  // consumers: warp rows 16 w .. 16 w + 15 of the item, k-half wk of each stage
+  const int g = lane >> 2, cq = lane & 3, warp = wid & 3, wk = wid >> 2;
+  int4 dc = make_int4(0, 0, 0, 0);  // the current item; the epilogue's inputs fetched at its first stages
   float ep_r[2] = {0.f, 0.f}, ep_s1[2] = {0.f, 0.f}, ep_s2[2] = {0.f, 0.f};
   auto fetch_epilogue = [&]() {
     const int el = dc.w % p.E;
@@ -300,24 +323,15 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
       ep_s2[h] = j < p.de ? p.s2[size_t(dc.w) * p.de + j] : 0.f;
     }
   };
-
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-  for (int i = 0; i < kStages - 1; ++i) {
-    if (i < total) load(i);
-    cp_async_commit();
-  }
   for (int i = 0; i < total; ++i) {
     const int mc = i / ns, ks = i - mc * ns;
     if (ks == 0) dc = desc[b + mc * G];
     if (ks == (ns > 1 ? 1 : 0)) fetch_epilogue();
-    cp_async_wait<kStages - 2>();
-    if (!mbar_wait_bounded(&full[i % kStages], uint32_t(i / kStages) & 1u, kFp8WaitNs))
-      atomicOr(&p.hdr->err, uint32_t(kErrRingWait));  // recorded; the CTA goes on without hanging
-    __syncthreads();  // stage i landed; stage i - 1 is no longer read
-    if (i + kStages - 1 < total) load(i + kStages - 1);
-    cp_async_commit();
-    const uint32_t ws = sbase + (i % kStages) * kUpStage, xs = ws + kWBytes;
+    const int slot = i % kStages;
+    if (!mbar_wait_bounded(&full[slot], uint32_t(i / kStages) & 1u, kFp8WaitNs))
+      atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
+    const uint32_t ws = sbase + slot * kStage, xs = ws + kWBytes;
     const uint32_t brow = xs + g * kAPitch + cq * 8;
 #pragma unroll
     for (int kq = 0; kq < kKB / 64; ++kq) {
@@ -330,52 +344,48 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
       mma_f16_16816(acc, a0, b00, b01);
       mma_f16_16816(acc, a1, b10, b11);
     }
-    if (ks == ns - 1) {  // the item's epilogue: the two halves of k added, then h'' by the k-half 0 warps
-      if (wk == 1) xchg[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      __syncthreads();
-      __half* hb = p.h + (size_t(dc.x - c0) * p.E + dc.y) * 2 * 8 * p.de;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[slot]);
+    if (ks == ns - 1) {  // the item's epilogue: the two halves of k added, then h'' by the k-half 0 warp
+      float4* xc = xchg[mc & 1];
+      if (wk == 1) xc[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      named_sync(1 + warp, 64);
       if (wk == 0) {
-        const float4 o = xchg[warp * 32 + lane];
-        acc[0] += o.x;
-        acc[1] += o.y;
-        acc[2] += o.z;
-        acc[3] += o.w;
-      }
+        const float4 o = xc[warp * 32 + lane];
+        const float sum[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};
+        __half* hb = p.h + (size_t(dc.x - c0) * p.E + dc.y) * 8 * p.de;
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        if (wk != 0) break;
-        const int h = v >> 1, t = 2 * cq + (v & 1);  // row g + 8 h, token t
-        const int j = dc.z * kRows + 16 * warp + g + 8 * h;
-        if (j >= p.de) continue;
-        const float uu = ep_s1[h] * acc[v];
-        const float r = (v & 1) ? ep_r[1] : ep_r[0];
-        const float hh = t < p.L ? ep_s2[h] * (r * (uu / (1.f + expf(-uu)))) : 0.f;
-        const __half hi = __float2half_rn(hh);
-        const __half lo = __float2half_rn(hh - __half2float(hi));
-        hb[size_t(t) * p.de + j] = hi;
-        hb[(8 + size_t(t)) * p.de + j] = lo;
+        for (int v = 0; v < 4; ++v) {
+          const int h = v >> 1, t = 2 * cq + (v & 1);  // row g + 8 h, token t
+          const int j = dc.z * kRows + 16 * warp + g + 8 * h;
+          if (j >= p.de) continue;
+          const float uu = ep_s1[h] * sum[v];
+          const float r = (v & 1) ? ep_r[1] : ep_r[0];
+          const float hh = t < p.L ? ep_s2[h] * (r * (uu / (1.f + expf(-uu)))) : 0.f;
+          hb[size_t(t) * p.de + j] = __float2half_rn(hh);
+        }
       }
       acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
     }
   }
-  cp_async_wait<0>();
 }
 
 // ------------------------------------------------------------------------------------ down-projection
 // Items of chunks [c0, c1): (chunk, 64-row block of d), output-stationary.  An item's stages run over the
-// chunk's active experts a and 256-wide blocks jk of de: 64 rows x 256 codes of W2 and the h hi and lo
-// planes (8 x 256 f16 each).  A chunk without active experts still takes one (empty) stage and writes
-// zeros.  The CTA's items are taken in groups of kItemTab: a group's per-item stage counts and layers go
-// to shared memory first; the expert of the stage after the one being loaded is fetched into a register
-// one stage early.  y[c][t][k] = t2 acc (one writer per element, a fixed order of terms).
+// chunk's active experts a and 256-wide blocks jk of de: 64 rows x 256 codes of W2 and the f16 h'' rows
+// (8 x 256).  A chunk without active experts still takes one (empty) stage and writes zeros.  The CTA's
+// items are taken in groups of kItemTab: a group's per-item stage counts and layers go to shared memory
+// first (the one CTA-wide barrier pair per group); the producer warp then walks the group's stages,
+// fetching the expert of the stage after the one it loads one stage early, while the consumers contract.
+// y[c][t][k] = t2 acc (one writer per element, a fixed order of terms).
 constexpr int kItemTab = 256;
 __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __grid_constant__ Maps mp, int c0, int c1) {
   extern __shared__ uint8_t smem_raw[];
   __shared__ int2 itab[kItemTab];  // per item of the group: {stages, layer (-1: none active)}
-  __shared__ float4 xchg[4 * 32];  // the k-half 1 warps' partial sums at an item's end
-  __shared__ __align__(8) uint64_t full[kStages];  // a stage's code boxes landed
-  const int tid = threadIdx.x, lane = tid & 31, g = lane >> 2, cq = lane & 3;
-  const int warp = (tid >> 5) & 3, wk = tid >> 7;  // row group, half of the stage's k
+  __shared__ float4 xchg[2][4 * 32];
+  __shared__ __align__(8) uint64_t full[kStages];
+  __shared__ __align__(8) uint64_t empty[kStages];
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int RB = (p.d + kRows - 1) / kRows, JK = (p.de + kKB - 1) / kKB;
   const int G = int(gridDim.x), b = int(blockIdx.x);
   const int n_items = (c1 - c0) * RB;
@@ -384,18 +394,23 @@ __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __gri
   uint8_t* const sgen = smem_raw + (sbase - smem_u32(smem_raw));
   if (tid == 0) {
     prefetch_tensormap(&mp.w2);
-    for (int q = 0; q < kStages; ++q) mbar_init(&full[q], 1);
+    for (int q = 0; q < kStages; ++q) {
+      mbar_init(&full[q], 1 + 32);
+      mbar_init(&empty[q], kCT / 32);
+    }
     fence_mbar_init();
   }
   __syncthreads();
+  const bool producer = wid == kCT / 32;
   const uint64_t pol = policy_evict_first();
   int base_use = 0;  // stages of earlier item groups: stage u of the CTA uses slot u % kStages, phase u / kStages
+  int items_done = 0;  // items finished by the consumers (the exchange buffer's parity)
   auto chunk_of = [&](int m) { return c0 + (b + m * G) / RB; };
   auto rb_of = [&](int m) { return (b + m * G) % RB; };
 
   for (int gb = 0; gb < mine; gb += kItemTab) {
     const int gn = min(kItemTab, mine - gb);
-    __syncthreads();  // the previous group's table and stages are no longer read
+    __syncthreads();  // the previous group's table is no longer read
     for (int k = tid; k < gn; k += kT) {
       const int c = chunk_of(gb + k), l = layer_of(p, c);
       const bool ok = l >= 0 && l < p.n_layers;
@@ -406,110 +421,105 @@ __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __gri
     int total = 0;
     for (int k = 0; k < gn; ++k) total += itab[k].x;
 
-    // the expert of stage s of group item k (0 when the item has no active expert)
-    auto expert_of = [&](int k, int s) -> int {
-      const int2 t = itab[k];
-      if (t.y < 0) return 0;
-      return t.y * p.E + p.active_idx[size_t(chunk_of(gb + k)) * p.E + s / JK];
-    };
-    // loader cursor: item k_l, stage s_l of it; e_l its expert, e_n the next stage's (in flight)
-    int k_l = 0, s_l = 0;
-    int e_l = expert_of(0, 0);
-    auto next_of = [&](int k, int s, int& kn, int& sn) {
-      if (s + 1 < itab[k].x) kn = k, sn = s + 1;
-      else kn = k + 1, sn = 0;
-    };
-    int k_n, s_n;
-    next_of(0, 0, k_n, s_n);
-    int e_n = k_n < gn ? expert_of(k_n, s_n) : 0;
-    auto load = [&](int slot) {
-      const int c = chunk_of(gb + k_l), rb = rb_of(gb + k_l);
-      const bool any = itab[k_l].y >= 0;
-      const int a = s_l / JK, j0 = (s_l - a * JK) * kKB;
-      const uint32_t st = sbase + slot * kDownStage;
-      if (tid == 0) {  // W2 codes: two boxes (an empty item's boxes come from expert 0 and meet zero h)
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&full[slot], kWBytes);
-        uint8_t* dst = sgen + slot * kDownStage;
-        tma_load_2d(dst, &mp.w2, j0, e_l * p.d + rb * kRows, &full[slot], pol);
-        tma_load_2d(dst + kWSub, &mp.w2, j0 + 128, e_l * p.d + rb * kRows, &full[slot], pol);
-      }
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {  // h'' hi and lo: 2 planes x 8 rows x 32 pieces
-        const int idx = tid + q * kT, plane = idx >> 8, t = (idx >> 5) & 7, ch = idx & 31;
-        const int j = j0 + ch * 8;
-        const bool ok = any && j < p.de;
-        const __half* src = ok ? p.h + (((size_t(c - c0) * p.E + a) * 2 + plane) * 8 + t) * p.de + j : p.h;
-        cp_async16(st + kWBytes + (plane * 8 + t) * kAPitch + ch * 16, src, ok ? 16 : 0);
-      }
-      // advance: the next stage's expert is in flight already; start fetching the one after it
-      k_l = k_n;
-      s_l = s_n;
-      e_l = e_n;
-      if (k_l < gn) {
-        next_of(k_l, s_l, k_n, s_n);
-        e_n = k_n < gn ? expert_of(k_n, s_n) : 0;
-      }
-    };
-
-#pragma unroll
-    for (int i = 0; i < kStages - 1; ++i) {
-      if (i < total) load((base_use + i) % kStages);
-      cp_async_commit();
-    }
-    int k_c = 0, s_c = 0;  // consumer cursor
-    float t2c = 0.f;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    for (int i = 0; i < total; ++i) {
-      if (s_c == 0) t2c = itab[k_c].y >= 0 ? p.t2[itab[k_c].y] : 0.f;  // used at the item's last stage
-      cp_async_wait<kStages - 2>();
-      if (!mbar_wait_bounded(&full[(base_use + i) % kStages], uint32_t((base_use + i) / kStages) & 1u, kFp8WaitNs))
-        atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
-      __syncthreads();
-      if (i + kStages - 1 < total) load((base_use + i + kStages - 1) % kStages);
-      cp_async_commit();
-      const uint32_t ws = sbase + ((base_use + i) % kStages) * kDownStage, hs = ws + kWBytes;
-      const uint32_t brow_hi = hs + g * kAPitch + cq * 8, brow_lo = brow_hi + 8 * kAPitch;
-      const bool work = itab[k_c].y >= 0;  // an empty item's stage is only waited for
-#pragma unroll
-      for (int kq = 0; kq < kKB / 64; ++kq) {
-        if (!work) break;
-        const int kb = wk * (kKB / 64) + kq;
-        uint32_t a0[4], a1[4];
-        load_a(ws, warp, lane, kb, a0, a1);
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "r"(brow_hi + kb * 64));
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h2), "=r"(h3) : "r"(brow_hi + kb * 64 + 32));
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(l0), "=r"(l1) : "r"(brow_lo + kb * 64));
-        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(l2), "=r"(l3) : "r"(brow_lo + kb * 64 + 32));
-        mma_f16_16816(acc, a0, h0, h1);
-        mma_f16_16816(acc, a0, l0, l1);
-        mma_f16_16816(acc, a1, h2, h3);
-        mma_f16_16816(acc, a1, l2, l3);
-      }
-      if (s_c + 1 == itab[k_c].x) {  // the item's last stage: the two halves of k added, then y rows
-        if (wk == 1) xchg[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-        __syncthreads();
-        const int c = chunk_of(gb + k_c), rb = rb_of(gb + k_c);
-        if (wk == 0) {
-          const float4 o = xchg[warp * 32 + lane];
-          const float sum[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const int k = rb * kRows + 16 * warp + g + (v >> 1) * 8, t = 2 * cq + (v & 1);
-            if (k < p.d && t < p.L) p.y[(size_t(c) * p.L + t) * p.d + k] = t2c * sum[v];
-          }
+    if (producer) {
+      // the expert of stage s of group item k (0 when the item has no active expert)
+      auto expert_of = [&](int k, int s) -> int {
+        const int2 t = itab[k];
+        if (t.y < 0) return 0;
+        return t.y * p.E + p.active_idx[size_t(chunk_of(gb + k)) * p.E + s / JK];
+      };
+      auto next_of = [&](int k, int s, int& kn, int& sn) {
+        if (s + 1 < itab[k].x) kn = k, sn = s + 1;
+        else kn = k + 1, sn = 0;
+      };
+      // cursor: item k_l, stage s_l of it; e_l its expert, e_n the next stage's (in flight)
+      int k_l = 0, s_l = 0, k_n, s_n;
+      int e_l = expert_of(0, 0);
+      next_of(0, 0, k_n, s_n);
+      int e_n = k_n < gn ? expert_of(k_n, s_n) : 0;
+      for (int i = 0; i < total; ++i) {
+        const int u = base_use + i, slot = u % kStages;
+        if (u >= kStages && !mbar_wait_bounded(&empty[slot], uint32_t(u / kStages - 1) & 1u, kFp8WaitNs))
+          atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
+        const int c = chunk_of(gb + k_l), rb = rb_of(gb + k_l);
+        const bool any = itab[k_l].y >= 0;
+        const int a = s_l / JK, j0 = (s_l - a * JK) * kKB;
+        if (lane == 0) {  // W2 codes: two boxes (an empty item's boxes come from expert 0 and meet zero h)
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&full[slot], kWBytes);
+          uint8_t* dst = sgen + slot * kStage;
+          tma_load_2d(dst, &mp.w2, j0, e_l * p.d + rb * kRows, &full[slot], pol);
+          tma_load_2d(dst + kWSub, &mp.w2, j0 + 128, e_l * p.d + rb * kRows, &full[slot], pol);
         }
-        acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-        ++k_c;
-        s_c = 0;
-      } else {
-        ++s_c;
+        const int j = j0 + lane * 8;  // h'' rows: 8 x this lane's 16-byte piece
+        const bool ok = any && j < p.de;
+        const __half* hsrc = p.h + (size_t(c - c0) * p.E + a) * 8 * p.de + j;
+        const uint32_t hs = sbase + slot * kStage + kWBytes + lane * 16;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) cp_async16(hs + t * kAPitch, ok ? hsrc + size_t(t) * p.de : p.h, ok ? 16 : 0);
+        cp_async_arrive_noinc(&full[slot]);
+        // advance: the next stage's expert is in flight already; start fetching the one after it
+        k_l = k_n;
+        s_l = s_n;
+        e_l = e_n;
+        if (k_l < gn) {
+          next_of(k_l, s_l, k_n, s_n);
+          e_n = k_n < gn ? expert_of(k_n, s_n) : 0;
+        }
+      }
+    } else {
+      const int g = lane >> 2, cq = lane & 3, warp = wid & 3, wk = wid >> 2;
+      int k_c = 0, s_c = 0;  // consumer cursor
+      float t2c = 0.f;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int i = 0; i < total; ++i) {
+        const int u = base_use + i, slot = u % kStages;
+        if (s_c == 0) t2c = itab[k_c].y >= 0 ? p.t2[itab[k_c].y] : 0.f;  // used at the item's last stage
+        if (!mbar_wait_bounded(&full[slot], uint32_t(u / kStages) & 1u, kFp8WaitNs))
+          atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
+        const uint32_t ws = sbase + slot * kStage, hs = ws + kWBytes;
+        const uint32_t brow = hs + g * kAPitch + cq * 8;
+        const bool work = itab[k_c].y >= 0;  // an empty item's stage is only waited for
+#pragma unroll
+        for (int kq = 0; kq < kKB / 64; ++kq) {
+          if (!work) break;
+          const int kb = wk * (kKB / 64) + kq;
+          uint32_t a0[4], a1[4];
+          load_a(ws, warp, lane, kb, a0, a1);
+          uint32_t h0, h1, h2, h3;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "r"(brow + kb * 64));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h2), "=r"(h3) : "r"(brow + kb * 64 + 32));
+          mma_f16_16816(acc, a0, h0, h1);
+          mma_f16_16816(acc, a1, h2, h3);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (s_c + 1 == itab[k_c].x) {  // the item's last stage: the two halves of k added, then y rows
+          float4* xc = xchg[items_done & 1];
+          if (wk == 1) xc[warp * 32 + lane] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+          named_sync(1 + warp, 64);
+          const int c = chunk_of(gb + k_c), rb = rb_of(gb + k_c);
+          if (wk == 0) {
+            const float4 o = xc[warp * 32 + lane];
+            const float sum[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int k = rb * kRows + 16 * warp + g + (v >> 1) * 8, t = 2 * cq + (v & 1);
+              if (k < p.d && t < p.L) p.y[(size_t(c) * p.L + t) * p.d + k] = t2c * sum[v];
+            }
+          }
+          acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+          ++items_done;
+          ++k_c;
+          s_c = 0;
+        } else {
+          ++s_c;
+        }
       }
     }
-    cp_async_wait<0>();
     base_use += total;
   }
+  if (producer) cp_async_wait_all();
 }
 
 }  // namespace
@@ -526,7 +536,7 @@ Fp8Layout layout(int C, int L, int d, int E, int de) {
   l.offs_off = l.bar_off + align256(size_t(C) * 4);
   l.xh_off = l.offs_off + align256(size_t(C + 1) * 4);
   l.h_off = l.xh_off + align256(size_t(C) * 8 * d * 2);
-  const size_t per_chunk = size_t(E) * 2 * 8 * de * 2;
+  const size_t per_chunk = size_t(E) * 8 * de * 2;  // f16 h'' rows of every active slot
   l.wave = int(std::max<size_t>(1, std::min<size_t>(size_t(C), kHBufBytes / per_chunk)));
   l.desc_off = l.h_off + align256(size_t(l.wave) * per_chunk);
   l.total = l.desc_off + align256(size_t(l.wave) * E * ((de + 63) / 64) * 16);
@@ -560,18 +570,17 @@ cudaError_t forward(const Fp8Params& p, const Maps& m, const batch::Params& rp, 
   }
   scan_items_kernel<<<1, 1024, 0, st>>>(p.n_active, p.C, p.JB, p.offs);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  if ((err = cudaFuncSetAttribute(up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpSmem)) != cudaSuccess)
+  if ((err = cudaFuncSetAttribute(up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem)) != cudaSuccess)
     return err;
-  if ((err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDownSmem)) !=
-      cudaSuccess)
+  if ((err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem)) != cudaSuccess)
     return err;
   const int grid = 2 * num_sms;
   const long long max_items = (long long)p.wave * p.E * p.JB;  // a wave's items when every expert is active
   for (int c0 = 0; c0 < p.C; c0 += p.wave) {
     const int c1 = std::min(p.C, c0 + p.wave);
     decode_items_kernel<<<unsigned((max_items + 255) / 256), 256, 0, st>>>(p, c0, c1, p.desc);
-    up_kernel<<<grid, kT, kUpSmem, st>>>(p, m, c0, c1, p.desc);
-    down_kernel<<<grid, kT, kDownSmem, st>>>(p, m, c0, c1);
+    up_kernel<<<grid, kT, kSmem, st>>>(p, m, c0, c1, p.desc);
+    down_kernel<<<grid, kT, kSmem, st>>>(p, m, c0, c1);
   }
   return cudaGetLastError();
 }
