@@ -161,11 +161,12 @@ __global__ void __launch_bounds__(256) prefill_fill_kernel(PrefillParams p) {
 namespace {
 
 // ---------------------------------------------------------------------------------- P4/P5 GEMMs
-constexpr int kGThreads = 192;   // warp 0: TMA producer, warp 1: MMA issuer (owns TMEM), warps 2-5: epilogue
-constexpr int kG1Threads = 320;  // GEMM1 adds warps 6-9: the gathered A rows, one token row per thread
+constexpr int kG1Threads = 320;  // GEMM1: warp 0 TMA producer, warp 1 MMA issuer (owns TMEM), warps 2-5
+                                 // epilogue, warps 6-9 the gathered A rows (one token row per thread)
+constexpr int kG2Threads = 320;  // GEMM2: warps 0, 1 as in GEMM1; warps 2-9 epilogue, two per lane quarter
 constexpr int kTileM = 128;
 constexpr int kPf1 = 12;  // GEMM1: W1 rows are prefetched into L2 this many stages ahead
-constexpr int kEpPitch = 36;  // GEMM2 epilogue block: 144-byte rows, so 8 lanes' 16-byte stores hit 32 banks
+constexpr int kEpBlock = 32 * 32;  // GEMM2 epilogue: a warp's 32 x 32 fp32 block, 16-byte pieces swizzled by row
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
@@ -184,14 +185,14 @@ struct GemmSmem {
   uint64_t* full;   // [S] operands of a stage landed
   uint64_t* empty;  // [S] MMAs of a stage done reading it
   uint64_t* accf;   // [2] accumulator buffer complete
-  uint64_t* acce;   // [2] accumulator buffer drained by the epilogue (4 warps)
+  uint64_t* acce;   // [2] accumulator buffer drained by the epilogue warps
   uint64_t* drain;  // every MMA of this CTA complete (before TMEM is freed)
   uint32_t* tmem_slot;
   volatile int* abort_flag;
   int* toff;        // [E+1] copies of the per-expert tile offsets, pair offsets and token counts
   int* off;         // [E+1]
   int* cnt;         // [E]
-  float* ep_buf;    // GEMM2: per epilogue warp a 32 x 32 fp32 block (row pitch kEpPitch)
+  float* ep_buf;    // GEMM2: per epilogue warp a 32 x 32 fp32 block (kEpBlock floats)
 };
 
 __device__ __forceinline__ GemmSmem carve(uint8_t* raw, int S, uint32_t stage_bytes, int E) {
@@ -289,7 +290,8 @@ __device__ __forceinline__ uint32_t tmem_cols(int n) {
   return c;
 }
 
-__device__ void gemm_setup(const PrefillParams& p, const GemmSmem& g, int S, int N, int full_count) {
+__device__ void gemm_setup(const PrefillParams& p, const GemmSmem& g, int S, int N, int full_count,
+                           int epilogue_warps) {
   const int tid = threadIdx.x, warp = tid >> 5;
   for (int i = tid; i <= p.E; i += blockDim.x) {  // the tables every tile lookup reads
     g.toff[i] = p.toff[i];
@@ -303,7 +305,7 @@ __device__ void gemm_setup(const PrefillParams& p, const GemmSmem& g, int S, int
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&g.accf[b], 1);
-      mbar_init(&g.acce[b], 4);
+      mbar_init(&g.acce[b], epilogue_warps);
     }
     mbar_init(g.drain, 1);
     *g.abort_flag = 0;
@@ -345,7 +347,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
   const GemmSmem g = carve(smem_raw, S, stage_bytes, p.E);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) prefetch_tensormap(&m.w1);
-  gemm_setup(p, g, S, N, 1 + kTileM);  // the W1 box (expect_tx) and one row-copy arrival per A row
+  gemm_setup(p, g, S, N, 1 + kTileM, 4);  // the W1 box (expect_tx) and one row-copy arrival per A row
   const uint32_t tmem = *g.tmem_slot;
   const int T = g.toff[p.E];
   const int KB = p.d / 64;
@@ -484,7 +486,7 @@ __global__ void __launch_bounds__(kG1Threads, 1)
 
 // GEMM2: per tile of 128 pairs of expert e and N2 columns of d, Y = H_hi W2_e^T + H_lo W2_e^T, added
 // into y[token] with vector reductions (every pair's row goes to its token's row).
-__global__ void __launch_bounds__(kGThreads, 1)
+__global__ void __launch_bounds__(kG2Threads, 1)
     prefill_gemm2_kernel(const __grid_constant__ PrefillParams p, const __grid_constant__ PrefillMaps m) {
   extern __shared__ uint8_t smem_raw[];
   const int N = p.N2, S = p.S2;
@@ -495,7 +497,7 @@ __global__ void __launch_bounds__(kGThreads, 1)
     prefetch_tensormap(&m.h);
     prefetch_tensormap(&m.w2);
   }
-  gemm_setup(p, g, S, N, 1);
+  gemm_setup(p, g, S, N, 1, 8);
   const uint32_t tmem = *g.tmem_slot;
   const int NT = p.d / N;
   const int T = g.toff[p.E] * NT;
@@ -553,12 +555,16 @@ __global__ void __launch_bounds__(kGThreads, 1)
       __syncwarp();
     }
   } else {
-    // Each 32-row x 32-column block leaves tensor memory one row per lane, goes through this warp's
-    // shared block, and is added into y by rows: 8 lanes cover one row's 128 bytes, so a reduction
-    // instruction writes 4 whole lines of y instead of 32 pieces of 32 different lines.
-    const int q = warp & 3;
+    // Two warps per lane quarter q, each over half of the tile's columns.  Each 32-row x 32-column block
+    // leaves tensor memory one row per lane, goes through this warp's shared block, and is added into y
+    // by rows: 8 lanes cover one row's 128 bytes, so a reduction instruction writes 4 whole lines of y
+    // instead of 32 pieces of 32 different lines.  The block's 16-byte pieces are swizzled by row (piece
+    // c of row r at c ^ (r & 7)), so both the row-per-lane writes and the 8-lanes-per-row reads are free
+    // of bank conflicts.
+    const int q = warp & 3, half = (warp - 2) >> 2;
     const uint64_t pol_y = policy_evict_last();
-    float* blk = g.ep_buf + q * 32 * kEpPitch;
+    float* blk = g.ep_buf + (warp - 2) * kEpBlock;
+    float4* mine = reinterpret_cast<float4*>(blk + lane * 32);
     int tcount = 0;
     for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++tcount) {
       const int ab = tcount & 1;
@@ -569,18 +575,18 @@ __global__ void __launch_bounds__(kGThreads, 1)
       const int row = q * 32 + lane;
       const int tok = m0 + row < ne ? p.tok[g.off[e] + m0 + row] : -1;  // this lane's row's token
       float* ycols = p.y + size_t(jn) * N + (lane & 7) * 4;
-      for (int c0 = 0; c0 < N; c0 += 32) {
+      for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
         float v[32];
         tc::ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * N + c0), v);
-        float4* mine = reinterpret_cast<float4*>(blk + lane * kEpPitch);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) mine[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        for (int k = 0; k < 8; ++k)
+          mine[k ^ (lane & 7)] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
         __syncwarp();
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const int r = 4 * i + (lane >> 3);
           const int tok_r = __shfl_sync(0xffffffffu, tok, r);
-          const float4 a = *reinterpret_cast<const float4*>(blk + r * kEpPitch + (lane & 7) * 4);
+          const float4 a = reinterpret_cast<const float4*>(blk + r * 32)[(lane & 7) ^ (r & 7)];
           if (tok_r >= 0) red_add_v4(ycols + size_t(tok_r) * p.d + c0, a.x, a.y, a.z, a.w, pol_y);
         }
         __syncwarp();  // the block is read before the next one overwrites it
@@ -604,7 +610,7 @@ bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, Prefil
   p->N2 = d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
   // alignment slack, barriers, tensor-memory slot, abort flag, the three per-expert tables
   const size_t fixed = 1024 + 256 + (3 * size_t(E) + 2) * 4;
-  const size_t fixed2 = fixed + 16 + 4 * 32 * kEpPitch * sizeof(float);  // + the epilogue blocks
+  const size_t fixed2 = fixed + 16 + 8 * kEpBlock * sizeof(float);  // + the eight epilogue blocks
   const size_t st1 = size_t(kTileM) * 128 + size_t(p->N1) * 128;
   const size_t st2 = 2 * size_t(kTileM) * 128 + size_t(p->N2) * 128;
   p->S1 = int((size_t(max_smem) - fixed) / st1);
@@ -638,7 +644,7 @@ cudaError_t prefill_launch(const PrefillParams& p, const PrefillMaps& m, const P
                                   int(pl.smem2))) != cudaSuccess)
     return err;
   prefill_gemm1_kernel<<<pl.grid, kG1Threads, pl.smem1, st>>>(p, m);
-  prefill_gemm2_kernel<<<pl.grid, kGThreads, pl.smem2, st>>>(p, m);
+  prefill_gemm2_kernel<<<pl.grid, kG2Threads, pl.smem2, st>>>(p, m);
   return cudaGetLastError();
 }
 
