@@ -20,8 +20,9 @@
 // turns each pair into its exact f16 values, and mma.sync f16 (fp32 accumulate) contracts them with the
 // activations in f16, read in the same order of k (a thread's pair of A slots 2c, 2c+1 holds codes 4c,
 // 4c+1 and slots 2c+8, 2c+9 codes 4c+2, 4c+3, so its B fragment is the activations at 4c .. 4c+3).  The
-// activations are x (bf16 values, exact in f16 in the normal range) and h'' rounded once to f16 (a
-// relative 2^-11 per element, the one rounding the fp8 path adds beyond fp32 accumulation).
+// activations are x (bf16 values, exact in f16 in the normal range) and h'' as an f16 hi + lo pair (h''
+// rounded once to f16 would leave y about 3e-4 rms(y) off per element, up to 0.75 of the tolerance's
+// 1e-3 rms(y) floor on the decode layer: too little margin).
 // Every sum runs in a fixed order: y is bit-reproducible.
 #include <algorithm>
 #include <cuda_fp16.h>
@@ -41,9 +42,11 @@ constexpr int kWSub = kRows * 128;  // one tensor box: 64 rows x 128 codes, 128-
 constexpr int kWBytes = 2 * kWSub;  // a stage's codes: two boxes side by side along k
 constexpr int kAPitch = 2 * kKB + 32;  // 544 B rows of 256 f16 activations: conflict-free 8-byte loads
 constexpr int kStages = 4;
-constexpr int kXBytes = 8 * kAPitch;                                // 4352 (8 token rows)
-constexpr int kStage = (kWBytes + kXBytes + 1023) / 1024 * 1024;  // 21504: boxes stay 1024-aligned
-constexpr int kSmem = kStages * kStage + 1024;                    // + alignment slack
+constexpr int kXBytes = 8 * kAPitch;                                      // 4352 (8 token rows)
+constexpr int kUpStage = (kWBytes + kXBytes + 1023) / 1024 * 1024;       // 21504: boxes stay 1024-aligned
+constexpr int kDownStage = (kWBytes + 2 * kXBytes + 1023) / 1024 * 1024;  // 25600 (h'' hi and lo planes)
+constexpr int kUpSmem = kStages * kUpStage + 1024;                       // + alignment slack
+constexpr int kDownSmem = kStages * kDownStage + 1024;
 constexpr uint64_t kFp8WaitNs = 2000000000ull;
 
 __device__ __forceinline__ int layer_of(const Fp8Params& p, int c) { return p.layer ? p.layer[c] : c % p.n_layers; }
@@ -247,7 +250,8 @@ __global__ void __launch_bounds__(256) decode_items_kernel(const Fp8Params p, in
 // (empty[s]), then issues the slot's two code boxes (TMA, transaction bytes on full[s]) and the x rows
 // (cp.async, one arrival per lane on full[s] once its copies land).  The consumers wait on full[s] only,
 // so no CTA-wide barrier sits between stages.  At an item's end the two k-halves of a row group meet at a
-// barrier of their own; the epilogue writes h'' = s2 r Swish(s1 u) as f16 into h[chunk - c0][a][t][j].
+// barrier of their own; the epilogue writes h'' = s2 r Swish(s1 u) as f16 hi + lo into
+// h[chunk - c0][a][plane][t][j].
 __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_constant__ Maps mp, int c0, int c1,
                                                const int4* __restrict__ desc) {
   extern __shared__ uint8_t smem_raw[];
@@ -293,13 +297,13 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
                         // stored; columns past d and rows past the last expert read as zeros)
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&full[slot], kWBytes);
-        uint8_t* dst = sgen + slot * kStage;
+        uint8_t* dst = sgen + slot * kUpStage;
         tma_load_2d(dst, &mp.w1, k0, dl.w * p.de + dl.z * kRows, &full[slot], pol);
         tma_load_2d(dst + kWSub, &mp.w1, k0 + 128, dl.w * p.de + dl.z * kRows, &full[slot], pol);
       }
       const int k = k0 + lane * 8;  // x in f16: 8 rows, this lane's 16-byte piece of each
       const bool ok = k < p.d;
-      const uint32_t xs = sbase + slot * kStage + kWBytes + lane * 16;
+      const uint32_t xs = sbase + slot * kUpStage + kWBytes + lane * 16;
 #pragma unroll
       for (int t = 0; t < 8; ++t)
         cp_async16(xs + t * kAPitch, ok ? p.xh + (size_t(dl.x) * 8 + t) * p.d + k : p.xh, ok ? 16 : 0);
@@ -331,7 +335,7 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
     const int slot = i % kStages;
     if (!mbar_wait_bounded(&full[slot], uint32_t(i / kStages) & 1u, kFp8WaitNs))
       atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
-    const uint32_t ws = sbase + slot * kStage, xs = ws + kWBytes;
+    const uint32_t ws = sbase + slot * kUpStage, xs = ws + kWBytes;
     const uint32_t brow = xs + g * kAPitch + cq * 8;
 #pragma unroll
     for (int kq = 0; kq < kKB / 64; ++kq) {
@@ -353,7 +357,7 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
       if (wk == 0) {
         const float4 o = xc[warp * 32 + lane];
         const float sum[4] = {acc[0] + o.x, acc[1] + o.y, acc[2] + o.z, acc[3] + o.w};
-        __half* hb = p.h + (size_t(dc.x - c0) * p.E + dc.y) * 8 * p.de;
+        __half* hb = p.h + (size_t(dc.x - c0) * p.E + dc.y) * 2 * 8 * p.de;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const int h = v >> 1, t = 2 * cq + (v & 1);  // row g + 8 h, token t
@@ -362,7 +366,9 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
           const float uu = ep_s1[h] * sum[v];
           const float r = (v & 1) ? ep_r[1] : ep_r[0];
           const float hh = t < p.L ? ep_s2[h] * (r * (uu / (1.f + expf(-uu)))) : 0.f;
-          hb[size_t(t) * p.de + j] = __float2half_rn(hh);
+          const __half hi = __float2half_rn(hh);
+          hb[size_t(t) * p.de + j] = hi;
+          hb[(8 + size_t(t)) * p.de + j] = __float2half_rn(hh - __half2float(hi));
         }
       }
       acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -372,8 +378,8 @@ __global__ void __launch_bounds__(kT) up_kernel(const Fp8Params p, const __grid_
 
 // ------------------------------------------------------------------------------------ down-projection
 // Items of chunks [c0, c1): (chunk, 64-row block of d), output-stationary.  An item's stages run over the
-// chunk's active experts a and 256-wide blocks jk of de: 64 rows x 256 codes of W2 and the f16 h'' rows
-// (8 x 256).  A chunk without active experts still takes one (empty) stage and writes zeros.  The CTA's
+// chunk's active experts a and 256-wide blocks jk of de: 64 rows x 256 codes of W2 and the h'' hi and lo
+// planes (8 x 256 f16 each).  A chunk without active experts still takes one (empty) stage and writes zeros.  The CTA's
 // items are taken in groups of kItemTab: a group's per-item stage counts and layers go to shared memory
 // first (the one CTA-wide barrier pair per group); the producer warp then walks the group's stages,
 // fetching the expert of the stage after the one it loads one stage early, while the consumers contract.
@@ -447,16 +453,16 @@ __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __gri
         if (lane == 0) {  // W2 codes: two boxes (an empty item's boxes come from expert 0 and meet zero h)
           fence_proxy_async_smem();
           mbar_arrive_expect_tx(&full[slot], kWBytes);
-          uint8_t* dst = sgen + slot * kStage;
+          uint8_t* dst = sgen + slot * kDownStage;
           tma_load_2d(dst, &mp.w2, j0, e_l * p.d + rb * kRows, &full[slot], pol);
           tma_load_2d(dst + kWSub, &mp.w2, j0 + 128, e_l * p.d + rb * kRows, &full[slot], pol);
         }
-        const int j = j0 + lane * 8;  // h'' rows: 8 x this lane's 16-byte piece
+        const int j = j0 + lane * 8;  // h'' hi and lo planes: 16 rows x this lane's 16-byte piece
         const bool ok = any && j < p.de;
-        const __half* hsrc = p.h + (size_t(c - c0) * p.E + a) * 8 * p.de + j;
-        const uint32_t hs = sbase + slot * kStage + kWBytes + lane * 16;
+        const __half* hsrc = p.h + (size_t(c - c0) * p.E + a) * 2 * 8 * p.de + j;
+        const uint32_t hs = sbase + slot * kDownStage + kWBytes + lane * 16;
 #pragma unroll
-        for (int t = 0; t < 8; ++t) cp_async16(hs + t * kAPitch, ok ? hsrc + size_t(t) * p.de : p.h, ok ? 16 : 0);
+        for (int t = 0; t < 16; ++t) cp_async16(hs + t * kAPitch, ok ? hsrc + size_t(t) * p.de : p.h, ok ? 16 : 0);
         cp_async_arrive_noinc(&full[slot]);
         // advance: the next stage's expert is in flight already; start fetching the one after it
         k_l = k_n;
@@ -477,8 +483,8 @@ __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __gri
         if (s_c == 0) t2c = itab[k_c].y >= 0 ? p.t2[itab[k_c].y] : 0.f;  // used at the item's last stage
         if (!mbar_wait_bounded(&full[slot], uint32_t(u / kStages) & 1u, kFp8WaitNs))
           atomicOr(&p.hdr->err, uint32_t(kErrRingWait));
-        const uint32_t ws = sbase + slot * kStage, hs = ws + kWBytes;
-        const uint32_t brow = hs + g * kAPitch + cq * 8;
+        const uint32_t ws = sbase + slot * kDownStage, hs = ws + kWBytes;
+        const uint32_t brow_hi = hs + g * kAPitch + cq * 8, brow_lo = brow_hi + 8 * kAPitch;
         const bool work = itab[k_c].y >= 0;  // an empty item's stage is only waited for
 #pragma unroll
         for (int kq = 0; kq < kKB / 64; ++kq) {
@@ -486,11 +492,15 @@ __global__ void __launch_bounds__(kT) down_kernel(const Fp8Params p, const __gri
           const int kb = wk * (kKB / 64) + kq;
           uint32_t a0[4], a1[4];
           load_a(ws, warp, lane, kb, a0, a1);
-          uint32_t h0, h1, h2, h3;
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "r"(brow + kb * 64));
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h2), "=r"(h3) : "r"(brow + kb * 64 + 32));
+          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h0), "=r"(h1) : "r"(brow_hi + kb * 64));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(h2), "=r"(h3) : "r"(brow_hi + kb * 64 + 32));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(l0), "=r"(l1) : "r"(brow_lo + kb * 64));
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(l2), "=r"(l3) : "r"(brow_lo + kb * 64 + 32));
           mma_f16_16816(acc, a0, h0, h1);
+          mma_f16_16816(acc, a0, l0, l1);
           mma_f16_16816(acc, a1, h2, h3);
+          mma_f16_16816(acc, a1, l2, l3);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[slot]);
@@ -536,7 +546,7 @@ Fp8Layout layout(int C, int L, int d, int E, int de) {
   l.offs_off = l.bar_off + align256(size_t(C) * 4);
   l.xh_off = l.offs_off + align256(size_t(C + 1) * 4);
   l.h_off = l.xh_off + align256(size_t(C) * 8 * d * 2);
-  const size_t per_chunk = size_t(E) * 8 * de * 2;  // f16 h'' rows of every active slot
+  const size_t per_chunk = size_t(E) * 2 * 8 * de * 2;  // f16 h'' hi and lo rows of every active slot
   l.wave = int(std::max<size_t>(1, std::min<size_t>(size_t(C), kHBufBytes / per_chunk)));
   l.desc_off = l.h_off + align256(size_t(l.wave) * per_chunk);
   l.total = l.desc_off + align256(size_t(l.wave) * E * ((de + 63) / 64) * 16);
@@ -570,17 +580,18 @@ cudaError_t forward(const Fp8Params& p, const Maps& m, const batch::Params& rp, 
   }
   scan_items_kernel<<<1, 1024, 0, st>>>(p.n_active, p.C, p.JB, p.offs);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
-  if ((err = cudaFuncSetAttribute(up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem)) != cudaSuccess)
+  if ((err = cudaFuncSetAttribute(up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kUpSmem)) != cudaSuccess)
     return err;
-  if ((err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem)) != cudaSuccess)
+  if ((err = cudaFuncSetAttribute(down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kDownSmem)) !=
+      cudaSuccess)
     return err;
   const int grid = 2 * num_sms;
   const long long max_items = (long long)p.wave * p.E * p.JB;  // a wave's items when every expert is active
   for (int c0 = 0; c0 < p.C; c0 += p.wave) {
     const int c1 = std::min(p.C, c0 + p.wave);
     decode_items_kernel<<<unsigned((max_items + 255) / 256), 256, 0, st>>>(p, c0, c1, p.desc);
-    up_kernel<<<grid, kT, kSmem, st>>>(p, m, c0, c1, p.desc);
-    down_kernel<<<grid, kT, kSmem, st>>>(p, m, c0, c1);
+    up_kernel<<<grid, kT, kUpSmem, st>>>(p, m, c0, c1, p.desc);
+    down_kernel<<<grid, kT, kDownSmem, st>>>(p, m, c0, c1);
   }
   return cudaGetLastError();
 }
