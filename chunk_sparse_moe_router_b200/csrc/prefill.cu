@@ -163,7 +163,8 @@ namespace {
 // ---------------------------------------------------------------------------------- P4/P5 GEMMs
 constexpr int kG1Threads = 320;  // GEMM1: warp 0 TMA producer, warp 1 MMA issuer (owns TMEM), warps 2-5
                                  // epilogue, warps 6-9 the gathered A rows (one token row per thread)
-constexpr int kG2Threads = 320;  // GEMM2: warps 0, 1 as in GEMM1; warps 2-9 epilogue, two per lane quarter
+constexpr int kG2EpWarps = 8;    // GEMM2 epilogue warps: a multiple of 4 (each lane quarter gets kG2EpWarps / 4)
+constexpr int kG2Threads = 64 + 32 * kG2EpWarps;  // GEMM2: warps 0, 1 as in GEMM1, then the epilogue
 constexpr int kTileM = 128;
 constexpr int kPf1 = 12;  // GEMM1: W1 rows are prefetched into L2 this many stages ahead
 constexpr int kEpBlock = 32 * 32;  // GEMM2 epilogue: a warp's 32 x 32 fp32 block, 16-byte pieces swizzled by row
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
     prefetch_tensormap(&m.h);
     prefetch_tensormap(&m.w2);
   }
-  gemm_setup(p, g, S, N, 1, 8);
+  gemm_setup(p, g, S, N, 1, kG2EpWarps);
   const uint32_t tmem = *g.tmem_slot;
   const int NT = p.d / N;
   const int T = g.toff[p.E] * NT;
@@ -555,13 +556,13 @@ __global__ void __launch_bounds__(kG2Threads, 1)
       __syncwarp();
     }
   } else {
-    // Two warps per lane quarter q, each over half of the tile's columns.  Each 32-row x 32-column block
+    // kG2EpWarps / 4 warps per lane quarter q, taking the tile's 32-column blocks in turn.  Each block
     // leaves tensor memory one row per lane, goes through this warp's shared block, and is added into y
     // by rows: 8 lanes cover one row's 128 bytes, so a reduction instruction writes 4 whole lines of y
     // instead of 32 pieces of 32 different lines.  The block's 16-byte pieces are swizzled by row (piece
     // c of row r at c ^ (r & 7)), so both the row-per-lane writes and the 8-lanes-per-row reads are free
     // of bank conflicts.
-    const int q = warp & 3, half = (warp - 2) >> 2;
+    const int q = warp & 3, set = (warp - 2) >> 2, nsets = kG2EpWarps / 4;
     const uint64_t pol_y = policy_evict_last();
     float* blk = g.ep_buf + (warp - 2) * kEpBlock;
     float4* mine = reinterpret_cast<float4*>(blk + lane * 32);
@@ -575,7 +576,7 @@ __global__ void __launch_bounds__(kG2Threads, 1)
       const int row = q * 32 + lane;
       const int tok = m0 + row < ne ? p.tok[g.off[e] + m0 + row] : -1;  // this lane's row's token
       float* ycols = p.y + size_t(jn) * N + (lane & 7) * 4;
-      for (int c0 = half * (N / 2); c0 < (half + 1) * (N / 2); c0 += 32) {
+      for (int c0 = 32 * set; c0 < N; c0 += 32 * nsets) {
         float v[32];
         tc::ld_32x32b_x32(tmem + (uint32_t(q * 32) << 16) + uint32_t(ab * N + c0), v);
 #pragma unroll
@@ -610,7 +611,7 @@ bool prefill_plan(int L, int d, int E, int de, int num_sms, int max_smem, Prefil
   p->N2 = d % 256 == 0 ? 256 : d % 128 == 0 ? 128 : 64;
   // alignment slack, barriers, tensor-memory slot, abort flag, the three per-expert tables
   const size_t fixed = 1024 + 256 + (3 * size_t(E) + 2) * 4;
-  const size_t fixed2 = fixed + 16 + 8 * kEpBlock * sizeof(float);  // + the eight epilogue blocks
+  const size_t fixed2 = fixed + 16 + kG2EpWarps * kEpBlock * sizeof(float);  // + the epilogue blocks
   const size_t st1 = size_t(kTileM) * 128 + size_t(p->N1) * 128;
   const size_t st2 = 2 * size_t(kTileM) * 128 + size_t(p->N2) * 128;
   p->S1 = int((size_t(max_smem) - fixed) / st1);
