@@ -835,9 +835,10 @@ def run_fp8(args):
 def run_backward(args):
     """The layer's backward (blockffn_layer_backward) for --chunks chunks of 8 tokens (default 512: 4096
     tokens) at the decode layer's shape (d = 2048, E = 64, de = 256) with a random upstream gradient.
-    Roofline: the dense contraction flops of the step (5 products of 2 T d E de: U, Q, dW2, dW1, dX; the
-    router's are 4 T d E) over its CUDA-event time, against the measured bf16 tensor peak; the MMAs
-    issued are about twice that (fp32 operands as bf16 hi + lo pairs)."""
+    Roofline: the contraction flops of the step over the P active (token, expert) pairs (5 products of
+    2 P d de: U, Q, dW2, dW1, dX; the router's are 4 T d E) over its CUDA-event time, against the measured
+    bf16 tensor peak; the MMAs issued are about twice that (fp32 operands as bf16 hi + lo pairs).  P is
+    counted on the host from the same inputs (every pre-activation keeps a margin from zero)."""
     import numpy as np
     import torch
 
@@ -880,20 +881,24 @@ def run_backward(args):
             e1.synchronize()
         del graph
     ms = e0.elapsed_time(e1) / args.steps
-    flops = 5 * 2.0 * T * d * E * de + 4.0 * T * d * E
+    s_host = gen.bf16_bits_to_f32(x_np).astype(np.float64) @ lay.Wr.astype(np.float64) + lay.br
+    P = int((s_host > 0).sum())
+    flops = 5 * 2.0 * P * d * de + 4.0 * T * d * E
     peak, peak_kind = measured_peaks("bf16_tflops")
     tf = flops / (ms * 1e-3) / 1e12
-    line = {"metric": "BlockFFN layer backward tokens/s and achieved TFLOP/s (dense over experts)",
+    line = {"metric": "BlockFFN layer backward tokens/s and achieved TFLOP/s (over the active pairs)",
             "value": round(T / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16 x and weights; fp32 dy and gradients (hi + lo bf16 pairs on warp MMAs)",
             "data": "synthetic",
-            "config": {"workload": f"backward_T{T}_d{d}_E{E}_de{de}", "tokens": T,
-                       "l2": "inputs larger than L2 (U, Q and the pairs: 1.1 GB of intermediates per step)"},
+            "config": {"workload": f"backward_T{T}_d{d}_E{E}_de{de}", "tokens": T, "active_pairs": P,
+                       "tls": round(1.0 - P / (T * E), 4),
+                       "l2": "inputs larger than L2 (x, dy, the weights and the pair rows: about "
+                             f"{(T * d * 6 + E * d * de * 4 + P * (de * 16 + d * 4)) / 1e9:.2f} GB per step)"},
             "roofline": {"bound": "tensor", "achieved": round(tf, 1), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(tf / peak, 4), "peak_kind": peak_kind, "traffic": None,
                          "flops_per_step": flops},
-            "gpu_launches": 14 * args.steps, "clocks": clocks.summary()}
+            "gpu_launches": 18 * args.steps, "clocks": clocks.summary()}
     if not args.no_cpu_baseline:
         import oracle
         w = lambda b: gen.bf16_bits_to_f32(b).astype(np.float64)

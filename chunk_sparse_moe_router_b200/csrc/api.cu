@@ -697,7 +697,7 @@ int blockffn_chunk_forward_batch_fp8(const void* x, int C, int L, int d, const i
 }
 
 size_t blockffn_layer_backward_workspace_size(int T, int d, int E, int de) {
-  if (T < 1 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
+  if (T < 1 || T > 65535 * 128 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
       1ll * T * E * de >= (1ll << 31) || 1ll * T * d >= (1ll << 31))
     return 0;
   DeviceInfo di;
@@ -710,7 +710,7 @@ int blockffn_layer_backward(const void* x, int T, int d, const float* Wr, const 
                             const void* W1, const void* W2, int E, int de, const float* dy, float* dx, float* dWr,
                             float* db, float* dg, float* dW1, float* dW2, void* workspace, size_t workspace_bytes,
                             void* stream) {
-  if (T < 1 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
+  if (T < 1 || T > 65535 * 128 || d < 8 || d % 8 != 0 || de < 8 || de % 8 != 0 || E < 1 || E > kMaxE ||
       1ll * T * E * de >= (1ll << 31) || 1ll * T * d >= (1ll << 31))
     return BFFN_EINVAL;
   const void* bulk[] = {x, W1, W2};

@@ -442,7 +442,7 @@ cudaError_t forward(const Fp8Params& p, const Maps& m, const batch::Params& rp, 
 // ---------------------------------------------------------------- layer backward (layer_backward.cu)
 namespace bwd {
 struct Layout {  // byte offsets into the workspace
-  size_t wsplit, sparts, s, r, rho, dyhl, U, Q, rhhl, duhl, dr, ds, dgc, dshl, total;
+  size_t wsplit, sparts, s, r, rho, dyhl, U, Q, rhhl, duhl, dr, ds, dgc, dshl, cnt, goff, tok, pexp, pidx, xp, total;
   int parts;
 };
 Layout layout(int T, int d, int E, int de, int num_sms);

@@ -199,12 +199,16 @@ BFFN_API int blockffn_union_overlap(const int32_t* active_idx_a, const int32_t* 
  *   dx fp32 [T, d], dWr fp32 [d, E], db fp32 [E], dg fp32 [E], dW1 fp32 [E, de, d], dW2 fp32 [E, d, de]
  * are written (overwritten), with Wr fp32 [d, E], br fp32 [E] or NULL, g fp32 [E], W1 bf16 [E, de, d],
  * W2 bf16 [E, d, de] as in the forward.  A token whose router outputs are all zero has r = 0 and passes no
- * gradient to the router.  The experts are evaluated densely (an inactive expert's terms are exact zeros
- * through r = 0); every contraction runs on the warp tensor cores, fp32 operands carried as bf16 hi + lo
- * pairs, with fp32 accumulation in a fixed order (bit-identical reruns).
+ * gradient to the router.  Only the (token, expert) pairs whose router pre-activation is positive are
+ * evaluated (every other pair's terms are exact zeros through a = 0 and r = 0): they are grouped by expert
+ * on the device and every expert contraction runs over its own pairs; every contraction runs on the warp
+ * tensor cores, fp32 operands carried as bf16 hi + lo pairs, with fp32 accumulation in a fixed order
+ * (bit-identical reruns).
  * workspace: device memory of at least blockffn_layer_backward_workspace_size(T, d, E, de) bytes, 256-byte
- * aligned (about 12 T E de bytes; its contents need not be initialised).
- * Requirements (BFFN_EINVAL otherwise): T >= 1, d and de multiples of 8, 1 <= E <= 1024, T E de < 2^31;
+ * aligned (about 12 T E de + 4 T E d bytes, sized for every pair active; its contents need not be
+ * initialised).
+ * Requirements (BFFN_EINVAL otherwise): T >= 1, T <= 8 388 480, d and de multiples of 8, 1 <= E <= 1024,
+ * T E de < 2^31, T d < 2^31;
  * x, W1, W2, dy 16-byte aligned, the rest 4-byte aligned, non-NULL except br.  A smaller workspace returns
  * BFFN_ENOMEM, a failed launch BFFN_ECUDA.
  */

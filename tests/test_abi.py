@@ -233,9 +233,9 @@ def test_batch_fp8_workspace_size(bffn):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(T=0), dict(d=12), dict(de=4), dict(E=0), dict(E=1025), dict(x=None), dict(x=FAKE + 8), dict(W1=FAKE + 2),
-    dict(dy=FAKE + 4), dict(dx=None), dict(dW2=FAKE + 2), dict(br=FAKE + 1), dict(workspace=None),
-    dict(workspace=FAKE + 16),
+    dict(T=0), dict(T=65535 * 128 + 1, d=8, E=1, de=8), dict(d=12), dict(de=4), dict(E=0), dict(E=1025),
+    dict(x=None), dict(x=FAKE + 8), dict(W1=FAKE + 2), dict(dy=FAKE + 4), dict(dx=None), dict(dW2=FAKE + 2),
+    dict(br=FAKE + 1), dict(workspace=None), dict(workspace=FAKE + 16),
 ])
 def test_layer_backward_validates(bffn, kw):
     a = dict(x=FAKE, T=64, d=256, Wr=FAKE, br=None, g=FAKE, W1=FAKE, W2=FAKE, E=16, de=64, dy=FAKE, dx=FAKE,
@@ -247,6 +247,9 @@ def test_layer_backward_validates(bffn, kw):
 
 
 def test_layer_backward_workspace_size(bffn):
-    assert bffn.blockffn_layer_backward_workspace_size(4096, 2048, 64, 256) > 4096 * 64 * 256 * 12
+    # sized for every pair active: the pair rows of U, Q, RH, DU and the per-pair dx terms
+    assert bffn.blockffn_layer_backward_workspace_size(4096, 2048, 64, 256) > 4096 * 64 * (256 * 12 + 2048 * 4)
+    assert bffn.blockffn_layer_backward_workspace_size(65535 * 128, 8, 1, 8) > 0
+    assert bffn.blockffn_layer_backward_workspace_size(65535 * 128 + 1, 8, 1, 8) == 0
     for bad in [(0, 256, 16, 64), (64, 250, 16, 64), (64, 256, 0, 64), (64, 256, 16, 60)]:
         assert bffn.blockffn_layer_backward_workspace_size(*bad) == 0

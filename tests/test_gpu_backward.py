@@ -76,3 +76,17 @@ def test_layer_backward_silent_token_and_reruns(bffn, cuda_device):
     for k in a:
         assert np.array_equal(a[k], b[k])
     _compare(a, _ref(lay, x, dy))
+
+
+def test_layer_backward_expert_never_and_always_active(bffn, cuda_device):
+    """An expert no token activates (its gradients are exact zeros: no pairs) and one every token activates
+    (its pairs span the whole token range)."""
+    base = gen.make_layer(9, 128, 16, 32, beta=0.84, var_x=1.09)
+    br = base.br.copy()
+    br[0], br[1] = -50.0, 50.0
+    lay, x, dy = _case(9, 96, 128, 16, 32, br=br)
+    got = _run(bffn, lay, x, dy)
+    for k in ("dW1", "dW2"):
+        assert np.all(got[k][0] == 0.0)
+    assert got["db"][0] == 0.0 and got["dg"][0] == 0.0
+    _compare(got, _ref(lay, x, dy))
