@@ -120,3 +120,52 @@ def test_planted_backward_mistake_is_caught(mutation):
     finally:
         oracle.set_mutation(0)
     assert caught, f"mutation {mutation} passed every backward pin"
+
+
+def _pairs_only(x, Wr, br, g, W1, W2, dy, active):
+    """The layer's gradients with the expert terms restricted to the (token, expert) pairs in `active`
+    (fp64 numpy, written out per pair); the router part as in the chain rule."""
+    T, d = x.shape
+    E, de, _ = W1.shape
+    s = x @ Wr + br
+    a = np.maximum(s, 0.0)
+    rho = np.sqrt((a * a).mean(axis=1))
+    r = np.where(rho[:, None] > 0, g * a / np.where(rho > 0, rho, 1.0)[:, None], 0.0)
+    dx = np.zeros((T, d)); dW1 = np.zeros_like(W1); dW2 = np.zeros_like(W2); dr = np.zeros((T, E))
+    for t, e in zip(*np.nonzero(active)):
+        u = W1[e] @ x[t]
+        sg = 1.0 / (1.0 + np.exp(-u))
+        h = u * sg
+        q = W2[e].T @ dy[t]
+        dr[t, e] = h @ q
+        du = r[t, e] * q * (sg * (1.0 + u * (1.0 - sg)))
+        dW2[e] += np.outer(dy[t], r[t, e] * h)
+        dW1[e] += np.outer(du, x[t])
+        dx[t] += W1[e].T @ du
+    c = (dr * g * a).sum(axis=1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        da = np.where(rho[:, None] > 0, g * dr / rho[:, None] - a * (c / (E * rho ** 3))[:, None], 0.0)
+    dS = np.where(s > 0, da, 0.0)
+    dg = np.where(rho[:, None] > 0, dr * a / np.where(rho > 0, rho, 1.0)[:, None], 0.0).sum(axis=0)
+    return dict(dx=dx + dS @ Wr.T, dWr=x.T @ dS, db=dS.sum(axis=0), dg=dg, dW1=dW1, dW2=dW2)
+
+
+def test_active_pairs_reading_equals_dense_backward():
+    """Evaluating the expert terms only over the pairs with s > 0 gives the dense backward (the other pairs'
+    terms are exact zeros through a = 0): pinned against the oracle, including an expert with g = 0, where
+    a pair can have r = 0 while a > 0 and its dr still enters dg.  Restricting to r > 0 instead loses dg there."""
+    oracle.set_mutation(0)
+    x, Wr, br, g, W1, W2, dy = _case(11, T=7, d=10, E=6, de=5)
+    g = g.copy()
+    g[2] = 0.0
+    s = x @ Wr + br
+    assert ((s[:, 2] > 0)).any(), "the g = 0 expert must be active somewhere for this pin to bite"
+    ref = oracle.layer_backward(x, Wr, br, g, W1, W2, dy)
+    got = _pairs_only(x, Wr, br, g, W1, W2, dy, s > 0)
+    for k, v in got.items():
+        assert np.allclose(v, ref[k], rtol=1e-10, atol=1e-12 * max(1.0, np.abs(ref[k]).max())), k
+    a = np.maximum(s, 0.0)
+    rho = np.sqrt((a * a).mean(axis=1))
+    r = np.where(rho[:, None] > 0, g * a / np.where(rho > 0, rho, 1.0)[:, None], 0.0)
+    wrong = _pairs_only(x, Wr, br, g, W1, W2, dy, r > 0)
+    assert not np.allclose(wrong["dg"][2], ref["dg"][2])
