@@ -1066,6 +1066,77 @@ def run_reference(args, w):
     print(json.dumps(out), flush=True)
 
 
+def _reference_line(args, metric, config, units_per_step, step, sample, cores):
+    """Times `step` (one bounded sample of the workload through the oracle) --steps times after one warm-up
+    call and prints the reference arm's JSON line (tokens/s)."""
+    world = dist_env()[0]
+    step()
+    t0 = time.time()
+    for _ in range(args.steps):
+        step()
+    dt = time.time() - t0
+    value = args.steps * units_per_step / dt
+    out = {"metric": metric, "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+           "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+           "config": {**config, "tokens_per_step": units_per_step},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def run_reference_workload(args):
+    """The reference arm (the fp64 oracle on the host) for the workloads with their own runners: the
+    CLS-aware losses, the fp8 decode layer (the oracle's forward on the dequantised weights) and the layer
+    backward.  Rank 0 only; the same metric and config names as the GPU runner."""
+    if dist_env()[1] != 0:
+        return
+    import copy
+
+    import numpy as np
+
+    import gen
+    import oracle
+
+    cores = oracle.available_cores()
+    if args.workload == "cls_losses":
+        C, L, d, E, alpha = args.chunks or 4096, 8, 2048, 64, 4.0
+        lay = gen.make_layer(0, d, E, 8, beta=1.04, var_x=1.09)
+        m = 64
+        x_np = gen.make_chunks(0, lay, m, L, 0.3).reshape(m * L, d)
+        _reference_line(args, "CLS-aware losses + router backward tokens/s and achieved HBM GB/s over the step's I/O",
+                        {"workload": f"cls_losses_C{C}_L{L}_d{d}_E{E}", "tokens": C * L, "alpha": alpha}, m * L,
+                        lambda: oracle.cls_losses(x_np, m, L, lay.Wr, lay.br, alpha),
+                        f"each step: {m} chunks of {L} tokens, the fp64 oracle's losses and gradients (one core)", 1)
+    elif args.workload == "fp8":
+        w = gen.workload("decode")
+        lay = copy.copy(w.layer(0))
+        q1, q2, s1, s2, t2 = oracle.quantize_fp8(lay.W1, lay.W2, 1)
+        lay.W1, lay.W2 = oracle.dequantize_fp8(q1, q2, s1, s2, t2)
+        n = max(1, args.ref_chunks) * w.L
+        xs = gen.make_chunks(w.seed, lay, max(1, args.ref_chunks), w.L, w.noise, stream=0).reshape(-1, w.d)[:n]
+        _reference_line(args, METRIC + " (fp8 e4m3 expert weights)",
+                        {**w.describe(), "chunks_per_step": args.chunks or w.n_chunks}, n,
+                        lambda: oracle.tokens_forward_mt(xs, lay.Wr, lay.br, lay.g, lay.W1, lay.W2, cores),
+                        f"each step: {n} tokens, dense fp64 oracle on the dequantised fp8 weights "
+                        f"(all {w.E} experts per token)", cores)
+    elif args.workload == "backward":
+        C, L, d, E, de = args.chunks or 512, 8, 2048, 64, 256
+        lay = gen.make_layer(0, d, E, de, beta=0.84, var_x=1.09)
+        n = 4
+        x_np = gen.make_chunks(0, lay, 1, L, 0.3).reshape(L, d)[:n]
+        dy_np = np.random.default_rng(1).standard_normal((n, d)).astype(np.float32)
+        wf = lambda b: gen.bf16_bits_to_f32(b).astype(np.float64)
+        W1f, W2f, xf = wf(lay.W1), wf(lay.W2), wf(x_np)
+        _reference_line(args, "BlockFFN layer backward tokens/s and achieved TFLOP/s (over the active pairs)",
+                        {"workload": f"backward_T{C * L}_d{d}_E{E}_de{de}", "tokens": C * L}, n,
+                        lambda: oracle.layer_backward(xf, lay.Wr, lay.br, lay.g, W1f, W2f, dy_np),
+                        f"each step: {n} tokens, the fp64 oracle's backward (dense over the experts, one core)", 1)
+    else:
+        raise ValueError(args.workload)
+
+
 def launch_local_ranks(n: int, argv: list[str]) -> int:
     """Run this script as n ranks on this node (one process per GPU, rendezvous on 127.0.0.1) when it
     was started without a launcher; returns the launcher's exit status."""
@@ -1123,6 +1194,12 @@ def main():
         kw["replicas"] = args.replicas
     if args.workload == "tls_sweep" and args.impl == "ours" and not args.tls:
         run_tls_sweep(args)
+        return
+    if args.impl == "reference" and args.workload in ("cls_losses", "fp8", "backward"):
+        run_reference_workload(args)
+        return
+    if args.impl == "reference" and args.workload == "reuse":  # the reuse runs are the decode layer's forward
+        run_reference(args, gen.workload("decode"))
         return
     if args.workload == "reuse":
         run_reuse(args)

@@ -73,6 +73,28 @@ def test_clock_summary_parses_samples(tmp_path):
     assert s["reasons"] == ["sw_power_cap"] and s["samples"] == 3
 
 
+@pytest.mark.parametrize("workload,prefix", [("cls_losses", "cls_losses_"), ("fp8", "decode_"),
+                                             ("backward", "backward_")])
+def test_reference_arm_of_the_other_workloads(workload, prefix):
+    # the workloads with runners of their own time the oracle too, under the GPU runner's metric and config
+    import json
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--impl", "reference", "--workload",
+                          workload, "--steps", "1", "--warmup", "3"], capture_output=True, text=True, cwd=root,
+                         timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    assert j["impl"] == "reference" and j["value"] > 0 and j["cpu_baseline"]["kind"] == "oracle"
+    assert j["config"]["workload"].startswith(prefix)
+    assert j["e2e"]["h2d_bytes_per_step"] == 0
+
+
 def test_reference_arm_prints_the_contract_line():
     # bench.py --impl reference times the fp64 oracle on the host cores (no GPU) and prints one JSON
     # line with the benchmark's keys, its own CPU-baseline record and a host-only end-to-end figure
