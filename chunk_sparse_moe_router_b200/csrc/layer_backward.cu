@@ -47,10 +47,10 @@ constexpr int kPlain = 0, kPairs = 1, kTokens = 2;
 // Grouping: none; M is batch z's pair count (C rows are pair rows); K is batch z's pair count.
 constexpr int kNoGroup = 0, kGroupM = 1, kGroupK = 2;
 
-// C[m][n] (+)= sum_k A[m][k] B[k][n].  A K-major: A[m][k] = a[m lda + k]; else A[k][m] = a[k lda + m].
+// C[m][n] = sum_k A[m][k] B[k][n].  A K-major: A[m][k] = a[m lda + k]; else A[k][m] = a[k lda + m].
 // B K-major: B[k][n] = b[n ldb + k]; else b[k ldb + n].  ASPLIT / BSPLIT: the operand is hi + lo.  The stored
 // row (m or n of a K-major operand, k otherwise) goes through the operand's mode AMODE / BMODE.
-template <bool AK, bool ASPLIT, bool BK, bool BSPLIT, bool ADD, int AMODE, int BMODE, int GRP>
+template <bool AK, bool ASPLIT, bool BK, bool BSPLIT, int AMODE, int BMODE, int GRP>
 __global__ void __launch_bounds__(kT) gemm_kernel(const GemmArgs g) {
   extern __shared__ __align__(128) uint8_t smem[];
   constexpr int kParts = (ASPLIT ? 2 : 1) + (BSPLIT ? 2 : 1);
@@ -182,19 +182,19 @@ __global__ void __launch_bounds__(kT) gemm_kernel(const GemmArgs g) {
         for (int q = 0; q < 2; ++q) {
           if (n + q >= g.N) continue;
           float* p = C + crow * g.ldc + n + q;
-          *p = ADD ? *p + acc[mt][nt][2 * h + q] : acc[mt][nt][2 * h + q];
+          *p = acc[mt][nt][2 * h + q];
         }
       }
     }
 }
 
 // M (for kGroupM: the largest batch's pair count, at most T) sets the grid's row tiles.
-template <bool AK, bool ASPLIT, bool BK, bool BSPLIT, bool ADD, int AMODE = kPlain, int BMODE = kPlain,
+template <bool AK, bool ASPLIT, bool BK, bool BSPLIT, int AMODE = kPlain, int BMODE = kPlain,
           int GRP = kNoGroup>
 cudaError_t gemm(const GemmArgs& g, int batch, cudaStream_t st) {
   constexpr int kParts = (ASPLIT ? 2 : 1) + (BSPLIT ? 2 : 1);
   const int smem = kStages * kParts * kPart;
-  auto fn = gemm_kernel<AK, ASPLIT, BK, BSPLIT, ADD, AMODE, BMODE, GRP>;
+  auto fn = gemm_kernel<AK, ASPLIT, BK, BSPLIT, AMODE, BMODE, GRP>;
   cudaError_t err = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (err != cudaSuccess) return err;
   fn<<<dim3((g.N + kBN - 1) / kBN, (g.M + kBM - 1) / kBM, batch), kT, smem, st>>>(g);
@@ -486,23 +486,23 @@ cudaError_t launch(const __nv_bfloat16* x, int T, int d, const float* Wr, const 
   GemmArgs a{};
   // U_e = X[T_e] W1_e^T: pair rows [|T_e|, de]; X rows gathered, W1_e [de][d] (K-major)
   a = GemmArgs{x, nullptr, W1, nullptr, F(l.U), T, de, d, d, d, de, 0, (long long)de * d, 0, goff, tok};
-  if ((err = gemm<true, false, true, false, false, kTokens, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
+  if ((err = gemm<true, false, true, false, kTokens, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
   // Q_e = dY[T_e] W2_e: pair rows [|T_e|, de]; dY rows gathered, W2_e [d][de] (N-major)
   a = GemmArgs{dy_hi, dy_lo, W2, nullptr, F(l.Q), T, de, d, d, de, de, 0, (long long)d * de, 0, goff, tok};
-  if ((err = gemm<true, true, false, false, false, kTokens, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
+  if ((err = gemm<true, true, false, false, kTokens, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
   // h, dr, RH, DU per pair (one warp per possible pair; the warps past the pair count return)
   expert_pointwise_kernel<<<unsigned((P * 32 + 255) / 256), 256, 0, st>>>(F(l.U), F(l.Q), F(l.r), tok, I(l.pexp),
                                                                           goff, E, de, F(l.dr), rh_hi, rh_lo, du_hi,
                                                                           du_lo);
   // dW2_e = dY[T_e]^T RH_e: [d, de]; A = dY (M-major, rows k gathered), B = RH_e (N-major pair rows)
   a = GemmArgs{dy_hi, dy_lo, rh_hi, rh_lo, dW2, d, de, 0, d, de, de, 0, 0, (long long)d * de, goff, tok};
-  if ((err = gemm<false, true, false, true, false, kTokens, kPairs, kGroupK>(a, E, st)) != cudaSuccess) return err;
+  if ((err = gemm<false, true, false, true, kTokens, kPairs, kGroupK>(a, E, st)) != cudaSuccess) return err;
   // dW1_e = DU_e^T X[T_e]: [de, d]; A = DU_e (M-major pair rows), B = X (N-major, rows k gathered)
   a = GemmArgs{du_hi, du_lo, x, nullptr, dW1, de, d, 0, de, d, d, 0, 0, (long long)de * d, goff, tok};
-  if ((err = gemm<false, true, false, false, false, kPairs, kTokens, kGroupK>(a, E, st)) != cudaSuccess) return err;
+  if ((err = gemm<false, true, false, false, kPairs, kTokens, kGroupK>(a, E, st)) != cudaSuccess) return err;
   // the expert terms of dX per pair: DU_e W1_e, [|T_e|, d]; A = DU_e (K-major pair rows), B = W1_e [de][d]
   a = GemmArgs{du_hi, du_lo, W1, nullptr, F(l.xp), T, d, de, de, d, d, 0, (long long)de * d, 0, goff, tok};
-  if ((err = gemm<true, true, false, false, false, kPairs, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
+  if ((err = gemm<true, true, false, false, kPairs, kPlain, kGroupM>(a, E, st)) != cudaSuccess) return err;
   // router backward
   router_bwd_kernel<<<(T + 7) / 8, 256, 0, st>>>(F(l.s), F(l.rho), F(l.dr), g, T, E, Ep, F(l.ds), F(l.dgc), ds_hi,
                                                  ds_lo);
@@ -510,10 +510,10 @@ cudaError_t launch(const __nv_bfloat16* x, int T, int d, const float* Wr, const 
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   // dWr = X^T dS: [d, E], A = X (M-major), B = dS [T][Ep] (N-major)
   a = GemmArgs{x, nullptr, ds_hi, ds_lo, dWr, d, E, T, d, Ep, E, 0, 0, 0, nullptr, nullptr};
-  if ((err = gemm<false, false, false, true, false>(a, 1, st)) != cudaSuccess) return err;
+  if ((err = gemm<false, false, false, true>(a, 1, st)) != cudaSuccess) return err;
   // dX = dS Wr^T: [T, d], A = dS [T][Ep] (K-major), B = Wr as [d][Ep] (K-major); then the pairs' terms
   a = GemmArgs{ds_hi, ds_lo, wsplit, wsplit + size_t(d) * Ep, dx, T, d, Ep, Ep, Ep, d, 0, 0, 0, nullptr, nullptr};
-  if ((err = gemm<true, true, true, true, false>(a, 1, st)) != cudaSuccess) return err;
+  if ((err = gemm<true, true, true, true>(a, 1, st)) != cudaSuccess) return err;
   pair_reduce_kernel<<<T, 256, size_t(E) * 4, st>>>(F(l.xp), I(l.pidx), T, E, d, dx);
   return cudaGetLastError();
 }
