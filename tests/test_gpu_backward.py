@@ -90,3 +90,19 @@ def test_layer_backward_expert_never_and_always_active(bffn, cuda_device):
         assert np.all(got[k][0] == 0.0)
     assert got["db"][0] == 0.0 and got["dg"][0] == 0.0
     _compare(got, _ref(lay, x, dy))
+
+
+def test_layer_backward_zero_gain(bffn, cuda_device):
+    """An expert with gain g = 0: its pairs have r = 0 while a > 0, so they pass no expert gradient but
+    their dr still enters dg (the pairs are grouped by s > 0, not by r > 0)."""
+    lay, x, dy = _case(13, 64, 128, 16, 32)
+    lay.g = lay.g.copy()
+    lay.g[3] = 0.0
+    s = gen.bf16_bits_to_f32(x).astype(np.float64) @ lay.Wr.astype(np.float64) + lay.br
+    assert (s[:, 3] > 0).any()
+    got = _run(bffn, lay, x, dy)
+    ref = _ref(lay, x, dy)
+    assert ref["dg"][3] != 0.0
+    for k in ("dW1", "dW2"):
+        assert np.all(got[k][3] == 0.0)
+    _compare(got, ref)
