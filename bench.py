@@ -632,6 +632,65 @@ def run_tls_sweep(args):
 
 
 # ---------------------------------------------------------------------------------- cross-chunk reuse
+def run_dense_ffn(args):
+    """The sweep's comparison point in a library: a dense FFN of the stacked model's shape (--replicas
+    layers, default 32, of d = 4096 and E de = 32768 hidden units, 17.2 GB of bf16 weights) as plain cuBLAS
+    bf16 GEMMs through torch, one chunk of L = 8 tokens at a time, 8 chunks per layer per step, as the sweep
+    visits them: y = Swish(x W1^T) W2^T.  Random weights (their values do not change the time); HBM-bound
+    like the sweep, so the line reports tokens/s and GB/s over the weight bytes."""
+    import torch
+
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    R, d, H, L = args.replicas or 32, 4096, 128 * 256, 8
+    per_layer = 8
+    gen_t = torch.Generator(device=device).manual_seed(0)
+    W1 = torch.randn((R, H, d), dtype=torch.bfloat16, device=device, generator=gen_t).mul_(d ** -0.5)
+    W2 = torch.randn((R, d, H), dtype=torch.bfloat16, device=device, generator=gen_t).mul_(256 ** -0.5)
+    x = torch.randn((R * per_layer, L, d), dtype=torch.bfloat16, device=device, generator=gen_t)
+    y = torch.empty_like(x)
+    s = torch.cuda.Stream(device)
+
+    def step():
+        for c in range(R * per_layer):
+            l = c % R
+            y[c] = torch.nn.functional.silu(x[c] @ W1[l].t()) @ W2[l].t()
+
+    with torch.cuda.stream(s):
+        step()
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        graph.capture_begin()
+        step()
+        graph.capture_end()
+        for _ in range(args.warmup):
+            graph.replay()
+        s.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(0) as clocks:
+            e0.record(s)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(s)
+            e1.synchronize()
+        del graph
+    ms = e0.elapsed_time(e1) / args.steps
+    chunks = R * per_layer
+    bytes_step = chunks * (2 * H * d * 2 + L * d * 2 * 2)
+    peak, peak_kind = measured_peaks()
+    gbs = bytes_step / (ms * 1e-3) / 1e9
+    line = {"metric": "dense FFN (cuBLAS bf16 through torch) tokens/s at chunk L=8, the stacked model's shape",
+            "value": round(chunks * L / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (random weights)",
+            "config": {"workload": f"dense_ffn_layers{R}_d{d}_hidden{H}_L{L}", "chunks_per_step": chunks,
+                       "l2": f"inputs larger than L2: {R * 2 * H * d * 2 / 1e9:.1f} GB of weights"},
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": peak_kind, "traffic": None},
+            "gpu_launches": 0, "library": "cuBLAS (torch.matmul) and a torch SiLU kernel", "clocks": clocks.summary()}
+    print(json.dumps(line), flush=True)
+
+
 def run_reuse(args):
     """Cross-chunk expert reuse on the per-chunk path (one chunk at a time on the whole GPU): the
     consecutive verification chunks of one sequence, as a drifting sequence of chunk bases (gen's
@@ -1157,7 +1216,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="decode",
-                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses", "fp8", "backward"])
+                    choices=["decode", "tiny", "lsweep", "tls_sweep", "prefill", "reuse", "cls_losses", "fp8", "backward",
+                             "dense_ffn"])
     ap.add_argument("--drift", default="0.0,0.9,0.97",
                     help="--workload reuse: drift of the chunk bases of a sequence (0: independent chunks)")
     ap.add_argument("--L", type=int, default=None, help="chunk length for --workload lsweep")
@@ -1200,6 +1260,13 @@ def main():
         return
     if args.impl == "reference" and args.workload == "reuse":  # the reuse runs are the decode layer's forward
         run_reference(args, gen.workload("decode"))
+        return
+    if args.workload == "dense_ffn":
+        if args.impl == "reference":
+            print(json.dumps({"impl": "reference", "unavailable": "the dense cuBLAS FFN is itself a comparison "
+                              "point; its oracle is the decode layer's (--workload tls_sweep --impl reference)"}))
+            return
+        run_dense_ffn(args)
         return
     if args.workload == "reuse":
         run_reuse(args)
